@@ -1,0 +1,354 @@
+"""Pins for the fp64 oracle: brute force, closed forms and the pages' invariants.
+
+None of these compares the oracle with a retyped copy of itself.  Each check is
+chosen so that a plausible slip (a dropped term, a sign, a swapped index or
+operand, head/tail order, target/candidate order) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as orc
+import synthetic as sy
+from tests import bruteforce as bf
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _tiny_inputs(seed, B=2, N=10, S=3, d=5):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((B, N, d))
+
+
+# ------------------------------------------------------------------ MaxSim --
+
+def test_maxsim_hand_example():
+    """Hand-derived MaxSim values on axis-aligned vectors (tests/golden)."""
+    g = json.load(open(os.path.join(GOLD, "maxsim_axes.json")))
+    X = np.array(g["X"], dtype=np.float64)[None]
+    S = g["S"]
+    _, scores, idx, w = orc.rank(X, S, g["k"])
+    # Expected values derived by hand (see the fixture's "derivation").
+    expect = np.array([[2.0, 1.0, 1.4, 0.0],
+                       [1.0, 2.0, 0.6, 0.0],
+                       [0.8, 0.6, 2.0, 0.0],
+                       [0.0, 0.0, 0.0, 1.0]])
+    np.testing.assert_allclose(scores, expect, atol=1e-12)
+    assert idx.tolist() == [[2, 1], [0, 2], [0, 1], [0, 1]]
+    np.testing.assert_allclose(w, [[1.0, 1.0 / 1.4], [1.0, 0.6], [1.0, 0.75], [0.0, 0.0]],
+                               atol=1e-12)
+
+
+@pytest.mark.parametrize("seed,N,S", [(0, 10, 3), (1, 12, 4), (2, 7, 2), (3, 9, 1)])
+def test_maxsim_matches_bruteforce(seed, N, S):
+    X = _tiny_inputs(seed, N=N, S=S)
+    B = X.shape[0]
+    n = -(-N // S)
+    ref = bf.maxsim_matrix(X.tolist(), S)
+    got = orc.maxsim_rows(X, S, orc.all_targets(B, n)).reshape(B, n, n)
+    np.testing.assert_allclose(got, np.array(ref), rtol=1e-12, atol=1e-12)
+
+
+def test_maxsim_s1_is_cosine_matrix():
+    """With S = 1 each split is one token, so MaxSim is the cosine matrix."""
+    X = _tiny_inputs(4, B=1, N=9, d=6)
+    got = orc.maxsim_rows(X, 1, orc.all_targets(1, 9))
+    Xn = X[0] / np.linalg.norm(X[0], axis=1, keepdims=True)
+    np.testing.assert_allclose(got, Xn @ Xn.T, atol=1e-12)
+
+
+def test_maxsim_is_asymmetric_in_the_right_direction():
+    """score(t, c) sums over the rows of t and maximises over the rows of c."""
+    # t = split 0: two identical rows e1; c = split 1: rows e1 and e2.
+    X = np.array([[[1, 0], [1, 0], [1, 0], [0, 1]]], dtype=np.float64)
+    sc = orc.maxsim_rows(X, 2, orc.all_targets(1, 2))
+    assert sc[0, 1] == pytest.approx(2.0)   # each row of t finds e1 in c
+    assert sc[1, 0] == pytest.approx(1.0)   # e1 finds e1, e2 finds only cos 0
+
+
+def test_planted_duplicate_scores_exactly_S_and_ranks_first():
+    w = sy.custom(B=2, N=64 * 16, S=64, d=48, k=3, centers=4, sigma=0.5, dup_frac=0.15)
+    E = sy.gen_embeddings(w)
+    must = [(b, t) for b in range(w.B) for t, _ in E.dup_pairs[b]]
+    sel = np.array(must, dtype=np.int32)
+    _, scores, idx, wt = orc.rank(E.X, w.S, w.k, sel)
+    for r, (b, t) in enumerate(must):
+        src = dict(E.dup_pairs[b])[t]
+        assert scores[r, src] == pytest.approx(w.S, abs=1e-9)
+        assert idx[r, 0] == src and wt[r, 0] == 1.0
+
+
+# ------------------------------------------------------------------- top-k --
+
+@pytest.mark.parametrize("seed", range(4))
+def test_topk_matches_full_sort(seed):
+    rng = np.random.default_rng(seed)
+    n, k = 23, 5
+    scores = rng.standard_normal((n, n)) + 3.0
+    scores[:, 7] = scores[:, 3]  # exact ties -> lower index first
+    idx, w = orc.topk(scores, np.arange(n), k)
+    for t in range(n):
+        order = sorted((c for c in range(n) if c != t), key=lambda c: (-scores[t, c], c))
+        assert idx[t].tolist() == order[:k]
+        assert t not in idx[t]
+        assert w[t, 0] == 1.0
+        assert np.all(w[t] <= 1.0) and np.all(w[t] > 0.0)
+        np.testing.assert_allclose(w[t], scores[t, order[:k]] / scores[t, order[0]], rtol=1e-15)
+
+
+def test_topk_all_others_when_k_is_n_minus_1():
+    rng = np.random.default_rng(5)
+    n = 9
+    scores = rng.random((n, n)) + 0.5
+    idx, _ = orc.topk(scores, np.arange(n), n - 1)
+    for t in range(n):
+        assert sorted(idx[t].tolist()) == [c for c in range(n) if c != t]
+
+
+def test_topk_short_candidate_list_pads():
+    scores = np.array([[5.0, 2.0, 1.0]])
+    idx, w = orc.topk(scores, [0], 4)
+    assert idx.tolist() == [[1, 2, -1, -1]]
+    np.testing.assert_allclose(w, [[1.0, 0.5, 0.0, 0.0]])
+
+
+# ------------------------------------------------------------- compression --
+
+def test_compress_hand_example():
+    g = json.load(open(os.path.join(GOLD, "maxsim_axes.json")))
+    X = np.array(g["X"], dtype=np.float64)[None]
+    S, k = g["S"], g["k"]
+    P = np.array(g["P"], dtype=np.float64)
+    sel, _, idx, w = orc.rank(X, S, k)
+    out = orc.compress(X, S, k, sel, idx, w, P)
+    wt = 1.0 / 1.4  # weight of split 1 for target 0 (derived in the fixture)
+    np.testing.assert_allclose(out[0], [[4 + wt / 2, 0, -2], [0, 4.5, -5 * wt]], atol=1e-12)
+
+
+def test_compress_identity_and_zero_P():
+    X = _tiny_inputs(6, B=1, N=12, S=3)
+    S, k = 3, 2
+    sel, _, idx, w = orc.rank(X, S, k)
+    P_id = np.zeros((S, (k + 1) * S))
+    P_id[:, :S] = np.eye(S)
+    xt = X[0].reshape(4, S, -1)
+    np.testing.assert_allclose(orc.compress(X, S, k, sel, idx, w, P_id), 2 * xt, atol=1e-12)
+    np.testing.assert_allclose(orc.compress(X, S, k, sel, idx, w, 0 * P_id), xt, atol=1e-15)
+
+
+def test_compress_is_linear_in_the_weights_and_picks_the_ranked_blocks():
+    X = _tiny_inputs(7, B=1, N=12, S=3)
+    S, k = 3, 2
+    sel, _, idx, w = orc.rank(X, S, k)
+    P = np.zeros((S, (k + 1) * S))
+    P[:, 2 * S:3 * S] = np.eye(S)  # select exactly the rank-2 block
+    out = orc.compress(X, S, k, sel, idx, w, P)
+    xt = X[0].reshape(4, S, -1)
+    for s in range(4):
+        c2 = idx[s, 1]
+        np.testing.assert_allclose(out[s], xt[s] + w[s, 1] * xt[c2], atol=1e-12)
+    out2 = orc.compress(X, S, k, sel, idx, 2 * w, P)
+    np.testing.assert_allclose(out2 - xt, 2 * (out - xt), atol=1e-12)
+
+
+def test_compress_matches_bruteforce_with_padding():
+    X = _tiny_inputs(8, B=2, N=10, S=3)
+    S, k = 3, 2
+    rng = np.random.default_rng(9)
+    P = rng.standard_normal((S, (k + 1) * S))
+    sel, _, idx, w = orc.rank(X, S, k)
+    got = orc.compress(X, S, k, sel, idx, w, P)
+    for r, (b, t) in enumerate(sel.tolist()):
+        ref = bf.compress(X.tolist(), S, k, b, t, idx[r].tolist(), w[r].tolist(), P.tolist())
+        np.testing.assert_allclose(got[r], np.array(ref), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------- the mixes --
+
+def test_static_mix_identity_and_permutation():
+    rng = np.random.default_rng(10)
+    zt = rng.random((5, 7))
+    np.testing.assert_allclose(orc.static_mix(np.eye(5), zt), zt, atol=0)
+    perm = np.eye(5)[[3, 0, 4, 1, 2]]
+    np.testing.assert_allclose(orc.static_mix(perm, zt), zt[[3, 0, 4, 1, 2]], atol=0)
+
+
+def test_dynamic_mix_hand_example():
+    """z1 = (1, 0), z2 = (1, 1): G = [[1, r], [r, 1]] with r = 1/sqrt 2; eps = 0."""
+    zt = np.array([[1.0, 0.0], [1.0, 1.0]])
+    c = orc.dynamic_mix(zt, 0.0)
+    s2 = math.sqrt(2.0)
+    np.testing.assert_allclose(c, [[1.0, s2 - 1.0], [1.0, 2.0 - s2]], atol=1e-15)
+
+
+def test_dynamic_rows_sum_to_one_when_positive():
+    """Eq. 6 makes each row sum to sum_j G_ij / (sum_j G_ij + eps) < 1, ~1."""
+    rng = np.random.default_rng(11)
+    eps = 1e-8
+    zt = rng.random((16, 24)) ** 2
+    Gt = orc.dynamic_weights(zt, eps)
+    rs = Gt.sum(axis=1)
+    assert np.all(rs < 1.0) and np.all(rs > 1.0 - 2 * eps)
+    assert np.all(Gt >= 0)
+    # G_ii = 1, so Gt_ii = 1 / (sum_j G_ij + eps) and the row sum is 1 - eps * Gt_ii
+    np.testing.assert_allclose(rs, 1.0 - eps * np.diag(Gt), rtol=0, atol=1e-15)
+    # ones column: c[:, -1] is the row sum of Gt
+    zt1 = np.concatenate([zt, np.ones((16, 1))], axis=1)
+    c = orc.dynamic_mix(zt1, eps)
+    np.testing.assert_allclose(c[:, -1], orc.dynamic_weights(zt1, eps).sum(1), rtol=1e-14)
+    assert np.all(np.abs(c[:, -1] - 1.0) < 2 * eps)
+
+
+def test_dynamic_identical_tokens_uniform():
+    z = np.random.default_rng(12).random(9) + 0.1
+    zt = np.tile(z, (6, 1))
+    eps = 1e-8
+    np.testing.assert_allclose(orc.dynamic_weights(zt, eps), np.full((6, 6), 1.0 / (6 + eps)),
+                               rtol=1e-14)
+    np.testing.assert_allclose(orc.dynamic_mix(zt, eps), np.tile(z * 6 / (6 + eps), (6, 1)),
+                               rtol=1e-14)
+
+
+def test_dynamic_zero_row_gets_zero_weights():
+    zt = np.array([[0.0, 0.0], [1.0, 2.0], [2.0, 1.0]])
+    Gt = orc.dynamic_weights(zt, 1e-8)
+    assert np.all(Gt[0] == 0.0) and np.all(Gt[:, 0] == 0.0)
+
+
+def test_dynamic_monotonicity_appendix_a():
+    """App. A: raising one token's similarity to the target raises its own
+    normalised weight and does not raise any other token's weight."""
+    rng = np.random.default_rng(13)
+    for _ in range(20):
+        zt = rng.random((6, 5)) ** 2
+        G0 = orc.dynamic_weights(zt, 1e-8)
+        # Move token 3 toward token 0 (target): its cosine to token 0 rises.
+        z2 = zt.copy()
+        z2[3] = 0.5 * z2[3] + 0.5 * z2[0] * (np.linalg.norm(z2[3]) / np.linalg.norm(z2[0]))
+        G1 = orc.dynamic_weights(z2, 1e-8)
+        u = zt / np.linalg.norm(zt, axis=1, keepdims=True)
+        u2 = z2 / np.linalg.norm(z2, axis=1, keepdims=True)
+        assert u2[3] @ u2[0] > u[3] @ u[0]
+        assert G1[0, 3] > G0[0, 3]
+        others = [j for j in range(6) if j != 3]
+        # the other raw similarities of row 0 are unchanged, so their weights fall
+        assert np.all(G1[0, others] <= G0[0, others] + 1e-15)
+
+
+def test_static_layer_gain_preserves_ratio_fig1a():
+    """Fig. 1(a) discussion: a static gain w scales both contributions, so
+    |w s21| / |w s31| = s21 / s31 (the order set by the similarities holds)."""
+    zt = np.array([[1.0, 0.2], [0.9, 0.3], [0.1, 1.0]])
+    Gt = orc.dynamic_weights(zt, 0.0)
+    s21, s31 = Gt[0, 1], Gt[0, 2]
+    assert s21 > s31
+    for wgain in (-3.0, -0.5, 0.7, 2.0):
+        V = wgain * np.eye(3)
+        c = orc.static_mix(V, Gt)  # static layer applied to the similarity rows
+        assert abs(c[0, 1]) / abs(c[0, 2]) == pytest.approx(s21 / s31, rel=1e-12)
+
+
+# ------------------------------------------------------------------ layers --
+
+def _layer_weights(rng, d, m, S, kind):
+    U = rng.standard_normal((d, m)) / math.sqrt(d)
+    bU = rng.standard_normal(m) / math.sqrt(d)
+    V = rng.standard_normal((S, S)) / math.sqrt(S) if kind == sy.STATIC else None
+    O = rng.standard_normal((m, d)) / math.sqrt(m)
+    return sy.LayerWeights(kind, U, bU, V, O)
+
+
+def test_layer_closed_form_one_token():
+    """x = (1, 2), U = [[1,0,1,1],[0,1,1,0]], b = (0,0,0.5,-1): Z = (1, 4, 12.25, 0);
+    S = 1 dynamic with eps = 0 keeps c = Z_t; O rows (1,0),(0,1),(1,1),(0,-1)."""
+    x = np.array([[[1.0, 2.0]]])
+    U = np.array([[1.0, 0.0, 1.0, 1.0], [0.0, 1.0, 1.0, 0.0]])
+    bU = np.array([0.0, 0.0, 0.5, -1.0])
+    O = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0], [0.0, -1.0]])
+    lw = sy.LayerWeights(sy.DYNAMIC, U, bU, None, O)
+    out = orc.layer(x, lw, 1, 2, 0.0, False)
+    # [Z_h || c] O = 1*(1,0) + 4*(0,1) + 12.25*(1,1) + 0*(0,-1) = (13.25, 16.25)
+    np.testing.assert_allclose(out[0, 0], [1 + 13.25, 2 + 16.25], atol=1e-12)
+    # head/tail order matters: static V = [[2]] doubles only the tail part
+    lw_s = sy.LayerWeights(sy.STATIC, U, bU, np.array([[2.0]]), O)
+    out_s = orc.layer(x, lw_s, 1, 2, 0.0, False)
+    np.testing.assert_allclose(out_s[0, 0], [1 + 1 + 24.5, 2 + 4 + 24.5], atol=1e-12)
+
+
+def test_layer_prenorm_closed_form():
+    """prenorm divides the enricher input by sqrt(mean(x^2) + 1e-6) only."""
+    x = np.array([[[3.0, 4.0]]])
+    r = math.sqrt((9 + 16) / 2 + 1e-6)
+    U = np.array([[1.0, 0.0], [0.0, 1.0]])
+    O = np.array([[1.0, 0.0], [0.0, 0.0]])
+    lw = sy.LayerWeights(sy.STATIC, U, np.zeros(2), np.array([[1.0]]), O)
+    out = orc.layer(x, lw, 1, 1, 0.0, True)
+    np.testing.assert_allclose(out[0, 0], [3.0 + (3.0 / r) ** 2, 4.0], rtol=1e-14)
+
+
+@pytest.mark.parametrize("kind", [sy.STATIC, sy.DYNAMIC])
+@pytest.mark.parametrize("prenorm", [False, True])
+def test_layer_matches_bruteforce(kind, prenorm):
+    rng = np.random.default_rng(20 + kind + 2 * prenorm)
+    S, d, m, m_h = 4, 5, 7, 3  # m_h != m_t, d != m != S: catches swapped operands
+    x = rng.standard_normal((3, S, d))
+    lw = _layer_weights(rng, d, m, S, kind)
+    got = orc.layer(x, lw, S, m_h, 1e-8, prenorm)
+    for sp in range(3):
+        ref = bf.layer(x[sp].tolist(), lw.U.tolist(), lw.bU.tolist(),
+                       None if lw.V is None else lw.V.tolist(), lw.O.tolist(), m_h, kind, 1e-8,
+                       prenorm)
+        np.testing.assert_allclose(got[sp], np.array(ref), rtol=1e-11, atol=1e-11)
+
+
+def test_layer_splits_are_independent():
+    """The processor treats each split independently (papernotes 关键设计 4)."""
+    rng = np.random.default_rng(30)
+    S, d, m = 4, 6, 8
+    x = rng.standard_normal((3, S, d))
+    lw = _layer_weights(rng, d, m, S, sy.DYNAMIC)
+    full = orc.layer(x, lw, S, 4, 1e-8, False)
+    x2 = x.copy()
+    x2[1] += 5.0
+    part = orc.layer(x2, lw, S, 4, 1e-8, False)
+    np.testing.assert_allclose(full[[0, 2]], part[[0, 2]], atol=0)
+
+
+def test_forward_matches_bruteforce_end_to_end():
+    w = sy.custom(B=2, N=22, S=4, d=6, m=8, m_h=3, k=2, pattern=(sy.STATIC, sy.DYNAMIC),
+                  dtype="f32", centers=3, sigma=0.4)
+    E = sy.gen_embeddings(w)
+    W = sy.gen_weights(w)
+    res = orc.forward(E.X, W, w)
+    Xl = E.X.astype(np.float64).tolist()
+    sc = bf.maxsim_matrix(Xl, w.S)
+    for r, (b, t) in enumerate(res["sel"].tolist()):
+        np.testing.assert_allclose(res["scores"][r], sc[b][t], rtol=1e-12, atol=1e-12)
+        idx, wt = bf.topk(sc[b][t], t, w.k)
+        assert res["idx"][r].tolist() == idx
+        x = bf.compress(Xl, w.S, w.k, b, t, idx, wt, W.P.astype(np.float64).tolist())
+        for lw in W.layers:
+            x = bf.layer(x, lw.U.tolist(), lw.bU.tolist(),
+                         None if lw.V is None else lw.V.tolist(), lw.O.tolist(), w.m_h, lw.kind,
+                         w.eps, w.prenorm)
+        np.testing.assert_allclose(res["layers"][-1][r], np.array(x), rtol=1e-10, atol=1e-10)
+
+
+def test_large_stack_needs_prenorm():
+    """The literal residual stack overflows within 12 layers at the large
+    workload's shapes; the prenorm reading keeps it finite."""
+    w = sy.WORKLOADS["large_bf16"]
+    W = sy.gen_weights(w)
+    x = np.random.default_rng(0).standard_normal((1, w.S, w.d))
+    with np.errstate(over="ignore", invalid="ignore"):
+        a = x.copy()
+        for lw in W.layers:
+            a = orc.layer(a, lw, w.S, w.m_h, w.eps, False)
+        assert not np.all(np.isfinite(a))
+    b = x.copy()
+    for lw in W.layers:
+        b = orc.layer(b, lw, w.S, w.m_h, w.eps, True)
+    assert np.all(np.isfinite(b)) and np.sqrt((b ** 2).mean()) < 100
