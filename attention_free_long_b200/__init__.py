@@ -1,0 +1,331 @@
+"""Python binding of libavey.so, the B200 (sm_100a) Avey-B ranker and
+neural-processor library.
+
+This module only marshals arguments: it takes torch CUDA tensors, allocates
+outputs and workspaces with torch (device memory and streams are all torch is
+used for), and calls the C ABI declared in ``include/avey.h`` on the current
+CUDA stream.  Every step of the computation runs in the library's kernels.
+There is no fallback: if ``libavey.so`` is missing, importing the functions
+raises.
+
+Entry points (same names as the C ABI):
+  avey_rank          MaxSim split scores -> top-k indices + divide-by-max weights
+  avey_compress      eq. 8 neural compression with residual
+  avey_dynamic_mix   eq. 6 row-normalised cosine mix of split blocks
+  avey_layer_forward enricher -> static/dynamic mix -> fuser + residual
+and ``encoder_forward`` which strings them together (ranker once, then every
+layer), the call a user of the encoder makes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import List, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libavey.so")
+
+AVEY_F32, AVEY_BF16, AVEY_BF16X2 = 0, 1, 2
+AVEY_STATIC, AVEY_DYNAMIC = 0, 1
+STATUS = {0: "AVEY_OK", 1: "AVEY_ERR_INVALID_ARG", 2: "AVEY_ERR_UNSUPPORTED", 3: "AVEY_ERR_CUDA",
+          4: "AVEY_ERR_DEVICE_TIMEOUT", 5: "AVEY_ERR_DEVICE_BOUNDS"}
+
+_lib = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+
+
+class AveyError(RuntimeError):
+    def __init__(self, fn: str, code: int, detail: str):
+        super().__init__(f"{fn}: {STATUS.get(code, code)}: {detail}")
+        self.code = code
+
+
+class LayerParams(ctypes.Structure):
+    _fields_ = [("kind", _i), ("d", _i), ("m", _i), ("m_h", _i), ("S", _i), ("eps", ctypes.c_float),
+                ("prenorm", _i), ("Ut", _vp), ("bU", _vp), ("V", _vp), ("Ot", _vp)]
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libavey.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              f"`python -m attention_free_long_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.avey_rank.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.avey_rank.restype = _i
+        L.avey_rank_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+        L.avey_rank_workspace_bytes.restype = _sz
+        L.avey_compress.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.avey_compress.restype = _i
+        L.avey_dynamic_mix.argtypes = [_vp, _i64, _i, _i, _i, _i, ctypes.c_float, _vp, _i64, _vp]
+        L.avey_dynamic_mix.restype = _i
+        L.avey_layer_forward.argtypes = [ctypes.POINTER(LayerParams), _i, _i, _vp, _vp, _vp, _vp,
+                                         _vp, _sz, _vp]
+        L.avey_layer_forward.restype = _i
+        L.avey_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+        L.avey_layer_workspace_bytes.restype = _sz
+        L.avey_device_status.argtypes = [_vp]
+        L.avey_device_status.restype = _i
+        L.avey_status_string.argtypes = [_i]
+        L.avey_status_string.restype = ctypes.c_char_p
+        L.avey_last_error_detail.argtypes = []
+        L.avey_last_error_detail.restype = ctypes.c_char_p
+        L.avey_kernel_launches.argtypes = []
+        L.avey_kernel_launches.restype = ctypes.c_uint64
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, code: int) -> None:
+    if code != 0:
+        raise AveyError(fn, code, lib().avey_last_error_detail().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return AVEY_F32
+    if t.dtype == torch.bfloat16:
+        return AVEY_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need(t: torch.Tensor, name: str):
+    if not (t.is_cuda and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def kernel_launches() -> int:
+    return int(lib().avey_kernel_launches())
+
+
+def device_status(stream=None) -> int:
+    s = _stream() if stream is None else ctypes.c_void_p(stream)
+    return int(lib().avey_device_status(s))
+
+
+# ------------------------------------------------------------------ ranker --
+
+def rank_workspace_bytes(dtype: int, B: int, N: int, d: int, S: int) -> int:
+    return int(lib().avey_rank_workspace_bytes(dtype, B, N, d, S))
+
+
+def avey_rank(x: torch.Tensor, S: int, k: int, return_scores: bool = False,
+              ws: Optional[torch.Tensor] = None):
+    """x [B, N, d] fp32 or bf16 -> (idx int32 [B, n, k], w fp32 [B, n, k][, scores])."""
+    _need(x, "x")
+    B, N, d = x.shape
+    n = -(-N // S)
+    dt = _dt(x)
+    idx = torch.empty((B, n, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((B, n, k), dtype=torch.float32, device=x.device)
+    scores = torch.empty((B, n, n), dtype=torch.float32, device=x.device) if return_scores else None
+    need = rank_workspace_bytes(dt, B, N, d, S)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, x.device)
+    _check("avey_rank", lib().avey_rank(_ptr(x), dt, B, N, d, S, k, _ptr(idx), _ptr(w),
+                                        _ptr(scores), _ptr(ws), ws.numel(), _stream()))
+    return (idx, w, scores) if return_scores else (idx, w)
+
+
+# ------------------------------------------------------------- compression --
+
+def avey_compress(x: torch.Tensor, S: int, k: int, idx: torch.Tensor, w: torch.Tensor,
+                  P: torch.Tensor, out: Optional[torch.Tensor] = None, lowp: bool = True):
+    """eq. 8 compression + residual.  Returns (out fp32 [B, n*S, d], pair or None).
+
+    For bf16 inputs the pair is the split activation [2, B*n*S, d] bf16.
+    """
+    for t, nm in ((x, "x"), (idx, "idx"), (w, "w"), (P, "P")):
+        _need(t, nm)
+    B, N, d = x.shape
+    n = -(-N // S)
+    dt = _dt(x)
+    if P.dtype != x.dtype:
+        raise TypeError("P must have the dtype of x")
+    if out is None:
+        out = torch.empty((B, n * S, d), dtype=torch.float32, device=x.device)
+    pair = None
+    if dt == AVEY_BF16 and lowp:
+        pair = torch.empty((2, B * n * S, d), dtype=torch.bfloat16, device=x.device)
+    _check("avey_compress", lib().avey_compress(_ptr(x), dt, B, N, d, S, k, _ptr(idx), _ptr(w),
+                                                _ptr(P), _ptr(out), _ptr(pair), _stream()))
+    return out, pair
+
+
+# ------------------------------------------------------------- dynamic mix --
+
+def avey_dynamic_mix(zt: torch.Tensor, S: int, eps: float, mt: Optional[int] = None,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Dynamic contextualizer on split blocks.
+
+    zt: fp32 [rows, ld] or a bf16 split pair [2, rows, ld]; rows = blocks * S;
+    the first ``mt`` (default ld) columns are mixed.  Returns out (same layout).
+    """
+    _need(zt, "zt")
+    if zt.dtype == torch.float32:
+        dt, rows, ld = AVEY_F32, zt.shape[0], zt.shape[1]
+    elif zt.dtype == torch.bfloat16 and zt.dim() == 3 and zt.shape[0] == 2:
+        dt, rows, ld = AVEY_BF16X2, zt.shape[1], zt.shape[2]
+    else:
+        raise TypeError("zt must be fp32 [rows, ld] or a bf16 pair [2, rows, ld]")
+    mt = ld if mt is None else mt
+    if out is None:
+        out = torch.empty_like(zt)
+    _need(out, "out")
+    _check("avey_dynamic_mix", lib().avey_dynamic_mix(_ptr(zt), ld, dt, rows // S, S, mt, eps,
+                                                      _ptr(out), out.shape[-1], _stream()))
+    return out
+
+
+# ------------------------------------------------------------------ layer --
+
+@dataclass
+class DeviceLayer:
+    """Device copies of one layer's weights in the layout the library takes."""
+    kind: int
+    Ut: torch.Tensor  # [m, d] (U transposed), bf16 or fp32
+    bU: torch.Tensor  # [m] fp32
+    V: Optional[torch.Tensor]  # [S, S] or None
+    Ot: torch.Tensor  # [d, m] (O transposed)
+
+
+def layer_workspace_bytes(dtype: int, T: int, d: int, m: int, prenorm: bool) -> int:
+    return int(lib().avey_layer_workspace_bytes(dtype, T, d, m, int(bool(prenorm))))
+
+
+def avey_layer_forward(layer: DeviceLayer, S: int, m_h: int, eps: float, prenorm: bool,
+                       x_in: torch.Tensor, x_in_lowp: Optional[torch.Tensor] = None,
+                       x_out: Optional[torch.Tensor] = None, lowp_out: bool = True,
+                       x_out_lowp: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None):
+    """One layer on x_in fp32 [T, d] (any leading shape that flattens to T rows).
+
+    Returns (x_out fp32, x_out_lowp pair or None).
+    """
+    _need(x_in, "x_in")
+    d = x_in.shape[-1]
+    T = x_in.numel() // d
+    m = layer.Ut.shape[0]
+    dt = _dt(layer.Ut)
+    if x_out is None:
+        x_out = torch.empty_like(x_in)
+    if dt == AVEY_BF16 and lowp_out and x_out_lowp is None:
+        x_out_lowp = torch.empty((2, T, d), dtype=torch.bfloat16, device=x_in.device)
+    need = layer_workspace_bytes(dt, T, d, m, prenorm)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, x_in.device)
+    p = LayerParams(layer.kind, d, m, m_h, S, eps, int(bool(prenorm)), layer.Ut.data_ptr(),
+                    layer.bU.data_ptr(), None if layer.V is None else layer.V.data_ptr(),
+                    layer.Ot.data_ptr())
+    _check("avey_layer_forward",
+           lib().avey_layer_forward(ctypes.byref(p), dt, T, _ptr(x_in), _ptr(x_in_lowp),
+                                    _ptr(x_out), _ptr(x_out_lowp if dt == AVEY_BF16 else None),
+                                    _ptr(ws), ws.numel(), _stream()))
+    return x_out, (x_out_lowp if dt == AVEY_BF16 else None)
+
+
+def device_layers(weights, dtype: torch.dtype, device) -> List[DeviceLayer]:
+    """Device copies of host weights (U [d, m], bU, V, O [m, d] numpy arrays)."""
+    out = []
+    for lw in weights.layers:
+        Ut = torch.from_numpy(lw.U.T.copy()).to(device=device, dtype=dtype).contiguous()
+        Ot = torch.from_numpy(lw.O.T.copy()).to(device=device, dtype=dtype).contiguous()
+        bU = torch.from_numpy(lw.bU).to(device=device, dtype=torch.float32).contiguous()
+        V = None if lw.V is None else torch.from_numpy(lw.V).to(device=device, dtype=dtype).contiguous()
+        out.append(DeviceLayer(int(lw.kind), Ut, bU, V, Ot))
+    return out
+
+
+@dataclass
+class EncoderWorkspace:
+    """Preallocated buffers for encoder_forward at one shape (reused per call)."""
+    rank_ws: torch.Tensor
+    layer_ws: torch.Tensor
+    idx: torch.Tensor
+    w: torch.Tensor
+    x0: torch.Tensor
+    x1: torch.Tensor
+    pair0: Optional[torch.Tensor]
+    pair1: Optional[torch.Tensor]
+
+
+def make_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: torch.dtype, prenorm: bool,
+                   device) -> EncoderWorkspace:
+    n = -(-N // S)
+    T = B * n * S
+    dt = AVEY_BF16 if dtype == torch.bfloat16 else AVEY_F32
+    rank_ws = _ws(rank_workspace_bytes(dt, B, N, d, S), device)
+    layer_ws = _ws(layer_workspace_bytes(dt, T, d, m, prenorm), device)
+    idx = torch.empty((B, n, k), dtype=torch.int32, device=device)
+    w = torch.empty((B, n, k), dtype=torch.float32, device=device)
+    x0 = torch.empty((T, d), dtype=torch.float32, device=device)
+    x1 = torch.empty((T, d), dtype=torch.float32, device=device)
+    pair0 = pair1 = None
+    if dt == AVEY_BF16:
+        pair0 = torch.empty((2, T, d), dtype=torch.bfloat16, device=device)
+        pair1 = torch.empty((2, T, d), dtype=torch.bfloat16, device=device)
+    return EncoderWorkspace(rank_ws, layer_ws, idx, w, x0, x1, pair0, pair1)
+
+
+def encoder_forward(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLayer], S: int, k: int,
+                    m_h: int, eps: float, prenorm: bool,
+                    ws: Optional[EncoderWorkspace] = None, marks=None) -> torch.Tensor:
+    """Ranker once, compression, then every layer (Avey-B paperlayer summary
+    App. H: the ranker runs once per forward).  Returns fp32 [B, n*S, d].
+
+    ``marks``: optional list of 3 + len(layers) torch.cuda.Event, recorded on
+    the current stream before the ranker and after every C-ABI call.
+    """
+    B, N, d = x.shape
+    n = -(-N // S)
+    T = B * n * S
+    dt = _dt(x)
+    m = layers[0].Ut.shape[0] if layers else d
+    if ws is None:
+        ws = make_workspace(B, N, d, S, k, m, x.dtype, prenorm, x.device)
+    L = lib()
+    st = _stream()
+    if marks is not None:
+        marks[0].record()
+    _check("avey_rank", L.avey_rank(_ptr(x), dt, B, N, d, S, k, _ptr(ws.idx), _ptr(ws.w), None,
+                                    _ptr(ws.rank_ws), ws.rank_ws.numel(), st))
+    if marks is not None:
+        marks[1].record()
+    _check("avey_compress", L.avey_compress(_ptr(x), dt, B, N, d, S, k, _ptr(ws.idx), _ptr(ws.w),
+                                            _ptr(P), _ptr(ws.x0), _ptr(ws.pair0), st))
+    if marks is not None:
+        marks[2].record()
+    cur, nxt = (ws.x0, ws.pair0), (ws.x1, ws.pair1)
+    for li, lay in enumerate(layers):
+        p = LayerParams(lay.kind, d, m, m_h, S, eps, int(bool(prenorm)), lay.Ut.data_ptr(),
+                        lay.bU.data_ptr(), None if lay.V is None else lay.V.data_ptr(),
+                        lay.Ot.data_ptr())
+        _check("avey_layer_forward",
+               L.avey_layer_forward(ctypes.byref(p), dt, T, _ptr(cur[0]), _ptr(cur[1]),
+                                    _ptr(nxt[0]), _ptr(nxt[1]), _ptr(ws.layer_ws),
+                                    ws.layer_ws.numel(), st))
+        if marks is not None:
+            marks[3 + li].record()
+        cur, nxt = nxt, cur
+    return cur[0].view(B, n * S, d)

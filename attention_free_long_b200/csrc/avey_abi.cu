@@ -1,0 +1,149 @@
+// avey_abi.cu -- host-side utilities of libavey.so: status reporting, error
+// details, launch counting, SM count, and TMA tensor-map encoding.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "avey_common.cuh"
+
+namespace avey {
+
+// Device status word: kernels record the first failure here (no trap, no
+// assert); avey_device_status() reads and clears it.
+static __device__ int g_status_word;
+
+namespace {
+thread_local char t_detail[512] = {0};
+std::atomic<uint64_t> g_launches{0};
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int *g_status_ptr[kMaxDevices] = {};
+int g_sms[kMaxDevices] = {};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+}  // namespace
+
+void set_detail(const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_detail, sizeof(t_detail), fmt, ap);
+  va_end(ap);
+}
+
+int *device_status_word() {
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) == cudaSuccess) g_status_ptr[dev] = static_cast<int *>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+int sm_count() {
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sms[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    g_sms[dev] = v > 0 ? v : 148;
+  }
+  return g_sms[dev];
+}
+
+bool encode_bf16_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                     uint64_t batch, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
+                     uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    set_detail("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  const cuuint64_t dims[3] = {inner, rows, batch};
+  const cuuint64_t strides[2] = {row_stride_bytes, batch_stride_bytes};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_detail("cuTensorMapEncodeTiled failed (%d): inner=%llu rows=%llu batch=%llu", int(r),
+               (unsigned long long)inner, (unsigned long long)rows, (unsigned long long)batch);
+    return false;
+  }
+  return true;
+}
+
+}  // namespace avey
+
+extern "C" {
+
+avey_status avey_device_status(avey_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    avey::set_detail("cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    return AVEY_ERR_CUDA;
+  }
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, avey::g_status_word, sizeof(int));
+  if (e != cudaSuccess) {
+    avey::set_detail("reading the device status word: %s", cudaGetErrorString(e));
+    return AVEY_ERR_CUDA;
+  }
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(avey::g_status_word, &zero, sizeof(int));
+    if (e != cudaSuccess) {
+      avey::set_detail("clearing the device status word: %s", cudaGetErrorString(e));
+      return AVEY_ERR_CUDA;
+    }
+  }
+  return static_cast<avey_status>(v);
+}
+
+const char *avey_status_string(avey_status s) {
+  switch (s) {
+    case AVEY_OK: return "AVEY_OK";
+    case AVEY_ERR_INVALID_ARG: return "AVEY_ERR_INVALID_ARG";
+    case AVEY_ERR_UNSUPPORTED: return "AVEY_ERR_UNSUPPORTED";
+    case AVEY_ERR_CUDA: return "AVEY_ERR_CUDA";
+    case AVEY_ERR_DEVICE_TIMEOUT: return "AVEY_ERR_DEVICE_TIMEOUT";
+    case AVEY_ERR_DEVICE_BOUNDS: return "AVEY_ERR_DEVICE_BOUNDS";
+  }
+  return "AVEY_ERR_UNKNOWN";
+}
+
+const char *avey_last_error_detail(void) { return avey::t_detail; }
+
+uint64_t avey_kernel_launches(void) { return avey::g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,339 @@
+// avey_compress.cu -- neural compression of each split with its retrieved
+// splits, plus the residual to the split's own tokens (papernotes 关键设计 4,
+// eq. 8; paperlayer summary §4.3, App. H):
+//   out(t) = sum_{r=0..k} w_r P_r X_{c_r} + X_t,   c_0 = t, w_0 = 1,
+// where P_r = P[:, rS:(r+1)S] is the r-th S x S block of P.  Writing the
+// product block by block is the same contraction as P X_cat with the weighted
+// blocks stacked in rank order; the weight multiplies the fp32 partial
+// product of its block, so the bf16 embeddings are never re-rounded.
+//
+// bf16 kernel: one CTA per (target split, column slab of d).  Each retrieved
+// block (S rows x slab) and its P_r are staged in shared memory with
+// cp.async, double-buffered over r; 8 warps compute the S x slab product with
+// mma.sync m16n8k16 (P_r from ldmatrix, X from ldmatrix.trans).  The kernel is
+// bound by HBM: it reads (k+1) S x d bf16 per split and writes S x d fp32 plus
+// the bf16 split pair.
+#include <algorithm>
+
+#include "avey_common.cuh"
+#include "avey_internal.h"
+
+namespace avey {
+namespace {
+
+template <int S>
+struct CompressTile {
+  static constexpr int WM = S >= 32 ? 32 : 16;         // rows per warp
+  static constexpr int WARPS_M = S / WM;
+  static constexpr int WARPS_N = 8 / WARPS_M;
+  static constexpr int WN = 32;                         // columns per warp
+  static constexpr int NS = WN * WARPS_N;               // slab width
+  static constexpr int MI = WM / 16, NI = WN / 8;
+  static constexpr int XLD = NS + 8;                    // padded smem row (elements)
+  static constexpr int PLD = S + 8;
+  static constexpr int XBYTES = S * XLD * 2;
+  static constexpr int PBYTES = S * PLD * 2;
+  static constexpr int STAGE = XBYTES + PBYTES;
+  static constexpr int SMEM = 2 * STAGE;
+};
+
+template <int S>
+__global__ void __launch_bounds__(256) compress_bf16(const bf16 *__restrict__ x, int N, int d,
+                                                     int n, int k, const int32_t *__restrict__ idx,
+                                                     const float *__restrict__ w,
+                                                     const bf16 *__restrict__ P,
+                                                     float *__restrict__ out,
+                                                     bf16 *__restrict__ out_hi,
+                                                     bf16 *__restrict__ out_lo, long long plane,
+                                                     int *status) {
+  using C = CompressTile<S>;
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ int s_c[33];
+  __shared__ float s_w[33];
+  const int slab = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
+  const int q0 = slab * C::NS;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp / C::WARPS_N, wn = warp % C::WARPS_N;
+  const long long R = static_cast<long long>(n) * S;
+
+  if (tid <= k) {
+    int c = t;
+    float wr = 1.f;
+    if (tid > 0) {
+      const long long o = (static_cast<long long>(b) * n + t) * k + (tid - 1);
+      c = idx[o];
+      wr = w[o];
+      if (c < -1 || c >= n) {
+        record_status(status, AVEY_ERR_DEVICE_BOUNDS);
+        c = -1;
+      }
+    }
+    s_c[tid] = c;
+    s_w[tid] = wr;
+  }
+  __syncthreads();
+
+  // Stage r: X block of split s_c[r] (rows, slab columns) and P_r.
+  auto load_stage = [&](int r, int buf) {
+    uint8_t *xs = smem + buf * C::STAGE;
+    uint8_t *ps = xs + C::XBYTES;
+    const int c = s_c[r];
+    constexpr int XCH = S * (C::NS / 8);  // 16-byte chunks
+    for (int e = tid; e < XCH; e += 256) {
+      const int row = e / (C::NS / 8), cc = e % (C::NS / 8);
+      const int tok = c * S + row, col = q0 + cc * 8;
+      const bool ok = c >= 0 && tok < N && col < d;
+      const bf16 *src = ok ? x + (static_cast<long long>(b) * N + tok) * d + col : x;
+      cp_async16(smem_u32(xs + (row * C::XLD + cc * 8) * 2), src, ok ? 16 : 0);
+    }
+    constexpr int PCH = S * (S / 8);
+    for (int e = tid; e < PCH; e += 256) {
+      const int row = e / (S / 8), cc = e % (S / 8);
+      const bf16 *src = P + static_cast<long long>(row) * (k + 1) * S + r * S + cc * 8;
+      cp_async16(smem_u32(ps + (row * C::PLD + cc * 8) * 2), src, 16);
+    }
+    cp_async_commit();
+  };
+
+  float acc[C::MI][C::NI][4];
+#pragma unroll
+  for (int i = 0; i < C::MI; ++i)
+#pragma unroll
+    for (int j = 0; j < C::NI; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[i][j][q] = 0.f;
+
+  load_stage(0, 0);
+  for (int r = 0; r <= k; ++r) {
+    if (r < k) {
+      load_stage(r + 1, (r + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint8_t *xs = smem + (r & 1) * C::STAGE;
+    const uint8_t *ps = xs + C::XBYTES;
+    float tmp[C::MI][C::NI][4];
+#pragma unroll
+    for (int i = 0; i < C::MI; ++i)
+#pragma unroll
+      for (int j = 0; j < C::NI; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmp[i][j][q] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < S; kk += 16) {
+      uint32_t af[C::MI][4];
+#pragma unroll
+      for (int i = 0; i < C::MI; ++i) {
+        const int row = wm * C::WM + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int col = kk + (lane >> 4) * 8;
+        ldsm_x4(smem_u32(ps + (row * C::PLD + col) * 2), af[i][0], af[i][1], af[i][2], af[i][3]);
+      }
+#pragma unroll
+      for (int j = 0; j < C::NI; j += 2) {
+        uint32_t b0, b1, b2, b3;
+        const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int ncol = wn * C::WN + j * 8 + (lane >> 4) * 8;
+        ldsm_x4_t(smem_u32(xs + (krow * C::XLD + ncol) * 2), b0, b1, b2, b3);
+        const uint32_t bA[2] = {b0, b1}, bB[2] = {b2, b3};
+#pragma unroll
+        for (int i = 0; i < C::MI; ++i) {
+          mma16816(tmp[i][j], af[i], bA);
+          mma16816(tmp[i][j + 1], af[i], bB);
+        }
+      }
+    }
+    const float wr = s_w[r];
+#pragma unroll
+    for (int i = 0; i < C::MI; ++i)
+#pragma unroll
+      for (int j = 0; j < C::NI; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][j][q] = fmaf(wr, tmp[i][j][q], acc[i][j][q]);
+    if (r == 0) {
+      // residual: the target split's own tokens (stage 0 holds X_t)
+#pragma unroll
+      for (int i = 0; i < C::MI; ++i)
+#pragma unroll
+        for (int j = 0; j < C::NI; ++j)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = wm * C::WM + i * 16 + (lane >> 2) + h * 8;
+            const int col = wn * C::WN + j * 8 + (lane & 3) * 2;
+            const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t *>(xs + (row * C::XLD + col) * 2));
+            acc[i][j][2 * h] += xv.x;
+            acc[i][j][2 * h + 1] += xv.y;
+          }
+    }
+    __syncthreads();
+  }
+
+  // store fp32 + split pair
+#pragma unroll
+  for (int i = 0; i < C::MI; ++i)
+#pragma unroll
+    for (int j = 0; j < C::NI; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = wm * C::WM + i * 16 + (lane >> 2) + h * 8;
+        const int col = q0 + wn * C::WN + j * 8 + (lane & 3) * 2;
+        if (col >= d) continue;
+        const long long o = (static_cast<long long>(b) * R + static_cast<long long>(t) * S + row) * d + col;
+        const float v0 = acc[i][j][2 * h], v1 = acc[i][j][2 * h + 1];
+        *reinterpret_cast<float2 *>(out + o) = make_float2(v0, v1);
+        if (out_hi != nullptr) {
+          uint32_t hi, lo;
+          split_pack(v0, v1, hi, lo);
+          *reinterpret_cast<uint32_t *>(out_hi + o) = hi;
+          *reinterpret_cast<uint32_t *>(out_lo + o) = lo;
+        }
+      }
+  (void)plane;
+}
+
+// fp32 SIMT compression: one CTA per (target split, 64-column slab).
+template <int S>
+__global__ void __launch_bounds__(256) compress_f32(const float *__restrict__ x, int N, int d,
+                                                    int n, int k, const int32_t *__restrict__ idx,
+                                                    const float *__restrict__ w,
+                                                    const float *__restrict__ P,
+                                                    float *__restrict__ out, int *status) {
+  constexpr int NSL = 64;
+  constexpr int PER = (S * NSL + 255) / 256;  // outputs per thread
+  __shared__ float xs[S][NSL];
+  __shared__ float ps[S][S];
+  __shared__ int s_c[33];
+  __shared__ float s_w[33];
+  const int slab = blockIdx.x, t = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int q0 = slab * NSL;
+  if (tid <= k) {
+    int c = t;
+    float wr = 1.f;
+    if (tid > 0) {
+      const long long o = (static_cast<long long>(b) * n + t) * k + (tid - 1);
+      c = idx[o];
+      wr = w[o];
+      if (c < -1 || c >= n) {
+        record_status(status, AVEY_ERR_DEVICE_BOUNDS);
+        c = -1;
+      }
+    }
+    s_c[tid] = c;
+    s_w[tid] = wr;
+  }
+  __syncthreads();
+  float acc[PER], res[PER];
+#pragma unroll
+  for (int p = 0; p < PER; ++p) acc[p] = res[p] = 0.f;
+  for (int r = 0; r <= k; ++r) {
+    const int c = s_c[r];
+    for (int e = tid; e < S * NSL; e += 256) {
+      const int row = e / NSL, col = e % NSL;
+      const int tok = c * S + row;
+      xs[row][col] = (c >= 0 && tok < N && q0 + col < d)
+                         ? x[(static_cast<long long>(b) * N + tok) * d + q0 + col]
+                         : 0.f;
+    }
+    for (int e = tid; e < S * S; e += 256) {
+      const int row = e / S, j = e % S;
+      ps[row][j] = P[static_cast<long long>(row) * (k + 1) * S + r * S + j];
+    }
+    __syncthreads();
+    const float wr = s_w[r];
+#pragma unroll
+    for (int p = 0; p < PER; ++p) {
+      const int e = tid + p * 256;
+      if (e < S * NSL) {
+        const int i = e / NSL, col = e % NSL;
+        float s = 0.f;
+        for (int j = 0; j < S; ++j) s = fmaf(ps[i][j], xs[j][col], s);
+        acc[p] = fmaf(wr, s, acc[p]);
+        if (r == 0) res[p] = xs[i][col];
+      }
+    }
+    __syncthreads();
+  }
+  const long long R = static_cast<long long>(n) * S;
+#pragma unroll
+  for (int p = 0; p < PER; ++p) {
+    const int e = tid + p * 256;
+    if (e < S * NSL) {
+      const int i = e / NSL, col = e % NSL;
+      if (q0 + col < d)
+        out[(static_cast<long long>(b) * R + static_cast<long long>(t) * S + i) * d + q0 + col] =
+            acc[p] + res[p];
+    }
+  }
+}
+
+template <int S>
+avey_status run_compress_bf16(const bf16 *x, int B, int N, int d, int n, int k, const int32_t *idx,
+                              const float *w, const bf16 *P, float *out, bf16 *hi, bf16 *lo,
+                              cudaStream_t s) {
+  using C = CompressTile<S>;
+  auto kern = compress_bf16<S>;
+  if (C::SMEM > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) {
+      set_detail("compress: %s", cudaGetErrorString(e));
+      return AVEY_ERR_CUDA;
+    }
+  }
+  const dim3 grid((d + C::NS - 1) / C::NS, n, B);
+  const long long plane = static_cast<long long>(B) * n * S * d;
+  kern<<<grid, 256, C::SMEM, s>>>(x, N, d, n, k, idx, w, P, out, hi, lo, plane,
+                                  device_status_word());
+  AVEY_CHECK_LAUNCH("compress_bf16");
+  return AVEY_OK;
+}
+
+}  // namespace
+}  // namespace avey
+
+using namespace avey;
+
+extern "C" avey_status avey_compress(const void *x, avey_dtype dt, int B, int N, int d, int S,
+                                     int k, const int32_t *idx, const float *w, const void *P,
+                                     float *out, void *out_lowp, avey_stream_t stream) {
+  AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
+               "avey_compress: dtype %d unsupported (F32 or BF16)", int(dt));
+  AVEY_REQUIRE(x && idx && w && P && out, AVEY_ERR_INVALID_ARG, "avey_compress: null pointer");
+  AVEY_REQUIRE(B >= 1 && N >= 1 && d >= 1 && S >= 1 && k >= 1, AVEY_ERR_INVALID_ARG,
+               "avey_compress: sizes must be >= 1");
+  AVEY_REQUIRE(d % 8 == 0, AVEY_ERR_INVALID_ARG, "avey_compress: d=%d must be a multiple of 8", d);
+  AVEY_REQUIRE(k <= 32, AVEY_ERR_UNSUPPORTED, "avey_compress: k=%d > 32", k);
+  AVEY_REQUIRE(aligned16(x) && aligned16(P) && aligned16(out) && (!out_lowp || aligned16(out_lowp)),
+               AVEY_ERR_INVALID_ARG, "avey_compress: pointers must be 16-byte aligned");
+  const int n = (N + S - 1) / S;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dt == AVEY_BF16) {
+    AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
+                 "avey_compress(BF16): S=%d unsupported (16, 32, 64 or 128)", S);
+    const bf16 *xb = static_cast<const bf16 *>(x);
+    const bf16 *Pb = static_cast<const bf16 *>(P);
+    bf16 *hi = static_cast<bf16 *>(out_lowp);
+    bf16 *lo = hi ? hi + static_cast<long long>(B) * n * S * d : nullptr;
+    switch (S) {
+      case 16: return run_compress_bf16<16>(xb, B, N, d, n, k, idx, w, Pb, out, hi, lo, s);
+      case 32: return run_compress_bf16<32>(xb, B, N, d, n, k, idx, w, Pb, out, hi, lo, s);
+      case 64: return run_compress_bf16<64>(xb, B, N, d, n, k, idx, w, Pb, out, hi, lo, s);
+      default: return run_compress_bf16<128>(xb, B, N, d, n, k, idx, w, Pb, out, hi, lo, s);
+    }
+  }
+  AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
+               "avey_compress(F32): S=%d unsupported (power of two <= 64)", S);
+  const dim3 grid((d + 63) / 64, n, B);
+  const float *xf = static_cast<const float *>(x);
+  const float *Pf = static_cast<const float *>(P);
+  int *st = device_status_word();
+  switch (S) {
+#define AVEY_CF_CASE(SS) \
+  case SS: compress_f32<SS><<<grid, 256, 0, s>>>(xf, N, d, n, k, idx, w, Pf, out, st); break;
+    AVEY_CF_CASE(1) AVEY_CF_CASE(2) AVEY_CF_CASE(4) AVEY_CF_CASE(8) AVEY_CF_CASE(16)
+    AVEY_CF_CASE(32) AVEY_CF_CASE(64)
+#undef AVEY_CF_CASE
+  }
+  AVEY_CHECK_LAUNCH("compress_f32");
+  return AVEY_OK;
+}

@@ -1,0 +1,51 @@
+// avey_internal.h -- launchers shared between the translation units of
+// libavey.so.  Not part of the public ABI (include/avey.h is).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "avey.h"
+
+namespace avey {
+
+using bf16 = __nv_bfloat16;
+
+// ---- tcgen05 contractions (avey_tc.cu) ----
+
+// MaxSim split scores: xhat [B, R = n*S, d] bf16 (unit rows, zero pad rows).
+avey_status launch_maxsim_tc(const bf16 *xhat, int B, int R, int d, int S, int n, float *scores,
+                             cudaStream_t s);
+
+// Enricher: Z = relu(scale_row * (X U) + b)^2, X given as a split pair
+// (xhi, xlo) [T, d]; Ut [m, d]; writes the split pair of Z (zhi, zlo) [T, m].
+// inv_rms may be null (scale 1).
+avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, const bf16 *Ut,
+                             int m, const float *bias, const float *inv_rms, bf16 *zhi,
+                             bf16 *zlo, cudaStream_t s);
+
+// Fuser: x_out = x_in + A O, A given as a split pair (ahi, alo) [T, m];
+// Ot [d, m]; writes fp32 x_out and (optionally) its split pair.
+avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
+                           const float *x_in, float *x_out, bf16 *xo_hi, bf16 *xo_lo,
+                           cudaStream_t s);
+
+// ---- ranker pieces (avey_rank.cu) ----
+avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, int S, void *xhat,
+                             cudaStream_t s);
+avey_status launch_topk(const float *scores, int B, int n, int k, int32_t *idx, float *w,
+                        cudaStream_t s);
+
+// ---- mixes (avey_mix.cu) ----
+avey_status launch_static_mix_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int S, int mt,
+                                 int64_t plane, cudaStream_t s);
+avey_status launch_dynamic_mix_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
+                                  int64_t ld_out, int64_t plane_out, int blocks, int S, int mt,
+                                  float eps, cudaStream_t s);
+avey_status launch_static_mix_f32(const float *V, const float *zt, int64_t ld_zt, float *out,
+                                  int64_t ld_out, int blocks, int S, int mt, cudaStream_t s);
+avey_status launch_dynamic_mix_f32(const float *zt, int64_t ld_zt, float *out, int64_t ld_out,
+                                   int blocks, int S, int mt, float eps, cudaStream_t s);
+
+}  // namespace avey

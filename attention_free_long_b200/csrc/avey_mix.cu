@@ -1,0 +1,541 @@
+// avey_mix.cu -- the contextualizer of a neural-processor layer, applied per
+// split block of S tokens (papernotes 关键设计 2 and 3; paperlayer summary §4.2):
+//   static:   c = V Z_t                      (learned S x S map, signed)
+//   dynamic:  G_ij = N(z_i).N(z_j);  Gt_ij = G_ij / (sum_j G_ij + eps)  (eq. 6)
+//             c = Gt Z_t
+// Identity activation, no bias.
+//
+// bf16 path: Z_t is an activation split pair (hi, lo bf16 planes).  Both
+// kernels are bound by HBM (read Z_t, write c, 8 bytes per element each way):
+//   static_mix_x2   one CTA per (block, feature slab); V and both planes of
+//                   the slab in shared memory; c = V Z_hi + V Z_lo with
+//                   mma.sync; written back in place as a split pair.
+//   dynamic_mix_x2  one CTA per block, two passes over Z_t in 64-feature
+//                   chunks (the second pass mostly hits L2):
+//                   1. Gram R = Z_hi Z_hi^T (mma.sync) and fp32 row sums of
+//                      squares of hi + lo;
+//                   2. G = R / (n_i n_j), row sums, Gt in fp32, split to bf16
+//                      hi/lo in shared memory;
+//                   3. c = Gt_hi Z_hi + Gt_lo Z_hi + Gt_hi Z_lo, split pair out.
+// fp32 path: plain SIMT kernels.
+#include <algorithm>
+
+#include "avey_common.cuh"
+#include "avey_internal.h"
+
+namespace avey {
+namespace {
+
+// ---------------------------------------------------------------- static --
+
+template <int S>
+struct StaticTile {
+  static constexpr int WM = S >= 32 ? 32 : 16;
+  static constexpr int WARPS_M = S / WM;
+  static constexpr int WARPS_N = 8 / WARPS_M;
+  static constexpr int WN = 32;
+  static constexpr int NS = WN * WARPS_N;
+  static constexpr int MI = WM / 16, NI = WN / 8;
+  static constexpr int ZLD = NS + 8, VLD = S + 8;
+  static constexpr int ZBYTES = S * ZLD * 2, VBYTES = S * VLD * 2;
+  static constexpr int SMEM = VBYTES + 2 * ZBYTES;
+};
+
+template <int S>
+__global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V, bf16 *zt,
+                                                     long long ld, int mt, long long plane) {
+  using C = StaticTile<S>;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t *vs = smem;
+  uint8_t *zh = smem + C::VBYTES;
+  uint8_t *zl = zh + C::ZBYTES;
+  const int slab = blockIdx.x, blk = blockIdx.y;
+  const int f0 = slab * C::NS;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp / C::WARPS_N, wn = warp % C::WARPS_N;
+  bf16 *zbase = zt + static_cast<long long>(blk) * S * ld;
+
+  for (int e = tid; e < S * (S / 8); e += 256) {
+    const int row = e / (S / 8), cc = e % (S / 8);
+    cp_async16(smem_u32(vs + (row * C::VLD + cc * 8) * 2), V + row * S + cc * 8, 16);
+  }
+  for (int e = tid; e < S * (C::NS / 8); e += 256) {
+    const int row = e / (C::NS / 8), cc = e % (C::NS / 8);
+    const int f = f0 + cc * 8;
+    const bool ok = f < mt;
+    const bf16 *src = ok ? zbase + row * ld + f : zbase;
+    cp_async16(smem_u32(zh + (row * C::ZLD + cc * 8) * 2), src, ok ? 16 : 0);
+    cp_async16(smem_u32(zl + (row * C::ZLD + cc * 8) * 2), ok ? src + plane : zbase, ok ? 16 : 0);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  float acc[C::MI][C::NI][4] = {};
+#pragma unroll
+  for (int kk = 0; kk < S; kk += 16) {
+    uint32_t af[C::MI][4];
+#pragma unroll
+    for (int i = 0; i < C::MI; ++i) {
+      const int row = wm * C::WM + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      ldsm_x4(smem_u32(vs + (row * C::VLD + kk + (lane >> 4) * 8) * 2), af[i][0], af[i][1], af[i][2],
+              af[i][3]);
+    }
+#pragma unroll
+    for (int j = 0; j < C::NI; j += 2) {
+      const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int ncol = wn * C::WN + j * 8 + (lane >> 4) * 8;
+#pragma unroll
+      for (int pl = 0; pl < 2; ++pl) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(smem_u32((pl ? zl : zh) + (krow * C::ZLD + ncol) * 2), b0, b1, b2, b3);
+        const uint32_t bA[2] = {b0, b1}, bB[2] = {b2, b3};
+#pragma unroll
+        for (int i = 0; i < C::MI; ++i) {
+          mma16816(acc[i][j], af[i], bA);
+          mma16816(acc[i][j + 1], af[i], bB);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < C::MI; ++i)
+#pragma unroll
+    for (int j = 0; j < C::NI; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = wm * C::WM + i * 16 + (lane >> 2) + h * 8;
+        const int f = f0 + wn * C::WN + j * 8 + (lane & 3) * 2;
+        if (f >= mt) continue;
+        uint32_t hi, lo;
+        split_pack(acc[i][j][2 * h], acc[i][j][2 * h + 1], hi, lo);
+        bf16 *dst = zbase + row * ld + f;
+        *reinterpret_cast<uint32_t *>(dst) = hi;
+        *reinterpret_cast<uint32_t *>(dst + plane) = lo;
+      }
+}
+
+// --------------------------------------------------------------- dynamic --
+
+template <int S>
+struct DynTile {
+  static constexpr int FC = 64;  // feature chunk
+  static constexpr int CLD = FC + 8;
+  static constexpr int CBYTES = S * CLD * 2;  // one plane of one chunk
+  static constexpr int BUF = 2 * CBYTES;      // hi + lo
+  // Gram tiling (S x S)
+  static constexpr int GW_M = S == 16 ? 1 : (S == 128 ? 4 : 2);
+  static constexpr int GW_N = S == 16 ? 2 : (S == 128 ? 2 : 4);
+  static constexpr int GMI = (S / GW_M) / 16, GNI = (S / GW_N) / 8;
+  // apply tiling (S x FC)
+  static constexpr int AW_M = S == 16 ? 1 : (S == 128 ? 4 : 2);
+  static constexpr int AW_N = S == 16 ? 4 : (S == 128 ? 2 : 4);
+  static constexpr int AMI = (S / AW_M) / 16, ANI = (FC / AW_N) / 8;
+  static constexpr int GLD = S + 8;             // bf16 Gt row
+  static constexpr int GBYTES = S * GLD * 2;
+  static constexpr int FLD = S + 4;             // fp32 G row
+  static constexpr int TR = 256 / S;            // threads per row for sums of squares
+  static constexpr int SMEM = 2 * BUF + 2 * GBYTES;
+  static_assert(S * FLD * 4 <= 2 * BUF, "fp32 G must fit in the chunk buffers");
+};
+
+template <int S>
+__global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long ld_zt,
+                                                      long long plane_zt, bf16 *out,
+                                                      long long ld_out, long long plane_out,
+                                                      int mt, float eps) {
+  using C = DynTile<S>;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t *bufs = smem;                       // 2 x (hi, lo) chunks; later fp32 G
+  uint8_t *gth = smem + 2 * C::BUF;           // Gt hi [S][GLD]
+  uint8_t *gtl = gth + C::GBYTES;             // Gt lo
+  __shared__ float s_ss[S * C::TR];
+  __shared__ float s_nf[S];
+  __shared__ float s_den[S];
+  const int blk = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bf16 *zb = zt + static_cast<long long>(blk) * S * ld_zt;
+  bf16 *ob = out + static_cast<long long>(blk) * S * ld_out;
+  const int nchunks = (mt + C::FC - 1) / C::FC;
+
+  auto load_chunk = [&](int ch, int buf) {
+    uint8_t *h = bufs + buf * C::BUF;
+    uint8_t *l = h + C::CBYTES;
+    for (int e = tid; e < S * (C::FC / 8); e += 256) {
+      const int row = e / (C::FC / 8), cc = e % (C::FC / 8);
+      const int f = ch * C::FC + cc * 8;
+      const bool ok = f < mt;
+      const bf16 *src = ok ? zb + row * ld_zt + f : zb;
+      cp_async16(smem_u32(h + (row * C::CLD + cc * 8) * 2), src, ok ? 16 : 0);
+      cp_async16(smem_u32(l + (row * C::CLD + cc * 8) * 2), ok ? src + plane_zt : zb, ok ? 16 : 0);
+    }
+    cp_async_commit();
+  };
+
+  // ---- pass 1: Gram of the hi plane and row sums of squares ----
+  const int gwm = warp / C::GW_N, gwn = warp % C::GW_N;
+  const bool gram_warp = warp < C::GW_M * C::GW_N;
+  float g[C::GMI][C::GNI][4] = {};
+  const int sr = tid % S, sp = tid / S;  // sum-of-squares row / part
+  float ss = 0.f;
+  load_chunk(0, 0);
+  for (int ch = 0; ch < nchunks; ++ch) {
+    if (ch + 1 < nchunks) {
+      load_chunk(ch + 1, (ch + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint8_t *h = bufs + (ch & 1) * C::BUF;
+    const uint8_t *l = h + C::CBYTES;
+    {
+      constexpr int FPT = C::FC / C::TR;  // features per thread
+#pragma unroll
+      for (int q = 0; q < FPT; q += 2) {
+        const int f = sp * FPT + q;
+        const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t *>(h + (sr * C::CLD + f) * 2));
+        const float2 b = unpack_bf16(*reinterpret_cast<const uint32_t *>(l + (sr * C::CLD + f) * 2));
+        const float v0 = a.x + b.x, v1 = a.y + b.y;
+        ss = fmaf(v0, v0, ss);
+        ss = fmaf(v1, v1, ss);
+      }
+    }
+    if (gram_warp) {
+#pragma unroll
+      for (int kk = 0; kk < C::FC; kk += 16) {
+        uint32_t af[C::GMI][4];
+#pragma unroll
+        for (int i = 0; i < C::GMI; ++i) {
+          const int row = gwm * (S / C::GW_M) + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          ldsm_x4(smem_u32(h + (row * C::CLD + kk + (lane >> 4) * 8) * 2), af[i][0], af[i][1],
+                  af[i][2], af[i][3]);
+        }
+#pragma unroll
+        for (int j = 0; j < C::GNI; ++j) {
+          uint32_t b0, b1;
+          const int jrow = gwn * (S / C::GW_N) + j * 8 + (lane & 7);
+          ldsm_x2(smem_u32(h + (jrow * C::CLD + kk + ((lane >> 3) & 1) * 8) * 2), b0, b1);
+          const uint32_t bb[2] = {b0, b1};
+#pragma unroll
+          for (int i = 0; i < C::GMI; ++i) mma16816(g[i][j], af[i], bb);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- pass 2: eq. 6 in fp32 ----
+  float *G = reinterpret_cast<float *>(bufs);
+  if (gram_warp) {
+#pragma unroll
+    for (int i = 0; i < C::GMI; ++i)
+#pragma unroll
+      for (int j = 0; j < C::GNI; ++j)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int row = gwm * (S / C::GW_M) + i * 16 + (lane >> 2) + hh * 8;
+          const int col = gwn * (S / C::GW_N) + j * 8 + (lane & 3) * 2;
+          G[row * C::FLD + col] = g[i][j][2 * hh];
+          G[row * C::FLD + col + 1] = g[i][j][2 * hh + 1];
+        }
+  }
+  s_ss[sr * C::TR + sp] = ss;
+  __syncthreads();
+  if (tid < S) {
+    float t2 = 0.f;
+    for (int p = 0; p < C::TR; ++p) t2 += s_ss[tid * C::TR + p];
+    s_nf[tid] = fmaxf(sqrtf(t2), 1e-12f);
+  }
+  __syncthreads();
+  if (tid < S) {
+    const float ni = s_nf[tid];
+    float rs = 0.f;
+    for (int j = 0; j < S; ++j) {
+      const float v = G[tid * C::FLD + j] / (ni * s_nf[j]);
+      G[tid * C::FLD + j] = v;
+      rs += v;
+    }
+    s_den[tid] = rs + eps;
+  }
+  __syncthreads();
+  for (int e = tid; e < S * S; e += 256) {
+    const int i = e / S, j = e % S;
+    const float v = G[i * C::FLD + j] / s_den[i];
+    float hi, lo;
+    split_bf16(v, hi, lo);
+    reinterpret_cast<bf16 *>(gth)[i * C::GLD + j] = __float2bfloat16_rn(hi);
+    reinterpret_cast<bf16 *>(gtl)[i * C::GLD + j] = __float2bfloat16_rn(lo);
+  }
+  __syncthreads();
+
+  // ---- pass 3: c = Gt Z_t ----
+  const int awm = warp / C::AW_N, awn = warp % C::AW_N;
+  const bool apply_warp = warp < C::AW_M * C::AW_N;
+  load_chunk(0, 0);
+  for (int ch = 0; ch < nchunks; ++ch) {
+    if (ch + 1 < nchunks) {
+      load_chunk(ch + 1, (ch + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint8_t *h = bufs + (ch & 1) * C::BUF;
+    const uint8_t *l = h + C::CBYTES;
+    if (apply_warp) {
+      float acc[C::AMI][C::ANI][4] = {};
+#pragma unroll
+      for (int kk = 0; kk < S; kk += 16) {
+        uint32_t ah[C::AMI][4], al[C::AMI][4];
+#pragma unroll
+        for (int i = 0; i < C::AMI; ++i) {
+          const int row = awm * (S / C::AW_M) + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int col = kk + (lane >> 4) * 8;
+          ldsm_x4(smem_u32(gth + (row * C::GLD + col) * 2), ah[i][0], ah[i][1], ah[i][2], ah[i][3]);
+          ldsm_x4(smem_u32(gtl + (row * C::GLD + col) * 2), al[i][0], al[i][1], al[i][2], al[i][3]);
+        }
+#pragma unroll
+        for (int j = 0; j < C::ANI; j += 2) {
+          const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int ncol = awn * (C::FC / C::AW_N) + j * 8 + (lane >> 4) * 8;
+          uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+          ldsm_x4_t(smem_u32(h + (krow * C::CLD + ncol) * 2), h0, h1, h2, h3);
+          ldsm_x4_t(smem_u32(l + (krow * C::CLD + ncol) * 2), l0, l1, l2, l3);
+          const uint32_t hA[2] = {h0, h1}, hB[2] = {h2, h3}, lA[2] = {l0, l1}, lB[2] = {l2, l3};
+#pragma unroll
+          for (int i = 0; i < C::AMI; ++i) {
+            mma16816(acc[i][j], ah[i], hA);
+            mma16816(acc[i][j + 1], ah[i], hB);
+            mma16816(acc[i][j], al[i], hA);
+            mma16816(acc[i][j + 1], al[i], hB);
+            mma16816(acc[i][j], ah[i], lA);
+            mma16816(acc[i][j + 1], ah[i], lB);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < C::AMI; ++i)
+#pragma unroll
+        for (int j = 0; j < C::ANI; ++j)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int row = awm * (S / C::AW_M) + i * 16 + (lane >> 2) + hh * 8;
+            const int f = ch * C::FC + awn * (C::FC / C::AW_N) + j * 8 + (lane & 3) * 2;
+            if (f >= mt) continue;
+            uint32_t hi, lo;
+            split_pack(acc[i][j][2 * hh], acc[i][j][2 * hh + 1], hi, lo);
+            bf16 *dst = ob + row * ld_out + f;
+            *reinterpret_cast<uint32_t *>(dst) = hi;
+            *reinterpret_cast<uint32_t *>(dst + plane_out) = lo;
+          }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ fp32 --
+
+template <int S>
+__global__ void __launch_bounds__(256) static_mix_f32(const float *__restrict__ V, const float *zt,
+                                                      long long ld_zt, float *out,
+                                                      long long ld_out, int mt) {
+  constexpr int NSL = 64;
+  __shared__ float vs[S][S];
+  __shared__ float zs[S][NSL];
+  const int slab = blockIdx.x, blk = blockIdx.y, tid = threadIdx.x;
+  const int f0 = slab * NSL;
+  const float *zb = zt + static_cast<long long>(blk) * S * ld_zt;
+  float *ob = out + static_cast<long long>(blk) * S * ld_out;
+  for (int e = tid; e < S * S; e += 256) vs[e / S][e % S] = V[e];
+  for (int e = tid; e < S * NSL; e += 256) {
+    const int r = e / NSL, c = e % NSL;
+    zs[r][c] = (f0 + c < mt) ? zb[r * ld_zt + f0 + c] : 0.f;
+  }
+  __syncthreads();
+  for (int e = tid; e < S * NSL; e += 256) {
+    const int i = e / NSL, c = e % NSL;
+    if (f0 + c >= mt) continue;
+    float s = 0.f;
+    for (int j = 0; j < S; ++j) s = fmaf(vs[i][j], zs[j][c], s);
+    ob[i * ld_out + f0 + c] = s;
+  }
+}
+
+template <int S>
+__global__ void __launch_bounds__(256) dynamic_mix_f32(const float *zt, long long ld_zt,
+                                                       float *out, long long ld_out, int mt,
+                                                       float eps) {
+  constexpr int NSL = 64;
+  __shared__ float Gt[S][S + 1];
+  __shared__ float nf[S];
+  __shared__ float zs[S][NSL];
+  const int blk = blockIdx.x, tid = threadIdx.x;
+  const float *zb = zt + static_cast<long long>(blk) * S * ld_zt;
+  float *ob = out + static_cast<long long>(blk) * S * ld_out;
+  if (tid < S) {
+    float ss = 0.f;
+    for (int f = 0; f < mt; ++f) ss = fmaf(zb[tid * ld_zt + f], zb[tid * ld_zt + f], ss);
+    nf[tid] = fmaxf(sqrtf(ss), 1e-12f);
+  }
+  __syncthreads();
+  for (int e = tid; e < S * S; e += 256) {
+    const int i = e / S, j = e % S;
+    float s = 0.f;
+    for (int f = 0; f < mt; ++f) s = fmaf(zb[i * ld_zt + f], zb[j * ld_zt + f], s);
+    Gt[i][j] = s / (nf[i] * nf[j]);
+  }
+  __syncthreads();
+  if (tid < S) {
+    float rs = 0.f;
+    for (int j = 0; j < S; ++j) rs += Gt[tid][j];
+    const float den = rs + eps;
+    for (int j = 0; j < S; ++j) Gt[tid][j] = Gt[tid][j] / den;
+  }
+  __syncthreads();
+  // c = Gt Z_t, slab by slab; every slab is read into shared memory before
+  // its outputs are written, so out may alias zt.
+  for (int f0 = 0; f0 < mt; f0 += NSL) {
+    for (int e = tid; e < S * NSL; e += 256) {
+      const int r = e / NSL, c = e % NSL;
+      zs[r][c] = (f0 + c < mt) ? zb[r * ld_zt + f0 + c] : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < S * NSL; e += 256) {
+      const int i = e / NSL, c = e % NSL;
+      if (f0 + c >= mt) continue;
+      float s = 0.f;
+      for (int j = 0; j < S; ++j) s = fmaf(Gt[i][j], zs[j][c], s);
+      ob[i * ld_out + f0 + c] = s;
+    }
+    __syncthreads();
+  }
+}
+
+template <typename K>
+avey_status set_smem(K kern, int bytes, const char *name) {
+  if (bytes <= 48 * 1024) return AVEY_OK;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    set_detail("%s: %s", name, cudaGetErrorString(e));
+    return AVEY_ERR_CUDA;
+  }
+  return AVEY_OK;
+}
+
+template <int S>
+avey_status run_static_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int mt, int64_t plane,
+                          cudaStream_t s) {
+  using C = StaticTile<S>;
+  if (avey_status st = set_smem(static_mix_x2<S>, C::SMEM, "static_mix_x2")) return st;
+  const dim3 grid((mt + C::NS - 1) / C::NS, blocks);
+  static_mix_x2<S><<<grid, 256, C::SMEM, s>>>(V, zt, ld, mt, plane);
+  AVEY_CHECK_LAUNCH("static_mix_x2");
+  return AVEY_OK;
+}
+
+template <int S>
+avey_status run_dynamic_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
+                           int64_t ld_out, int64_t plane_out, int blocks, int mt, float eps,
+                           cudaStream_t s) {
+  using C = DynTile<S>;
+  if (avey_status st = set_smem(dynamic_mix_x2<S>, C::SMEM, "dynamic_mix_x2")) return st;
+  dynamic_mix_x2<S><<<blocks, 256, C::SMEM, s>>>(zt, ld_zt, plane_zt, out, ld_out, plane_out, mt, eps);
+  AVEY_CHECK_LAUNCH("dynamic_mix_x2");
+  return AVEY_OK;
+}
+
+}  // namespace
+
+avey_status launch_static_mix_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int S, int mt,
+                                 int64_t plane, cudaStream_t s) {
+  switch (S) {
+    case 16: return run_static_x2<16>(V, zt, ld, blocks, mt, plane, s);
+    case 32: return run_static_x2<32>(V, zt, ld, blocks, mt, plane, s);
+    case 64: return run_static_x2<64>(V, zt, ld, blocks, mt, plane, s);
+    case 128: return run_static_x2<128>(V, zt, ld, blocks, mt, plane, s);
+  }
+  set_detail("static mix: S=%d unsupported", S);
+  return AVEY_ERR_UNSUPPORTED;
+}
+
+avey_status launch_dynamic_mix_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
+                                  int64_t ld_out, int64_t plane_out, int blocks, int S, int mt,
+                                  float eps, cudaStream_t s) {
+  switch (S) {
+    case 16: return run_dynamic_x2<16>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, s);
+    case 32: return run_dynamic_x2<32>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, s);
+    case 64: return run_dynamic_x2<64>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, s);
+    case 128: return run_dynamic_x2<128>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, s);
+  }
+  set_detail("dynamic mix: S=%d unsupported", S);
+  return AVEY_ERR_UNSUPPORTED;
+}
+
+avey_status launch_static_mix_f32(const float *V, const float *zt, int64_t ld_zt, float *out,
+                                  int64_t ld_out, int blocks, int S, int mt, cudaStream_t s) {
+  const dim3 grid((mt + 63) / 64, blocks);
+  switch (S) {
+#define AVEY_SF(SS) \
+  case SS: static_mix_f32<SS><<<grid, 256, 0, s>>>(V, zt, ld_zt, out, ld_out, mt); break;
+    AVEY_SF(1) AVEY_SF(2) AVEY_SF(4) AVEY_SF(8) AVEY_SF(16) AVEY_SF(32) AVEY_SF(64)
+#undef AVEY_SF
+    default: set_detail("static mix (F32): S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
+  }
+  AVEY_CHECK_LAUNCH("static_mix_f32");
+  return AVEY_OK;
+}
+
+avey_status launch_dynamic_mix_f32(const float *zt, int64_t ld_zt, float *out, int64_t ld_out,
+                                   int blocks, int S, int mt, float eps, cudaStream_t s) {
+  switch (S) {
+#define AVEY_DF(SS) \
+  case SS: dynamic_mix_f32<SS><<<blocks, 256, 0, s>>>(zt, ld_zt, out, ld_out, mt, eps); break;
+    AVEY_DF(1) AVEY_DF(2) AVEY_DF(4) AVEY_DF(8) AVEY_DF(16) AVEY_DF(32) AVEY_DF(64)
+#undef AVEY_DF
+    default: set_detail("dynamic mix (F32): S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
+  }
+  AVEY_CHECK_LAUNCH("dynamic_mix_f32");
+  return AVEY_OK;
+}
+
+}  // namespace avey
+
+using namespace avey;
+
+extern "C" avey_status avey_dynamic_mix(const void *zt, int64_t ld_zt, avey_dtype dt, int blocks,
+                                        int S, int mt, float eps, void *out, int64_t ld_out,
+                                        avey_stream_t stream) {
+  AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16X2, AVEY_ERR_UNSUPPORTED,
+               "avey_dynamic_mix: dtype %d unsupported (F32 or BF16X2)", int(dt));
+  AVEY_REQUIRE(zt && out, AVEY_ERR_INVALID_ARG, "avey_dynamic_mix: null pointer");
+  AVEY_REQUIRE(blocks >= 0 && S >= 1 && mt >= 1 && ld_zt >= mt && ld_out >= mt && eps >= 0.f,
+               AVEY_ERR_INVALID_ARG, "avey_dynamic_mix: bad sizes");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (blocks == 0) return AVEY_OK;
+  const char *zb = static_cast<const char *>(zt);
+  const char *obp = static_cast<const char *>(out);
+  const size_t es = dt == AVEY_F32 ? 4 : 2;
+  const size_t zspan = static_cast<size_t>(blocks) * S * ld_zt * es;
+  const size_t ospan = static_cast<size_t>(blocks) * S * ld_out * es;
+  const bool same = zt == out && ld_zt == ld_out;
+  const bool overlap = !same && zb < obp + ospan * (dt == AVEY_BF16X2 ? 2 : 1) &&
+                       obp < zb + zspan * (dt == AVEY_BF16X2 ? 2 : 1);
+  AVEY_REQUIRE(!overlap, AVEY_ERR_INVALID_ARG,
+               "avey_dynamic_mix: out overlaps zt without aliasing it exactly");
+  if (dt == AVEY_BF16X2) {
+    AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
+                 "avey_dynamic_mix(BF16X2): S=%d unsupported (16, 32, 64 or 128)", S);
+    AVEY_REQUIRE(mt % 8 == 0 && ld_zt % 8 == 0 && ld_out % 8 == 0 && aligned16(zt) && aligned16(out),
+                 AVEY_ERR_INVALID_ARG,
+                 "avey_dynamic_mix(BF16X2): mt and ld must be multiples of 8, pointers 16-byte aligned");
+    const int64_t pz = static_cast<int64_t>(blocks) * S * ld_zt;
+    const int64_t po = static_cast<int64_t>(blocks) * S * ld_out;
+    return launch_dynamic_mix_x2(static_cast<const bf16 *>(zt), ld_zt, pz, static_cast<bf16 *>(out),
+                                 ld_out, po, blocks, S, mt, eps, s);
+  }
+  AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
+               "avey_dynamic_mix(F32): S=%d unsupported (power of two <= 64)", S);
+  return launch_dynamic_mix_f32(static_cast<const float *>(zt), ld_zt, static_cast<float *>(out),
+                                ld_out, blocks, S, mt, eps, s);
+}

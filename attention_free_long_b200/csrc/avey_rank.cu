@@ -1,0 +1,303 @@
+// avey_rank.cu -- the Avey-B ranker: row normalisation, MaxSim split scores,
+// top-k selection with divide-by-max weights (Avey-B paperlayer summary §3
+// Background and App. H; papernotes 整体框架).
+//
+//   normalize_rows   N(x) = x / max(||x||, 1e-12) per token, padded to n*S
+//                    rows per sequence (pad rows zero); bf16 or fp32 out.
+//   maxsim (bf16)    tcgen05 kernel in avey_tc.cu.
+//   maxsim_f32       SIMT fp32 version (one CTA per target/candidate pair).
+//   topk_warp        one warp per target split: k rounds of a warp-wide
+//                    argmax over the split's score row held in shared memory,
+//                    order (score desc, index asc), self excluded, then
+//                    w_r = s_r / s_1 with IEEE division (s_1 / s_1 == 1).
+#include <algorithm>
+
+#include "avey_common.cuh"
+#include "avey_internal.h"
+
+namespace avey {
+namespace {
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) normalize_rows(const Tin *__restrict__ x, int B, int N,
+                                                      int d, int R, Tout *__restrict__ xhat) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(B) * R) return;
+  const int b = static_cast<int>(row / R);
+  const int tok = static_cast<int>(row - static_cast<long long>(b) * R);
+  Tout *dst = xhat + row * d;
+  if (tok >= N) {  // pad row
+    for (int j = lane * 8; j < d; j += 256) {
+      if constexpr (sizeof(Tout) == 2) {
+        *reinterpret_cast<uint4 *>(dst + j) = make_uint4(0, 0, 0, 0);
+      } else {
+        *reinterpret_cast<float4 *>(dst + j) = make_float4(0, 0, 0, 0);
+        *reinterpret_cast<float4 *>(dst + j + 4) = make_float4(0, 0, 0, 0);
+      }
+    }
+    return;
+  }
+  const Tin *src = x + (static_cast<long long>(b) * N + tok) * d;
+  float v[8];
+  auto load8 = [&](int j) {
+    if constexpr (sizeof(Tin) == 2) {
+      const uint4 u = *reinterpret_cast<const uint4 *>(src + j);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = unpack_bf16(w4[q]);
+        v[2 * q] = f.x;
+        v[2 * q + 1] = f.y;
+      }
+    } else {
+      const float4 a = *reinterpret_cast<const float4 *>(src + j);
+      const float4 c = *reinterpret_cast<const float4 *>(src + j + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+    }
+  };
+  float ss = 0.f;
+  for (int j = lane * 8; j < d; j += 256) {
+    load8(j);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) ss = fmaf(v[q], v[q], ss);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+  for (int j = lane * 8; j < d; j += 256) {
+    load8(j);
+    if constexpr (sizeof(Tout) == 2) {
+      *reinterpret_cast<uint4 *>(dst + j) =
+          make_uint4(pack_bf16(v[0] * inv, v[1] * inv), pack_bf16(v[2] * inv, v[3] * inv),
+                     pack_bf16(v[4] * inv, v[5] * inv), pack_bf16(v[6] * inv, v[7] * inv));
+    } else {
+      *reinterpret_cast<float4 *>(dst + j) = make_float4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+      *reinterpret_cast<float4 *>(dst + j + 4) =
+          make_float4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
+    }
+  }
+}
+
+// fp32 MaxSim: one CTA per (target t, candidate c, sequence b).  Thread
+// layout: TPR = 256/S threads per target row, each covering S/TPR candidate
+// rows; the d-loop is staged through shared memory in chunks of 32.
+template <int S>
+__global__ void __launch_bounds__(256) maxsim_f32(const float *__restrict__ xhat, int R, int d,
+                                                  int n, float *__restrict__ scores) {
+  constexpr int TPR = (256 / S) < S ? (256 / S) : S;  // threads per target row
+  constexpr int CPT = S / TPR;                         // candidate rows per thread
+  __shared__ float st[S][33];
+  __shared__ float sc[S][33];
+  __shared__ float rowmax[S][TPR];
+  const int c = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
+  const float *xt = xhat + (static_cast<long long>(b) * R + static_cast<long long>(t) * S) * d;
+  const float *xc = xhat + (static_cast<long long>(b) * R + static_cast<long long>(c) * S) * d;
+  const int tid = threadIdx.x;
+  const int i = tid % S;          // target row
+  const int part = tid / S;       // which slice of candidate rows
+  const bool active = tid < S * TPR;
+  float acc[CPT];
+#pragma unroll
+  for (int q = 0; q < CPT; ++q) acc[q] = 0.f;
+  for (int k0 = 0; k0 < d; k0 += 32) {
+    for (int e = tid; e < S * 32; e += 256) {
+      const int r = e / 32, kk = e % 32;
+      st[r][kk] = (k0 + kk < d) ? xt[static_cast<long long>(r) * d + k0 + kk] : 0.f;
+      sc[r][kk] = (k0 + kk < d) ? xc[static_cast<long long>(r) * d + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+    if (active) {
+#pragma unroll
+      for (int q = 0; q < CPT; ++q) {
+        const int j = part * CPT + q;
+        float s = acc[q];
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) s = fmaf(st[i][kk], sc[j][kk], s);
+        acc[q] = s;
+      }
+    }
+    __syncthreads();
+  }
+  if (active) {
+    float m = acc[0];
+#pragma unroll
+    for (int q = 1; q < CPT; ++q) m = fmaxf(m, acc[q]);
+    rowmax[i][part] = m;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float total = 0.f;
+    for (int r = 0; r < S; ++r) {
+      float m = rowmax[r][0];
+      for (int p = 1; p < TPR; ++p) m = fmaxf(m, rowmax[r][p]);
+      total += m;
+    }
+    scores[(static_cast<long long>(b) * n + t) * n + c] = total;
+  }
+}
+
+constexpr int kTopkWarps = 4;
+
+__global__ void __launch_bounds__(kTopkWarps * 32)
+    topk_warp(const float *__restrict__ scores, int B, int n, int k, int32_t *__restrict__ idx,
+              float *__restrict__ w) {
+  extern __shared__ float srow_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long rowid = static_cast<long long>(blockIdx.x) * kTopkWarps + warp;
+  if (rowid >= static_cast<long long>(B) * n) return;
+  const int t = static_cast<int>(rowid % n);
+  float *srow = srow_all + static_cast<long long>(warp) * n;
+  const float *src = scores + rowid * n;
+  for (int c = lane; c < n; c += 32) srow[c] = (c == t) ? -INFINITY : src[c];
+  __syncwarp();
+  float s1 = 1.f;
+  for (int r = 0; r < k; ++r) {
+    float best = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int c = lane; c < n; c += 32) {
+      const float v = srow[c];
+      if (v > best) {  // increasing c per lane: ties keep the lower index
+        best = v;
+        bi = c;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ob > best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    const long long o = rowid * k + r;
+    if (r < n - 1 && bi != 0x7fffffff && best != -INFINITY) {
+      if (r == 0) s1 = best > 1e-30f ? best : 1e-30f;
+      if (lane == 0) {
+        idx[o] = bi;
+        w[o] = best / s1;
+        srow[bi] = -INFINITY;
+      }
+    } else if (lane == 0) {
+      idx[o] = -1;
+      w[o] = 0.f;
+    }
+    __syncwarp();
+  }
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, int S, void *xhat,
+                             cudaStream_t s) {
+  const int n = (N + S - 1) / S, R = n * S;
+  const long long rows = static_cast<long long>(B) * R;
+  const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+  if (dt == AVEY_BF16)
+    normalize_rows<bf16, bf16><<<grid, 256, 0, s>>>(static_cast<const bf16 *>(x), B, N, d, R,
+                                                    static_cast<bf16 *>(xhat));
+  else
+    normalize_rows<float, float><<<grid, 256, 0, s>>>(static_cast<const float *>(x), B, N, d, R,
+                                                      static_cast<float *>(xhat));
+  AVEY_CHECK_LAUNCH("normalize_rows");
+  return AVEY_OK;
+}
+
+avey_status launch_topk(const float *scores, int B, int n, int k, int32_t *idx, float *w,
+                        cudaStream_t s) {
+  const long long rows = static_cast<long long>(B) * n;
+  const size_t smem = static_cast<size_t>(kTopkWarps) * n * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(topk_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) {
+      set_detail("topk: %s", cudaGetErrorString(e));
+      return AVEY_ERR_CUDA;
+    }
+  }
+  const unsigned grid = static_cast<unsigned>((rows + kTopkWarps - 1) / kTopkWarps);
+  topk_warp<<<grid, kTopkWarps * 32, smem, s>>>(scores, B, n, k, idx, w);
+  AVEY_CHECK_LAUNCH("topk_warp");
+  return AVEY_OK;
+}
+
+static avey_status launch_maxsim_f32(const float *xhat, int B, int R, int d, int S, int n,
+                                     float *scores, cudaStream_t s) {
+  const dim3 grid(n, n, B);
+  switch (S) {
+#define AVEY_MS_CASE(SS)                                                          \
+  case SS:                                                                        \
+    maxsim_f32<SS><<<grid, 256, 0, s>>>(xhat, R, d, n, scores);                   \
+    break;
+    AVEY_MS_CASE(1) AVEY_MS_CASE(2) AVEY_MS_CASE(4) AVEY_MS_CASE(8) AVEY_MS_CASE(16)
+    AVEY_MS_CASE(32) AVEY_MS_CASE(64) AVEY_MS_CASE(128)
+#undef AVEY_MS_CASE
+    default:
+      set_detail("avey_rank(F32): S=%d unsupported (powers of two up to 128)", S);
+      return AVEY_ERR_UNSUPPORTED;
+  }
+  AVEY_CHECK_LAUNCH("maxsim_f32");
+  return AVEY_OK;
+}
+
+}  // namespace avey
+
+using namespace avey;
+
+extern "C" size_t avey_rank_workspace_bytes(avey_dtype dt, int B, int N, int d, int S) {
+  if (B <= 0 || N <= 0 || d <= 0 || S <= 0) return 0;
+  const long long n = (N + S - 1) / S, R = n * S;
+  const size_t es = dt == AVEY_F32 ? 4 : 2;
+  return align256(static_cast<size_t>(B) * R * d * es) + align256(static_cast<size_t>(B) * n * n * 4);
+}
+
+extern "C" avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
+                                 int32_t *idx, float *w, float *scores, void *ws, size_t ws_bytes,
+                                 avey_stream_t stream) {
+  AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
+               "avey_rank: dtype %d unsupported (F32 or BF16)", int(dt));
+  AVEY_REQUIRE(x && idx && w && ws, AVEY_ERR_INVALID_ARG, "avey_rank: null pointer");
+  AVEY_REQUIRE(B >= 1 && N >= 1 && d >= 1 && S >= 1 && k >= 1, AVEY_ERR_INVALID_ARG,
+               "avey_rank: sizes must be >= 1 (B=%d N=%d d=%d S=%d k=%d)", B, N, d, S, k);
+  AVEY_REQUIRE(d % 8 == 0, AVEY_ERR_INVALID_ARG, "avey_rank: d=%d must be a multiple of 8", d);
+  AVEY_REQUIRE(k <= 32, AVEY_ERR_UNSUPPORTED, "avey_rank: k=%d > 32", k);
+  AVEY_REQUIRE(aligned16(x) && aligned16(ws) && (!scores || aligned16(scores)),
+               AVEY_ERR_INVALID_ARG, "avey_rank: pointers must be 16-byte aligned");
+  AVEY_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255) == 0, AVEY_ERR_INVALID_ARG,
+               "avey_rank: workspace must be 256-byte aligned");
+  if (dt == AVEY_BF16)
+    AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
+                 "avey_rank(BF16): S=%d unsupported (16, 32, 64 or 128)", S);
+  else
+    AVEY_REQUIRE(S <= 128 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
+                 "avey_rank(F32): S=%d unsupported (power of two <= 128)", S);
+  const long long n = (N + S - 1) / S, R = n * S;
+  AVEY_REQUIRE(n <= 46340 && static_cast<long long>(B) * R <= (1ll << 31) - 1,
+               AVEY_ERR_UNSUPPORTED, "avey_rank: problem too large");
+  const size_t need = avey_rank_workspace_bytes(dt, B, N, d, S);
+  AVEY_REQUIRE(ws_bytes >= need, AVEY_ERR_INVALID_ARG,
+               "avey_rank: workspace %zu bytes < %zu required", ws_bytes, need);
+  AVEY_REQUIRE(static_cast<size_t>(n) * 4 * 4 <= 200 * 1024, AVEY_ERR_UNSUPPORTED,
+               "avey_rank: n=%lld too large for the top-k kernel", n);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = dt == AVEY_F32 ? 4 : 2;
+  char *wsb = static_cast<char *>(ws);
+  void *xhat = wsb;
+  float *sc = scores ? scores : reinterpret_cast<float *>(wsb + align256(static_cast<size_t>(B) * R * d * es));
+
+  avey_status st = launch_normalize(x, dt, B, N, d, S, xhat, s);
+  if (st != AVEY_OK) return st;
+  if (dt == AVEY_BF16)
+    st = launch_maxsim_tc(static_cast<const bf16 *>(xhat), B, static_cast<int>(R), d, S,
+                          static_cast<int>(n), sc, s);
+  else
+    st = launch_maxsim_f32(static_cast<const float *>(xhat), B, static_cast<int>(R), d, S,
+                           static_cast<int>(n), sc, s);
+  if (st != AVEY_OK) return st;
+  return launch_topk(sc, B, static_cast<int>(n), k, idx, w, s);
+}

@@ -1,0 +1,530 @@
+// avey_tc.cu -- tcgen05 / TMEM / TMA contractions of the Avey-B hot path.
+//
+// One persistent, warp-specialised kernel template serves three contractions:
+//
+//   MaxSim  (ranker, Avey-B paperlayer summary §3 and papernotes 整体框架):
+//           D = Xhat_tile(128 rows) . Xhat_tile(256 rows)^T per sequence; the
+//           epilogue takes, per row, the max over each candidate split's S
+//           columns, then sums those maxima over the S rows of each target
+//           split, so only the [B, n, n] split scores reach HBM.
+//   Enricher (papernotes 整体框架, Z = sigma(XU+b); ReLU^2 per the paperlayer
+//           summary App. A): D = X U with X as a bf16 split pair (two MMAs per
+//           K step); epilogue scale (optional prenorm) + bias + ReLU^2, Z
+//           written as a bf16 split pair.
+//   Fuser   (papernotes 整体框架, f = [Z_h || c] O plus residual):
+//           D = [Z_h || c] O with the activation as a split pair; epilogue adds
+//           the fp32 residual and writes fp32 plus the next layer's split pair.
+//
+// Roles (192 threads, one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: K-chunks of 64 bf16 (128-byte swizzle) of the A
+//               plane(s) and B into a ring of shared-memory stages.
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
+//               and, from one thread, issues tcgen05.mma (M=128, N=256, K=16)
+//               and tcgen05.commit to release stages / publish accumulators.
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes (rows), fused
+//               reduction / activation / residual, stores to HBM.
+// The two TMEM accumulators let the epilogue of tile i overlap the MMAs of
+// tile i+1.  Every barrier wait is bounded (see avey_common.cuh).
+#include <algorithm>
+
+#include "avey_common.cuh"
+#include "avey_internal.h"
+
+namespace avey {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kRedGroups = 8, kRedCands = 16;
+
+enum { MODE_MAXSIM = 0, MODE_ENRICH = 1, MODE_FUSE = 2 };
+
+struct TcArgs {
+  int rows;  // A rows per batch
+  int cols;  // B rows (output columns)
+  int kdim;  // contraction length
+  int tiles_m, tiles_n, num_tiles, group_m;
+  // MaxSim
+  int S, n;
+  float *scores;
+  // enricher
+  const float *bias;
+  const float *inv_rms;
+  bf16 *out_hi;
+  bf16 *out_lo;
+  long long ld_out;
+  // fuser
+  const float *x_in;
+  float *x_out;
+  int *status;
+};
+
+template <int A_PLANES>
+struct Layout {
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_PLANES * A_BYTES + B_BYTES;
+  static constexpr int STAGES = A_PLANES == 1 ? 4 : 3;
+  static constexpr uint32_t TILES_BYTES = STAGES * STAGE_BYTES;
+  static constexpr uint32_t CTRL_BYTES = 256 + 2 * kRedGroups * kRedCands * 4;
+  static constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + 1024;
+};
+
+template <int MODE>
+__device__ __forceinline__ void decode_tile(const TcArgs &a, int tile, int &b, int &mt, int &nt) {
+  if (MODE == MODE_MAXSIM) {
+    // Groups of group_m row tiles walk the column tiles together so that the
+    // group's rows stay in L2 while every column tile streams past once.
+    const int per_b = a.tiles_m * a.tiles_n;
+    b = tile / per_b;
+    const int local = tile - b * per_b;
+    const int gsz = a.group_m * a.tiles_n;
+    const int g = local / gsz;
+    const int rem = local - g * gsz;
+    const int rows_g = min(a.group_m, a.tiles_m - g * a.group_m);
+    nt = rem / rows_g;
+    mt = g * a.group_m + (rem - nt * rows_g);
+  } else {
+    b = 0;
+    mt = tile / a.tiles_n;
+    nt = tile - mt * a.tiles_n;
+  }
+}
+
+// Time-bounded wait that ignores the abort flag (used to drain in-flight work).
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// ---- epilogues -------------------------------------------------------------
+
+// Per-row maxima over each candidate split's columns, summed over the rows of
+// each target split inside this warp; partial sums go to red[group][cand].
+template <int S>
+__device__ __forceinline__ void epi_maxsim_rows(uint32_t taddr, int lane, int quarter,
+                                                float *red) {
+  constexpr int NC = BN / S;
+  float mx[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) mx[c] = -INFINITY;
+#pragma unroll
+  for (int ch = 0; ch < BN / 32; ++ch) {
+    float v[32];
+    tmem_ld32(taddr + ch * 32, v);
+    tmem_ld_wait();
+    if constexpr (S >= 32) {
+      float m = v[0];
+#pragma unroll
+      for (int i = 1; i < 32; ++i) m = fmaxf(m, v[i]);
+      constexpr int per = S / 32;
+      mx[ch / per] = fmaxf(mx[ch / per], m);
+    } else {
+      float m0 = v[0], m1 = v[16];
+#pragma unroll
+      for (int i = 1; i < 16; ++i) {
+        m0 = fmaxf(m0, v[i]);
+        m1 = fmaxf(m1, v[16 + i]);
+      }
+      mx[2 * ch] = m0;
+      mx[2 * ch + 1] = m1;
+    }
+  }
+  if constexpr (S >= 32) {
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx[c] += __shfl_xor_sync(0xffffffffu, mx[c], off);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int c = 0; c < NC; ++c) red[quarter * kRedCands + c] = mx[c];
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) mx[c] += __shfl_xor_sync(0xffffffffu, mx[c], off);
+    }
+    if ((lane & 15) == 0) {
+      const int g = quarter * 2 + (lane >> 4);
+#pragma unroll
+      for (int c = 0; c < NC; ++c) red[g * kRedCands + c] = mx[c];
+    }
+  }
+}
+
+// Final split scores of one tile, from the per-warp partial sums.
+template <int S>
+__device__ __forceinline__ void epi_maxsim_write(const TcArgs &a, const float *red, int lane,
+                                                 int b, int mt, int nt) {
+  constexpr int TS = BM / S, NC = BN / S;
+  for (int e = lane; e < TS * NC; e += 32) {
+    const int ts = e / NC, cs = e - (e / NC) * NC;
+    float sc = 0.f;
+    if constexpr (S >= 32) {
+      constexpr int per = S / 32;
+#pragma unroll
+      for (int q = 0; q < per; ++q) sc += red[(ts * per + q) * kRedCands + cs];
+    } else {
+      sc = red[ts * kRedCands + cs];
+    }
+    const int t = mt * TS + ts, c = nt * NC + cs;
+    if (t < a.n && c < a.n) a.scores[(static_cast<long long>(b) * a.n + t) * a.n + c] = sc;
+  }
+}
+
+__device__ __forceinline__ void epi_enrich(const TcArgs &a, uint32_t taddr, int row, int nt) {
+  const bool valid = row < a.rows;
+  const float scale = (a.inv_rms != nullptr && valid) ? a.inv_rms[row] : 1.f;
+#pragma unroll 1
+  for (int ch = 0; ch < BN / 32; ++ch) {
+    float v[32];
+    tmem_ld32(taddr + ch * 32, v);
+    tmem_ld_wait();
+    const int col0 = nt * BN + ch * 32;
+    if (!valid || col0 >= a.cols) continue;
+    bf16 *ph = a.out_hi + static_cast<long long>(row) * a.ld_out + col0;
+    bf16 *pl = a.out_lo + static_cast<long long>(row) * a.ld_out + col0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (col0 + g * 8 >= a.cols) break;
+      const float4 b0 = __ldg(reinterpret_cast<const float4 *>(a.bias + col0 + g * 8));
+      const float4 b1 = __ldg(reinterpret_cast<const float4 *>(a.bias + col0 + g * 8 + 4));
+      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        float z0 = fmaxf(fmaf(v[g * 8 + j], scale, bb[j]), 0.f);
+        float z1 = fmaxf(fmaf(v[g * 8 + j + 1], scale, bb[j + 1]), 0.f);
+        split_pack(z0 * z0, z1 * z1, hi[j / 2], lo[j / 2]);
+      }
+      *reinterpret_cast<uint4 *>(ph + g * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4 *>(pl + g * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_fuse(const TcArgs &a, uint32_t taddr, int row, int nt) {
+  const bool valid = row < a.rows;
+#pragma unroll 1
+  for (int ch = 0; ch < BN / 32; ++ch) {
+    float v[32];
+    tmem_ld32(taddr + ch * 32, v);
+    tmem_ld_wait();
+    const int col0 = nt * BN + ch * 32;
+    if (!valid || col0 >= a.cols) continue;
+    const long long off = static_cast<long long>(row) * a.cols + col0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (col0 + g * 8 >= a.cols) break;
+      const float4 x0 = *reinterpret_cast<const float4 *>(a.x_in + off + g * 8);
+      const float4 x1 = *reinterpret_cast<const float4 *>(a.x_in + off + g * 8 + 4);
+      float o[8] = {x0.x + v[g * 8 + 0], x0.y + v[g * 8 + 1], x0.z + v[g * 8 + 2],
+                    x0.w + v[g * 8 + 3], x1.x + v[g * 8 + 4], x1.y + v[g * 8 + 5],
+                    x1.z + v[g * 8 + 6], x1.w + v[g * 8 + 7]};
+      *reinterpret_cast<float4 *>(a.x_out + off + g * 8) = make_float4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<float4 *>(a.x_out + off + g * 8 + 4) = make_float4(o[4], o[5], o[6], o[7]);
+      if (a.out_hi != nullptr) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) split_pack(o[j], o[j + 1], hi[j / 2], lo[j / 2]);
+        *reinterpret_cast<uint4 *>(a.out_hi + off + g * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(a.out_lo + off + g * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+  }
+}
+
+// ---- the kernel ------------------------------------------------------------
+
+template <int MODE, int A_PLANES, int SPLIT_S>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+              const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
+  using L = Layout<A_PLANES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t *ctrl = smem_raw + pad + L::TILES_BYTES;
+  const uint32_t sbase = raw_s + pad;
+  const uint32_t cbase = sbase + L::TILES_BYTES;
+  // control block: full[4] @0, empty[4] @64, tfull[2] @128, tempty[2] @144,
+  // redbar[2] @160, drain @176, tmem base @192, abort flag @196, red @256
+  auto full_bar = [&](int s) { return cbase + 8u * s; };
+  auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
+  auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
+  auto tempty_bar = [&](int i) { return cbase + 144u + 8u * i; };
+  auto red_bar = [&](int i) { return cbase + 160u + 8u * i; };
+  const uint32_t drain_bar = cbase + 176u;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 192);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 196);
+  float *red = reinterpret_cast<float *>(ctrl + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), 4);
+      mbar_init(red_bar(i), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(ctrl + 192), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA0);
+    if (A_PLANES == 2) prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int kchunks = (a.kdim + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        int b, mt, nt;
+        decode_tile<MODE>(a, tile, b, mt, nt);
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = sbase + stage * L::STAGE_BYTES;
+          mbar_arrive_expect_tx(full_bar(stage), L::STAGE_BYTES);
+          tma_load_3d(st, &tmA0, full_bar(stage), kc * BK, mt * BM, b);
+          if (A_PLANES == 2) tma_load_3d(st + L::A_BYTES, &tmA1, full_bar(stage), kc * BK, mt * BM, b);
+          tma_load_3d(st + A_PLANES * L::A_BYTES, &tmB, full_bar(stage), kc * BK, nt * BN, b);
+          ++issued;
+          if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      // Drain: every load issued must land before the CTA may exit.
+      for (int s = 0; s < L::STAGES; ++s) {
+        if (issued > s) {
+          const long long last = ((issued - 1 - s) / L::STAGES) * L::STAGES + s;
+          mbar_wait_drain(full_bar(s), static_cast<uint32_t>((last / L::STAGES) & 1));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + stage * L::STAGE_BYTES;
+          const uint64_t da0 = sdesc_k_sw128(st);
+          const uint64_t da1 = sdesc_k_sw128(st + L::A_BYTES);
+          const uint64_t db = sdesc_k_sw128(st + A_PLANES * L::A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // +32 bytes along K inside the 128-byte swizzled row = +2 in the
+            // descriptor's 16-byte address units.
+            tc_mma_bf16(d_tmem, da0 + 2u * kk, db + 2u * kk, idesc, (kc | kk) != 0);
+            if (A_PLANES == 2) tc_mma_bf16(d_tmem, da1 + 2u * kk, db + 2u * kk, idesc, 1u);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      tc_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+      int b, mt, nt;
+      decode_tile<MODE>(a, tile, b, mt, nt);
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr =
+          tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int row = mt * BM + quarter * 32 + lane;
+      if constexpr (MODE == MODE_MAXSIM) {
+        float *red_acc = red + acc * kRedGroups * kRedCands;
+        epi_maxsim_rows<SPLIT_S>(taddr, lane, quarter, red_acc);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(red_bar(acc));
+        if (warp == 2) {
+          // leader warp: combine the four warps' partial sums
+          if (!mbar_wait(red_bar(acc), acc_phase, abort_flag)) {
+            ok = false;
+          } else {
+            epi_maxsim_write<SPLIT_S>(a, red_acc, lane, b, mt, nt);
+          }
+        }
+      } else if constexpr (MODE == MODE_ENRICH) {
+        epi_enrich(a, taddr, row, nt);
+      } else {
+        epi_fuse(a, taddr, row, nt);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (!ok) break;
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int MODE, int A_PLANES, int SPLIT_S>
+avey_status run_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b, TcArgs args,
+                   cudaStream_t st, const char *name) {
+  using L = Layout<A_PLANES>;
+  if (args.num_tiles <= 0) return AVEY_OK;
+  auto kern = tc_kernel<MODE, A_PLANES, SPLIT_S>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::SMEM_BYTES));
+  if (e != cudaSuccess) {
+    set_detail("%s: cudaFuncSetAttribute: %s", name, cudaGetErrorString(e));
+    return AVEY_ERR_CUDA;
+  }
+  const int grid = std::min(args.num_tiles, sm_count());
+  kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(a0, a1, b, args);
+  AVEY_CHECK_LAUNCH(name);
+  return AVEY_OK;
+}
+
+TcArgs base_args(int rows, int cols, int kdim) {
+  TcArgs a{};
+  a.rows = rows;
+  a.cols = cols;
+  a.kdim = kdim;
+  a.tiles_m = (rows + BM - 1) / BM;
+  a.tiles_n = (cols + BN - 1) / BN;
+  a.num_tiles = a.tiles_m * a.tiles_n;
+  a.group_m = 1;
+  a.status = device_status_word();
+  return a;
+}
+
+}  // namespace
+
+avey_status launch_maxsim_tc(const bf16 *xhat, int B, int R, int d, int S, int n, float *scores,
+                             cudaStream_t s) {
+  CUtensorMap ma, mb;
+  const uint64_t rs = static_cast<uint64_t>(d) * 2, bs = rs * static_cast<uint64_t>(R);
+  if (!encode_bf16_map(&ma, xhat, d, R, B, rs, bs, BM)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&mb, xhat, d, R, B, rs, bs, BN)) return AVEY_ERR_CUDA;
+  TcArgs a = base_args(R, R, d);
+  a.num_tiles = a.tiles_m * a.tiles_n * B;
+  a.group_m = 16;
+  a.S = S;
+  a.n = n;
+  a.scores = scores;
+  switch (S) {
+    case 16: return run_tc<MODE_MAXSIM, 1, 16>(ma, ma, mb, a, s, "maxsim_tc");
+    case 32: return run_tc<MODE_MAXSIM, 1, 32>(ma, ma, mb, a, s, "maxsim_tc");
+    case 64: return run_tc<MODE_MAXSIM, 1, 64>(ma, ma, mb, a, s, "maxsim_tc");
+    case 128: return run_tc<MODE_MAXSIM, 1, 128>(ma, ma, mb, a, s, "maxsim_tc");
+    default: set_detail("maxsim_tc: S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
+  }
+}
+
+avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, const bf16 *Ut,
+                             int m, const float *bias, const float *inv_rms, bf16 *zhi,
+                             bf16 *zlo, cudaStream_t s) {
+  CUtensorMap a0, a1, mb;
+  const uint64_t rs = static_cast<uint64_t>(d) * 2;
+  if (!encode_bf16_map(&a0, xhi, d, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&a1, xlo, d, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&mb, Ut, d, m, 1, rs, rs * m, BN)) return AVEY_ERR_CUDA;
+  TcArgs a = base_args(T, m, d);
+  a.bias = bias;
+  a.inv_rms = inv_rms;
+  a.out_hi = zhi;
+  a.out_lo = zlo;
+  a.ld_out = m;
+  return run_tc<MODE_ENRICH, 2, 0>(a0, a1, mb, a, s, "enrich_tc");
+}
+
+avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
+                           const float *x_in, float *x_out, bf16 *xo_hi, bf16 *xo_lo,
+                           cudaStream_t s) {
+  CUtensorMap a0, a1, mb;
+  const uint64_t rs = static_cast<uint64_t>(m) * 2;
+  if (!encode_bf16_map(&a0, ahi, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&a1, alo, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&mb, Ot, m, d, 1, rs, rs * d, BN)) return AVEY_ERR_CUDA;
+  TcArgs a = base_args(T, d, m);
+  a.x_in = x_in;
+  a.x_out = x_out;
+  a.out_hi = xo_hi;
+  a.out_lo = xo_lo;
+  a.ld_out = d;
+  return run_tc<MODE_FUSE, 2, 0>(a0, a1, mb, a, s, "fuse_tc");
+}
+
+}  // namespace avey

@@ -1,0 +1,400 @@
+"""Benchmark of the Avey-B ranker + neural-processor hot path on B200.
+
+One step = one full encoder forward of the long-context workload (batch 1,
+N = 98304 tokens, S = 64, d = 768, m = 1536 (768/768), k = 7, four layers
+S,D,S,D): avey_rank (normalise, MaxSim, top-k) -> avey_compress -> 4 x
+avey_layer_forward, through the C ABI, on inputs already resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torchrun: every rank encodes its own sequence (weak
+scaling, no data-path collective; NCCL carries only the barrier and the
+max-over-ranks of the timings).  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference this build
+has) on the host cores, on a bounded sample of target splits of the same
+workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic as sy  # noqa: E402
+
+WORKLOAD = "long_bf16"
+METRIC = "encoder tokens/sec at N=96K d=768 (1 B200); MaxSim % tensor peak, mix % HBM BW"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+THROTTLE_BAD = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+REASONS = ("gpu_idle", "applications_clocks_setting", "sw_power_cap", "hw_slowdown",
+           "hw_thermal_slowdown", "hw_power_brake_slowdown", "sw_thermal_slowdown", "sync_boost")
+
+
+# ------------------------------------------------------------- utilities ---
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def workload_desc(wl) -> str:
+    kinds = ",".join("S" if k == sy.STATIC else "D" for k in wl.pattern)
+    return (f"{wl.name}: B={wl.B} N={wl.N} S={wl.S} d={wl.d} m={wl.m} ({wl.m_h}/{wl.m_t}) "
+            f"k={wl.k} layers={kinds} prenorm={int(wl.prenorm)}")
+
+
+def maxsim_flops(wl) -> float:
+    """Algorithmic MaxSim work per forward: 2 * (n S)^2 * d per sequence."""
+    R = wl.n * wl.S
+    return 2.0 * wl.B * R * R * wl.d
+
+
+def layer_flops(wl) -> float:
+    """Enricher + fuser GEMMs, 2 T d m each, per layer."""
+    return wl.layers * 2 * (2.0 * wl.T * wl.d * wl.m)
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"avey_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        q = "clocks.sm,clocks.max.sm," + ",".join(f"clocks_event_reasons.{r}" for r in REASONS)
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, active = [], [], set()
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 2 + len(REASONS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for r, v in zip(REASONS, parts[2:]):
+                if v.lower().startswith("active"):
+                    active.add(r)
+        # samples taken while the GPU idled at the edges are not "under load"
+        busy = [s for s in sm if smax and s > 0.3 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(active - {"gpu_idle"}), "samples": len(sm)}
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(backend: str, world: int):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Embedding seed of the sequence a rank encodes (rank 0 = the parity seed)."""
+    return rank
+
+
+def traffic_from_profile(kernel_src: str):
+    """DRAM bytes per MaxSim launch from the committed ncu summary, or None when
+    the kernel source changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "maxsim_long_bf16.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m1 = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    m2 = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    if not (m1 and m2):
+        return None
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    return float(m1.group(1)) if sha == m2.group(1) else None
+
+
+# ----------------------------------------------------------- CPU baseline ---
+
+def cpu_baseline(wl, E, W, budget_s: float = 15.0, max_splits: int = 64):
+    """The fp64 oracle as it stands, on this host's cores, on a bounded sample
+    of target splits of the same workload (rank, compression, every layer)."""
+    import oracle as orc
+    X64 = E.X.astype(np.float64)
+    one = sy.sample_targets(wl, 1, seed=100)[:1]
+    t0 = time.perf_counter()
+    orc.forward(X64, W, wl, sel=one)
+    t_one = time.perf_counter() - t0
+    count = int(max(1, min(max_splits, budget_s / max(t_one, 1e-3))))
+    sel = sy.sample_targets(wl, count, seed=101)[:count]
+    t0 = time.perf_counter()
+    orc.forward(X64, W, wl, sel=sel)
+    el = time.perf_counter() - t0
+    toks = sel.shape[0] * wl.S
+    return {"value": toks / el, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+            "sample": f"{sel.shape[0]} seeded target splits x {wl.S} tokens of {wl.name} "
+                      f"(full rank row, compression, {wl.layers} layers each), {el:.1f} s"}
+
+
+# -------------------------------------------------------------- our arm ---
+
+def run_ours(args):
+    import torch
+    import attention_free_long_b200 as av
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl", world)
+    barrier = (lambda: dist.barrier(device_ids=[local])) if world > 1 else (lambda: None)
+
+    wl = sy.WORKLOADS[args.workload]
+    E = sy.gen_embeddings(wl, seed=rank_seed(rank))
+    W = sy.gen_weights(wl)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    x = torch.from_numpy(E.X).to(dev, dt)
+    P = torch.from_numpy(W.P).to(dev, dt)
+    layers = av.device_layers(W, dt, dev)
+    ws = av.make_workspace(wl.B, wl.N, wl.d, wl.S, wl.k, wl.m, dt, wl.prenorm, dev)
+
+    def step(marks=None):
+        return av.encoder_forward(x, P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm, ws, marks)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = av.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after warm-up")
+
+    # ---- device-timed region: inputs resident in HBM (X is 151 MB > L2) ----
+    n_marks = 2 + wl.layers
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks + 1)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    l0 = av.kernel_launches()
+    with ClockSampler(local) as clk:
+        start.record()
+        for s in range(args.steps):
+            step(marks[s])
+        end.record()
+        torch.cuda.synchronize()
+    launches = av.kernel_launches() - l0
+    barrier()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / args.steps
+    ms_max = max_over_ranks(ms, dev)
+    stage = np.array([[marks[s][i].elapsed_time(marks[s][i + 1]) for i in range(n_marks)]
+                      for s in range(args.steps)]).mean(axis=0)
+    rank_ms, compress_ms, layer_ms = float(stage[0]), float(stage[1]), stage[2:].tolist()
+    st = av.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after the timed region")
+
+    # ---- dynamic mix alone at the layer's shape (HBM-bound kernel) ----
+    T, mt = wl.T, wl.m_t
+    zpair = torch.rand((2, T, wl.m), device=dev).to(torch.bfloat16)
+    zt = zpair[:, :, wl.m_h:]
+    L = av.lib()
+    import ctypes
+    mix_call = lambda: L.avey_dynamic_mix(ctypes.c_void_p(zt.data_ptr()), wl.m, av.AVEY_BF16X2,
+                                          T // wl.S, wl.S, mt, wl.eps,
+                                          ctypes.c_void_p(zt.data_ptr()), wl.m, av._stream())
+    for _ in range(3):
+        assert mix_call() == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(10, args.steps)
+    e0.record()
+    for _ in range(reps):
+        mix_call()
+    e1.record()
+    torch.cuda.synchronize()
+    mix_ms = e0.elapsed_time(e1) / reps
+    del zpair, zt
+
+    # ---- end to end through the public API with host buffers ----
+    xh = torch.from_numpy(E.X).to(dt).pin_memory()
+    outh = torch.empty((wl.B, wl.n * wl.S, wl.d), dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(x)
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        out = av.encoder_forward(xd, P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm, ws)
+        outh.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(args.steps):
+        e2e_step()
+    end.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
+
+    tokens = wl.B * wl.N * world
+    peaks, peak_kind = load_peaks()
+    sustained = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    achieved = maxsim_flops(wl) / (rank_ms * 1e-3) / 1e12
+    mix_bytes = 2.0 * T * mt * 4  # read Z_t pair, write c pair
+    comp_bytes = (wl.k + 1) * wl.T * wl.d * 2.0 + wl.T * wl.d * 8.0
+    kernel_src = os.path.join(ROOT, "attention_free_long_b200", "csrc", "avey_tc.cu")
+    result = {
+        "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian mixture, random N(0,1/fan_in) weights)",
+        "config": {"workload": workload_desc(wl), "global_batch": wl.B * world, "seq_len": wl.N,
+                   "parallelism": f"dp{world} (one sequence per GPU, no collective)",
+                   "l2": "inputs larger than L2 (X is 151 MB bf16, 126 MB L2); no flush"},
+        "roofline": {"bound": "tensor", "kernel": "maxsim (avey_rank call)",
+                     "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                     "frac": achieved / sustained,
+                     "peak_kind": f"{peak_kind} bf16 sustained (kernel inside a long step)",
+                     "algorithmic_flop_per_launch": maxsim_flops(wl),
+                     "traffic": traffic_from_profile(kernel_src),
+                     "note": "duration is the whole avey_rank call (normalise + MaxSim + top-k)"},
+        "kernels_ms": {"rank": rank_ms, "compress": compress_ms, "layers": layer_ms},
+        "hbm": {"dynamic_mix": {"ms": mix_ms, "gbs": mix_bytes / (mix_ms * 1e-3) / 1e9,
+                                "frac": mix_bytes / (mix_ms * 1e-3) / 1e9 / hbm,
+                                "peak": hbm, "bytes": mix_bytes},
+                "compress": {"ms": compress_ms, "gbs": comp_bytes / (compress_ms * 1e-3) / 1e9,
+                             "frac": comp_bytes / (compress_ms * 1e-3) / 1e9 / hbm,
+                             "bytes": comp_bytes}},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
+                "d2h_bytes_per_step": int(outh.numel() * outh.element_size())},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, E, W)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# -------------------------------------------------------- reference arm ---
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle as orc
+    wl = sy.WORKLOADS[args.workload]
+    E, W = sy.gen_embeddings(wl, seed=0), sy.gen_weights(wl)
+    X64 = E.X.astype(np.float64)
+    t0 = time.perf_counter()
+    orc.forward(X64, W, wl, sel=sy.sample_targets(wl, 1, seed=200)[:1])
+    t_one = time.perf_counter() - t0
+    budget = 150.0
+    per_step = int(max(1, min(16, budget / max(1, args.steps + args.warmup) / max(t_one, 1e-3))))
+    for i in range(args.warmup):
+        orc.forward(X64, W, wl, sel=sy.sample_targets(wl, per_step, seed=300 + i)[:per_step])
+    el = 0.0
+    for i in range(args.steps):
+        sel = sy.sample_targets(wl, per_step, seed=400 + i)[:per_step]
+        t0 = time.perf_counter()
+        orc.forward(X64, W, wl, sel=sel)
+        el += time.perf_counter() - t0
+    toks = args.steps * per_step * wl.S
+    value = toks / el
+    sample = (f"{per_step} seeded target splits x {wl.S} tokens of {wl.name} per step "
+              f"(full rank row, compression, {wl.layers} layers each)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Gaussian mixture, random N(0,1/fan_in) weights)",
+        "config": {"workload": workload_desc(wl), "global_batch": wl.B, "seq_len": wl.N,
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(sy.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    _, world, _ = dist_env()
+    if world != args.gpus:
+        if args.gpus > 1:
+            ap.error(f"--gpus {args.gpus} needs torchrun with {args.gpus} ranks (WORLD_SIZE={world})")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,215 @@
+/*
+ * avey.h -- C ABI of the B200 (sm_100a) Avey-B ranker and neural-processor
+ * library (libavey.so).
+ *
+ * Pages defining the operations (cited by title and section):
+ *   [AB-notes] "Avey-B: 把无注意力架构改造成双向编码器" (papernotes.org ICLR 2026
+ *              note): 方法详解 整体框架 (splits, MaxSim ranker, top-k,
+ *              divide-by-max weights, enricher Z = sigma(XU+b), fuser
+ *              f = [Z_h || c(Z_t)] O plus residual); 关键设计 2 (static layer
+ *              c = V Z_t, dynamic layer N(Z_t) N(Z_t)^T); 关键设计 3 (eq. 6,
+ *              divide by row sum + eps); 关键设计 4 (eq. 8, X_hat = P X_cat,
+ *              residual to the split's own tokens).
+ *   [AB-sum]   "Avey-B" (paperlayer.ai summary of arXiv 2602.15814v1): §3
+ *              Background (ranker, enricher/contextualizer/fuser), §4
+ *              (bidirectional, decoupled layers, compression), App. A (ReLU^2
+ *              enricher), App. B (S -> D interleaving), App. H (ranker once,
+ *              on the initial embeddings).
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers unless a parameter says otherwise.  The
+ *     caller allocates and owns every buffer, including workspaces; the
+ *     library never allocates device memory and keeps no per-call state.
+ *   - Row-major, densely packed tensors unless an leading dimension ("ld",
+ *     in elements) is given.  Base addresses must be 16-byte aligned.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *     Argument errors are detected on the host BEFORE any launch and return
+ *     AVEY_ERR_INVALID_ARG / AVEY_ERR_UNSUPPORTED with nothing enqueued.
+ *     Launch failures return AVEY_ERR_CUDA.
+ *   - Kernel-side failures (a bounded wait that ran out, a failed bounds
+ *     check) never trap: the kernel records a code in a device status word
+ *     and returns.  Read it with avey_device_status().
+ *   - Padding: a sequence of N tokens is cut into n = ceil(N/S) splits of S
+ *     tokens; the last split is zero-padded ([AB-notes] 整体框架).  Outputs
+ *     that are per token have n*S rows per sequence; the caller keeps the
+ *     first N.
+ *
+ * Types
+ *   AVEY_F32    fp32 everywhere (SIMT kernels, fp32 accumulate).
+ *   AVEY_BF16   bf16 embeddings and weights; tensor-core contractions with
+ *               fp32 accumulation; fp32 residual stream.
+ *   AVEY_BF16X2 a "split" activation: an fp32 value x held as two bf16 planes,
+ *               hi = bf16(x) and lo = bf16(x - hi), the lo plane directly
+ *               after the hi plane (plane stride = rows * ld elements).  Layer
+ *               activations use it so that products against bf16 weights
+ *               keep about 16 significant bits.
+ */
+#ifndef AVEY_H_
+#define AVEY_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AVEY_API __attribute__((visibility("default")))
+#else
+#define AVEY_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *avey_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  AVEY_OK = 0,
+  AVEY_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer, too-small workspace */
+  AVEY_ERR_UNSUPPORTED = 2,    /* valid but not implemented shape/dtype combination */
+  AVEY_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+  AVEY_ERR_DEVICE_TIMEOUT = 4, /* a kernel's bounded wait ran out (reported by avey_device_status) */
+  AVEY_ERR_DEVICE_BOUNDS = 5   /* a kernel's bounds check failed (reported by avey_device_status) */
+} avey_status;
+
+typedef enum { AVEY_F32 = 0, AVEY_BF16 = 1, AVEY_BF16X2 = 2 } avey_dtype;
+
+typedef enum { AVEY_STATIC = 0, AVEY_DYNAMIC = 1 } avey_ctx_kind;
+
+/* ------------------------------------------------------------------ ranker --
+ * avey_rank: the ranker, run once per forward on the input embeddings
+ * ([AB-sum] App. H).
+ *   1. N(x) = x / max(||x||_2, 1e-12) per token (pad rows are zero).
+ *   2. MaxSim score(t, c) = sum_{i in split t} max_{j in split c} N(x_i).N(x_j)
+ *      for every ordered pair of splits of the same sequence (bidirectional:
+ *      [AB-sum] §4; definition: [AB-sum] §3, [AB-notes] 整体框架).  The
+ *      (n*S) x (n*S) similarity matrix is never materialised.
+ *   3. Top-k per target split over c != t, ordered by (score desc, index asc);
+ *      w_r = s_r / s_1 so the best selected split has weight exactly 1
+ *      ([AB-notes] 整体框架: "divide by the largest").
+ *
+ * x       [B, N, d], dtype dt (AVEY_F32 or AVEY_BF16), read only.
+ * idx     [B, n, k] int32 out: selected splits in rank order; -1 where n-1 < k.
+ * w       [B, n, k] fp32 out: normalised weights (0 where idx is -1).
+ * scores  [B, n, n] fp32 out, or NULL: the full split-score matrix (diagonal
+ *         included), written when non-NULL.
+ * ws      device workspace of at least avey_rank_workspace_bytes(...) bytes,
+ *         256-byte aligned.  Contents are scratch (undefined afterwards).
+ * Constraints: B, N, d, S, k >= 1; d % 8 == 0; k <= 32.  AVEY_BF16 needs S in
+ * {16, 32, 64, 128}; AVEY_F32 needs S a power of two <= 128.
+ */
+AVEY_API avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
+                      int32_t *idx, float *w, float *scores, void *ws, size_t ws_bytes,
+                      avey_stream_t stream);
+
+AVEY_API size_t avey_rank_workspace_bytes(avey_dtype dt, int B, int N, int d, int S);
+
+/* ---------------------------------------------------------- compression --
+ * avey_compress: neural compression of each split with its retrieved splits
+ * plus the residual to the split's own tokens ([AB-notes] 关键设计 4, eq. 8):
+ *   X_cat(t) = [X_t ; w_1 X_c1 ; ... ; w_k X_ck]   ((k+1)S x d, rank order)
+ *   out(t)   = P X_cat(t) + X_t,   P in R^{S x (k+1)S}, shared by all splits.
+ * A candidate index of -1 contributes a zero block.
+ *
+ * x        [B, N, d] embeddings, dtype dt (AVEY_F32 or AVEY_BF16).
+ * idx, w   [B, n, k] from avey_rank (any int32 in [-1, n) is accepted; out of
+ *          range indices are rejected on the device as AVEY_ERR_DEVICE_BOUNDS
+ *          and their block is treated as zero).
+ * P        [S, (k+1)S], dtype dt.
+ * out      [B, n*S, d] fp32 out (the residual stream entering layer 0).
+ * out_lowp for AVEY_BF16: NULL or an AVEY_BF16X2 pair [2][B*n*S][d] of `out`
+ *          (what avey_layer_forward reads as x_in_lowp).  Ignored for F32.
+ * Constraints: d % 8 == 0; k <= 32; AVEY_BF16 needs S in {16, 32, 64, 128};
+ * AVEY_F32 needs S a power of two <= 64.
+ */
+AVEY_API avey_status avey_compress(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
+                          const int32_t *idx, const float *w, const void *P, float *out,
+                          void *out_lowp, avey_stream_t stream);
+
+/* ----------------------------------------------------------- dynamic mix --
+ * avey_dynamic_mix: the dynamic contextualizer of one layer on `blocks`
+ * independent split blocks of S tokens ([AB-notes] 关键设计 2 and 3):
+ *   G_ij  = N(z_i) . N(z_j)              (cosine, N(z) = z / max(||z||, 1e-12))
+ *   Gt_ij = G_ij / (sum_j G_ij + eps)    (eq. 6)
+ *   c     = Gt Z_t                        (identity activation, no bias)
+ * zt   block b, token i, feature f at zt[(b*S + i) * ld_zt + f], f < mt.
+ *      AVEY_F32: fp32.  AVEY_BF16X2: split pair, lo plane at
+ *      zt + blocks*S*ld_zt elements.
+ * out  same layout and dtype with ld_out (lo plane at out + blocks*S*ld_out).
+ *      out may alias zt exactly (in place); partial overlap is not allowed.
+ * Constraints: S in {16, 32, 64, 128} for AVEY_BF16X2 (a power of two <= 64
+ * for F32);
+ * mt % 8 == 0 and ld % 8 == 0 for AVEY_BF16X2; eps >= 0.
+ */
+AVEY_API avey_status avey_dynamic_mix(const void *zt, int64_t ld_zt, avey_dtype dt, int blocks, int S,
+                             int mt, float eps, void *out, int64_t ld_out, avey_stream_t stream);
+
+/* ----------------------------------------------------------------- layer --
+ * avey_layer_forward: one neural-processor layer on T = blocks * S tokens
+ * ([AB-notes] 整体框架, 关键设计 2-3; [AB-sum] §3, App. A):
+ *   xin = prenorm ? x / sqrt(mean(x^2) + 1e-6) : x   (per token; see below)
+ *   Z   = relu(xin U + b)^2                          (enricher, ReLU^2)
+ *   Z_h = Z[:, :m_h],  Z_t = Z[:, m_h:]              (head bypass / tail)
+ *   c   = V Z_t (static) or Gt Z_t (dynamic), per split of S tokens
+ *   x'  = x + [Z_h || c] O                           (fuser + residual)
+ * `prenorm` is an option of this library, not of the pages: a gain-free RMS
+ * norm of the enricher input that keeps deep stacks finite.  It leaves the
+ * residual path untouched.
+ *
+ * Weights (dtype = dt: AVEY_F32, or AVEY_BF16 for the tensor-core path):
+ *   Ut [m, d]  the enricher matrix U stored transposed (row f holds U[:, f])
+ *   bU [m]     fp32 enricher bias (fp32 for both dtypes)
+ *   V  [S, S]  static map (AVEY_STATIC), NULL for AVEY_DYNAMIC
+ *   Ot [d, m]  the fuser matrix O stored transposed (row q holds O[:, q])
+ * Activations:
+ *   x_in      [T, d] fp32 residual stream in.
+ *   x_in_lowp AVEY_BF16 only: NULL or the AVEY_BF16X2 pair of x_in (as
+ *             written by avey_compress / the previous layer).  When NULL the
+ *             pair is built in the workspace.
+ *   x_out     [T, d] fp32 out (may alias x_in exactly).
+ *   x_out_lowp AVEY_BF16 only: NULL or an AVEY_BF16X2 pair [2][T][d] out.
+ *   ws        >= avey_layer_workspace_bytes(...) bytes, 256-byte aligned.
+ * Constraints: T % S == 0; d, m, m_h multiples of 8 with 0 < m_h < m;
+ * S in {16, 32, 64, 128} for AVEY_BF16 (a power of two <= 64 for F32); eps >= 0.
+ */
+typedef struct {
+  avey_ctx_kind kind;
+  int d, m, m_h, S;
+  float eps;
+  int prenorm;
+  const void *Ut;
+  const float *bU;
+  const void *V;
+  const void *Ot;
+} avey_layer_params;
+
+AVEY_API avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype dt, int T,
+                               const float *x_in, const void *x_in_lowp, float *x_out,
+                               void *x_out_lowp, void *ws, size_t ws_bytes,
+                               avey_stream_t stream);
+
+AVEY_API size_t avey_layer_workspace_bytes(avey_dtype dt, int T, int d, int m, int prenorm);
+
+/* ------------------------------------------------------------- utilities --
+ * avey_device_status: synchronises `stream`, returns the first kernel-side
+ * failure recorded since the previous call (AVEY_ERR_DEVICE_TIMEOUT or
+ * AVEY_ERR_DEVICE_BOUNDS) or AVEY_OK, and clears it.  Returns AVEY_ERR_CUDA
+ * if the synchronisation itself fails.
+ */
+AVEY_API avey_status avey_device_status(avey_stream_t stream);
+
+/* avey_status_string: static, never NULL. */
+AVEY_API const char *avey_status_string(avey_status s);
+
+/* avey_last_error_detail: a static description of the last host-side
+ * rejection or CUDA error in this thread (empty string if none). */
+AVEY_API const char *avey_last_error_detail(void);
+
+/* avey_kernel_launches: number of kernels this library has launched since it
+ * was loaded, in this process (all threads). */
+AVEY_API uint64_t avey_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AVEY_H_ */
