@@ -14,9 +14,11 @@ using bf16 = __nv_bfloat16;
 
 // ---- tcgen05 contractions (avey_tc.cu) ----
 
-// MaxSim split scores: xhat [B, R = n*S, d] bf16 (unit rows, zero pad rows).
-avey_status launch_maxsim_tc(const bf16 *xhat, int B, int R, int d, int S, int n, float *scores,
-                             cudaStream_t s);
+// MaxSim split scores from the raw embeddings x [B, N, d] bf16 and the
+// inverse row norms inv_norm [B, rs_ld] (rs_ld >= R rounded up to 256, zero
+// past N); R = n*S.
+avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N, int R, int rs_ld,
+                             int d, int S, int n, float *scores, cudaStream_t s);
 
 // Enricher: Z = relu(scale_row * (X U) + b)^2, X given as a split pair
 // (xhi, xlo) [T, d]; Ut [m, d]; writes the split pair of Z (zhi, zlo) [T, m].
@@ -33,6 +35,8 @@ avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const
 
 // ---- ranker pieces (avey_rank.cu) ----
 avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, int S, void *xhat,
+                             cudaStream_t s);
+avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, float *inv,
                              cudaStream_t s);
 avey_status launch_topk(const float *scores, int B, int n, int k, int32_t *idx, float *w,
                         cudaStream_t s);

@@ -2,9 +2,11 @@
 // top-k selection with divide-by-max weights (Avey-B paperlayer summary §3
 // Background and App. H; papernotes 整体框架).
 //
-//   normalize_rows   N(x) = x / max(||x||, 1e-12) per token, padded to n*S
-//                    rows per sequence (pad rows zero); bf16 or fp32 out.
-//   maxsim (bf16)    tcgen05 kernel in avey_tc.cu.
+//   inv_norms        (bf16) 1/max(||x||, 1e-12) per token, 0 for the pad rows
+//                    of the last split; the tcgen05 MaxSim (avey_tc.cu) reads
+//                    the raw bf16 rows and applies these scales in its epilogue.
+//   normalize_rows   (fp32) N(x) = x / max(||x||, 1e-12) per token, padded to
+//                    n*S rows per sequence (pad rows zero).
 //   maxsim_f32       SIMT fp32 version (one CTA per target/candidate pair).
 //   topk_warp        one warp per target split: k rounds of a warp-wide
 //                    argmax over the split's score row held in shared memory,
@@ -138,6 +140,36 @@ __global__ void __launch_bounds__(256) maxsim_f32(const float *__restrict__ xhat
   }
 }
 
+// One warp per row of inv [B, rs_ld]: rows < N get 1/max(||x||, 1e-12),
+// rows >= N (split padding and tile padding) get 0.
+__global__ void __launch_bounds__(256) inv_norms(const bf16 *__restrict__ x, int B, int N, int d,
+                                                 int rs_ld, float *__restrict__ inv) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(B) * rs_ld) return;
+  const int b = static_cast<int>(row / rs_ld);
+  const int tok = static_cast<int>(row - static_cast<long long>(b) * rs_ld);
+  if (tok >= N) {
+    if (lane == 0) inv[row] = 0.f;
+    return;
+  }
+  const bf16 *src = x + (static_cast<long long>(b) * N + tok) * d;
+  float ss = 0.f;
+  for (int j = lane * 8; j < d; j += 256) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(src + j);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = unpack_bf16(w4[q]);
+      ss = fmaf(f.x, f.x, ss);
+      ss = fmaf(f.y, f.y, ss);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if (lane == 0) inv[row] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+}
+
 constexpr int kTopkWarps = 4;
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
@@ -207,6 +239,14 @@ avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, 
   return AVEY_OK;
 }
 
+avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, float *inv,
+                             cudaStream_t s) {
+  const long long rows = static_cast<long long>(B) * rs_ld;
+  inv_norms<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(x, B, N, d, rs_ld, inv);
+  AVEY_CHECK_LAUNCH("inv_norms");
+  return AVEY_OK;
+}
+
 avey_status launch_topk(const float *scores, int B, int n, int k, int32_t *idx, float *w,
                         cudaStream_t s) {
   const long long rows = static_cast<long long>(B) * n;
@@ -248,11 +288,16 @@ static avey_status launch_maxsim_f32(const float *xhat, int B, int R, int d, int
 
 using namespace avey;
 
+// Padded row count of the inverse-norm table: a multiple of the MaxSim
+// column tile (256) so that every tile's scale loads stay in bounds.
+static inline long long scale_ld(long long R) { return (R + 255) / 256 * 256; }
+
 extern "C" size_t avey_rank_workspace_bytes(avey_dtype dt, int B, int N, int d, int S) {
   if (B <= 0 || N <= 0 || d <= 0 || S <= 0) return 0;
   const long long n = (N + S - 1) / S, R = n * S;
-  const size_t es = dt == AVEY_F32 ? 4 : 2;
-  return align256(static_cast<size_t>(B) * R * d * es) + align256(static_cast<size_t>(B) * n * n * 4);
+  const size_t first = dt == AVEY_F32 ? static_cast<size_t>(B) * R * d * 4   // normalised copy
+                                      : static_cast<size_t>(B) * scale_ld(R) * 4;  // 1/||x||
+  return align256(first) + align256(static_cast<size_t>(B) * n * n * 4);
 }
 
 extern "C" avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
@@ -285,19 +330,26 @@ extern "C" avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int
                "avey_rank: n=%lld too large for the top-k kernel", n);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const size_t es = dt == AVEY_F32 ? 4 : 2;
   char *wsb = static_cast<char *>(ws);
-  void *xhat = wsb;
-  float *sc = scores ? scores : reinterpret_cast<float *>(wsb + align256(static_cast<size_t>(B) * R * d * es));
+  const size_t first = dt == AVEY_F32 ? static_cast<size_t>(B) * R * d * 4
+                                      : static_cast<size_t>(B) * scale_ld(R) * 4;
+  float *sc = scores ? scores : reinterpret_cast<float *>(wsb + align256(first));
 
-  avey_status st = launch_normalize(x, dt, B, N, d, S, xhat, s);
-  if (st != AVEY_OK) return st;
-  if (dt == AVEY_BF16)
-    st = launch_maxsim_tc(static_cast<const bf16 *>(xhat), B, static_cast<int>(R), d, S,
+  avey_status st;
+  if (dt == AVEY_BF16) {
+    float *inv = reinterpret_cast<float *>(wsb);
+    const int ld = static_cast<int>(scale_ld(R));
+    st = launch_inv_norms(static_cast<const bf16 *>(x), B, N, d, ld, inv, s);
+    if (st != AVEY_OK) return st;
+    st = launch_maxsim_tc(static_cast<const bf16 *>(x), inv, B, N, static_cast<int>(R), ld, d, S,
                           static_cast<int>(n), sc, s);
-  else
+  } else {
+    void *xhat = wsb;
+    st = launch_normalize(x, dt, B, N, d, S, xhat, s);
+    if (st != AVEY_OK) return st;
     st = launch_maxsim_f32(static_cast<const float *>(xhat), B, static_cast<int>(R), d, S,
                            static_cast<int>(n), sc, s);
+  }
   if (st != AVEY_OK) return st;
   return launch_topk(sc, B, static_cast<int>(n), k, idx, w, s);
 }

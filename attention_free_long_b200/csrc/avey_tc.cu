@@ -3,10 +3,13 @@
 // One persistent, warp-specialised kernel template serves three contractions:
 //
 //   MaxSim  (ranker, Avey-B paperlayer summary §3 and papernotes 整体框架):
-//           D = Xhat_tile(128 rows) . Xhat_tile(256 rows)^T per sequence; the
-//           epilogue takes, per row, the max over each candidate split's S
-//           columns, then sums those maxima over the S rows of each target
-//           split, so only the [B, n, n] split scores reach HBM.
+//           D = X_tile(128 rows) . X_tile(256 rows)^T per sequence on the raw
+//           bf16 embeddings (exact products, fp32 accumulation); the epilogue
+//           scales each column by 1/||x_j||, takes per row the max over each
+//           candidate split's S columns, scales it by 1/||x_i|| (a positive
+//           factor commutes with the max), then sums the maxima over the S
+//           rows of each target split.  Only the [B, n, n] split scores reach
+//           HBM; neither the N x N cosines nor a normalised copy of X exist.
 //   Enricher (papernotes 整体框架, Z = sigma(XU+b); ReLU^2 per the paperlayer
 //           summary App. A): D = X U with X as a bf16 split pair (two MMAs per
 //           K step); epilogue scale (optional prenorm) + bias + ReLU^2, Z
@@ -48,6 +51,8 @@ struct TcArgs {
   // MaxSim
   int S, n;
   float *scores;
+  const float *inv_norm;  // [batch][rs_ld] 1/max(||x||, 1e-12), 0 for pad rows
+  int rs_ld;
   // enricher
   const float *bias;
   const float *inv_rms;
@@ -105,17 +110,28 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
 // Per-row maxima over each candidate split's columns, summed over the rows of
 // each target split inside this warp; partial sums go to red[group][cand].
 template <int S>
-__device__ __forceinline__ void epi_maxsim_rows(uint32_t taddr, int lane, int quarter,
-                                                float *red) {
+__device__ __forceinline__ void epi_maxsim_rows(uint32_t taddr, int lane, int quarter, float *red,
+                                                const float *__restrict__ col_scale,
+                                                float row_scale) {
   constexpr int NC = BN / S;
   float mx[NC];
 #pragma unroll
   for (int c = 0; c < NC; ++c) mx[c] = -INFINITY;
 #pragma unroll
   for (int ch = 0; ch < BN / 32; ++ch) {
+    const float4 *cs4 = reinterpret_cast<const float4 *>(col_scale + ch * 32);
+    float4 c4[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) c4[q] = __ldg(cs4 + q);
     float v[32];
     tmem_ld32(taddr + ch * 32, v);
-    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      v[4 * q] *= c4[q].x;
+      v[4 * q + 1] *= c4[q].y;
+      v[4 * q + 2] *= c4[q].z;
+      v[4 * q + 3] *= c4[q].w;
+    }
     if constexpr (S >= 32) {
       float m = v[0];
 #pragma unroll
@@ -133,6 +149,8 @@ __device__ __forceinline__ void epi_maxsim_rows(uint32_t taddr, int lane, int qu
       mx[2 * ch + 1] = m1;
     }
   }
+#pragma unroll
+  for (int c = 0; c < NC; ++c) mx[c] *= row_scale;
   if constexpr (S >= 32) {
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
@@ -184,7 +202,6 @@ __device__ __forceinline__ void epi_enrich(const TcArgs &a, uint32_t taddr, int 
   for (int ch = 0; ch < BN / 32; ++ch) {
     float v[32];
     tmem_ld32(taddr + ch * 32, v);
-    tmem_ld_wait();
     const int col0 = nt * BN + ch * 32;
     if (!valid || col0 >= a.cols) continue;
     bf16 *ph = a.out_hi + static_cast<long long>(row) * a.ld_out + col0;
@@ -214,7 +231,6 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, uint32_t taddr, int ro
   for (int ch = 0; ch < BN / 32; ++ch) {
     float v[32];
     tmem_ld32(taddr + ch * 32, v);
-    tmem_ld_wait();
     const int col0 = nt * BN + ch * 32;
     if (!valid || col0 >= a.cols) continue;
     const long long off = static_cast<long long>(row) * a.cols + col0;
@@ -402,7 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = mt * BM + quarter * 32 + lane;
       if constexpr (MODE == MODE_MAXSIM) {
         float *red_acc = red + acc * kRedGroups * kRedCands;
-        epi_maxsim_rows<SPLIT_S>(taddr, lane, quarter, red_acc);
+        const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
+        epi_maxsim_rows<SPLIT_S>(taddr, lane, quarter, red_acc, rs + nt * BN, rs[row]);
         __syncwarp();
         if (lane == 0) mbar_arrive(red_bar(acc));
         if (warp == 2) {
@@ -472,18 +489,22 @@ TcArgs base_args(int rows, int cols, int kdim) {
 
 }  // namespace
 
-avey_status launch_maxsim_tc(const bf16 *xhat, int B, int R, int d, int S, int n, float *scores,
-                             cudaStream_t s) {
+avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N, int R, int rs_ld,
+                             int d, int S, int n, float *scores, cudaStream_t s) {
+  // The maps cover the unpadded [B, N, d] embeddings: rows N..R-1 of the last
+  // split (and any tile rows past R) read as zeros, which is the padding.
   CUtensorMap ma, mb;
-  const uint64_t rs = static_cast<uint64_t>(d) * 2, bs = rs * static_cast<uint64_t>(R);
-  if (!encode_bf16_map(&ma, xhat, d, R, B, rs, bs, BM)) return AVEY_ERR_CUDA;
-  if (!encode_bf16_map(&mb, xhat, d, R, B, rs, bs, BN)) return AVEY_ERR_CUDA;
+  const uint64_t rs = static_cast<uint64_t>(d) * 2, bs = rs * static_cast<uint64_t>(N);
+  if (!encode_bf16_map(&ma, x, d, N, B, rs, bs, BM)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&mb, x, d, N, B, rs, bs, BN)) return AVEY_ERR_CUDA;
   TcArgs a = base_args(R, R, d);
   a.num_tiles = a.tiles_m * a.tiles_n * B;
   a.group_m = 16;
   a.S = S;
   a.n = n;
   a.scores = scores;
+  a.inv_norm = inv_norm;
+  a.rs_ld = rs_ld;
   switch (S) {
     case 16: return run_tc<MODE_MAXSIM, 1, 16>(ma, ma, mb, a, s, "maxsim_tc");
     case 32: return run_tc<MODE_MAXSIM, 1, 32>(ma, ma, mb, a, s, "maxsim_tc");

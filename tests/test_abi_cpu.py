@@ -52,10 +52,13 @@ def test_status_strings():
 
 
 def test_workspace_sizes():
-    # X_hat bf16 + scores fp32, each rounded up to 256 bytes
+    # bf16: 1/||x|| per padded row (rows rounded up to 256) + scores fp32
     n, R = 64, 64 * 64
-    expect = (8 * R * 768 * 2 + 255) // 256 * 256 + (8 * n * n * 4 + 255) // 256 * 256
+    expect = (8 * R * 4 + 255) // 256 * 256 + (8 * n * n * 4 + 255) // 256 * 256
     assert av.rank_workspace_bytes(av.AVEY_BF16, 8, 4096, 768, 64) == expect
+    # fp32: a normalised copy X_hat + scores
+    expect32 = (8 * R * 768 * 4 + 255) // 256 * 256 + (8 * n * n * 4 + 255) // 256 * 256
+    assert av.rank_workspace_bytes(av.AVEY_F32, 8, 4096, 768, 64) == expect32
     assert av.rank_workspace_bytes(av.AVEY_BF16, 0, 4096, 768, 64) == 0
     T, d, m = 4096, 768, 1536
     b = av.layer_workspace_bytes(av.AVEY_BF16, T, d, m, False)

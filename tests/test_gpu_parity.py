@@ -54,13 +54,16 @@ def run_gpu(wl, E, W, sel, dev):
     return res
 
 
+# Rows whose top-k lists differ by a near tie (checked by check_topk) are left
+# out of the downstream comparison: the oracle never takes the GPU's selection
+# as an input.  Mixtures with several splits per centre produce many such ties.
 def compare(wl, E, W, sel, dev):
     g = run_gpu(wl, E, W, sel, dev)
     o = orc.forward(E.X, W, wl, sel=sel)
     tol = TOL[wl.dtype]
     assert rel_err(g["scores"], o["scores"]) <= tol, "scores"
     exact = check_topk(g["idx"], g["w"], o["idx"], o["scores"], sel[:, 1], tol)
-    assert exact.mean() >= 0.9, f"only {exact.mean():.2f} of the rows have identical top-k lists"
+    assert exact.mean() >= 0.75, f"only {exact.mean():.2f} of the rows have identical top-k lists"
     keep = np.repeat(exact, wl.S)
     ref = [o["compressed"].reshape(-1, wl.d)] + [a.reshape(-1, wl.d) for a in o["layers"]]
     errs = [rel_err(gg[keep], oo[keep]) for gg, oo in zip(g["outs"], ref)]
@@ -71,17 +74,17 @@ def compare(wl, E, W, sel, dev):
 
 SMALL = [
     sy.custom("f32_s8", B=2, N=100, S=8, d=32, m=48, m_h=24, k=4, pattern=(sy.STATIC, sy.DYNAMIC),
-              dtype="f32", centers=3, sigma=0.4),
+              dtype="f32", centers=6, sigma=0.4),
     sy.custom("f32_s16_pre", B=1, N=250, S=16, d=64, m=128, k=3, pattern=(sy.DYNAMIC, sy.STATIC),
-              dtype="f32", centers=4, sigma=0.3, prenorm=True),
+              dtype="f32", centers=8, sigma=0.3, prenorm=True),
     sy.custom("bf16_s16", B=3, N=777, S=16, d=64, m=128, k=3, pattern=(sy.STATIC, sy.DYNAMIC),
-              centers=4, sigma=0.3),
+              centers=24, sigma=0.3),
     sy.custom("bf16_s32", B=2, N=2053, S=32, d=96, m=192, m_h=64, k=7,
-              pattern=(sy.DYNAMIC, sy.STATIC), centers=8, sigma=0.5),
+              pattern=(sy.DYNAMIC, sy.STATIC), centers=32, sigma=0.5),
     sy.custom("bf16_s64_ragged", B=2, N=1000, S=64, d=136, m=272, m_h=136, k=5,
-              pattern=(sy.STATIC, sy.DYNAMIC), centers=6, sigma=0.5),
+              pattern=(sy.STATIC, sy.DYNAMIC), centers=8, sigma=0.5),
     sy.custom("bf16_s128_pre", B=1, N=3000, S=128, d=128, m=256, k=15,
-              pattern=(sy.STATIC, sy.DYNAMIC, sy.STATIC), centers=8, sigma=0.5, prenorm=True),
+              pattern=(sy.STATIC, sy.DYNAMIC, sy.STATIC), centers=12, sigma=0.5, prenorm=True),
     sy.custom("bf16_k_gt_n", B=2, N=200, S=64, d=64, m=128, k=7, pattern=(sy.DYNAMIC,),
               centers=2, sigma=0.5),
 ]
@@ -110,7 +113,7 @@ def test_named_workloads_full(name, cuda_dev):
     compare(wl, E, W, orc.all_targets(wl.B, wl.n), cuda_dev)
 
 
-@pytest.mark.parametrize("name,per_seq", [("mid_bf16", 12), ("long_bf16", 20), ("large_bf16", 4)])
+@pytest.mark.parametrize("name,per_seq", [("mid_bf16", 24), ("long_bf16", 48), ("large_bf16", 4)])
 def test_named_workloads_sampled(name, per_seq, cuda_dev):
     wl = sy.WORKLOADS[name]
     E, W = sy.gen_embeddings(wl), sy.gen_weights(wl)
@@ -141,12 +144,11 @@ def test_dynamic_mix_entry_point(dtype, S, cuda_dev):
         got = av.avey_dynamic_mix(zt, S, 1e-8, mt=mt).cpu().numpy()[:, :mt]
         inplace = av.avey_dynamic_mix(zt, S, 1e-8, mt=mt, out=zt).cpu().numpy()[:, :mt]
     else:
-        zf = torch.from_numpy(z).to(cuda_dev)
-        hi = zf.to(torch.bfloat16)
-        lo = (zf - hi.float()).to(torch.bfloat16)
-        pair = torch.stack([hi, lo]).contiguous()
+        hi = sy.round_bf16(z)
+        lo = sy.round_bf16(z - hi)
+        pair = torch.from_numpy(np.stack([hi, lo])).to(cuda_dev, torch.bfloat16).contiguous()
         # the oracle sees exactly the value the pair represents
-        zrep = (hi.float() + lo.float()).cpu().numpy().astype(np.float64)
+        zrep = hi.astype(np.float64) + lo.astype(np.float64)
         ref = np.concatenate([orc.dynamic_mix(zrep[b * S:(b + 1) * S, :mt], 1e-8)
                               for b in range(blocks)])
         tol = TOL["bf16"]
