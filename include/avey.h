@@ -103,6 +103,28 @@ AVEY_API avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int d
 
 AVEY_API size_t avey_rank_workspace_bytes(avey_dtype dt, int B, int N, int d, int S);
 
+/* avey_rank_static: avey_rank for callers that cannot allocate device memory
+ * (a plugin interface that hands over only input and output buffers, or a
+ * host that forbids cudaMalloc on the calling path).  The pages have no
+ * counterpart: this is a deployment variant of the ranker, not a step of the
+ * method.  It computes exactly what avey_rank computes, with the same kernels,
+ * but its scratch lives in a fixed device array inside the library
+ * (avey_rank_static_max_scratch_bytes(), 16 MiB, held by every GPU that loads
+ * the library until the process exits) instead of a caller workspace.
+ *   - It allocates nothing.  A shape whose scratch
+ *     (avey_rank_workspace_bytes) exceeds the array is rejected with
+ *     AVEY_ERR_UNSUPPORTED before anything is enqueued.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array, which keeps the previous call's contents; every
+ *     call rewrites what it reads.  Calls whose kernels overlap on the GPU
+ *     (e.g. on two unordered streams) race on it: order them.
+ * Arguments and constraints as for avey_rank, without scores and workspace. */
+AVEY_API avey_status avey_rank_static(const void *x, avey_dtype dt, int B, int N, int d, int S,
+                                      int k, int32_t *idx, float *w, avey_stream_t stream);
+
+AVEY_API size_t avey_rank_static_max_scratch_bytes(void);
+
 /* ---------------------------------------------------------- compression --
  * avey_compress: neural compression of each split with its retrieved splits
  * plus the residual to the split's own tokens ([AB-notes] 关键设计 4, eq. 8):
