@@ -80,9 +80,9 @@ int sm_count() {
   return g_sms[dev];
 }
 
-bool encode_bf16_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
-                     uint64_t batch, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
-                     uint32_t box_rows) {
+bool encode_map(CUtensorMap *map, bool fp32, const void *base, uint64_t inner, uint64_t rows,
+                uint64_t batch, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
+                uint32_t box_inner, uint32_t box_rows, int swizzle_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     set_detail("cuTensorMapEncodeTiled is not available from the driver");
@@ -90,17 +90,29 @@ bool encode_bf16_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_
   }
   const cuuint64_t dims[3] = {inner, rows, batch};
   const cuuint64_t strides[2] = {row_stride_bytes, batch_stride_bytes};
-  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
-    set_detail("cuTensorMapEncodeTiled failed (%d): inner=%llu rows=%llu batch=%llu", int(r),
-               (unsigned long long)inner, (unsigned long long)rows, (unsigned long long)batch);
+    set_detail("cuTensorMapEncodeTiled failed (%d): inner=%llu rows=%llu batch=%llu box=%ux%u", int(r),
+               (unsigned long long)inner, (unsigned long long)rows, (unsigned long long)batch,
+               box_inner, box_rows);
     return false;
   }
   return true;
+}
+
+bool encode_bf16_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                     uint64_t batch, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
+                     uint32_t box_rows) {
+  return encode_map(map, false, base, inner, rows, batch, row_stride_bytes, batch_stride_bytes, 64,
+                    box_rows, 128);
 }
 
 }  // namespace avey

@@ -33,6 +33,11 @@ int sm_count();
 bool encode_bf16_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                      uint64_t batch, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
                      uint32_t box_rows);
+// General 3-D tiled map: element type (bf16 or fp32), box {box_inner,
+// box_rows, 1}, swizzle 64 or 128 (bytes of the swizzle span).
+bool encode_map(CUtensorMap *map, bool fp32, const void *base, uint64_t inner, uint64_t rows,
+                uint64_t batch, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
+                uint32_t box_inner, uint32_t box_rows, int swizzle_bytes);
 
 #define AVEY_CHECK_LAUNCH(name)                                             \
   do {                                                                      \
@@ -125,6 +130,34 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// TMA: 3-D tiled store from shared memory (bulk-group completion).  Out of
+// range parts of the box are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y,
+                                             int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until at most N committed bulk groups still read their shared source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Waits until every committed bulk group has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {

@@ -72,8 +72,12 @@ struct Layout {
   static constexpr uint32_t STAGE_BYTES = A_PLANES * A_BYTES + B_BYTES;
   static constexpr int STAGES = A_PLANES == 1 ? 4 : 3;
   static constexpr uint32_t TILES_BYTES = STAGES * STAGE_BYTES;
-  static constexpr uint32_t CTRL_BYTES = 256 + 2 * kRedGroups * kRedCands * 4;
-  static constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + 1024;
+  // barriers etc. (+ the MaxSim partial sums), rounded up to 1 KB
+  static constexpr uint32_t CTRL_BYTES = A_PLANES == 1 ? 2048 : 1024;
+  // layer GEMMs: per epilogue warp 8 KB of swizzled output staging for TMA stores
+  static constexpr uint32_t STAGING_BYTES = A_PLANES == 1 ? 0 : 4 * 8192;
+  static constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + STAGING_BYTES + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 template <int MODE>
@@ -113,12 +117,15 @@ template <int S>
 __device__ __forceinline__ void epi_maxsim_rows(uint32_t taddr, int lane, int quarter, float *red,
                                                 const float *__restrict__ col_scale,
                                                 float row_scale) {
-  constexpr int NC = BN / S;
-  float mx[NC];
-#pragma unroll
-  for (int c = 0; c < NC; ++c) mx[c] = -INFINITY;
-#pragma unroll
-  for (int ch = 0; ch < BN / 32; ++ch) {
+  // One 32-column TMEM chunk at a time: scale the columns by 1/||x_j||, take
+  // the running row max of the candidate split, and once a candidate split is
+  // complete scale by 1/||x_i|| and sum over the warp's rows.
+  constexpr int CH_PER_CAND = S >= 32 ? S / 32 : 1;
+  constexpr int CANDS_PER_CH = S >= 32 ? 1 : 32 / S;
+  constexpr int NCH = BN / 32;
+  float m[CANDS_PER_CH];
+#pragma unroll 1
+  for (int ch = 0; ch < NCH; ++ch) {
     const float4 *cs4 = reinterpret_cast<const float4 *>(col_scale + ch * 32);
     float4 c4[8];
 #pragma unroll
@@ -132,45 +139,31 @@ __device__ __forceinline__ void epi_maxsim_rows(uint32_t taddr, int lane, int qu
       v[4 * q + 2] *= c4[q].z;
       v[4 * q + 3] *= c4[q].w;
     }
-    if constexpr (S >= 32) {
-      float m = v[0];
+    if (ch % CH_PER_CAND == 0) {
 #pragma unroll
-      for (int i = 1; i < 32; ++i) m = fmaxf(m, v[i]);
-      constexpr int per = S / 32;
-      mx[ch / per] = fmaxf(mx[ch / per], m);
-    } else {
-      float m0 = v[0], m1 = v[16];
+      for (int u = 0; u < CANDS_PER_CH; ++u) m[u] = -INFINITY;
+    }
 #pragma unroll
-      for (int i = 1; i < 16; ++i) {
-        m0 = fmaxf(m0, v[i]);
-        m1 = fmaxf(m1, v[16 + i]);
+    for (int u = 0; u < CANDS_PER_CH; ++u) {
+      constexpr int W = 32 / CANDS_PER_CH;
+#pragma unroll
+      for (int i = 0; i < W; ++i) m[u] = fmaxf(m[u], v[u * W + i]);
+    }
+    if (ch % CH_PER_CAND == CH_PER_CAND - 1) {
+#pragma unroll
+      for (int u = 0; u < CANDS_PER_CH; ++u) {
+        const int cand = (ch / CH_PER_CAND) * CANDS_PER_CH + u;
+        float t = m[u] * row_scale;
+        if constexpr (S >= 32) {
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+          if (lane == 0) red[quarter * kRedCands + cand] = t;
+        } else {
+#pragma unroll
+          for (int off = 8; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+          if ((lane & 15) == 0) red[(quarter * 2 + (lane >> 4)) * kRedCands + cand] = t;
+        }
       }
-      mx[2 * ch] = m0;
-      mx[2 * ch + 1] = m1;
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < NC; ++c) mx[c] *= row_scale;
-  if constexpr (S >= 32) {
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mx[c] += __shfl_xor_sync(0xffffffffu, mx[c], off);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int c = 0; c < NC; ++c) red[quarter * kRedCands + c] = mx[c];
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-#pragma unroll
-      for (int off = 8; off > 0; off >>= 1) mx[c] += __shfl_xor_sync(0xffffffffu, mx[c], off);
-    }
-    if ((lane & 15) == 0) {
-      const int g = quarter * 2 + (lane >> 4);
-#pragma unroll
-      for (int c = 0; c < NC; ++c) red[g * kRedCands + c] = mx[c];
     }
   }
 }
@@ -195,63 +188,131 @@ __device__ __forceinline__ void epi_maxsim_write(const TcArgs &a, const float *r
   }
 }
 
-__device__ __forceinline__ void epi_enrich(const TcArgs &a, uint32_t taddr, int row, int nt) {
+// Output staging for TMA stores.  Each epilogue warp owns 8 KB and writes
+// one 32-row x 32-column chunk at a time: row r (lane r) of an fp32 chunk is
+// 128 bytes with its 16-byte pieces in the 128-byte swizzle order, a bf16
+// chunk row is 64 bytes in the 64-byte swizzle order; the TMA store unswizzles
+// them.  Both orders keep each shared-memory store conflict free.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+__device__ __forceinline__ uint32_t sw64_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+// Enricher epilogue: Z = relu(scale * acc + b)^2 as a split pair, two staging
+// buffers of 4 KB (hi 2 KB + lo 2 KB) alternate so that the TMA store of one
+// chunk overlaps the math of the next.  `it` counts chunks across tiles.
+__device__ __forceinline__ void epi_enrich(const TcArgs &a, const CUtensorMap *mhi,
+                                           const CUtensorMap *mlo, uint32_t taddr, int row0,
+                                           int lane, int nt, uint32_t stg, int &it) {
+  const int row = row0 + lane;
   const bool valid = row < a.rows;
   const float scale = (a.inv_rms != nullptr && valid) ? a.inv_rms[row] : 1.f;
 #pragma unroll 1
   for (int ch = 0; ch < BN / 32; ++ch) {
+    const int col0 = nt * BN + ch * 32;
+    if (col0 >= a.cols) break;  // warp-uniform
+    float4 bb[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      bb[q] = (col0 + 4 * q < a.cols) ? __ldg(reinterpret_cast<const float4 *>(a.bias + col0) + q)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
     float v[32];
     tmem_ld32(taddr + ch * 32, v);
-    const int col0 = nt * BN + ch * 32;
-    if (!valid || col0 >= a.cols) continue;
-    bf16 *ph = a.out_hi + static_cast<long long>(row) * a.ld_out + col0;
-    bf16 *pl = a.out_lo + static_cast<long long>(row) * a.ld_out + col0;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      if (col0 + g * 8 >= a.cols) break;
-      const float4 b0 = __ldg(reinterpret_cast<const float4 *>(a.bias + col0 + g * 8));
-      const float4 b1 = __ldg(reinterpret_cast<const float4 *>(a.bias + col0 + g * 8 + 4));
-      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        float z0 = fmaxf(fmaf(v[g * 8 + j], scale, bb[j]), 0.f);
-        float z1 = fmaxf(fmaf(v[g * 8 + j + 1], scale, bb[j + 1]), 0.f);
-        split_pack(z0 * z0, z1 * z1, hi[j / 2], lo[j / 2]);
-      }
-      *reinterpret_cast<uint4 *>(ph + g * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4 *>(pl + g * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    const uint32_t buf = stg + (it & 1) * 4096;
+    if (it >= 2) {  // the store issued from this buffer two chunks ago must have read it
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
     }
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float b4[4] = {bb[q].x, bb[q].y, bb[q].z, bb[q].w};
+#pragma unroll
+      for (int j = 0; j < 4; j += 2) {
+        float z0 = fmaxf(fmaf(v[4 * q + j], scale, b4[j]), 0.f);
+        float z1 = fmaxf(fmaf(v[4 * q + j + 1], scale, b4[j + 1]), 0.f);
+        split_pack(z0 * z0, z1 * z1, hi[2 * q + j / 2], lo[2 * q + j / 2]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      st_shared_v4(buf + sw64_off(lane, c), hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+      st_shared_v4(buf + 2048 + sw64_off(lane, c), lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(mhi, buf, col0, row0, 0);
+      tma_store_3d(mlo, buf + 2048, col0, row0, 0);
+      bulk_commit();
+    }
+    (void)valid;
+    ++it;
   }
 }
 
-__device__ __forceinline__ void epi_fuse(const TcArgs &a, uint32_t taddr, int row, int nt) {
+// Fuser epilogue: x_out = x_in + acc (fp32) and its split pair; one 8 KB
+// staging buffer (fp32 4 KB, hi 2 KB, lo 2 KB).  The residual loads are
+// issued before the TMEM load so that their latency overlaps it.
+__device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mout,
+                                         const CUtensorMap *mhi, const CUtensorMap *mlo,
+                                         uint32_t taddr, int row0, int lane, int nt, uint32_t stg,
+                                         int &it) {
+  const int row = row0 + lane;
   const bool valid = row < a.rows;
+  const bool pair = a.out_hi != nullptr;
 #pragma unroll 1
   for (int ch = 0; ch < BN / 32; ++ch) {
+    const int col0 = nt * BN + ch * 32;
+    if (col0 >= a.cols) break;  // warp-uniform
+    const float4 *src = reinterpret_cast<const float4 *>(a.x_in + static_cast<long long>(row) * a.cols + col0);
+    float4 xi[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      xi[q] = (valid && col0 + 4 * q < a.cols) ? src[q] : make_float4(0.f, 0.f, 0.f, 0.f);
     float v[32];
     tmem_ld32(taddr + ch * 32, v);
-    const int col0 = nt * BN + ch * 32;
-    if (!valid || col0 >= a.cols) continue;
-    const long long off = static_cast<long long>(row) * a.cols + col0;
+    if (it >= 1) {  // the previous chunk's stores must have read the buffer
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+    }
+    float o[32];
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      if (col0 + g * 8 >= a.cols) break;
-      const float4 x0 = *reinterpret_cast<const float4 *>(a.x_in + off + g * 8);
-      const float4 x1 = *reinterpret_cast<const float4 *>(a.x_in + off + g * 8 + 4);
-      float o[8] = {x0.x + v[g * 8 + 0], x0.y + v[g * 8 + 1], x0.z + v[g * 8 + 2],
-                    x0.w + v[g * 8 + 3], x1.x + v[g * 8 + 4], x1.y + v[g * 8 + 5],
-                    x1.z + v[g * 8 + 6], x1.w + v[g * 8 + 7]};
-      *reinterpret_cast<float4 *>(a.x_out + off + g * 8) = make_float4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<float4 *>(a.x_out + off + g * 8 + 4) = make_float4(o[4], o[5], o[6], o[7]);
-      if (a.out_hi != nullptr) {
-        uint32_t hi[4], lo[4];
+    for (int q = 0; q < 8; ++q) {
+      o[4 * q] = xi[q].x + v[4 * q];
+      o[4 * q + 1] = xi[q].y + v[4 * q + 1];
+      o[4 * q + 2] = xi[q].z + v[4 * q + 2];
+      o[4 * q + 3] = xi[q].w + v[4 * q + 3];
+    }
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) split_pack(o[j], o[j + 1], hi[j / 2], lo[j / 2]);
-        *reinterpret_cast<uint4 *>(a.out_hi + off + g * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(a.out_lo + off + g * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    for (int c = 0; c < 8; ++c)
+      st_shared_v4(stg + sw128_off(lane, c), __float_as_uint(o[4 * c]), __float_as_uint(o[4 * c + 1]),
+                   __float_as_uint(o[4 * c + 2]), __float_as_uint(o[4 * c + 3]));
+    if (pair) {
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) split_pack(o[2 * j], o[2 * j + 1], hi[j], lo[j]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        st_shared_v4(stg + 4096 + sw64_off(lane, c), hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+        st_shared_v4(stg + 6144 + sw64_off(lane, c), lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
       }
     }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(mout, stg, col0, row0, 0);
+      if (pair) {
+        tma_store_3d(mhi, stg + 4096, col0, row0, 0);
+        tma_store_3d(mlo, stg + 6144, col0, row0, 0);
+      }
+      bulk_commit();
+    }
+    ++it;
   }
 }
 
@@ -260,7 +321,9 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, uint32_t taddr, int ro
 template <int MODE, int A_PLANES, int SPLIT_S>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-              const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
+              const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmO0,
+              const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2,
+              const TcArgs a) {
   using L = Layout<A_PLANES>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -304,6 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmA0);
     if (A_PLANES == 2) prefetch_tmap(&tmA1);
     prefetch_tmap(&tmB);
+    if (MODE != MODE_MAXSIM) {
+      prefetch_tmap(&tmO0);
+      prefetch_tmap(&tmO1);
+      if (MODE == MODE_FUSE) prefetch_tmap(&tmO2);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -402,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-    int acc = 0;
+    const uint32_t stg = cbase + L::CTRL_BYTES + static_cast<uint32_t>(warp - 2) * 8192u;
+    int acc = 0, it = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
@@ -431,9 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if constexpr (MODE == MODE_ENRICH) {
-        epi_enrich(a, taddr, row, nt);
+        epi_enrich(a, &tmO0, &tmO1, taddr, row - lane, lane, nt, stg, it);
       } else {
-        epi_fuse(a, taddr, row, nt);
+        epi_fuse(a, &tmO0, &tmO1, &tmO2, taddr, row - lane, lane, nt, stg, it);
       }
       tc_fence_before();
       __syncwarp();
@@ -446,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       *abort_flag = 1;
       record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
     }
+    if (MODE != MODE_MAXSIM && lane == 0) bulk_wait_all();  // outputs written before exit
   }
 
   tc_fence_before();
@@ -457,7 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int MODE, int A_PLANES, int SPLIT_S>
-avey_status run_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b, TcArgs args,
+avey_status run_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+                   const CUtensorMap &o0, const CUtensorMap &o1, const CUtensorMap &o2, TcArgs args,
                    cudaStream_t st, const char *name) {
   using L = Layout<A_PLANES>;
   if (args.num_tiles <= 0) return AVEY_OK;
@@ -469,7 +540,7 @@ avey_status run_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorM
     return AVEY_ERR_CUDA;
   }
   const int grid = std::min(args.num_tiles, sm_count());
-  kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(a0, a1, b, args);
+  kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(a0, a1, b, o0, o1, o2, args);
   AVEY_CHECK_LAUNCH(name);
   return AVEY_OK;
 }
@@ -506,10 +577,10 @@ avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N,
   a.inv_norm = inv_norm;
   a.rs_ld = rs_ld;
   switch (S) {
-    case 16: return run_tc<MODE_MAXSIM, 1, 16>(ma, ma, mb, a, s, "maxsim_tc");
-    case 32: return run_tc<MODE_MAXSIM, 1, 32>(ma, ma, mb, a, s, "maxsim_tc");
-    case 64: return run_tc<MODE_MAXSIM, 1, 64>(ma, ma, mb, a, s, "maxsim_tc");
-    case 128: return run_tc<MODE_MAXSIM, 1, 128>(ma, ma, mb, a, s, "maxsim_tc");
+    case 16: return run_tc<MODE_MAXSIM, 1, 16>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
+    case 32: return run_tc<MODE_MAXSIM, 1, 32>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
+    case 64: return run_tc<MODE_MAXSIM, 1, 64>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
+    case 128: return run_tc<MODE_MAXSIM, 1, 128>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
     default: set_detail("maxsim_tc: S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
   }
 }
@@ -517,35 +588,45 @@ avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N,
 avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, const bf16 *Ut,
                              int m, const float *bias, const float *inv_rms, bf16 *zhi,
                              bf16 *zlo, cudaStream_t s) {
-  CUtensorMap a0, a1, mb;
-  const uint64_t rs = static_cast<uint64_t>(d) * 2;
+  CUtensorMap a0, a1, mb, o0, o1;
+  const uint64_t rs = static_cast<uint64_t>(d) * 2, zs = static_cast<uint64_t>(m) * 2;
   if (!encode_bf16_map(&a0, xhi, d, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&a1, xlo, d, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&mb, Ut, d, m, 1, rs, rs * m, BN)) return AVEY_ERR_CUDA;
+  if (!encode_map(&o0, false, zhi, m, T, 1, zs, zs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
+  if (!encode_map(&o1, false, zlo, m, T, 1, zs, zs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
   TcArgs a = base_args(T, m, d);
   a.bias = bias;
   a.inv_rms = inv_rms;
   a.out_hi = zhi;
   a.out_lo = zlo;
   a.ld_out = m;
-  return run_tc<MODE_ENRICH, 2, 0>(a0, a1, mb, a, s, "enrich_tc");
+  return run_tc<MODE_ENRICH, 2, 0>(a0, a1, mb, o0, o1, o1, a, s, "enrich_tc");
 }
 
 avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
                            const float *x_in, float *x_out, bf16 *xo_hi, bf16 *xo_lo,
                            cudaStream_t s) {
-  CUtensorMap a0, a1, mb;
+  CUtensorMap a0, a1, mb, o0, o1, o2;
   const uint64_t rs = static_cast<uint64_t>(m) * 2;
+  const uint64_t fs = static_cast<uint64_t>(d) * 4, hs = static_cast<uint64_t>(d) * 2;
   if (!encode_bf16_map(&a0, ahi, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&a1, alo, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&mb, Ot, m, d, 1, rs, rs * d, BN)) return AVEY_ERR_CUDA;
+  if (!encode_map(&o0, true, x_out, d, T, 1, fs, fs * T, 32, 32, 128)) return AVEY_ERR_CUDA;
+  o1 = o0;
+  o2 = o0;
+  if (xo_hi != nullptr) {
+    if (!encode_map(&o1, false, xo_hi, d, T, 1, hs, hs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
+    if (!encode_map(&o2, false, xo_lo, d, T, 1, hs, hs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
+  }
   TcArgs a = base_args(T, d, m);
   a.x_in = x_in;
   a.x_out = x_out;
   a.out_hi = xo_hi;
   a.out_lo = xo_lo;
   a.ld_out = d;
-  return run_tc<MODE_FUSE, 2, 0>(a0, a1, mb, a, s, "fuse_tc");
+  return run_tc<MODE_FUSE, 2, 0>(a0, a1, mb, o0, o1, o2, a, s, "fuse_tc");
 }
 
 }  // namespace avey
