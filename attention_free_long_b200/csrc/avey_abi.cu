@@ -115,9 +115,41 @@ bool encode_bf16_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_
                     box_rows, 128);
 }
 
+// Self-test of the bounded waits: one warp waits on an mbarrier that nothing
+// ever arrives on, through the same wait routine the tcgen05 kernels use,
+// with a short limit; on expiry it records the timeout and returns.
+__global__ void wait_timeout_probe(uint64_t limit_ns, int *status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    if (!mbar_wait_limit(smem_u32(&bar), 0, &abort_flag, limit_ns))
+      record_status(status, AVEY_ERR_DEVICE_TIMEOUT);
+    // complete the barrier's phase so nothing is left pending
+    mbar_arrive(smem_u32(&bar));
+  }
+}
+
 }  // namespace avey
 
 extern "C" {
+
+avey_status avey_selftest_wait_timeout(uint32_t limit_us, avey_stream_t stream) {
+  AVEY_REQUIRE(limit_us >= 1 && limit_us <= 2000000, AVEY_ERR_INVALID_ARG,
+               "avey_selftest_wait_timeout: limit_us must be in [1, 2000000]");
+  int *st = avey::device_status_word();
+  AVEY_REQUIRE(st != nullptr, AVEY_ERR_CUDA, "avey_selftest_wait_timeout: no device status word");
+  avey::wait_timeout_probe<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull, st);
+  AVEY_CHECK_LAUNCH("wait_timeout_probe");
+  return AVEY_OK;
+}
+
 
 avey_status avey_device_status(avey_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

@@ -226,6 +226,14 @@ AVEY_API const char *avey_status_string(avey_status s);
  * rejection or CUDA error in this thread (empty string if none). */
 AVEY_API const char *avey_last_error_detail(void);
 
+/* avey_selftest_wait_timeout: diagnostic with no counterpart on the pages.
+ * Launches one warp that waits, through the same bounded wait the tcgen05
+ * kernels use, on a barrier nothing arrives on, for limit_us microseconds
+ * (1 .. 2e6); the wait then gives up, records AVEY_ERR_DEVICE_TIMEOUT in the
+ * device status word and the kernel returns.  The next avey_device_status()
+ * reports it; the context stays usable. */
+AVEY_API avey_status avey_selftest_wait_timeout(uint32_t limit_us, avey_stream_t stream);
+
 /* avey_kernel_launches: number of kernels this library has launched since it
  * was loaded, in this process (all threads). */
 AVEY_API uint64_t avey_kernel_launches(void);
