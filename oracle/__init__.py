@@ -57,6 +57,11 @@ def lib():
                                                ctypes.c_int, _I, _I, ctypes.c_int, _D]
             L.avey_orc_topk_row.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _D]
             L.avey_orc_topk_row.restype = ctypes.c_int
+            L.avey_orc_topk_row_dir.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, _I, _D]
+            L.avey_orc_topk_row_dir.restype = ctypes.c_int
+            L.avey_orc_coupled_causal_mix.argtypes = [_D, _D, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_longlong, _D, ctypes.c_longlong]
             L.avey_orc_compress_rows.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int, _I, _I, ctypes.c_int, _I, _D, _D,
                                                  _D]
@@ -129,11 +134,13 @@ def all_targets(B: int, n: int) -> np.ndarray:
     return np.stack([bb.ravel(), tt.ravel()], axis=1).astype(np.int32)
 
 
-def topk(scores_rows, targets, k: int):
+def topk(scores_rows, targets, k: int, causal: bool = False):
     """Top-k (self excluded, ties -> lower index) and w = s / s_best.
 
-    scores_rows [n_sel, n]; targets [n_sel] target split index of each row.
-    Returns idx int32 [n_sel, k] (-1 where n-1 < k) and w float64 [n_sel, k].
+    scores_rows [n_sel, n]; targets [n_sel] target split index of each row;
+    causal: candidates only c < t (unidirectional ranker).
+    Returns idx int32 [n_sel, k] (-1 where fewer than k candidates) and
+    w float64 [n_sel, k].
     """
     sc = _f64(scores_rows)
     n_sel, n = sc.shape
@@ -142,11 +149,12 @@ def topk(scores_rows, targets, k: int):
     L = lib()
     for s in range(n_sel):
         row = np.ascontiguousarray(sc[s])
-        L.avey_orc_topk_row(_pd(row), n, int(targets[s]), k, _pi(idx[s]), _pd(w[s]))
+        L.avey_orc_topk_row_dir(_pd(row), n, int(targets[s]), k, int(bool(causal)), _pi(idx[s]),
+                                _pd(w[s]))
     return idx, w
 
 
-def rank(X, S: int, k: int, sel=None):
+def rank(X, S: int, k: int, sel=None, causal: bool = False):
     """Ranker for the selected (b, t) targets (all targets when sel is None).
 
     Returns (sel, scores [n_sel, n], idx [n_sel, k], w [n_sel, k]).
@@ -156,7 +164,7 @@ def rank(X, S: int, k: int, sel=None):
     n = -(-N // S)
     sel = all_targets(B, n) if sel is None else _i32(sel).reshape(-1, 2)
     scores = maxsim_rows(X, S, sel)
-    idx, w = topk(scores, sel[:, 1], k)
+    idx, w = topk(scores, sel[:, 1], k, causal)
     return sel, scores, idx, w
 
 
@@ -181,6 +189,15 @@ def static_mix(V, zt) -> np.ndarray:
     S, mt = zt.shape
     c = np.empty((S, mt), dtype=np.float64)
     lib().avey_orc_static_mix(_pd(V), _pd(zt), S, mt, mt, _pd(c), mt)
+    return c
+
+
+def coupled_causal_mix(V, zt) -> np.ndarray:
+    """c = (V * N(Z)N(Z)^T, masked to j <= i) Z_t for one split (original Avey)."""
+    V, zt = _f64(V), _f64(zt)
+    S, mt = zt.shape
+    c = np.empty((S, mt), dtype=np.float64)
+    lib().avey_orc_coupled_causal_mix(_pd(V), _pd(zt), S, mt, mt, _pd(c), mt)
     return c
 
 
@@ -224,7 +241,7 @@ def layer(x_splits, lw, S: int, m_h: int, eps: float, prenorm: bool) -> np.ndarr
     return x
 
 
-def forward(X, weights, wl, sel=None, idx=None, w=None):
+def forward(X, weights, wl, sel=None, idx=None, w=None, causal: bool = False):
     """Ranker once, compression, then every layer, for selected targets.
 
     X [B, N, d]; weights: synthetic.Weights; wl: synthetic.Workload.
@@ -233,7 +250,7 @@ def forward(X, weights, wl, sel=None, idx=None, w=None):
     Returns dict(sel, scores, idx, w, compressed, layers=[per-layer outputs]).
     """
     X = _f64(X)
-    sel, scores, oidx, ow = rank(X, wl.S, wl.k, sel)
+    sel, scores, oidx, ow = rank(X, wl.S, wl.k, sel, causal)
     use_idx = oidx if idx is None else _i32(idx)
     use_w = ow if w is None else _f64(w)
     xc = compress(X, wl.S, wl.k, sel, use_idx, use_w, weights.P)

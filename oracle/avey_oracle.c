@@ -42,6 +42,9 @@
 
 #define NORM_FLOOR 1e-12
 
+void avey_orc_coupled_causal_mix(const double *V, const double *zt, int S, int mt, long long ld,
+                                 double *c, long long ldc);
+
 int avey_orc_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
@@ -141,11 +144,22 @@ static int cand_cmp(const void *pa, const void *pb) {
  * ([AB-notes] 整体框架: "divide by the largest of them"; [AB-sum] §3).
  * Returns the number of real candidates k' = min(k, n-1); positions >= k' get
  * idx -1 and weight 0. */
+int avey_orc_topk_row_dir(const double *scores, int n, int t, int k, int causal, int *idx,
+                          double *w);
+
 int avey_orc_topk_row(const double *scores, int n, int t, int k, int *idx, double *w) {
+  return avey_orc_topk_row_dir(scores, n, t, k, 0, idx, w);
+}
+
+/* As above; with causal != 0 the candidates are only the preceding splits
+ * c < t (the unidirectional ranker of the original Avey, and the ablation
+ * setting of [AB-sum] App. B "Ranker direction"). */
+int avey_orc_topk_row_dir(const double *scores, int n, int t, int k, int causal, int *idx,
+                          double *w) {
   cand_t *cand = (cand_t *)malloc(sizeof(cand_t) * (size_t)(n > 0 ? n : 1));
   int m = 0;
   for (int c = 0; c < n; ++c)
-    if (c != t) {
+    if (c != t && (!causal || c < t)) {
       cand[m].score = scores[c];
       cand[m].idx = c;
       ++m;
@@ -247,7 +261,9 @@ void avey_orc_dynamic_mix(const double *zt, int S, int mt, long long ld, double 
  *   head/tail Z_h = Z[:, :m_h], Z_t = Z[:, m_h:]   ([AB-notes] 整体框架)
  *   context   c = V Z_t (static) or Gt Z_t (dynamic)
  *   fuser     X' = X + [Z_h || c] O               ([AB-notes] 整体框架)
- * U is [d, m], bU [m], V [S, S] (static only), O [m, d]. */
+ * kind: 0 static, 1 dynamic, 2 coupled causal (original Avey, see
+ * avey_orc_coupled_causal_mix).
+ * U is [d, m], bU [m], V [S, S] (static and coupled), O [m, d]. */
 void avey_orc_layer(double *x, int n_splits, int S, int d, int m, int m_h, int kind, int prenorm,
                     double eps, const double *U, const double *bU, const double *V,
                     const double *O) {
@@ -285,8 +301,10 @@ void avey_orc_layer(double *x, int n_splits, int S, int d, int m, int m_h, int k
     }
     if (kind == 0)
       avey_orc_static_mix(V, Z + m_h, S, mt, m, c, mt);
-    else
+    else if (kind == 1)
       avey_orc_dynamic_mix(Z + m_h, S, mt, m, eps, c, mt);
+    else
+      avey_orc_coupled_causal_mix(V, Z + m_h, S, mt, m, c, mt);
     /* X'[i, q] = X[i, q] + sum_f [Z_h || c][i, f] O[f, q], the sum over f in
      * order (f outer so that the q loop walks contiguous rows of O) */
     for (int i = 0; i < S; ++i) {
@@ -313,4 +331,25 @@ void avey_orc_compress_rows(const double *x, int N, int d, int S, int k, const i
   for (int s = 0; s < n_sel; ++s)
     avey_orc_compress_split(x, N, d, S, k, sel_b[s], sel_t[s], idx + (long long)s * k,
                             w + (long long)s * k, P, out + (long long)s * S * d);
+}
+
+/* Coupled contextualizer of the original Avey ([AB-notes] 关键设计 2: the
+ * learned static matrix V multiplied element-wise with the input-dependent
+ * cosine matrix N(Z_t)N(Z_t)^T, the result combining the embeddings), with the
+ * autoregressive (causal) mask of the original Avey ([AB-sum] §3, §4: Avey-B
+ * removes that mask):
+ *   M_ij = V_ij * N(z_i).N(z_j) for j <= i, 0 for j > i;   c = M Z_t.
+ * Identity activation, no bias, no row normalisation. */
+void avey_orc_coupled_causal_mix(const double *V, const double *zt, int S, int mt, long long ld,
+                                 double *c, long long ldc) {
+  double *u = (double *)malloc(sizeof(double) * (size_t)S * (size_t)mt);
+  double *M = (double *)malloc(sizeof(double) * (size_t)S * (size_t)S);
+  for (int i = 0; i < S; ++i) l2_normalize_row(zt + (long long)i * ld, mt, u + (long long)i * mt);
+  for (int i = 0; i < S; ++i)
+    for (int j = 0; j < S; ++j)
+      M[(long long)i * S + j] =
+          j <= i ? V[(long long)i * S + j] * dot(u + (long long)i * mt, u + (long long)j * mt, mt) : 0.0;
+  avey_orc_static_mix(M, zt, S, mt, ld, c, ldc); /* same product, with M as the map */
+  free(u);
+  free(M);
 }

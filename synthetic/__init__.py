@@ -43,6 +43,7 @@ import numpy as np
 
 STATIC = 0
 DYNAMIC = 1
+COUPLED = 2  # original Avey: V * cosine, causal mask (not in the named workloads)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -149,10 +150,10 @@ def gen_embeddings(w: Workload, seed: int = 0) -> Embeddings:
 
 @dataclasses.dataclass
 class LayerWeights:
-    kind: int  # STATIC or DYNAMIC
+    kind: int  # STATIC, DYNAMIC or COUPLED
     U: np.ndarray  # [d, m]   enricher weight (Z = X U + b)
     bU: np.ndarray  # [m]
-    V: Optional[np.ndarray]  # [S, S] for static layers, None for dynamic
+    V: Optional[np.ndarray]  # [S, S] for static and coupled layers, None for dynamic
     O: np.ndarray  # [m, d]   fuser weight
 
 
@@ -174,7 +175,7 @@ def gen_weights(w: Workload, seed: int = 1) -> Weights:
     for kind in w.pattern:
         U = draw((w.d, w.m), w.d)
         bU = draw((w.m,), w.d)
-        V = draw((w.S, w.S), w.S) if kind == STATIC else None
+        V = draw((w.S, w.S), w.S) if kind in (STATIC, COUPLED) else None
         O = draw((w.m, w.d), w.m)
         layers.append(LayerWeights(kind, U, bU, V, O))
     return Weights(P, layers)

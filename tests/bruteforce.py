@@ -42,8 +42,8 @@ def maxsim_matrix(X, S):
     return out
 
 
-def topk(scores_row, t, k):
-    cands = sorted(((-s, c) for c, s in enumerate(scores_row) if c != t))
+def topk(scores_row, t, k, causal=False):
+    cands = sorted(((-s, c) for c, s in enumerate(scores_row) if c != t and (not causal or c < t)))
     picked = cands[:k]
     s1 = -picked[0][0] if picked else 1.0
     s1 = s1 if s1 > 1e-30 else 1e-30
@@ -87,6 +87,11 @@ def layer(x, U, bU, V, O, m_h, kind, eps, prenorm):
     mt = m - m_h
     if kind == 0:
         c = [[sum(V[i][j] * Zt[j][f] for j in range(S)) for f in range(mt)] for i in range(S)]
+    elif kind == 2:  # coupled causal (original Avey)
+        u = [_unit(r) for r in Zt]
+        M = [[V[i][j] * sum(p * q for p, q in zip(u[i], u[j])) if j <= i else 0.0
+              for j in range(S)] for i in range(S)]
+        c = [[sum(M[i][j] * Zt[j][f] for j in range(S)) for f in range(mt)] for i in range(S)]
     else:
         u = [_unit(r) for r in Zt]
         G = [[sum(p * q for p, q in zip(u[i], u[j])) for j in range(S)] for i in range(S)]

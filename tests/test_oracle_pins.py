@@ -352,3 +352,65 @@ def test_large_stack_needs_prenorm():
     for lw in W.layers:
         b = orc.layer(b, lw, w.S, w.m_h, w.eps, True)
     assert np.all(np.isfinite(b)) and np.sqrt((b ** 2).mean()) < 100
+
+
+# ------------------------------------------------ next: f2 and f4 variants --
+
+@pytest.mark.parametrize("seed", range(3))
+def test_causal_topk_matches_bruteforce(seed):
+    rng = np.random.default_rng(40 + seed)
+    n, k = 13, 4
+    scores = rng.standard_normal((n, n)) + 2.0
+    idx, w = orc.topk(scores, np.arange(n), k, causal=True)
+    for t in range(n):
+        ref_idx, ref_w = bf.topk(scores[t].tolist(), t, k, causal=True)
+        assert idx[t].tolist() == ref_idx
+        np.testing.assert_allclose(w[t], ref_w, rtol=1e-15)
+        assert all(c < t for c in idx[t] if c >= 0)
+    assert idx[0].tolist() == [-1] * k  # the first split has no predecessor
+
+
+def test_coupled_causal_mix_closed_forms():
+    rng = np.random.default_rng(50)
+    S, mt = 5, 6
+    zt = rng.random((S, mt)) + 0.1
+    V = rng.standard_normal((S, S))
+    c = orc.coupled_causal_mix(V, zt)
+    # row 0 sees only itself: c_0 = V_00 cos(z0, z0) z0 = V_00 z0
+    np.testing.assert_allclose(c[0], V[0, 0] * zt[0], rtol=1e-14)
+    # identical tokens: cos = 1, so c_i = sum_{j<=i} V_ij z
+    z = rng.random(mt) + 0.1
+    ci = orc.coupled_causal_mix(V, np.tile(z, (S, 1)))
+    for i in range(S):
+        np.testing.assert_allclose(ci[i], V[i, :i + 1].sum() * z, rtol=1e-13, atol=1e-14)
+    # causality: changing a later token leaves earlier outputs unchanged
+    z2 = zt.copy()
+    z2[3] = rng.random(mt) + 5.0
+    c2 = orc.coupled_causal_mix(V, z2)
+    np.testing.assert_allclose(c2[:3], c[:3], rtol=0, atol=0)
+    assert not np.allclose(c2[3], c[3])
+
+
+@pytest.mark.parametrize("prenorm", [False, True])
+def test_coupled_layer_matches_bruteforce(prenorm):
+    rng = np.random.default_rng(60 + prenorm)
+    S, d, m, m_h = 4, 5, 7, 3
+    x = rng.standard_normal((2, S, d))
+    lw = _layer_weights(rng, d, m, S, sy.STATIC)
+    lw = sy.LayerWeights(sy.COUPLED, lw.U, lw.bU, lw.V, lw.O)
+    got = orc.layer(x, lw, S, m_h, 1e-8, prenorm)
+    for sp in range(2):
+        ref = bf.layer(x[sp].tolist(), lw.U.tolist(), lw.bU.tolist(), lw.V.tolist(), lw.O.tolist(),
+                       m_h, sy.COUPLED, 1e-8, prenorm)
+        np.testing.assert_allclose(got[sp], np.array(ref), rtol=1e-11, atol=1e-11)
+
+
+def test_causal_forward_matches_bruteforce():
+    w = sy.custom(B=1, N=22, S=4, d=6, m=8, m_h=3, k=2, pattern=(sy.STATIC, sy.DYNAMIC),
+                  dtype="f32", centers=3, sigma=0.4)
+    E, W = sy.gen_embeddings(w), sy.gen_weights(w)
+    res = orc.forward(E.X, W, w, causal=True)
+    sc = bf.maxsim_matrix(E.X.astype(np.float64).tolist(), w.S)
+    for r, (b, t) in enumerate(res["sel"].tolist()):
+        idx, _ = bf.topk(sc[b][t], t, w.k, causal=True)
+        assert res["idx"][r].tolist() == idx
