@@ -29,7 +29,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libavey.so")
 
 AVEY_F32, AVEY_BF16, AVEY_BF16X2 = 0, 1, 2
-AVEY_STATIC, AVEY_DYNAMIC = 0, 1
+AVEY_STATIC, AVEY_DYNAMIC, AVEY_COUPLED_CAUSAL = 0, 1, 2
+AVEY_RANK_UNIDIRECTIONAL = 1
 STATUS = {0: "AVEY_OK", 1: "AVEY_ERR_INVALID_ARG", 2: "AVEY_ERR_UNSUPPORTED", 3: "AVEY_ERR_CUDA",
           4: "AVEY_ERR_DEVICE_TIMEOUT", 5: "AVEY_ERR_DEVICE_BOUNDS"}
 
@@ -61,6 +62,9 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         L.avey_rank.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]
         L.avey_rank.restype = _i
+        L.avey_rank_ex.argtypes = [_vp, _i, _i, _i, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _vp,
+                                   _vp, _sz, _vp]
+        L.avey_rank_ex.restype = _i
         L.avey_rank_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.avey_rank_workspace_bytes.restype = _sz
         L.avey_compress.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
@@ -131,8 +135,11 @@ def rank_workspace_bytes(dtype: int, B: int, N: int, d: int, S: int) -> int:
 
 
 def avey_rank(x: torch.Tensor, S: int, k: int, return_scores: bool = False,
-              ws: Optional[torch.Tensor] = None):
-    """x [B, N, d] fp32 or bf16 -> (idx int32 [B, n, k], w fp32 [B, n, k][, scores])."""
+              ws: Optional[torch.Tensor] = None, causal: bool = False):
+    """x [B, N, d] fp32 or bf16 -> (idx int32 [B, n, k], w fp32 [B, n, k][, scores]).
+
+    causal: candidates only the preceding splits (AVEY_RANK_UNIDIRECTIONAL).
+    """
     _need(x, "x")
     B, N, d = x.shape
     n = -(-N // S)
@@ -143,8 +150,9 @@ def avey_rank(x: torch.Tensor, S: int, k: int, return_scores: bool = False,
     need = rank_workspace_bytes(dt, B, N, d, S)
     if ws is None or ws.numel() < need:
         ws = _ws(need, x.device)
-    _check("avey_rank", lib().avey_rank(_ptr(x), dt, B, N, d, S, k, _ptr(idx), _ptr(w),
-                                        _ptr(scores), _ptr(ws), ws.numel(), _stream()))
+    flags = AVEY_RANK_UNIDIRECTIONAL if causal else 0
+    _check("avey_rank", lib().avey_rank_ex(_ptr(x), dt, B, N, d, S, k, flags, _ptr(idx), _ptr(w),
+                                           _ptr(scores), _ptr(ws), ws.numel(), _stream()))
     return (idx, w, scores) if return_scores else (idx, w)
 
 
@@ -290,7 +298,8 @@ def make_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: torch.
 
 def encoder_forward(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLayer], S: int, k: int,
                     m_h: int, eps: float, prenorm: bool,
-                    ws: Optional[EncoderWorkspace] = None, marks=None) -> torch.Tensor:
+                    ws: Optional[EncoderWorkspace] = None, marks=None,
+                    causal: bool = False) -> torch.Tensor:
     """Ranker once, compression, then every layer (Avey-B paperlayer summary
     App. H: the ranker runs once per forward).  Returns fp32 [B, n*S, d].
 
@@ -308,8 +317,9 @@ def encoder_forward(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLay
     st = _stream()
     if marks is not None:
         marks[0].record()
-    _check("avey_rank", L.avey_rank(_ptr(x), dt, B, N, d, S, k, _ptr(ws.idx), _ptr(ws.w), None,
-                                    _ptr(ws.rank_ws), ws.rank_ws.numel(), st))
+    _check("avey_rank", L.avey_rank_ex(_ptr(x), dt, B, N, d, S, k,
+                                       AVEY_RANK_UNIDIRECTIONAL if causal else 0, _ptr(ws.idx),
+                                       _ptr(ws.w), None, _ptr(ws.rank_ws), ws.rank_ws.numel(), st))
     if marks is not None:
         marks[1].record()
     _check("avey_compress", L.avey_compress(_ptr(x), dt, B, N, d, S, k, _ptr(ws.idx), _ptr(ws.w),

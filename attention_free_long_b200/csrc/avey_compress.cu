@@ -35,7 +35,10 @@ struct CompressTile {
   static constexpr int PBYTES = S * PLD * 2;
   static constexpr int STAGE = XBYTES + PBYTES;
   static constexpr int NST = S >= 128 ? 2 : 3;  // cp.async pipeline depth over the k+1 blocks
-  static constexpr int SMEM = NST * STAGE;
+  // output staging (reuses the pipeline buffers): fp32 [S][NS+4], hi/lo [S][NS+8]
+  static constexpr int OLD32 = NS + 4;
+  static constexpr int OUT_BYTES = S * OLD32 * 4 + 2 * S * XLD * 2;
+  static constexpr int SMEM = NST * STAGE > OUT_BYTES ? NST * STAGE : OUT_BYTES;
 };
 
 template <int S>
@@ -176,7 +179,13 @@ __global__ void __launch_bounds__(256) compress_bf16(const bf16 *__restrict__ x,
     __syncthreads();
   }
 
-  // store fp32 + split pair
+  // Stage the fp32 result and its split pair in shared memory (the pipeline
+  // buffers are free after the last block), then write them with coalesced
+  // 16-byte stores.
+  float *o32 = reinterpret_cast<float *>(smem);
+  uint8_t *ohi = smem + S * C::OLD32 * 4;
+  uint8_t *olo = ohi + S * C::XLD * 2;
+  const bool pair = out_hi != nullptr;
 #pragma unroll
   for (int i = 0; i < C::MI; ++i)
 #pragma unroll
@@ -184,18 +193,35 @@ __global__ void __launch_bounds__(256) compress_bf16(const bf16 *__restrict__ x,
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int row = wm * C::WM + i * 16 + (lane >> 2) + h * 8;
-        const int col = q0 + wn * C::WN + j * 8 + (lane & 3) * 2;
-        if (col >= d) continue;
-        const long long o = (static_cast<long long>(b) * R + static_cast<long long>(t) * S + row) * d + col;
+        const int col = wn * C::WN + j * 8 + (lane & 3) * 2;
         const float v0 = acc[i][j][2 * h], v1 = acc[i][j][2 * h + 1];
-        *reinterpret_cast<float2 *>(out + o) = make_float2(v0, v1);
-        if (out_hi != nullptr) {
+        *reinterpret_cast<float2 *>(o32 + row * C::OLD32 + col) = make_float2(v0, v1);
+        if (pair) {
           uint32_t hi, lo;
           split_pack(v0, v1, hi, lo);
-          *reinterpret_cast<uint32_t *>(out_hi + o) = hi;
-          *reinterpret_cast<uint32_t *>(out_lo + o) = lo;
+          *reinterpret_cast<uint32_t *>(ohi + (row * C::XLD + col) * 2) = hi;
+          *reinterpret_cast<uint32_t *>(olo + (row * C::XLD + col) * 2) = lo;
         }
       }
+  __syncthreads();
+  const long long row0 = static_cast<long long>(b) * R + static_cast<long long>(t) * S;
+  for (int e = tid; e < S * (C::NS / 4); e += 256) {
+    const int row = e / (C::NS / 4), cc = e % (C::NS / 4);
+    const int col = q0 + cc * 4;
+    if (col >= d) continue;
+    *reinterpret_cast<float4 *>(out + (row0 + row) * d + col) =
+        *reinterpret_cast<const float4 *>(o32 + row * C::OLD32 + cc * 4);
+  }
+  if (pair) {
+    for (int e = tid; e < S * (C::NS / 8); e += 256) {
+      const int row = e / (C::NS / 8), cc = e % (C::NS / 8);
+      const int col = q0 + cc * 8;
+      if (col >= d) continue;
+      const long long o = (row0 + row) * d + col;
+      *reinterpret_cast<uint4 *>(out_hi + o) = *reinterpret_cast<const uint4 *>(ohi + (row * C::XLD + cc * 8) * 2);
+      *reinterpret_cast<uint4 *>(out_lo + o) = *reinterpret_cast<const uint4 *>(olo + (row * C::XLD + cc * 8) * 2);
+    }
+  }
   (void)plane;
 }
 

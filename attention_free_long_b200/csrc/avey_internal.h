@@ -38,8 +38,8 @@ avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, 
                              cudaStream_t s);
 avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, float *inv,
                              cudaStream_t s);
-avey_status launch_topk(const float *scores, int B, int n, int k, int32_t *idx, float *w,
-                        cudaStream_t s);
+avey_status launch_topk(const float *scores, int B, int n, int k, int causal, int32_t *idx,
+                        float *w, cudaStream_t s);
 
 // ---- mixes (avey_mix.cu) ----
 avey_status launch_static_mix_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int S, int mt,
@@ -47,6 +47,12 @@ avey_status launch_static_mix_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks
 avey_status launch_dynamic_mix_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
                                   int64_t ld_out, int64_t plane_out, int blocks, int S, int mt,
                                   float eps, cudaStream_t s);
+// Coupled causal contextualizer (original Avey): c = (V * cos, j <= i) Z_t.
+avey_status launch_coupled_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld_zt, int64_t plane_zt,
+                                  bf16 *out, int64_t ld_out, int64_t plane_out, int blocks, int S,
+                                  int mt, cudaStream_t s);
+avey_status launch_coupled_mix_f32(const float *V, const float *zt, int64_t ld_zt, float *out,
+                                   int64_t ld_out, int blocks, int S, int mt, cudaStream_t s);
 avey_status launch_static_mix_f32(const float *V, const float *zt, int64_t ld_zt, float *out,
                                   int64_t ld_out, int blocks, int S, int mt, cudaStream_t s);
 avey_status launch_dynamic_mix_f32(const float *zt, int64_t ld_zt, float *out, int64_t ld_out,

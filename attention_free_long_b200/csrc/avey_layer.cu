@@ -139,10 +139,11 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   const int mt = m - m_h;
   AVEY_REQUIRE(x_in && x_out && ws && p->Ut && p->bU && p->Ot, AVEY_ERR_INVALID_ARG,
                "avey_layer_forward: null pointer");
-  AVEY_REQUIRE(p->kind == AVEY_STATIC || p->kind == AVEY_DYNAMIC, AVEY_ERR_INVALID_ARG,
-               "avey_layer_forward: bad kind %d", int(p->kind));
+  AVEY_REQUIRE(p->kind == AVEY_STATIC || p->kind == AVEY_DYNAMIC ||
+                   p->kind == AVEY_COUPLED_CAUSAL,
+               AVEY_ERR_INVALID_ARG, "avey_layer_forward: bad kind %d", int(p->kind));
   AVEY_REQUIRE(p->kind == AVEY_DYNAMIC || p->V != nullptr, AVEY_ERR_INVALID_ARG,
-               "avey_layer_forward: static layer needs V");
+               "avey_layer_forward: static and coupled layers need V");
   AVEY_REQUIRE(T >= 1 && S >= 1 && T % S == 0, AVEY_ERR_INVALID_ARG,
                "avey_layer_forward: T=%d must be a positive multiple of S=%d", T, S);
   AVEY_REQUIRE(d >= 8 && d % 8 == 0 && m % 8 == 0 && m_h % 8 == 0 && m_h > 0 && m_h < m,
@@ -182,8 +183,11 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
     if (p->kind == AVEY_STATIC)
       st = launch_static_mix_f32(static_cast<const float *>(p->V), Z + m_h, m, Z + m_h, m, blocks, S,
                                  mt, s);
-    else
+    else if (p->kind == AVEY_DYNAMIC)
       st = launch_dynamic_mix_f32(Z + m_h, m, Z + m_h, m, blocks, S, mt, p->eps, s);
+    else
+      st = launch_coupled_mix_f32(static_cast<const float *>(p->V), Z + m_h, m, Z + m_h, m, blocks,
+                                  S, mt, s);
     if (st != AVEY_OK) return st;
     gemm_f32<F32_FUSE><<<dim3((d + 63) / 64, (T + 63) / 64), 256, 0, s>>>(
         Z, static_cast<const float *>(p->Ot), T, d, m, nullptr, nullptr, x_in, x_out);
@@ -220,8 +224,11 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   const int64_t plane = static_cast<int64_t>(T) * m;
   if (p->kind == AVEY_STATIC)
     st = launch_static_mix_x2(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane, s);
-  else
+  else if (p->kind == AVEY_DYNAMIC)
     st = launch_dynamic_mix_x2(Zhi + m_h, m, plane, Zhi + m_h, m, plane, blocks, S, mt, p->eps, s);
+  else
+    st = launch_coupled_mix_x2(static_cast<const bf16 *>(p->V), Zhi + m_h, m, plane, Zhi + m_h, m,
+                               plane, blocks, S, mt, s);
   if (st != AVEY_OK) return st;
   bf16 *ohi = static_cast<bf16 *>(x_out_lowp);
   bf16 *olo = ohi ? ohi + static_cast<long long>(T) * d : nullptr;

@@ -12,8 +12,9 @@
 //                   mma.sync; written back in place as a split pair.
 //   dynamic_mix_x2  one CTA per block, two passes over Z_t in 64-feature
 //                   chunks (the second pass mostly hits L2):
-//                   1. Gram R = Z_hi Z_hi^T (mma.sync) and fp32 row sums of
-//                      squares of hi + lo;
+//                   1. from the hi plane only: Gram R = Z_hi Z_hi^T (mma.sync)
+//                      and fp32 row sums of squares, so G is the cosine matrix
+//                      of the hi vectors (within about 1e-4 of the exact one);
 //                   2. G = R / (n_i n_j), row sums, Gt in fp32, split to bf16
 //                      hi/lo in shared memory;
 //                   3. c = Gt_hi Z_hi + Gt_lo Z_hi + Gt_hi Z_lo, split pair out.
@@ -98,6 +99,9 @@ __global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V,
       }
     }
   }
+  // c as a split pair, staged over the (now consumed) input slab, then written
+  // back with coalesced 16-byte stores.
+  __syncthreads();
 #pragma unroll
   for (int i = 0; i < C::MI; ++i)
 #pragma unroll
@@ -105,14 +109,21 @@ __global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V,
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int row = wm * C::WM + i * 16 + (lane >> 2) + h * 8;
-        const int f = f0 + wn * C::WN + j * 8 + (lane & 3) * 2;
-        if (f >= mt) continue;
+        const int fl = wn * C::WN + j * 8 + (lane & 3) * 2;
         uint32_t hi, lo;
         split_pack(acc[i][j][2 * h], acc[i][j][2 * h + 1], hi, lo);
-        bf16 *dst = zbase + row * ld + f;
-        *reinterpret_cast<uint32_t *>(dst) = hi;
-        *reinterpret_cast<uint32_t *>(dst + plane) = lo;
+        *reinterpret_cast<uint32_t *>(zh + (row * C::ZLD + fl) * 2) = hi;
+        *reinterpret_cast<uint32_t *>(zl + (row * C::ZLD + fl) * 2) = lo;
       }
+  __syncthreads();
+  for (int e = tid; e < S * (C::NS / 8); e += 256) {
+    const int row = e / (C::NS / 8), cc = e % (C::NS / 8);
+    const int f = f0 + cc * 8;
+    if (f >= mt) continue;
+    bf16 *dst = zbase + row * ld + f;
+    *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(zh + (row * C::ZLD + cc * 8) * 2);
+    *reinterpret_cast<uint4 *>(dst + plane) = *reinterpret_cast<const uint4 *>(zl + (row * C::ZLD + cc * 8) * 2);
+  }
 }
 
 // --------------------------------------------------------------- dynamic --
@@ -139,11 +150,15 @@ struct DynTile {
   static_assert(S * FLD * 4 <= 2 * BUF, "fp32 G must fit in the chunk buffers");
 };
 
-template <int S>
+// COUPLED = false: eq. 6 (Avey-B dynamic layer).  COUPLED = true: the
+// original Avey's coupled causal map M_ij = V_ij G_ij (j <= i), no row
+// normalisation; everything else is shared.
+template <int S, bool COUPLED>
 __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long ld_zt,
                                                       long long plane_zt, bf16 *out,
                                                       long long ld_out, long long plane_out,
-                                                      int mt, float eps) {
+                                                      int mt, float eps,
+                                                      const bf16 *__restrict__ V) {
   using C = DynTile<S>;
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t *bufs = smem;                       // 2 x (hi, lo) chunks; later fp32 G
@@ -158,7 +173,7 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
   bf16 *ob = out + static_cast<long long>(blk) * S * ld_out;
   const int nchunks = (mt + C::FC - 1) / C::FC;
 
-  auto load_chunk = [&](int ch, int buf) {
+  auto load_chunk = [&](int ch, int buf, bool with_lo) {
     uint8_t *h = bufs + buf * C::BUF;
     uint8_t *l = h + C::CBYTES;
     for (int e = tid; e < S * (C::FC / 8); e += 256) {
@@ -167,7 +182,8 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
       const bool ok = f < mt;
       const bf16 *src = ok ? zb + row * ld_zt + f : zb;
       cp_async16(smem_u32(h + (row * C::CLD + cc * 8) * 2), src, ok ? 16 : 0);
-      cp_async16(smem_u32(l + (row * C::CLD + cc * 8) * 2), ok ? src + plane_zt : zb, ok ? 16 : 0);
+      if (with_lo)
+        cp_async16(smem_u32(l + (row * C::CLD + cc * 8) * 2), ok ? src + plane_zt : zb, ok ? 16 : 0);
     }
     cp_async_commit();
   };
@@ -178,27 +194,24 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
   float g[C::GMI][C::GNI][4] = {};
   const int sr = tid % S, sp = tid / S;  // sum-of-squares row / part
   float ss = 0.f;
-  load_chunk(0, 0);
+  load_chunk(0, 0, false);
   for (int ch = 0; ch < nchunks; ++ch) {
     if (ch + 1 < nchunks) {
-      load_chunk(ch + 1, (ch + 1) & 1);
+      load_chunk(ch + 1, (ch + 1) & 1, false);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
     __syncthreads();
     const uint8_t *h = bufs + (ch & 1) * C::BUF;
-    const uint8_t *l = h + C::CBYTES;
     {
       constexpr int FPT = C::FC / C::TR;  // features per thread
 #pragma unroll
       for (int q = 0; q < FPT; q += 2) {
         const int f = sp * FPT + q;
         const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t *>(h + (sr * C::CLD + f) * 2));
-        const float2 b = unpack_bf16(*reinterpret_cast<const uint32_t *>(l + (sr * C::CLD + f) * 2));
-        const float v0 = a.x + b.x, v1 = a.y + b.y;
-        ss = fmaf(v0, v0, ss);
-        ss = fmaf(v1, v1, ss);
+        ss = fmaf(a.x, a.x, ss);
+        ss = fmaf(a.y, a.y, ss);
       }
     }
     if (gram_warp) {
@@ -261,7 +274,11 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
   __syncthreads();
   for (int e = tid; e < S * S; e += 256) {
     const int i = e / S, j = e % S;
-    const float v = G[i * C::FLD + j] / s_den[i];
+    float v;
+    if constexpr (COUPLED)
+      v = j <= i ? __bfloat162float(V[i * S + j]) * G[i * C::FLD + j] : 0.f;
+    else
+      v = G[i * C::FLD + j] / s_den[i];
     float hi, lo;
     split_bf16(v, hi, lo);
     reinterpret_cast<bf16 *>(gth)[i * C::GLD + j] = __float2bfloat16_rn(hi);
@@ -272,19 +289,19 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
   // ---- pass 3: c = Gt Z_t ----
   const int awm = warp / C::AW_N, awn = warp % C::AW_N;
   const bool apply_warp = warp < C::AW_M * C::AW_N;
-  load_chunk(0, 0);
+  load_chunk(0, 0, true);
   for (int ch = 0; ch < nchunks; ++ch) {
     if (ch + 1 < nchunks) {
-      load_chunk(ch + 1, (ch + 1) & 1);
+      load_chunk(ch + 1, (ch + 1) & 1, true);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
     __syncthreads();
-    const uint8_t *h = bufs + (ch & 1) * C::BUF;
-    const uint8_t *l = h + C::CBYTES;
+    uint8_t *h = bufs + (ch & 1) * C::BUF;
+    uint8_t *l = h + C::CBYTES;
+    float acc[C::AMI][C::ANI][4] = {};
     if (apply_warp) {
-      float acc[C::AMI][C::ANI][4] = {};
 #pragma unroll
       for (int kk = 0; kk < S; kk += 16) {
         uint32_t ah[C::AMI][4], al[C::AMI][4];
@@ -314,6 +331,10 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
           }
         }
       }
+    }
+    // stage c (split pair) over the consumed chunk, then coalesced stores
+    __syncthreads();
+    if (apply_warp) {
 #pragma unroll
       for (int i = 0; i < C::AMI; ++i)
 #pragma unroll
@@ -321,14 +342,22 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int row = awm * (S / C::AW_M) + i * 16 + (lane >> 2) + hh * 8;
-            const int f = ch * C::FC + awn * (C::FC / C::AW_N) + j * 8 + (lane & 3) * 2;
-            if (f >= mt) continue;
+            const int fl = awn * (C::FC / C::AW_N) + j * 8 + (lane & 3) * 2;
             uint32_t hi, lo;
             split_pack(acc[i][j][2 * hh], acc[i][j][2 * hh + 1], hi, lo);
-            bf16 *dst = ob + row * ld_out + f;
-            *reinterpret_cast<uint32_t *>(dst) = hi;
-            *reinterpret_cast<uint32_t *>(dst + plane_out) = lo;
+            *reinterpret_cast<uint32_t *>(h + (row * C::CLD + fl) * 2) = hi;
+            *reinterpret_cast<uint32_t *>(l + (row * C::CLD + fl) * 2) = lo;
           }
+    }
+    __syncthreads();
+    for (int e = tid; e < S * (C::FC / 8); e += 256) {
+      const int row = e / (C::FC / 8), cc = e % (C::FC / 8);
+      const int f = ch * C::FC + cc * 8;
+      if (f >= mt) continue;
+      bf16 *dst = ob + row * ld_out + f;
+      *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(h + (row * C::CLD + cc * 8) * 2);
+      *reinterpret_cast<uint4 *>(dst + plane_out) =
+          *reinterpret_cast<const uint4 *>(l + (row * C::CLD + cc * 8) * 2);
     }
     __syncthreads();
   }
@@ -362,10 +391,10 @@ __global__ void __launch_bounds__(256) static_mix_f32(const float *__restrict__ 
   }
 }
 
-template <int S>
+template <int S, bool COUPLED>
 __global__ void __launch_bounds__(256) dynamic_mix_f32(const float *zt, long long ld_zt,
                                                        float *out, long long ld_out, int mt,
-                                                       float eps) {
+                                                       float eps, const float *__restrict__ V) {
   constexpr int NSL = 64;
   __shared__ float Gt[S][S + 1];
   __shared__ float nf[S];
@@ -387,10 +416,14 @@ __global__ void __launch_bounds__(256) dynamic_mix_f32(const float *zt, long lon
   }
   __syncthreads();
   if (tid < S) {
-    float rs = 0.f;
-    for (int j = 0; j < S; ++j) rs += Gt[tid][j];
-    const float den = rs + eps;
-    for (int j = 0; j < S; ++j) Gt[tid][j] = Gt[tid][j] / den;
+    if constexpr (COUPLED) {
+      for (int j = 0; j < S; ++j) Gt[tid][j] = j <= tid ? V[tid * S + j] * Gt[tid][j] : 0.f;
+    } else {
+      float rs = 0.f;
+      for (int j = 0; j < S; ++j) rs += Gt[tid][j];
+      const float den = rs + eps;
+      for (int j = 0; j < S; ++j) Gt[tid][j] = Gt[tid][j] / den;
+    }
   }
   __syncthreads();
   // c = Gt Z_t, slab by slab; every slab is read into shared memory before
@@ -434,14 +467,15 @@ avey_status run_static_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int m
   return AVEY_OK;
 }
 
-template <int S>
+template <int S, bool COUPLED>
 avey_status run_dynamic_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
                            int64_t ld_out, int64_t plane_out, int blocks, int mt, float eps,
-                           cudaStream_t s) {
+                           const bf16 *V, cudaStream_t s) {
   using C = DynTile<S>;
-  if (avey_status st = set_smem(dynamic_mix_x2<S>, C::SMEM, "dynamic_mix_x2")) return st;
-  dynamic_mix_x2<S><<<blocks, 256, C::SMEM, s>>>(zt, ld_zt, plane_zt, out, ld_out, plane_out, mt, eps);
-  AVEY_CHECK_LAUNCH("dynamic_mix_x2");
+  if (avey_status st = set_smem(dynamic_mix_x2<S, COUPLED>, C::SMEM, "dynamic_mix_x2")) return st;
+  dynamic_mix_x2<S, COUPLED><<<blocks, 256, C::SMEM, s>>>(zt, ld_zt, plane_zt, out, ld_out,
+                                                          plane_out, mt, eps, V);
+  AVEY_CHECK_LAUNCH(COUPLED ? "coupled_mix_x2" : "dynamic_mix_x2");
   return AVEY_OK;
 }
 
@@ -463,12 +497,25 @@ avey_status launch_dynamic_mix_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_z
                                   int64_t ld_out, int64_t plane_out, int blocks, int S, int mt,
                                   float eps, cudaStream_t s) {
   switch (S) {
-    case 16: return run_dynamic_x2<16>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, s);
-    case 32: return run_dynamic_x2<32>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, s);
-    case 64: return run_dynamic_x2<64>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, s);
-    case 128: return run_dynamic_x2<128>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, s);
+    case 16: return run_dynamic_x2<16, false>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, nullptr, s);
+    case 32: return run_dynamic_x2<32, false>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, nullptr, s);
+    case 64: return run_dynamic_x2<64, false>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, nullptr, s);
+    case 128: return run_dynamic_x2<128, false>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, nullptr, s);
   }
   set_detail("dynamic mix: S=%d unsupported", S);
+  return AVEY_ERR_UNSUPPORTED;
+}
+
+avey_status launch_coupled_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld_zt, int64_t plane_zt,
+                                  bf16 *out, int64_t ld_out, int64_t plane_out, int blocks, int S,
+                                  int mt, cudaStream_t s) {
+  switch (S) {
+    case 16: return run_dynamic_x2<16, true>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, 0.f, V, s);
+    case 32: return run_dynamic_x2<32, true>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, 0.f, V, s);
+    case 64: return run_dynamic_x2<64, true>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, 0.f, V, s);
+    case 128: return run_dynamic_x2<128, true>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, 0.f, V, s);
+  }
+  set_detail("coupled mix: S=%d unsupported", S);
   return AVEY_ERR_UNSUPPORTED;
 }
 
@@ -490,12 +537,25 @@ avey_status launch_dynamic_mix_f32(const float *zt, int64_t ld_zt, float *out, i
                                    int blocks, int S, int mt, float eps, cudaStream_t s) {
   switch (S) {
 #define AVEY_DF(SS) \
-  case SS: dynamic_mix_f32<SS><<<blocks, 256, 0, s>>>(zt, ld_zt, out, ld_out, mt, eps); break;
+  case SS: dynamic_mix_f32<SS, false><<<blocks, 256, 0, s>>>(zt, ld_zt, out, ld_out, mt, eps, nullptr); break;
     AVEY_DF(1) AVEY_DF(2) AVEY_DF(4) AVEY_DF(8) AVEY_DF(16) AVEY_DF(32) AVEY_DF(64)
 #undef AVEY_DF
     default: set_detail("dynamic mix (F32): S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
   }
   AVEY_CHECK_LAUNCH("dynamic_mix_f32");
+  return AVEY_OK;
+}
+
+avey_status launch_coupled_mix_f32(const float *V, const float *zt, int64_t ld_zt, float *out,
+                                   int64_t ld_out, int blocks, int S, int mt, cudaStream_t s) {
+  switch (S) {
+#define AVEY_CF(SS) \
+  case SS: dynamic_mix_f32<SS, true><<<blocks, 256, 0, s>>>(zt, ld_zt, out, ld_out, mt, 0.f, V); break;
+    AVEY_CF(1) AVEY_CF(2) AVEY_CF(4) AVEY_CF(8) AVEY_CF(16) AVEY_CF(32) AVEY_CF(64)
+#undef AVEY_CF
+    default: set_detail("coupled mix (F32): S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
+  }
+  AVEY_CHECK_LAUNCH("coupled_mix_f32");
   return AVEY_OK;
 }
 

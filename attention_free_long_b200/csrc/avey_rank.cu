@@ -173,8 +173,8 @@ __global__ void __launch_bounds__(256) inv_norms(const bf16 *__restrict__ x, int
 constexpr int kTopkWarps = 4;
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
-    topk_warp(const float *__restrict__ scores, int B, int n, int k, int32_t *__restrict__ idx,
-              float *__restrict__ w) {
+    topk_warp(const float *__restrict__ scores, int B, int n, int k, int causal,
+              int32_t *__restrict__ idx, float *__restrict__ w) {
   extern __shared__ float srow_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long rowid = static_cast<long long>(blockIdx.x) * kTopkWarps + warp;
@@ -182,7 +182,9 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
   const int t = static_cast<int>(rowid % n);
   float *srow = srow_all + static_cast<long long>(warp) * n;
   const float *src = scores + rowid * n;
-  for (int c = lane; c < n; c += 32) srow[c] = (c == t) ? -INFINITY : src[c];
+  // candidates: every other split, or only the preceding ones when causal
+  for (int c = lane; c < n; c += 32) srow[c] = (c == t || (causal && c > t)) ? -INFINITY : src[c];
+  const int avail = causal ? t : n - 1;
   __syncwarp();
   float s1 = 1.f;
   for (int r = 0; r < k; ++r) {
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
       }
     }
     const long long o = rowid * k + r;
-    if (r < n - 1 && bi != 0x7fffffff && best != -INFINITY) {
+    if (r < avail && bi != 0x7fffffff && best != -INFINITY) {
       if (r == 0) s1 = best > 1e-30f ? best : 1e-30f;
       if (lane == 0) {
         idx[o] = bi;
@@ -247,8 +249,8 @@ avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, floa
   return AVEY_OK;
 }
 
-avey_status launch_topk(const float *scores, int B, int n, int k, int32_t *idx, float *w,
-                        cudaStream_t s) {
+avey_status launch_topk(const float *scores, int B, int n, int k, int causal, int32_t *idx,
+                        float *w, cudaStream_t s) {
   const long long rows = static_cast<long long>(B) * n;
   const size_t smem = static_cast<size_t>(kTopkWarps) * n * sizeof(float);
   if (smem > 48 * 1024) {
@@ -260,7 +262,7 @@ avey_status launch_topk(const float *scores, int B, int n, int k, int32_t *idx, 
     }
   }
   const unsigned grid = static_cast<unsigned>((rows + kTopkWarps - 1) / kTopkWarps);
-  topk_warp<<<grid, kTopkWarps * 32, smem, s>>>(scores, B, n, k, idx, w);
+  topk_warp<<<grid, kTopkWarps * 32, smem, s>>>(scores, B, n, k, causal, idx, w);
   AVEY_CHECK_LAUNCH("topk_warp");
   return AVEY_OK;
 }
@@ -303,6 +305,14 @@ extern "C" size_t avey_rank_workspace_bytes(avey_dtype dt, int B, int N, int d, 
 extern "C" avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
                                  int32_t *idx, float *w, float *scores, void *ws, size_t ws_bytes,
                                  avey_stream_t stream) {
+  return avey_rank_ex(x, dt, B, N, d, S, k, 0u, idx, w, scores, ws, ws_bytes, stream);
+}
+
+extern "C" avey_status avey_rank_ex(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
+                                    uint32_t flags, int32_t *idx, float *w, float *scores, void *ws,
+                                    size_t ws_bytes, avey_stream_t stream) {
+  AVEY_REQUIRE((flags & ~static_cast<uint32_t>(AVEY_RANK_UNIDIRECTIONAL)) == 0u,
+               AVEY_ERR_INVALID_ARG, "avey_rank: unknown flags 0x%x", flags);
   AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
                "avey_rank: dtype %d unsupported (F32 or BF16)", int(dt));
   AVEY_REQUIRE(x && idx && w && ws, AVEY_ERR_INVALID_ARG, "avey_rank: null pointer");
@@ -351,5 +361,6 @@ extern "C" avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int
                            static_cast<int>(n), sc, s);
   }
   if (st != AVEY_OK) return st;
-  return launch_topk(sc, B, static_cast<int>(n), k, idx, w, s);
+  return launch_topk(sc, B, static_cast<int>(n), k,
+                     (flags & AVEY_RANK_UNIDIRECTIONAL) ? 1 : 0, idx, w, s);
 }

@@ -204,38 +204,34 @@ __device__ __forceinline__ void epi_maxsim_rows(uint32_t taddr, int lane, int qu
   }
 }
 
-// Max over the warp's 32 lanes (rows) of each of the 32 columns in v, as a
-// reduce-scatter: after five exchange steps lane l holds the maximum of
-// column l (v is consumed).
-__device__ __forceinline__ float colmax32(float (&v)[32], int lane) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < o; ++i) {
-      const float send = up ? v[i] : v[i + o];
-      const float keep = up ? v[i + o] : v[i];
-      v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
-    }
-  }
-  return v[0];
-}
-
 // Triangular MaxSim, one tile (row block I = mt, column blocks 2nt, 2nt+1 of
 // 128 columns).  Per 32-column chunk the cosines are formed in full (column
 // and row scale); chunks of a block left of the diagonal (K < I) are skipped
 // because the tile (K, I/2) covers that pair; for blocks right of it (K > I)
 // the column maxima over this warp's rows are kept in cm as well, which give
 // the mirrored scores score(c -> t).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Max of the 32 values (a tree of three-input maxima).
 __device__ __forceinline__ float max32(const float (&v)[32]) {
-  float a[16];
+  float a[11];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) a[i] = fmaxf(v[i], v[i + 16]);
-#pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) a[i] = fmaxf(a[i], a[i + w]);
-  return a[0];
+  for (int i = 0; i < 10; ++i) a[i] = max3f(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  a[10] = fmaxf(v[30], v[31]);
+  const float b0 = max3f(a[0], a[1], a[2]), b1 = max3f(a[3], a[4], a[5]);
+  const float b2 = max3f(a[6], a[7], a[8]), b3 = fmaxf(a[9], a[10]);
+  return max3f(b0, b1, fmaxf(b2, b3));
+}
+
+// Max over the warp's 32 lanes, delivered to every lane.
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
 }
 
 template <int S>
@@ -249,29 +245,47 @@ __device__ __forceinline__ void epi_maxsim_sym_rows(uint32_t taddr, int lane, in
   if (K < mt) return;           // left of the diagonal: covered by tile (K, mt/2)
   float m = -INFINITY;
 #pragma unroll 1
-  for (int ch = 4 * half; ch < 4 * half + 4; ++ch) {
-    const float4 *cs4 = reinterpret_cast<const float4 *>(col_scale + ch * 32);
-    float4 c4[8];
+  for (int pr = 0; pr < 2; ++pr) {  // two 64-column pieces of the block
+    const int ch0 = 4 * half + 2 * pr;
+    const float4 *cs4 = reinterpret_cast<const float4 *>(col_scale + ch0 * 32);
+    float4 c4[16];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) c4[q] = __ldg(cs4 + q);
-    float v[32];
-    tmem_ld32(taddr + ch * 32, v);
+    for (int q = 0; q < 16; ++q) c4[q] = __ldg(cs4 + q);
+    float v[64];
+    tmem_ld64(taddr + ch0 * 32, v);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < 16; ++q) {
       v[4 * q] *= c4[q].x * row_scale;
       v[4 * q + 1] *= c4[q].y * row_scale;
       v[4 * q + 2] *= c4[q].z * row_scale;
       v[4 * q + 3] *= c4[q].w * row_scale;
     }
-    if (ch % CH_PER_CAND == 0) m = -INFINITY;
-    m = fmaxf(m, max32(v));
-    if (ch % CH_PER_CAND == CH_PER_CAND - 1) {
-      float t = m;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-      if (lane == 0) red[quarter * kRedCands + ch / CH_PER_CAND] = t;
+    for (int u = 0; u < 2; ++u) {
+      const int ch = ch0 + u;
+      if (ch % CH_PER_CAND == 0) m = -INFINITY;
+      float part[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) part[j] = v[32 * u + j];
+      m = fmaxf(m, max32(part));
+      if (ch % CH_PER_CAND == CH_PER_CAND - 1) {
+        float t = m;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+        if (lane == 0) red[quarter * kRedCands + ch / CH_PER_CAND] = t;
+      }
     }
-    if (K > mt) cm[(quarter * 8 + ch) * 32 + lane] = colmax32(v, lane);
+    if (K > mt) {
+      // column maxima over this warp's 32 rows: one warp reduction per column
+      float c[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) c[j] = warp_max(v[j]);
+      if (lane == 0) {
+        float4 *dst = reinterpret_cast<float4 *>(cm + (quarter * 8 + ch0) * 32);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) dst[q] = make_float4(c[4 * q], c[4 * q + 1], c[4 * q + 2], c[4 * q + 3]);
+      }
+    }
   }
 }
 
@@ -482,12 +496,13 @@ __global__ void __launch_bounds__(Roles<MODE>::THREADS, 1)
   const uint32_t cbase = sbase + L::TILES_BYTES;
   // control block: full[4] @0, empty[4] @64, tfull[2] @128, tempty[2] @144,
   // redbar[2 acc][2 halves] @160, drain @192, tmem base @200, abort flag @204,
-  // red @256, column maxima @2048
+  // redfree[2 acc][2 halves] @224, red @256, column maxima @2048
   auto full_bar = [&](int s) { return cbase + 8u * s; };
   auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
   auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
   auto tempty_bar = [&](int i) { return cbase + 144u + 8u * i; };
   auto red_bar = [&](int i) { return cbase + 160u + 8u * i; };
+  auto red_free = [&](int i) { return cbase + 224u + 8u * i; };
   const uint32_t drain_bar = cbase + 192u;
   volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 200);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 204);
@@ -506,7 +521,10 @@ __global__ void __launch_bounds__(Roles<MODE>::THREADS, 1)
       mbar_init(tfull_bar(i), 1);
       mbar_init(tempty_bar(i), EPI);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(red_bar(i), 4);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(red_bar(i), 4);
+      mbar_init(red_free(i), 1);
+    }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -643,21 +661,38 @@ __global__ void __launch_bounds__(Roles<MODE>::THREADS, 1)
       const int row = mt * BM + quarter * 32 + lane;
       if constexpr (MODE == MODE_MAXSIM_SYM) {
         const int half = (warp - 2) >> 2;  // warps 2-5: block 2nt, warps 6-9: block 2nt+1
+        const int rb = acc * 2 + half;
         float *red_acc = red + acc * kRedGroups * kRedCands;
         float *cm_acc = cmx + acc * (4 * 8 * 32);
         const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
+        // the leader must have consumed the partials this buffer held two tiles ago
+        if (!mbar_wait(red_free(rb), acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         epi_maxsim_sym_rows<SPLIT_S>(taddr, lane, quarter, half, red_acc, cm_acc, rs + nt * BN,
                                      rs[row], mt, nt);
+        // TMEM is no longer needed by this warp: release it before the combine
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(red_bar(acc * 2 + half));
+        if (lane == 0) {
+          mbar_arrive(tempty_bar(acc));
+          mbar_arrive(red_bar(rb));
+        }
         if (warp == 2 + 4 * half) {
           // leader of this half: combine its four warps' partial results
-          if (!mbar_wait(red_bar(acc * 2 + half), acc_phase, abort_flag)) {
+          if (!mbar_wait(red_bar(rb), acc_phase, abort_flag)) {
             ok = false;
           } else {
             epi_maxsim_sym_write<SPLIT_S>(a, red_acc, cm_acc, lane, b, mt, nt, half);
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(red_free(rb));
         }
+        if (!ok) break;
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        continue;
       } else if constexpr (MODE == MODE_MAXSIM) {
         float *red_acc = red + acc * kRedGroups * kRedCands;
         const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;

@@ -73,7 +73,12 @@ typedef enum {
 
 typedef enum { AVEY_F32 = 0, AVEY_BF16 = 1, AVEY_BF16X2 = 2 } avey_dtype;
 
-typedef enum { AVEY_STATIC = 0, AVEY_DYNAMIC = 1 } avey_ctx_kind;
+/* Contextualizer kinds: the two Avey-B layers, plus the coupled causal layer
+ * of the original (autoregressive) Avey for comparison. */
+typedef enum { AVEY_STATIC = 0, AVEY_DYNAMIC = 1, AVEY_COUPLED_CAUSAL = 2 } avey_ctx_kind;
+
+/* avey_rank_ex flags */
+enum { AVEY_RANK_UNIDIRECTIONAL = 1 };
 
 /* ------------------------------------------------------------------ ranker --
  * avey_rank: the ranker, run once per forward on the input embeddings
@@ -102,6 +107,15 @@ AVEY_API avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int d
                       avey_stream_t stream);
 
 AVEY_API size_t avey_rank_workspace_bytes(avey_dtype dt, int B, int N, int d, int S);
+
+/* avey_rank_ex: avey_rank with flags.  AVEY_RANK_UNIDIRECTIONAL restricts the
+ * candidates of target split t to the preceding splits c < t (the ranker of
+ * the original Avey; [AB-sum] App. B "Ranker direction" compares both), so
+ * split t gets min(k, t) real candidates and the rest are -1 / 0.  Scores are
+ * computed for every pair either way.  flags = 0 is avey_rank. */
+AVEY_API avey_status avey_rank_ex(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
+                                  uint32_t flags, int32_t *idx, float *w, float *scores, void *ws,
+                                  size_t ws_bytes, avey_stream_t stream);
 
 /* avey_rank_static: avey_rank for callers that cannot allocate device memory
  * (a plugin interface that hands over only input and output buffers, or a
@@ -171,7 +185,10 @@ AVEY_API avey_status avey_dynamic_mix(const void *zt, int64_t ld_zt, avey_dtype 
  *   xin = prenorm ? x / sqrt(mean(x^2) + 1e-6) : x   (per token; see below)
  *   Z   = relu(xin U + b)^2                          (enricher, ReLU^2)
  *   Z_h = Z[:, :m_h],  Z_t = Z[:, m_h:]              (head bypass / tail)
- *   c   = V Z_t (static) or Gt Z_t (dynamic), per split of S tokens
+ *   c   = V Z_t (static) or Gt Z_t (dynamic), per split of S tokens; for
+ *         AVEY_COUPLED_CAUSAL, c = M Z_t with M_ij = V_ij N(z_i).N(z_j) for
+ *         j <= i and 0 otherwise (the original Avey's coupled contextualizer,
+ *         [AB-notes] 关键设计 2, with its causal mask; no row normalisation)
  *   x'  = x + [Z_h || c] O                           (fuser + residual)
  * `prenorm` is an option of this library, not of the pages: a gain-free RMS
  * norm of the enricher input that keeps deep stacks finite.  It leaves the
@@ -180,7 +197,7 @@ AVEY_API avey_status avey_dynamic_mix(const void *zt, int64_t ld_zt, avey_dtype 
  * Weights (dtype = dt: AVEY_F32, or AVEY_BF16 for the tensor-core path):
  *   Ut [m, d]  the enricher matrix U stored transposed (row f holds U[:, f])
  *   bU [m]     fp32 enricher bias (fp32 for both dtypes)
- *   V  [S, S]  static map (AVEY_STATIC), NULL for AVEY_DYNAMIC
+ *   V  [S, S]  static map (AVEY_STATIC, AVEY_COUPLED_CAUSAL), NULL for AVEY_DYNAMIC
  *   Ot [d, m]  the fuser matrix O stored transposed (row q holds O[:, q])
  * Activations:
  *   x_in      [T, d] fp32 residual stream in.

@@ -32,12 +32,12 @@ def _rows_of(wl, sel):
                            for b, t in sel.tolist()])
 
 
-def run_gpu(wl, E, W, sel, dev):
+def run_gpu(wl, E, W, sel, dev, causal=False):
     dt = _tdtype(wl)
     x = torch.from_numpy(E.X).to(dev, dtype=dt)
     P = torch.from_numpy(W.P).to(dev, dtype=dt)
     layers = av.device_layers(W, dt, dev)
-    idx, w, scores = av.avey_rank(x, wl.S, wl.k, return_scores=True)
+    idx, w, scores = av.avey_rank(x, wl.S, wl.k, return_scores=True, causal=causal)
     out, pair = av.avey_compress(x, wl.S, wl.k, idx, w, P)
     rows = torch.from_numpy(_rows_of(wl, sel)).to(dev)
     cur, cp = out.view(-1, wl.d), pair
@@ -57,13 +57,18 @@ def run_gpu(wl, E, W, sel, dev):
 # Rows whose top-k lists differ by a near tie (checked by check_topk) are left
 # out of the downstream comparison: the oracle never takes the GPU's selection
 # as an input.  Mixtures with several splits per centre produce many such ties.
-def compare(wl, E, W, sel, dev):
-    g = run_gpu(wl, E, W, sel, dev)
-    o = orc.forward(E.X, W, wl, sel=sel)
+def compare(wl, E, W, sel, dev, causal=False):
+    g = run_gpu(wl, E, W, sel, dev, causal)
+    o = orc.forward(E.X, W, wl, sel=sel, causal=causal)
     tol = TOL[wl.dtype]
     assert rel_err(g["scores"], o["scores"]) <= tol, "scores"
     exact = check_topk(g["idx"], g["w"], o["idx"], o["scores"], sel[:, 1], tol)
     assert exact.mean() >= 0.75, f"only {exact.mean():.2f} of the rows have identical top-k lists"
+    # a best score <= 0 makes the weights divide by the 1e-30 floor: such a
+    # split's compressed output is meaningless, so it is not compared further
+    best = np.array([o["scores"][r, o["idx"][r, 0]] if o["idx"][r, 0] >= 0 else 1.0
+                     for r in range(sel.shape[0])])
+    exact &= best > 1e-30
     keep = np.repeat(exact, wl.S)
     ref = [o["compressed"].reshape(-1, wl.d)] + [a.reshape(-1, wl.d) for a in o["layers"]]
     errs = [rel_err(gg[keep], oo[keep]) for gg, oo in zip(g["outs"], ref)]
@@ -169,3 +174,27 @@ def test_kernels_launched_through_the_library(cuda_dev):
     run_gpu(wl, E, W, orc.all_targets(1, 2), cuda_dev)
     # rank: normalize + maxsim + topk; compress; per layer: enrich + mix + fuse
     assert av.kernel_launches() - before == 3 + 1 + 3 * len(W.layers)
+
+
+# ---- the variants of the pages' ablations: unidirectional ranker (candidates
+# c < t) and the original Avey's coupled causal contextualizer
+
+NEXT = [
+    sy.custom("uni_coupled_s64", B=2, N=1500, S=64, d=128, m=256, k=5,
+              pattern=(sy.COUPLED, sy.DYNAMIC, sy.STATIC), centers=12, sigma=0.5),
+    sy.custom("uni_coupled_s32", B=1, N=2000, S=32, d=96, m=192, m_h=64, k=7,
+              pattern=(sy.STATIC, sy.COUPLED), centers=32, sigma=0.5),
+    sy.custom("uni_coupled_f32", B=1, N=300, S=16, d=64, m=128, k=3, pattern=(sy.COUPLED,),
+              dtype="f32", centers=10, sigma=0.3),
+]
+
+
+@pytest.mark.parametrize("wl", NEXT, ids=lambda w: w.name)
+def test_unidirectional_ranker_and_coupled_layers(wl, cuda_dev):
+    E, W = sy.gen_embeddings(wl), sy.gen_weights(wl)
+    g, o, _ = compare(wl, E, W, orc.all_targets(wl.B, wl.n), cuda_dev, causal=True)
+    idx = g["idx_full"]
+    for t in range(wl.n):
+        real = idx[:, t][idx[:, t] >= 0]
+        assert np.all(real < t)
+        assert (idx[:, t] >= 0).sum(axis=-1).max() == min(wl.k, t)
