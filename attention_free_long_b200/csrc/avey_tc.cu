@@ -48,7 +48,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kRedGroups = 8, kRedCands = 16;
 
 enum { MODE_MAXSIM = 0, MODE_ENRICH = 1, MODE_FUSE = 2, MODE_MAXSIM_SYM = 3 };
-constexpr int kSymGroup = 16;  // row tiles per L2 group of the triangular MaxSim order
+constexpr int kSymGroup = 64;  // row tiles per L2 group of the triangular MaxSim order
 
 struct TcArgs {
   int rows;  // A rows per batch

@@ -13,7 +13,7 @@ import math
 
 import pytest
 
-G = 16  # row tiles per group
+G = 64  # row tiles per group (kSymGroup)
 
 
 def _prefix(g, tn):
