@@ -20,6 +20,11 @@ using bf16 = __nv_bfloat16;
 avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N, int R, int rs_ld,
                              int d, int S, int n, float *scores, cudaStream_t s);
 
+// The same scores from 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2),
+// avey_maxsim2.cu; S in {32, 64, 128}, rs_ld >= R rounded up to 256.
+avey_status launch_maxsim_pair(const bf16 *x, const float *inv_norm, int B, int N, int R, int rs_ld,
+                               int d, int S, int n, float *scores, cudaStream_t s);
+
 // Enricher: Z = relu(scale_row * (X U) + b)^2, X given as a split pair
 // (xhi, xlo) [T, d]; Ut [m, d]; writes the split pair of Z (zhi, zlo) [T, m].
 // inv_rms may be null (scale 1).

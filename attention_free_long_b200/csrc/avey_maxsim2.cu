@@ -1,0 +1,454 @@
+// avey_maxsim2.cu -- MaxSim split scores on CTA pairs (tcgen05 cta_group::2).
+//
+// Same computation as the triangular MaxSim of avey_tc.cu (Avey-B paperlayer
+// summary §3 and papernotes 整体框架: score(t, c) = sum over the rows of split t
+// of the max cosine to a row of split c), laid out for two SMs per tile:
+//
+//   * A cluster of two CTAs owns a 256 x 256 tile of G = X X^T: each CTA
+//     holds 128 of its rows in TMEM (fp32), loads those 128 rows of X (A) and
+//     one half (128 rows) of the column tile (B) with TMA; CTA 0 issues
+//     tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), which reads A and
+//     both halves of B across the pair.  Per FLOP each SM moves a third fewer
+//     bytes from L2 than with 128 x 256 tiles on one SM.
+//   * Tiles are square in 256-row blocks, so the triangular order is simply
+//     nt >= mt: the diagonal tile yields the scores of its own splits from
+//     row maxima; a tile right of the diagonal yields score(t -> c) from row
+//     maxima and score(c -> t) from column maxima over each target split's
+//     rows (a target split never straddles the two CTAs).
+//   * Roles per CTA (320 threads): warp 0 TMA producer; warp 1 TMEM
+//     allocation (both CTAs) and the MMA issue (CTA 0); warps 2-9 epilogue,
+//     two per TMEM lane quarter, one per 128-column half.
+//   * Barriers: each CTA's loads complete on CTA 0's "full" barrier; the MMA
+//     commit frees the stage in both CTAs and publishes the accumulator to
+//     both; both CTAs' epilogue warps release the accumulator to CTA 0.
+//     Every wait is bounded (avey_common.cuh); no load uses multicast.
+#include <algorithm>
+
+#include "avey_common.cuh"
+#include "avey_internal.h"
+
+namespace avey {
+namespace {
+
+constexpr int PT = 256;                       // tile edge (rows and columns)
+constexpr int BK = 64;                        // K chunk (128-byte swizzled rows)
+constexpr int kStages = 6;
+constexpr int kEpi = 8;
+constexpr int kThreads = 64 + 32 * kEpi;
+constexpr uint32_t kTmemCols = 512;           // two 128 x 256 fp32 accumulators per CTA
+constexpr int kGroup = 32;                    // 256-row tiles per L2 group
+constexpr int kRedCands = 16;
+constexpr uint32_t HALF_BYTES = 128 * BK * 2;  // 16 KB: 128 rows x 64 bf16
+constexpr uint32_t STAGE_BYTES = 2 * HALF_BYTES;
+constexpr uint32_t TILES_BYTES = kStages * STAGE_BYTES;
+constexpr uint32_t CTRL_BYTES = 10240;
+constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct PairArgs {
+  int n;              // splits per sequence
+  int tiles;          // 256-blocks per sequence (rows = columns)
+  long long slots;    // triangular-order slots per sequence
+  int num_tiles;      // B * slots
+  int kchunks;
+  float *scores;      // [B, n, n]
+  const float *inv_norm;
+  int rs_ld;
+  int *status;
+};
+
+__device__ __forceinline__ long long pair_prefix(long long g, long long tn) {
+  return kGroup * g * tn - static_cast<long long>(kGroup) * kGroup * g * (g - 1) / 2;
+}
+
+// Slot -> (sequence, row block, column block).  Group g holds row blocks
+// 32g .. 32g+31 and column blocks 32g .. tiles-1; slots left of the diagonal
+// (nt < mt) hold no work and every role skips them alike.
+__device__ __forceinline__ bool decode_pair(const PairArgs &a, int tile, int &b, int &mt, int &nt) {
+  b = static_cast<int>(tile / a.slots);
+  const long long x = tile - static_cast<long long>(b) * a.slots;
+  const long long tn = a.tiles;
+  const double A = static_cast<double>(kGroup) * tn + kGroup * kGroup / 2.0;
+  const double disc = A * A - 2.0 * kGroup * kGroup * static_cast<double>(x);
+  long long g = static_cast<long long>((A - sqrt(disc > 0 ? disc : 0)) / (kGroup * kGroup));
+  if (g < 0) g = 0;
+  while (g > 0 && pair_prefix(g, tn) > x) --g;
+  while (pair_prefix(g + 1, tn) <= x && (g + 1) * kGroup < a.tiles) ++g;
+  const long long rem = x - pair_prefix(g, tn);
+  const int rows_g = min(kGroup, a.tiles - static_cast<int>(g) * kGroup);
+  nt = static_cast<int>(g * kGroup + rem / rows_g);
+  mt = static_cast<int>(g * kGroup + rem % rows_g);
+  return nt >= mt;
+}
+
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// One epilogue warp: its 32 rows (TMEM lanes) x its 128 columns.  Row maxima
+// per candidate split -> red; column maxima over the warp's rows -> cm (only
+// right of the diagonal).  Cosines are formed in full: dot * 1/|x_i| * 1/|x_j|.
+template <int S>
+__device__ __forceinline__ void pair_rows(uint32_t taddr, int lane, int quarter, int half, float *red,
+                                          float *cm, const float *__restrict__ col_scale,
+                                          float row_scale, bool need_col) {
+  constexpr int CH_PER_CAND = S / 32;
+  float m = -INFINITY;
+#pragma unroll 1
+  for (int pr = 0; pr < 2; ++pr) {
+    const int ch0 = 4 * half + 2 * pr;  // 32-column chunk index inside the 256-column tile
+    const float4 *cs4 = reinterpret_cast<const float4 *>(col_scale + ch0 * 32);
+    float4 c4[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) c4[q] = __ldg(cs4 + q);
+    float v[64];
+    tmem_ld64(taddr + ch0 * 32, v);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      v[4 * q] *= c4[q].x * row_scale;
+      v[4 * q + 1] *= c4[q].y * row_scale;
+      v[4 * q + 2] *= c4[q].z * row_scale;
+      v[4 * q + 3] *= c4[q].w * row_scale;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int ch = ch0 + u;
+      if (ch % CH_PER_CAND == 0) m = -INFINITY;
+      m = fmaxf(m, max32(v + 32 * u));
+      if (ch % CH_PER_CAND == CH_PER_CAND - 1) {
+        float t = m;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+        if (lane == 0) red[quarter * kRedCands + ch / CH_PER_CAND] = t;
+      }
+    }
+    if (need_col) {
+      float c[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) c[j] = warp_max(v[j]);
+      if (lane == 0) {
+        float4 *dst = reinterpret_cast<float4 *>(cm + (quarter * 8 + ch0) * 32);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) dst[q] = make_float4(c[4 * q], c[4 * q + 1], c[4 * q + 2], c[4 * q + 3]);
+      }
+    }
+  }
+}
+
+// Leader warp of one half: scores of this CTA's target splits against the
+// half's candidate splits (row maxima), and, right of the diagonal, of the
+// half's splits as targets against this CTA's splits (column maxima).
+template <int S>
+__device__ __forceinline__ void pair_write(const PairArgs &a, const float *red, const float *cm,
+                                           int lane, int b, int t0, int c0, int half,
+                                           bool need_col) {
+  constexpr int TS = 128 / S, PER = S / 32, CB = 128 / S;
+  float *scores = a.scores + static_cast<long long>(b) * a.n * a.n;
+  for (int e = lane; e < TS * CB; e += 32) {
+    const int ts = e / CB, cl = e - (e / CB) * CB;
+    float sc = 0.f;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) sc += red[(ts * PER + q) * kRedCands + half * CB + cl];
+    const int t = t0 + ts, c = c0 + cl;
+    if (t < a.n && c < a.n) scores[static_cast<long long>(t) * a.n + c] = sc;
+  }
+  if (!need_col) return;
+  for (int ts = 0; ts < TS; ++ts) {
+    for (int cl = 0; cl < CB; ++cl) {
+      float sum = 0.f;
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int ch = half * 4 + cl * PER + u;
+        float mx = cm[((ts * PER) * 8 + ch) * 32 + lane];
+#pragma unroll
+        for (int q = 1; q < PER; ++q) mx = fmaxf(mx, cm[((ts * PER + q) * 8 + ch) * 32 + lane]);
+        sum += mx;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      const int t = t0 + ts, c = c0 + cl;
+      if (lane == 0 && t < a.n && c < a.n) scores[static_cast<long long>(c) * a.n + t] = sum;
+    }
+  }
+}
+
+template <int S>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    maxsim_pair_kernel(const __grid_constant__ CUtensorMap tmX, const PairArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t *ctrl = smem_raw + pad + TILES_BYTES;
+  const uint32_t sbase = raw_s + pad;
+  const uint32_t cbase = sbase + TILES_BYTES;
+  // control block: full[6] @0, empty[6] @64, tfull[2] @128, tempty[2] @144,
+  // redbar[4] @160, redfree[4] @192, drain @224, tmem base @232, abort @236,
+  // red @256, column maxima @2048
+  auto full_bar = [&](int s) { return cbase + 8u * s; };
+  auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
+  auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
+  auto tempty_bar = [&](int i) { return cbase + 144u + 8u * i; };
+  auto red_bar = [&](int i) { return cbase + 160u + 8u * i; };
+  auto red_free = [&](int i) { return cbase + 192u + 8u * i; };
+  const uint32_t drain_bar = cbase + 224u;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 232);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 236);
+  float *red = reinterpret_cast<float *>(ctrl + 256);
+  float *cmx = reinterpret_cast<float *>(ctrl + 2048);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), 2 * kEpi);  // both CTAs' epilogue warps (used in CTA 0)
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(red_bar(i), 4);
+      mbar_init(red_free(i), 1);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tmX);
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote use
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(ctrl + 232), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // -------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < a.num_tiles && ok; tile += npairs) {
+        int b, mt, nt;
+        if (!decode_pair(a, tile, b, mt, nt)) continue;
+        for (int kc = 0; kc < a.kchunks; ++kc) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          const uint32_t full0 = mapa_shared(full_bar(stage), 0);
+          const uint32_t st = sbase + stage * STAGE_BYTES;
+          tma_load_3d_pair(st, &tmX, full0, kc * BK, mt * PT + rank * 128, b);
+          tma_load_3d_pair(st + HALF_BYTES, &tmX, full0, kc * BK, nt * PT + rank * 128, b);
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      // Drain: the pair's MMA has consumed (so the loads have landed in) every
+      // stage this CTA filled once its last use is released.
+      for (int s = 0; s < kStages; ++s) {
+        if (issued > s) {
+          const long long last = ((issued - 1 - s) / kStages) * kStages + s;
+          wait_drain(empty_bar(s), static_cast<uint32_t>((last / kStages) & 1));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------- MMA issue (CTA 0)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * 128, PT);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < a.num_tiles && ok; tile += npairs) {
+        int b, mt, nt;
+        if (!decode_pair(a, tile, b, mt, nt)) continue;
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * PT);
+        for (int kc = 0; kc < a.kchunks; ++kc) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + stage * STAGE_BYTES;
+          const uint64_t da = sdesc_k_sw128(st);
+          const uint64_t db = sdesc_k_sw128(st + HALF_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_bf16_pair(d_tmem, da + 2u * kk, db + 2u * kk, idesc, (kc | kk) != 0);
+          tc_commit_pair_both(empty_bar(stage));
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(tfull_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      tc_commit_pair_both(drain_bar);
+      wait_drain(drain_bar, 0);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t tempty_r0 = mapa_shared(tempty_bar(0), 0), tempty_r1 = mapa_shared(tempty_bar(1), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < a.num_tiles; tile += npairs) {
+      int b, mt, nt;
+      if (!decode_pair(a, tile, b, mt, nt)) continue;
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int rb = acc * 2 + half;
+      if (!mbar_wait(red_free(rb), acc_phase ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint32_t taddr =
+          tmem_base + static_cast<uint32_t>(acc * PT) + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int row0 = mt * PT + static_cast<int>(rank) * 128;  // this CTA's rows of the tile
+      const bool need_col = nt > mt;
+      float *red_acc = red + acc * 8 * kRedCands;
+      float *cm_acc = cmx + acc * (4 * 8 * 32);
+      const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
+      pair_rows<S>(taddr, lane, quarter, half, red_acc, cm_acc, rs + nt * PT, rs[row0 + quarter * 32 + lane],
+                   need_col);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(acc ? tempty_r1 : tempty_r0);  // release this accumulator to the MMA issuer
+        mbar_arrive(red_bar(rb));
+      }
+      if (warp == 2 + 4 * half) {
+        if (!mbar_wait(red_bar(rb), acc_phase, abort_flag)) {
+          ok = false;
+        } else {
+          pair_write<S>(a, red_acc, cm_acc, lane, b, row0 / S, (nt * PT + half * 128) / S, half,
+                        need_col);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(red_free(rb));
+      }
+      if (!ok) break;
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // Both CTAs past their loops: the pair's MMAs have drained (CTA 0 waited on
+  // the drain commit) and no remote arrival is still on its way.
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+  cluster_sync_all();
+}
+
+template <int S>
+avey_status run_pair(const CUtensorMap &mx, PairArgs a, cudaStream_t st) {
+  auto kern = maxsim_pair_kernel<S>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(SMEM_BYTES));
+  if (e != cudaSuccess) {
+    set_detail("maxsim_pair: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return AVEY_ERR_CUDA;
+  }
+  // Persistent grid: as many pairs as can be resident at once (a pair needs
+  // two SMs of one GPC, so this can be below half the SM count).
+  static int resident[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &cap = resident[dev & 63];
+  if (cap == 0) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * (sm_count() / 2));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    if (e != cudaSuccess || clusters < 1) {
+      set_detail("maxsim_pair: no resident CTA pair (%s)", cudaGetErrorString(e));
+      return AVEY_ERR_CUDA;
+    }
+    cap = std::min(clusters, sm_count() / 2);
+  }
+  const int pairs = std::max(1, std::min(a.num_tiles, cap));
+  kern<<<2 * pairs, kThreads, SMEM_BYTES, st>>>(mx, a);
+  AVEY_CHECK_LAUNCH("maxsim_pair");
+  return AVEY_OK;
+}
+
+}  // namespace
+
+avey_status launch_maxsim_pair(const bf16 *x, const float *inv_norm, int B, int N, int R, int rs_ld,
+                               int d, int S, int n, float *scores, cudaStream_t s) {
+  CUtensorMap mx;
+  const uint64_t rs = static_cast<uint64_t>(d) * 2, bs = rs * static_cast<uint64_t>(N);
+  if (!encode_bf16_map(&mx, x, d, N, B, rs, bs, 128)) return AVEY_ERR_CUDA;
+  PairArgs a{};
+  a.n = n;
+  a.tiles = (R + PT - 1) / PT;
+  long long slots = 0;
+  for (long long g = 0; g * kGroup < a.tiles; ++g)
+    slots += std::min<long long>(kGroup, a.tiles - g * kGroup) * (a.tiles - g * kGroup);
+  a.slots = slots;
+  if (slots * B > 0x7fffffffll || rs_ld < a.tiles * PT) {
+    set_detail("maxsim_pair: problem too large");
+    return AVEY_ERR_UNSUPPORTED;
+  }
+  a.num_tiles = static_cast<int>(slots * B);
+  a.kchunks = (d + BK - 1) / BK;
+  a.scores = scores;
+  a.inv_norm = inv_norm;
+  a.rs_ld = rs_ld;
+  a.status = device_status_word();
+  switch (S) {
+    case 32: return run_pair<32>(mx, a, s);
+    case 64: return run_pair<64>(mx, a, s);
+    case 128: return run_pair<128>(mx, a, s);
+    default: set_detail("maxsim_pair: S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace avey

@@ -351,8 +351,12 @@ extern "C" avey_status avey_rank_ex(const void *x, avey_dtype dt, int B, int N, 
     const int ld = static_cast<int>(scale_ld(R));
     st = launch_inv_norms(static_cast<const bf16 *>(x), B, N, d, ld, inv, s);
     if (st != AVEY_OK) return st;
-    st = launch_maxsim_tc(static_cast<const bf16 *>(x), inv, B, N, static_cast<int>(R), ld, d, S,
-                          static_cast<int>(n), sc, s);
+    if (S >= 32)
+      st = launch_maxsim_pair(static_cast<const bf16 *>(x), inv, B, N, static_cast<int>(R), ld, d,
+                              S, static_cast<int>(n), sc, s);
+    else
+      st = launch_maxsim_tc(static_cast<const bf16 *>(x), inv, B, N, static_cast<int>(R), ld, d, S,
+                            static_cast<int>(n), sc, s);
   } else {
     void *xhat = wsb;
     st = launch_normalize(x, dt, B, N, d, S, xhat, s);

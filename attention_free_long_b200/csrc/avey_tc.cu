@@ -10,6 +10,8 @@
 //           factor commutes with the max), then sums the maxima over the S
 //           rows of each target split.  Only the [B, n, n] split scores reach
 //           HBM; neither the N x N cosines nor a normalised copy of X exist.
+//           Full grid of tiles; serves S = 16 (for S >= 32 the triangular
+//           CTA-pair kernel of avey_maxsim2.cu computes half the tiles).
 //   Enricher (papernotes 整体框架, Z = sigma(XU+b); ReLU^2 per the paperlayer
 //           summary App. A): D = X U with X as a bf16 split pair (two MMAs per
 //           K step); epilogue scale (optional prenorm) + bias + ReLU^2, Z
@@ -37,25 +39,17 @@ namespace avey {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64;
-// Epilogue warps: 8 for the triangular MaxSim (two per TMEM lane quarter, one
-// per 128-column block), 4 otherwise.
-template <int MODE>
-struct Roles {
-  static constexpr int EPI = MODE == 3 ? 8 : 4;
-  static constexpr int THREADS = 64 + 32 * EPI;
-};
+constexpr int kEpi = 4, kThreads = 64 + 32 * kEpi;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRedGroups = 8, kRedCands = 16;
 
-enum { MODE_MAXSIM = 0, MODE_ENRICH = 1, MODE_FUSE = 2, MODE_MAXSIM_SYM = 3 };
-constexpr int kSymGroup = 64;  // row tiles per L2 group of the triangular MaxSim order
+enum { MODE_MAXSIM = 0, MODE_ENRICH = 1, MODE_FUSE = 2 };
 
 struct TcArgs {
   int rows;  // A rows per batch
   int cols;  // B rows (output columns)
   int kdim;  // contraction length
   int tiles_m, tiles_n, num_tiles, group_m;
-  long long sym_slots;  // triangular MaxSim: tile slots per sequence
   // MaxSim
   int S, n;
   float *scores;
@@ -80,43 +74,17 @@ struct Layout {
   static constexpr uint32_t STAGE_BYTES = A_PLANES * A_BYTES + B_BYTES;
   static constexpr int STAGES = A_PLANES == 1 ? 4 : 3;
   static constexpr uint32_t TILES_BYTES = STAGES * STAGE_BYTES;
-  // barriers etc. (+ the MaxSim partial sums and column maxima), 1 KB units
-  static constexpr uint32_t CTRL_BYTES = A_PLANES == 1 ? 2048 + 8192 : 1024;
+  // barriers etc. (+ the MaxSim partial sums), 1 KB units
+  static constexpr uint32_t CTRL_BYTES = A_PLANES == 1 ? 2048 : 1024;
   // layer GEMMs: per epilogue warp 8 KB of swizzled output staging for TMA stores
   static constexpr uint32_t STAGING_BYTES = A_PLANES == 1 ? 0 : 4 * 8192;
   static constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + STAGING_BYTES + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// Tile slots of the triangular MaxSim order before row-tile group g (all
-// earlier groups are full): group g holds rows 16g..16g+15 and column tiles
-// 8g..tiles_n-1, i.e. every column tile that reaches the group's diagonal.
-__device__ __forceinline__ long long sym_prefix(long long g, long long tn) {
-  return kSymGroup * g * tn - (kSymGroup / 2) * kSymGroup * g * (g - 1) / 2;
-}
-
-// Decodes a tile index into (sequence, row tile, column tile).  Returns false
-// for slots of the triangular order that hold no work (column tile entirely
-// left of the row tile's diagonal); every role skips the same slots.
+// Decodes a tile index into (sequence, row tile, column tile).
 template <int MODE>
 __device__ __forceinline__ bool decode_tile(const TcArgs &a, int tile, int &b, int &mt, int &nt) {
-  if (MODE == MODE_MAXSIM_SYM) {
-    b = static_cast<int>(tile / a.sym_slots);
-    const long long x = tile - static_cast<long long>(b) * a.sym_slots;
-    const long long tn = a.tiles_n;
-    // smallest root of P(g) = x, then integer correction
-    const double A = static_cast<double>(kSymGroup) * tn + (kSymGroup / 2) * kSymGroup / 2.0;
-    const double disc = A * A - 2.0 * (kSymGroup / 2) * kSymGroup * static_cast<double>(x);
-    long long g = static_cast<long long>((A - sqrt(disc > 0 ? disc : 0)) / ((kSymGroup / 2) * kSymGroup));
-    if (g < 0) g = 0;
-    while (g > 0 && sym_prefix(g, tn) > x) --g;
-    while (sym_prefix(g + 1, tn) <= x && (g + 1) * kSymGroup < a.tiles_m) ++g;
-    const long long rem = x - sym_prefix(g, tn);
-    const int rows_g = min(kSymGroup, a.tiles_m - static_cast<int>(g) * kSymGroup);
-    nt = static_cast<int>(g * (kSymGroup / 2) + rem / rows_g);
-    mt = static_cast<int>(g * kSymGroup + rem % rows_g);
-    return 2 * nt + 1 >= mt;
-  }
   if (MODE == MODE_MAXSIM) {
     // Groups of group_m row tiles walk the column tiles together so that the
     // group's rows stay in L2 while every column tile streams past once.
@@ -200,133 +168,6 @@ __device__ __forceinline__ void epi_maxsim_rows(uint32_t taddr, int lane, int qu
           if ((lane & 15) == 0) red[(quarter * 2 + (lane >> 4)) * kRedCands + cand] = t;
         }
       }
-    }
-  }
-}
-
-// Triangular MaxSim, one tile (row block I = mt, column blocks 2nt, 2nt+1 of
-// 128 columns).  Per 32-column chunk the cosines are formed in full (column
-// and row scale); chunks of a block left of the diagonal (K < I) are skipped
-// because the tile (K, I/2) covers that pair; for blocks right of it (K > I)
-// the column maxima over this warp's rows are kept in cm as well, which give
-// the mirrored scores score(c -> t).
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// Max of the 32 values (a tree of three-input maxima).
-__device__ __forceinline__ float max32(const float (&v)[32]) {
-  float a[11];
-#pragma unroll
-  for (int i = 0; i < 10; ++i) a[i] = max3f(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-  a[10] = fmaxf(v[30], v[31]);
-  const float b0 = max3f(a[0], a[1], a[2]), b1 = max3f(a[3], a[4], a[5]);
-  const float b2 = max3f(a[6], a[7], a[8]), b3 = fmaxf(a[9], a[10]);
-  return max3f(b0, b1, fmaxf(b2, b3));
-}
-
-// Max over the warp's 32 lanes, delivered to every lane.
-__device__ __forceinline__ float warp_max(float v) {
-  float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
-}
-
-template <int S>
-__device__ __forceinline__ void epi_maxsim_sym_rows(uint32_t taddr, int lane, int quarter, int half,
-                                                    float *red, float *cm,
-                                                    const float *__restrict__ col_scale,
-                                                    float row_scale, int mt, int nt) {
-  static_assert(S >= 32, "the triangular MaxSim needs S >= 32");
-  constexpr int CH_PER_CAND = S / 32;
-  const int K = 2 * nt + half;  // this warp's 128-column block
-  if (K < mt) return;           // left of the diagonal: covered by tile (K, mt/2)
-  float m = -INFINITY;
-#pragma unroll 1
-  for (int pr = 0; pr < 2; ++pr) {  // two 64-column pieces of the block
-    const int ch0 = 4 * half + 2 * pr;
-    const float4 *cs4 = reinterpret_cast<const float4 *>(col_scale + ch0 * 32);
-    float4 c4[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) c4[q] = __ldg(cs4 + q);
-    float v[64];
-    tmem_ld64(taddr + ch0 * 32, v);
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      v[4 * q] *= c4[q].x * row_scale;
-      v[4 * q + 1] *= c4[q].y * row_scale;
-      v[4 * q + 2] *= c4[q].z * row_scale;
-      v[4 * q + 3] *= c4[q].w * row_scale;
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int ch = ch0 + u;
-      if (ch % CH_PER_CAND == 0) m = -INFINITY;
-      float part[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) part[j] = v[32 * u + j];
-      m = fmaxf(m, max32(part));
-      if (ch % CH_PER_CAND == CH_PER_CAND - 1) {
-        float t = m;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-        if (lane == 0) red[quarter * kRedCands + ch / CH_PER_CAND] = t;
-      }
-    }
-    if (K > mt) {
-      // column maxima over this warp's 32 rows: one warp reduction per column
-      float c[64];
-#pragma unroll
-      for (int j = 0; j < 64; ++j) c[j] = warp_max(v[j]);
-      if (lane == 0) {
-        float4 *dst = reinterpret_cast<float4 *>(cm + (quarter * 8 + ch0) * 32);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) dst[q] = make_float4(c[4 * q], c[4 * q + 1], c[4 * q + 2], c[4 * q + 3]);
-      }
-    }
-  }
-}
-
-// Leader warp of the triangular MaxSim: row-direction scores for the blocks on
-// or right of the diagonal, column-direction (mirrored) scores for the blocks
-// right of it.
-template <int S>
-__device__ __forceinline__ void epi_maxsim_sym_write(const TcArgs &a, const float *red,
-                                                     const float *cm, int lane, int b, int mt,
-                                                     int nt, int half) {
-  constexpr int TS = BM / S, PER = S / 32, CB = 128 / S;
-  const int K = 2 * nt + half;
-  if (K < mt) return;
-  float *scores = a.scores + static_cast<long long>(b) * a.n * a.n;
-  // row direction: targets of this row block against the candidates of block K
-  for (int e = lane; e < TS * CB; e += 32) {
-    const int ts = e / CB, cl = e - (e / CB) * CB;
-    const int cs = half * CB + cl;  // candidate index inside the 256-column tile
-    float sc = 0.f;
-#pragma unroll
-    for (int q = 0; q < PER; ++q) sc += red[(ts * PER + q) * kRedCands + cs];
-    const int t = mt * TS + ts, c = K * CB + cl;
-    if (t < a.n && c < a.n) scores[static_cast<long long>(t) * a.n + c] = sc;
-  }
-  if (K == mt) return;
-  // column direction: candidates of block K as targets against this row block
-  for (int ts = 0; ts < TS; ++ts) {
-    for (int cl = 0; cl < CB; ++cl) {
-      float sum = 0.f;
-#pragma unroll
-      for (int u = 0; u < PER; ++u) {
-        const int ch = half * 4 + cl * PER + u;
-        float mx = cm[((ts * PER) * 8 + ch) * 32 + lane];
-#pragma unroll
-        for (int q = 1; q < PER; ++q) mx = fmaxf(mx, cm[((ts * PER + q) * 8 + ch) * 32 + lane]);
-        sum += mx;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      const int t = mt * TS + ts, c = K * CB + cl;
-      if (lane == 0 && t < a.n && c < a.n) scores[static_cast<long long>(c) * a.n + t] = sum;
     }
   }
 }
@@ -482,7 +323,7 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mou
 // ---- the kernel ------------------------------------------------------------
 
 template <int MODE, int A_PLANES, int SPLIT_S>
-__global__ void __launch_bounds__(Roles<MODE>::THREADS, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmO0,
               const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2,
@@ -495,20 +336,17 @@ __global__ void __launch_bounds__(Roles<MODE>::THREADS, 1)
   const uint32_t sbase = raw_s + pad;
   const uint32_t cbase = sbase + L::TILES_BYTES;
   // control block: full[4] @0, empty[4] @64, tfull[2] @128, tempty[2] @144,
-  // redbar[2 acc][2 halves] @160, drain @192, tmem base @200, abort flag @204,
-  // redfree[2 acc][2 halves] @224, red @256, column maxima @2048
+  // redbar[2 acc] @160, drain @192, tmem base @200, abort flag @204,
+  // MaxSim partial sums [2 acc][8 groups][16 candidates] @256
   auto full_bar = [&](int s) { return cbase + 8u * s; };
   auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
   auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
   auto tempty_bar = [&](int i) { return cbase + 144u + 8u * i; };
   auto red_bar = [&](int i) { return cbase + 160u + 8u * i; };
-  auto red_free = [&](int i) { return cbase + 224u + 8u * i; };
   const uint32_t drain_bar = cbase + 192u;
   volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 200);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 204);
-  constexpr int EPI = Roles<MODE>::EPI;
   float *red = reinterpret_cast<float *>(ctrl + 256);
-  float *cmx = reinterpret_cast<float *>(ctrl + 2048);  // [2][4 warps][8 chunks][32] column maxima
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -519,12 +357,9 @@ __global__ void __launch_bounds__(Roles<MODE>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull_bar(i), 1);
-      mbar_init(tempty_bar(i), EPI);
+      mbar_init(tempty_bar(i), kEpi);
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(red_bar(i), 4);
-      mbar_init(red_free(i), 1);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(red_bar(i), 4);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -596,10 +431,6 @@ __global__ void __launch_bounds__(Roles<MODE>::THREADS, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
-        if (MODE == MODE_MAXSIM_SYM) {
-          int b_, mt_, nt_;
-          if (!decode_tile<MODE>(a, tile, b_, mt_, nt_)) continue;
-        }
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -659,41 +490,7 @@ __global__ void __launch_bounds__(Roles<MODE>::THREADS, 1)
       const uint32_t taddr =
           tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
       const int row = mt * BM + quarter * 32 + lane;
-      if constexpr (MODE == MODE_MAXSIM_SYM) {
-        const int half = (warp - 2) >> 2;  // warps 2-5: block 2nt, warps 6-9: block 2nt+1
-        const int rb = acc * 2 + half;
-        float *red_acc = red + acc * kRedGroups * kRedCands;
-        float *cm_acc = cmx + acc * (4 * 8 * 32);
-        const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
-        // the leader must have consumed the partials this buffer held two tiles ago
-        if (!mbar_wait(red_free(rb), acc_phase ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        epi_maxsim_sym_rows<SPLIT_S>(taddr, lane, quarter, half, red_acc, cm_acc, rs + nt * BN,
-                                     rs[row], mt, nt);
-        // TMEM is no longer needed by this warp: release it before the combine
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(tempty_bar(acc));
-          mbar_arrive(red_bar(rb));
-        }
-        if (warp == 2 + 4 * half) {
-          // leader of this half: combine its four warps' partial results
-          if (!mbar_wait(red_bar(rb), acc_phase, abort_flag)) {
-            ok = false;
-          } else {
-            epi_maxsim_sym_write<SPLIT_S>(a, red_acc, cm_acc, lane, b, mt, nt, half);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(red_free(rb));
-        }
-        if (!ok) break;
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-        continue;
-      } else if constexpr (MODE == MODE_MAXSIM) {
+      if constexpr (MODE == MODE_MAXSIM) {
         float *red_acc = red + acc * kRedGroups * kRedCands;
         const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
         epi_maxsim_rows<SPLIT_S>(taddr, lane, quarter, red_acc, rs + nt * BN, rs[row]);
@@ -748,7 +545,7 @@ avey_status run_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorM
     return AVEY_ERR_CUDA;
   }
   const int grid = std::min(args.num_tiles, sm_count());
-  kern<<<grid, Roles<MODE>::THREADS, L::SMEM_BYTES, st>>>(a0, a1, b, o0, o1, o2, args);
+  kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(a0, a1, b, o0, o1, o2, args);
   AVEY_CHECK_LAUNCH(name);
   return AVEY_OK;
 }
@@ -779,23 +576,6 @@ avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N,
   TcArgs a = base_args(R, R, d);
   a.num_tiles = a.tiles_m * a.tiles_n * B;
   a.group_m = 16;
-  if (S >= 32) {
-    // triangular order: group g of kSymGroup row tiles takes the column tiles
-    // from 8g on (those that reach the group's diagonal)
-    const long long tn = a.tiles_n;
-    const long long groups = (a.tiles_m + kSymGroup - 1) / kSymGroup;
-    long long slots = 0;
-    for (long long g = 0; g < groups; ++g) {
-      const long long rows = std::min<long long>(kSymGroup, a.tiles_m - g * kSymGroup);
-      slots += rows * (tn - g * (kSymGroup / 2));
-    }
-    a.sym_slots = slots;
-    if (slots * B > 0x7fffffffll) {
-      set_detail("maxsim_tc: too many tiles");
-      return AVEY_ERR_UNSUPPORTED;
-    }
-    a.num_tiles = static_cast<int>(slots * B);
-  }
   a.S = S;
   a.n = n;
   a.scores = scores;
@@ -803,9 +583,9 @@ avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N,
   a.rs_ld = rs_ld;
   switch (S) {
     case 16: return run_tc<MODE_MAXSIM, 1, 16>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
-    case 32: return run_tc<MODE_MAXSIM_SYM, 1, 32>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
-    case 64: return run_tc<MODE_MAXSIM_SYM, 1, 64>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
-    case 128: return run_tc<MODE_MAXSIM_SYM, 1, 128>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
+    case 32: return run_tc<MODE_MAXSIM, 1, 32>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
+    case 64: return run_tc<MODE_MAXSIM, 1, 64>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
+    case 128: return run_tc<MODE_MAXSIM, 1, 128>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
     default: set_detail("maxsim_tc: S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
   }
 }

@@ -69,13 +69,15 @@ def maxsim_flops(wl) -> float:
 
 
 def maxsim_executed_flops(wl) -> float:
-    """MMA work the MaxSim kernel executes: 128x256 tiles of the (nS) x (nS)
-    product, only those on or right of each row tile's diagonal block when
-    S >= 32 (the mirrored scores come from the same tile), all tiles for S = 16."""
+    """MMA work the MaxSim kernel executes: for S >= 32, the 256x256 tiles on or
+    right of the diagonal of 256-row blocks (the mirrored scores come from the
+    same tile); for S = 16, every 128x256 tile of the (nS) x (nS) product."""
     R = wl.n * wl.S
-    tm, tn = -(-R // 128), -(-R // 256)
-    tiles = tm * tn if wl.S < 32 else sum(tn - mt // 2 for mt in range(tm))
-    return 2.0 * wl.B * tiles * 128 * 256 * (-(-wl.d // 64) * 64)
+    kpad = -(-wl.d // 64) * 64
+    if wl.S >= 32:
+        t = -(-R // 256)
+        return 2.0 * wl.B * (t * (t + 1) // 2) * 256 * 256 * kpad
+    return 2.0 * wl.B * (-(-R // 128)) * (-(-R // 256)) * 128 * 256 * kpad
 
 
 def layer_flops(wl) -> float:
@@ -339,7 +341,7 @@ def run_ours(args):
     achieved = maxsim_flops(wl) / (rank_ms * 1e-3) / 1e12
     mix_bytes = 2.0 * T * mt * 4  # read Z_t pair, write c pair
     comp_bytes = (wl.k + 1) * wl.T * wl.d * 2.0 + wl.T * wl.d * 8.0
-    kernel_src = os.path.join(ROOT, "attention_free_long_b200", "csrc", "avey_tc.cu")
+    kernel_src = os.path.join(ROOT, "attention_free_long_b200", "csrc", "avey_maxsim2.cu")
     result = {
         "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
