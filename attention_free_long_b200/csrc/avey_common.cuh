@@ -339,6 +339,15 @@ __device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
       : "memory");
 }
 
+// Two fp32 products in one instruction (round to nearest), sm_100.
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
+  return *reinterpret_cast<const float2 *>(&r);
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

@@ -88,51 +88,58 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-// One epilogue warp: its 32 rows (TMEM lanes) x its 128 columns.  Row maxima
-// per candidate split -> red; column maxima over the warp's rows -> cm (only
-// right of the diagonal).  Cosines are formed in full: dot * 1/|x_i| * 1/|x_j|.
+// One epilogue warp: its 32 rows (TMEM lanes) x its 128 columns.  With
+// v = x_i . x_j, r_i = 1/|x_i| and c_j = 1/|x_j| (both >= 0), the cosine's
+// row maximum is r_i * max_j (v c_j) and its column maximum c_j * max_i (v r_i);
+// each direction takes one packed product per two entries.  Row maxima per
+// candidate split, summed over the warp's rows -> red; column maxima of v r_i
+// over the warp's rows -> cm (only right of the diagonal; c_j is applied when
+// they are summed).
 template <int S>
 __device__ __forceinline__ void pair_rows(uint32_t taddr, int lane, int quarter, int half, float *red,
                                           float *cm, const float *__restrict__ col_scale,
                                           float row_scale, bool need_col) {
   constexpr int CH_PER_CAND = S / 32;
+  const float2 r2 = make_float2(row_scale, row_scale);
   float m = -INFINITY;
 #pragma unroll 1
   for (int pr = 0; pr < 2; ++pr) {
     const int ch0 = 4 * half + 2 * pr;  // 32-column chunk index inside the 256-column tile
     const float4 *cs4 = reinterpret_cast<const float4 *>(col_scale + ch0 * 32);
-    float4 c4[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) c4[q] = __ldg(cs4 + q);
     float v[64];
     tmem_ld64(taddr + ch0 * 32, v);
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      v[4 * q] *= c4[q].x * row_scale;
-      v[4 * q + 1] *= c4[q].y * row_scale;
-      v[4 * q + 2] *= c4[q].z * row_scale;
-      v[4 * q + 3] *= c4[q].w * row_scale;
-    }
-#pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int ch = ch0 + u;
+      float p[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 c = __ldg(cs4 + 8 * u + q);
+        const float2 a = fmul2(make_float2(v[32 * u + 4 * q], v[32 * u + 4 * q + 1]), make_float2(c.x, c.y));
+        const float2 b = fmul2(make_float2(v[32 * u + 4 * q + 2], v[32 * u + 4 * q + 3]), make_float2(c.z, c.w));
+        p[4 * q] = a.x;
+        p[4 * q + 1] = a.y;
+        p[4 * q + 2] = b.x;
+        p[4 * q + 3] = b.y;
+      }
       if (ch % CH_PER_CAND == 0) m = -INFINITY;
-      m = fmaxf(m, max32(v + 32 * u));
+      m = fmaxf(m, max32(p));
       if (ch % CH_PER_CAND == CH_PER_CAND - 1) {
-        float t = m;
+        float t = m * row_scale;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
         if (lane == 0) red[quarter * kRedCands + ch / CH_PER_CAND] = t;
       }
-    }
-    if (need_col) {
-      float c[64];
+      if (need_col) {
+        // column maxima of v r_i over this warp's 32 rows: one warp reduction per column
+        float4 *dst = reinterpret_cast<float4 *>(cm + (quarter * 8 + ch) * 32);
 #pragma unroll
-      for (int j = 0; j < 64; ++j) c[j] = warp_max(v[j]);
-      if (lane == 0) {
-        float4 *dst = reinterpret_cast<float4 *>(cm + (quarter * 8 + ch0) * 32);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) dst[q] = make_float4(c[4 * q], c[4 * q + 1], c[4 * q + 2], c[4 * q + 3]);
+        for (int g = 0; g < 8; ++g) {
+          const float2 a = fmul2(make_float2(v[32 * u + 4 * g], v[32 * u + 4 * g + 1]), r2);
+          const float2 b = fmul2(make_float2(v[32 * u + 4 * g + 2], v[32 * u + 4 * g + 3]), r2);
+          const float4 mx = make_float4(warp_max(a.x), warp_max(a.y), warp_max(b.x), warp_max(b.y));
+          if (lane == 0) dst[g] = mx;
+        }
       }
     }
   }
@@ -140,11 +147,12 @@ __device__ __forceinline__ void pair_rows(uint32_t taddr, int lane, int quarter,
 
 // Leader warp of one half: scores of this CTA's target splits against the
 // half's candidate splits (row maxima), and, right of the diagonal, of the
-// half's splits as targets against this CTA's splits (column maxima).
+// half's splits as targets against this CTA's splits (column maxima times
+// 1/|x_j|, summed over the candidate's columns).
 template <int S>
 __device__ __forceinline__ void pair_write(const PairArgs &a, const float *red, const float *cm,
-                                           int lane, int b, int t0, int c0, int half,
-                                           bool need_col) {
+                                           const float *__restrict__ col_scale, int lane, int b,
+                                           int t0, int c0, int half, bool need_col) {
   constexpr int TS = 128 / S, PER = S / 32, CB = 128 / S;
   float *scores = a.scores + static_cast<long long>(b) * a.n * a.n;
   for (int e = lane; e < TS * CB; e += 32) {
@@ -165,7 +173,7 @@ __device__ __forceinline__ void pair_write(const PairArgs &a, const float *red, 
         float mx = cm[((ts * PER) * 8 + ch) * 32 + lane];
 #pragma unroll
         for (int q = 1; q < PER; ++q) mx = fmaxf(mx, cm[((ts * PER + q) * 8 + ch) * 32 + lane]);
-        sum += mx;
+        sum += mx * __ldg(col_scale + ch * 32 + lane);
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
@@ -357,8 +365,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!mbar_wait(red_bar(rb), acc_phase, abort_flag)) {
           ok = false;
         } else {
-          pair_write<S>(a, red_acc, cm_acc, lane, b, row0 / S, (nt * PT + half * 128) / S, half,
-                        need_col);
+          pair_write<S>(a, red_acc, cm_acc, rs + nt * PT, lane, b, row0 / S,
+                        (nt * PT + half * 128) / S, half, need_col);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(red_free(rb));
