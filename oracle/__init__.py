@@ -65,6 +65,8 @@ def lib():
             L.avey_orc_compress_rows.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int, _I, _I, ctypes.c_int, _I, _D, _D,
                                                  _D]
+            L.avey_orc_context_rows.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, _I, _I, ctypes.c_int, _I, _D, _D]
             L.avey_orc_static_mix.argtypes = [_D, _D, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_longlong, _D, ctypes.c_longlong]
             L.avey_orc_dynamic_weights.argtypes = [_D, ctypes.c_int, ctypes.c_int,
@@ -181,6 +183,20 @@ def compress(X, S: int, k: int, sel, idx, w, P) -> np.ndarray:
     return out
 
 
+def context(X, S: int, k: int, sel, idx, w) -> np.ndarray:
+    """Uncompressed context of each selected target: [n_sel, (k+1)S, d] with
+    rows [X_t ; w_1 X_c1 ; ... ; w_k X_ck] (the compressor's input, eq. 8)."""
+    X = _f64(X)
+    B, N, d = X.shape
+    sel = _i32(sel).reshape(-1, 2)
+    sb, st = _i32(sel[:, 0]), _i32(sel[:, 1])
+    idx, w = _i32(idx), _f64(w)
+    out = np.empty((sel.shape[0], (k + 1) * S, d), dtype=np.float64)
+    lib().avey_orc_context_rows(_pd(X), N, d, S, k, _pi(sb), _pi(st), sel.shape[0], _pi(idx),
+                                _pd(w), _pd(out))
+    return out
+
+
 # ----------------------------------------------------------------- layer ----
 
 def static_mix(V, zt) -> np.ndarray:
@@ -260,3 +276,30 @@ def forward(X, weights, wl, sel=None, idx=None, w=None, causal: bool = False):
         x = layer(x, lw, wl.S, wl.m_h, wl.eps, wl.prenorm)
         outs.append(x)
     return dict(sel=sel, scores=scores, idx=oidx, w=ow, compressed=xc, layers=outs)
+
+
+def forward_uncompressed(X, weights, wl, sel=None, idx=None, w=None, causal: bool = False):
+    """The processor without neural compression ([AB-sum] §4.3: the ablation
+    that the 4.37x throughput figure compares against).
+
+    Ranker once; each selected target's (k+1)S-token context
+    [X_t ; w_1 X_c1 ; ... ; w_k X_ck] goes through every layer as one block, so
+    the contextualizer mixes all (k+1)S tokens (V is (k+1)S x (k+1)S, from
+    synthetic.gen_weights(wl, block=(k+1)S)); the first S rows of the last
+    layer's block are the target split's output.
+    Returns dict(sel, scores, idx, w, context, layers=[per-layer [n_sel, (k+1)S, d]],
+    out [n_sel, S, d]).
+    """
+    X = _f64(X)
+    sel, scores, oidx, ow = rank(X, wl.S, wl.k, sel, causal)
+    use_idx = oidx if idx is None else _i32(idx)
+    use_w = ow if w is None else _f64(w)
+    ctx = context(X, wl.S, wl.k, sel, use_idx, use_w)
+    L = (wl.k + 1) * wl.S
+    outs = []
+    x = ctx
+    for lw in weights.layers:
+        x = layer(x, lw, L, wl.m_h, wl.eps, wl.prenorm)
+        outs.append(x)
+    return dict(sel=sel, scores=scores, idx=oidx, w=ow, context=ctx, layers=outs,
+                out=x[:, :wl.S, :].copy())

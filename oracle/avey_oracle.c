@@ -323,6 +323,34 @@ void avey_orc_layer(double *x, int n_splits, int S, int d, int m, int m_h, int k
   }
 }
 
+/* Uncompressed context of target split t of sequence b (the tensor that the
+ * compressor of [AB-notes] 关键设计 4 maps from (k+1)S tokens to S, and that
+ * the neural processor sees in full without it, [AB-sum] §4.3):
+ *   X_cat = [X_t ; w_1 X_c1 ; ... ; w_k X_ck]          ((k+1)S x d)
+ * in rank order, the target block unweighted; a missing candidate (-1) and the
+ * pad rows of a ragged last split are zero rows. */
+void avey_orc_context_split(const double *x, int N, int d, int S, int k, int b, int t,
+                            const int *idx, const double *w, double *out) {
+  for (int r = 0; r <= k; ++r) {
+    int c = (r == 0) ? t : idx[r - 1];
+    double wr = (r == 0) ? 1.0 : w[r - 1];
+    for (int j = 0; j < S; ++j) {
+      double *o = out + ((long long)r * S + j) * d;
+      const double *xc_j = c < 0 ? 0 : split_row(x, N, d, S, b, c, j);
+      for (int q = 0; q < d; ++q) o[q] = xc_j ? wr * xc_j[q] : 0.0;
+    }
+  }
+}
+
+void avey_orc_context_rows(const double *x, int N, int d, int S, int k, const int *sel_b,
+                           const int *sel_t, int n_sel, const int *idx, const double *w,
+                           double *out) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int s = 0; s < n_sel; ++s)
+    avey_orc_context_split(x, N, d, S, k, sel_b[s], sel_t[s], idx + (long long)s * k,
+                           w + (long long)s * k, out + (long long)s * (k + 1) * S * d);
+}
+
 /* Compression of several target splits (independent; one split per thread). */
 void avey_orc_compress_rows(const double *x, int N, int d, int S, int k, const int *sel_b,
                             const int *sel_t, int n_sel, const int *idx, const double *w,

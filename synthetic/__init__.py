@@ -163,8 +163,17 @@ class Weights:
     layers: List[LayerWeights]
 
 
-def gen_weights(w: Workload, seed: int = 1) -> Weights:
+def gen_weights(w: Workload, seed: int = 1, block: int = 0) -> Weights:
+    """Seeded weights in a fixed draw order (P, then per layer U, bU, V, O).
+
+    ``block`` is the contextualizer's token block (V is block x block); the
+    default is the split size S.  The uncompressed processor mixes blocks of
+    (k+1)S tokens and takes block=(k+1)S: its V are drawn from a second stream
+    (seed, 1000 + layer), while the main stream makes the same draws as for
+    block=S, so P, U, bU and O are identical.
+    """
     rng = np.random.Generator(np.random.PCG64(seed))
+    blk = block if block else w.S
 
     def draw(shape, fan_in):
         a = (rng.standard_normal(shape, dtype=np.float32) * np.float32(1.0 / math.sqrt(fan_in)))
@@ -172,10 +181,14 @@ def gen_weights(w: Workload, seed: int = 1) -> Weights:
 
     P = draw((w.S, (w.k + 1) * w.S), (w.k + 1) * w.S)
     layers = []
-    for kind in w.pattern:
+    for li, kind in enumerate(w.pattern):
         U = draw((w.d, w.m), w.d)
         bU = draw((w.m,), w.d)
         V = draw((w.S, w.S), w.S) if kind in (STATIC, COUPLED) else None
+        if V is not None and blk != w.S:
+            r2 = np.random.Generator(np.random.PCG64([seed, 1000 + li]))
+            a = r2.standard_normal((blk, blk), dtype=np.float32) * np.float32(1.0 / math.sqrt(blk))
+            V = round_bf16(a) if w.dtype == "bf16" else a.astype(np.float32)
         O = draw((w.m, w.d), w.m)
         layers.append(LayerWeights(kind, U, bU, V, O))
     return Weights(P, layers)

@@ -102,3 +102,14 @@ def layer(x, U, bU, V, O, m_h, kind, eps, prenorm):
         cat = Zh[i] + c[i]
         out.append([x[i][q] + sum(cat[f] * O[f][q] for f in range(m)) for q in range(d)])
     return out
+
+
+def context(X, S, k, b, t, idx, w):
+    """[X_t ; w_1 X_c1 ; ... ; w_k X_ck] as a list of (k+1)S rows."""
+    N, d = len(X[0]), len(X[0][0])
+    rows = [_row(X, b, N, S, t, j, d) for j in range(S)]
+    for r in range(k):
+        c = idx[r]
+        for j in range(S):
+            rows.append([w[r] * a for a in _row(X, b, N, S, c, j, d)] if c >= 0 else [0.0] * d)
+    return rows
