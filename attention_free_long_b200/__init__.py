@@ -76,6 +76,10 @@ def lib() -> ctypes.CDLL:
         L.avey_layer_forward.restype = _i
         L.avey_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.avey_layer_workspace_bytes.restype = _sz
+        L.avey_layer_workspace_bytes_ex.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+        L.avey_layer_workspace_bytes_ex.restype = _sz
+        L.avey_context.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]
+        L.avey_context.restype = _i
         L.avey_device_status.argtypes = [_vp]
         L.avey_device_status.restype = _i
         L.avey_status_string.argtypes = [_i]
@@ -181,6 +185,28 @@ def avey_compress(x: torch.Tensor, S: int, k: int, idx: torch.Tensor, w: torch.T
     return out, pair
 
 
+def avey_context(x: torch.Tensor, S: int, k: int, idx: torch.Tensor, w: torch.Tensor,
+                 out: Optional[torch.Tensor] = None, lowp: bool = True):
+    """Uncompressed context [X_t ; w_1 X_c1 ; ... ; w_k X_ck] of every split.
+
+    Returns (out fp32 [B, n, (k+1)S, d], pair [2, B*n*(k+1)S, d] bf16 or None).
+    """
+    for t, nm in ((x, "x"), (idx, "idx"), (w, "w")):
+        _need(t, nm)
+    B, N, d = x.shape
+    n = -(-N // S)
+    dt = _dt(x)
+    L = (k + 1) * S
+    if out is None:
+        out = torch.empty((B, n, L, d), dtype=torch.float32, device=x.device)
+    pair = None
+    if dt == AVEY_BF16 and lowp:
+        pair = torch.empty((2, B * n * L, d), dtype=torch.bfloat16, device=x.device)
+    _check("avey_context", lib().avey_context(_ptr(x), dt, B, N, d, S, k, _ptr(idx), _ptr(w),
+                                              _ptr(out), _ptr(pair), _stream()))
+    return out, pair
+
+
 # ------------------------------------------------------------- dynamic mix --
 
 def avey_dynamic_mix(zt: torch.Tensor, S: int, eps: float, mt: Optional[int] = None,
@@ -218,7 +244,12 @@ class DeviceLayer:
     Ot: torch.Tensor  # [d, m] (O transposed)
 
 
-def layer_workspace_bytes(dtype: int, T: int, d: int, m: int, prenorm: bool) -> int:
+def layer_workspace_bytes(dtype: int, T: int, d: int, m: int, prenorm: bool, S: int = 0,
+                          kind: int = 1) -> int:
+    """Workspace of one layer; S > 128 (blocks of (k+1)S tokens) adds what a
+    dynamic layer over such blocks needs."""
+    if S > 128:
+        return int(lib().avey_layer_workspace_bytes_ex(dtype, T, d, m, int(bool(prenorm)), S, kind))
     return int(lib().avey_layer_workspace_bytes(dtype, T, d, m, int(bool(prenorm))))
 
 
@@ -240,7 +271,7 @@ def avey_layer_forward(layer: DeviceLayer, S: int, m_h: int, eps: float, prenorm
         x_out = torch.empty_like(x_in)
     if dt == AVEY_BF16 and lowp_out and x_out_lowp is None:
         x_out_lowp = torch.empty((2, T, d), dtype=torch.bfloat16, device=x_in.device)
-    need = layer_workspace_bytes(dt, T, d, m, prenorm)
+    need = layer_workspace_bytes(dt, T, d, m, prenorm, S, layer.kind)
     if ws is None or ws.numel() < need:
         ws = _ws(need, x_in.device)
     p = LayerParams(layer.kind, d, m, m_h, S, eps, int(bool(prenorm)), layer.Ut.data_ptr(),
@@ -279,12 +310,15 @@ class EncoderWorkspace:
 
 
 def make_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: torch.dtype, prenorm: bool,
-                   device) -> EncoderWorkspace:
+                   device, uncompressed: bool = False) -> EncoderWorkspace:
+    """Buffers for encoder_forward, or (uncompressed=True) for
+    encoder_forward_uncompressed, whose layers run on B*n*(k+1)S tokens."""
     n = -(-N // S)
-    T = B * n * S
+    blk = (k + 1) * S if uncompressed else S
+    T = B * n * blk
     dt = AVEY_BF16 if dtype == torch.bfloat16 else AVEY_F32
     rank_ws = _ws(rank_workspace_bytes(dt, B, N, d, S), device)
-    layer_ws = _ws(layer_workspace_bytes(dt, T, d, m, prenorm), device)
+    layer_ws = _ws(layer_workspace_bytes(dt, T, d, m, prenorm, blk, AVEY_DYNAMIC), device)
     idx = torch.empty((B, n, k), dtype=torch.int32, device=device)
     w = torch.empty((B, n, k), dtype=torch.float32, device=device)
     x0 = torch.empty((T, d), dtype=torch.float32, device=device)
@@ -339,3 +373,52 @@ def encoder_forward(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLay
             marks[3 + li].record()
         cur, nxt = nxt, cur
     return cur[0].view(B, n * S, d)
+
+
+def encoder_forward_uncompressed(x: torch.Tensor, layers: Sequence[DeviceLayer], S: int, k: int,
+                                 m_h: int, eps: float, prenorm: bool,
+                                 ws: Optional[EncoderWorkspace] = None, marks=None,
+                                 causal: bool = False) -> torch.Tensor:
+    """The processor without neural compression (Avey-B paperlayer summary
+    §4.3): ranker once, then each split's (k+1)S-token context
+    [X_t ; w_1 X_c1 ; ... ; w_k X_ck] goes through every layer as one block
+    (the layers' V are (k+1)S x (k+1)S).  Returns fp32 [B, n, S, d], the first
+    S rows of every block (a view).
+
+    ``marks``: optional list of 3 + len(layers) torch.cuda.Event, recorded on
+    the current stream before the ranker and after every C-ABI call.
+    """
+    B, N, d = x.shape
+    n = -(-N // S)
+    L_ = (k + 1) * S
+    T = B * n * L_
+    dt = _dt(x)
+    m = layers[0].Ut.shape[0] if layers else d
+    if ws is None:
+        ws = make_workspace(B, N, d, S, k, m, x.dtype, prenorm, x.device, uncompressed=True)
+    L = lib()
+    st = _stream()
+    if marks is not None:
+        marks[0].record()
+    _check("avey_rank", L.avey_rank_ex(_ptr(x), dt, B, N, d, S, k,
+                                       AVEY_RANK_UNIDIRECTIONAL if causal else 0, _ptr(ws.idx),
+                                       _ptr(ws.w), None, _ptr(ws.rank_ws), ws.rank_ws.numel(), st))
+    if marks is not None:
+        marks[1].record()
+    _check("avey_context", L.avey_context(_ptr(x), dt, B, N, d, S, k, _ptr(ws.idx), _ptr(ws.w),
+                                          _ptr(ws.x0), _ptr(ws.pair0), st))
+    if marks is not None:
+        marks[2].record()
+    cur, nxt = (ws.x0, ws.pair0), (ws.x1, ws.pair1)
+    for li, lay in enumerate(layers):
+        p = LayerParams(lay.kind, d, m, m_h, L_, eps, int(bool(prenorm)), lay.Ut.data_ptr(),
+                        lay.bU.data_ptr(), None if lay.V is None else lay.V.data_ptr(),
+                        lay.Ot.data_ptr())
+        _check("avey_layer_forward",
+               L.avey_layer_forward(ctypes.byref(p), dt, T, _ptr(cur[0]), _ptr(cur[1]),
+                                    _ptr(nxt[0]), _ptr(nxt[1]), _ptr(ws.layer_ws),
+                                    ws.layer_ws.numel(), st))
+        if marks is not None:
+            marks[3 + li].record()
+        cur, nxt = nxt, cur
+    return cur[0].view(B, n, L_, d)[:, :, :S, :]

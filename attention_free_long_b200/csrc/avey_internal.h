@@ -63,4 +63,13 @@ avey_status launch_static_mix_f32(const float *V, const float *zt, int64_t ld_zt
 avey_status launch_dynamic_mix_f32(const float *zt, int64_t ld_zt, float *out, int64_t ld_out,
                                    int blocks, int S, int mt, float eps, cudaStream_t s);
 
+// ---- mixes over long blocks of 256 or 512 tokens (avey_mix_long.cu) ----
+// In place on the split pair Z_t (hi at zt, lo at zt + plane).  The dynamic
+// mix needs long_dynamic_ws_bytes(blocks, SL) bytes of workspace.
+size_t long_dynamic_ws_bytes(int blocks, int SL);
+avey_status launch_long_static_mix(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int SL, int mt,
+                                   int64_t plane, cudaStream_t s);
+avey_status launch_long_dynamic_mix(bf16 *zt, int64_t ld, int64_t plane, int blocks, int SL, int mt,
+                                    float eps, void *ws, cudaStream_t s);
+
 }  // namespace avey

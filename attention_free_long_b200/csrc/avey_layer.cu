@@ -128,6 +128,14 @@ extern "C" size_t avey_layer_workspace_bytes(avey_dtype dt, int T, int d, int m,
   return b;
 }
 
+extern "C" size_t avey_layer_workspace_bytes_ex(avey_dtype dt, int T, int d, int m, int prenorm,
+                                                int S, avey_ctx_kind kind) {
+  size_t b = avey_layer_workspace_bytes(dt, T, d, m, prenorm);
+  if (b && dt == AVEY_BF16 && kind == AVEY_DYNAMIC && S > 128 && S > 0 && T % S == 0)
+    b += align256(long_dynamic_ws_bytes(T / S, S));
+  return b;
+}
+
 extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype dt, int T,
                                           const float *x_in, const void *x_in_lowp, float *x_out,
                                           void *x_out_lowp, void *ws, size_t ws_bytes,
@@ -155,12 +163,15 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
                AVEY_ERR_INVALID_ARG, "avey_layer_forward: pointers must be 16-byte aligned");
   AVEY_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255) == 0, AVEY_ERR_INVALID_ARG,
                "avey_layer_forward: workspace must be 256-byte aligned");
-  const size_t need = avey_layer_workspace_bytes(dt, T, d, m, p->prenorm);
+  const size_t need = avey_layer_workspace_bytes_ex(dt, T, d, m, p->prenorm, S, p->kind);
   AVEY_REQUIRE(ws_bytes >= need, AVEY_ERR_INVALID_ARG,
                "avey_layer_forward: workspace %zu bytes < %zu required", ws_bytes, need);
   if (dt == AVEY_BF16)
-    AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
-                 "avey_layer_forward(BF16): S=%d unsupported (16, 32, 64 or 128)", S);
+    AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128 ||
+                     ((S == 256 || S == 512) && p->kind != AVEY_COUPLED_CAUSAL),
+                 AVEY_ERR_UNSUPPORTED,
+                 "avey_layer_forward(BF16): S=%d unsupported (16, 32, 64 or 128; 256 or 512 for "
+                 "static and dynamic layers)", S);
   else
     AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
                  "avey_layer_forward(F32): S=%d unsupported (power of two <= 64)", S);
@@ -222,7 +233,14 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   st = launch_enrich_tc(xhi, xlo, T, d, static_cast<const bf16 *>(p->Ut), m, p->bU, inv, Zhi, Zlo, s);
   if (st != AVEY_OK) return st;
   const int64_t plane = static_cast<int64_t>(T) * m;
-  if (p->kind == AVEY_STATIC)
+  if (S > 128) {
+    // blocks of (k+1)S tokens (the processor without compression)
+    if (p->kind == AVEY_STATIC)
+      st = launch_long_static_mix(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane, s);
+    else
+      st = launch_long_dynamic_mix(Zhi + m_h, m, plane, blocks, S, mt, p->eps,
+                                   w + avey_layer_workspace_bytes(dt, T, d, m, p->prenorm), s);
+  } else if (p->kind == AVEY_STATIC)
     st = launch_static_mix_x2(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane, s);
   else if (p->kind == AVEY_DYNAMIC)
     st = launch_dynamic_mix_x2(Zhi + m_h, m, plane, Zhi + m_h, m, plane, blocks, S, mt, p->eps, s);

@@ -333,6 +333,54 @@ def run_ours(args):
     st = av.device_status()
     if st != 0:
         raise RuntimeError(f"device status {av.STATUS.get(st, st)} after the e2e region")
+    h2d_bytes = int(xh.numel() * xh.element_size())
+    d2h_bytes = int(outh[0].numel() * outh[0].element_size())
+    del wss, xd, outh, xh
+    torch.cuda.empty_cache()
+
+    # ---- the processor without neural compression, same workload ----
+    # Every split's (k+1)S-token context goes through the layers as one block
+    # (Avey-B paperlayer summary §4.3); the pages report compression as a
+    # 4.37x throughput gain over this.
+    unc = None
+    if not args.no_uncompressed:
+        Wu = sy.gen_weights(wl, block=(wl.k + 1) * wl.S)
+        layers_u = av.device_layers(Wu, dt, dev)
+        ws_u = av.make_workspace(wl.B, wl.N, wl.d, wl.S, wl.k, wl.m, dt, wl.prenorm, dev,
+                                 uncompressed=True)
+
+        def step_u(m=None):
+            return av.encoder_forward_uncompressed(x, layers_u, wl.S, wl.k, wl.m_h, wl.eps,
+                                                   wl.prenorm, ws_u, m)
+
+        for _ in range(2):
+            step_u()
+        torch.cuda.synchronize()
+        st = av.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {av.STATUS.get(st, st)} in the uncompressed run")
+        reps_u = max(3, min(10, args.steps))
+        marks_u = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks + 1)]
+                   for _ in range(reps_u)]
+        barrier()
+        torch.cuda.synchronize()
+        start.record()
+        for r_ in range(reps_u):
+            step_u(marks_u[r_])
+        end.record()
+        torch.cuda.synchronize()
+        ms_u = max_over_ranks(start.elapsed_time(end) / reps_u, dev)
+        st_u = np.array([[marks_u[r_][i].elapsed_time(marks_u[r_][i + 1]) for i in range(n_marks)]
+                         for r_ in range(reps_u)]).mean(axis=0)
+        unc = {"ms_per_step": ms_u, "value": wl.B * wl.N * world / (ms_u * 1e-3), "unit": UNIT,
+               "steps": reps_u, "compression_speedup": ms_u / ms_max, "pages_speedup": 4.37,
+               "kernels_ms": {"rank": float(st_u[0]), "context": float(st_u[1]),
+                              "layers": st_u[2:].tolist()},
+               "note": ("each split's (k+1)S-token context through every layer as one block; "
+                        "compression_speedup = uncompressed / compressed ms per step on this GPU; "
+                        "pages_speedup is the pages' figure (their hardware and code)")}
+        del ws_u, layers_u
+        torch.cuda.empty_cache()
 
     tokens = wl.B * wl.N * world
     peaks, peak_kind = load_peaks()
@@ -371,12 +419,14 @@ def run_ours(args):
                              "frac": comp_bytes / (compress_ms * 1e-3) / 1e9 / hbm,
                              "bytes": comp_bytes}},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
-                "d2h_bytes_per_step": int(outh[0].numel() * outh[0].element_size()),
+                "h2d_bytes_per_step": h2d_bytes,
+                "d2h_bytes_per_step": d2h_bytes,
                 "note": "copies of neighbouring steps overlap compute (two buffers, copy streams)"},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
+    if unc is not None:
+        result["uncompressed"] = unc
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, E, W)
     if world > 1:
@@ -434,6 +484,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(sy.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-uncompressed", action="store_true",
+                    help="skip the measurement of the processor without compression")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -161,6 +161,28 @@ AVEY_API avey_status avey_compress(const void *x, avey_dtype dt, int B, int N, i
                           const int32_t *idx, const float *w, const void *P, float *out,
                           void *out_lowp, avey_stream_t stream);
 
+/* --------------------------------------------------- uncompressed context --
+ * avey_context: the context of every split without neural compression, for
+ * the processor variant that contextualizes all (k+1)S tokens of each split
+ * ([AB-sum] §4.3, the ablation behind the 4.37x throughput figure; the
+ * tensor is the compressor's input of eq. 8, [AB-notes] 关键设计 4):
+ *   ctx(b, t) = [X_t ; w_1 X_c1 ; ... ; w_k X_ck]   ((k+1)S x d, rank order)
+ * The target block is unweighted; a candidate of -1 and the pad rows of a
+ * ragged last split are zero rows.
+ *
+ * x, idx, w as for avey_compress (out of range indices are rejected on the
+ *          device as AVEY_ERR_DEVICE_BOUNDS and their block is zero).
+ * out      [B, n, (k+1)S, d] fp32 (caller-owned).
+ * out_lowp for AVEY_BF16: NULL or an AVEY_BF16X2 pair [2][B*n*(k+1)S][d] of
+ *          `out`.  Ignored for F32.
+ * The processor then runs avey_layer_forward on T = B*n*(k+1)S tokens with
+ * S = (k+1)S (one block per split); rows [0, S) of each block are the split's
+ * output.  Constraints: d % 8 == 0; k <= 32.
+ */
+AVEY_API avey_status avey_context(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
+                                  const int32_t *idx, const float *w, float *out, void *out_lowp,
+                                  avey_stream_t stream);
+
 /* ----------------------------------------------------------- dynamic mix --
  * avey_dynamic_mix: the dynamic contextualizer of one layer on `blocks`
  * independent split blocks of S tokens ([AB-notes] 关键设计 2 and 3):
@@ -208,7 +230,9 @@ AVEY_API avey_status avey_dynamic_mix(const void *zt, int64_t ld_zt, avey_dtype 
  *   x_out_lowp AVEY_BF16 only: NULL or an AVEY_BF16X2 pair [2][T][d] out.
  *   ws        >= avey_layer_workspace_bytes(...) bytes, 256-byte aligned.
  * Constraints: T % S == 0; d, m, m_h multiples of 8 with 0 < m_h < m;
- * S in {16, 32, 64, 128} for AVEY_BF16 (a power of two <= 64 for F32); eps >= 0.
+ * S in {16, 32, 64, 128} for AVEY_BF16, and also 256 or 512 for static and
+ * dynamic layers (the blocks of (k+1)S tokens of the uncompressed processor,
+ * see avey_context); a power of two <= 64 for F32; eps >= 0.
  */
 typedef struct {
   avey_ctx_kind kind;
@@ -226,7 +250,14 @@ AVEY_API avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype d
                                void *x_out_lowp, void *ws, size_t ws_bytes,
                                avey_stream_t stream);
 
+/* Workspace of avey_layer_forward for S <= 128 (any kind). */
 AVEY_API size_t avey_layer_workspace_bytes(avey_dtype dt, int T, int d, int m, int prenorm);
+
+/* Workspace of avey_layer_forward for any supported S and kind: a dynamic
+ * layer over blocks of 256 or 512 tokens also holds each block's Gt (as a
+ * bf16 split pair, 4 S^2 bytes per block) and two fp32 scales per token. */
+AVEY_API size_t avey_layer_workspace_bytes_ex(avey_dtype dt, int T, int d, int m, int prenorm, int S,
+                                              avey_ctx_kind kind);
 
 /* ------------------------------------------------------------- utilities --
  * avey_device_status: synchronises `stream`, returns the first kernel-side
