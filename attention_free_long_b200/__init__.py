@@ -80,6 +80,10 @@ def lib() -> ctypes.CDLL:
         L.avey_layer_workspace_bytes_ex.restype = _sz
         L.avey_context.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]
         L.avey_context.restype = _i
+        L.avey_topk.argtypes = [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _vp]
+        L.avey_topk.restype = _i
+        L.avey_static_mix.argtypes = [_vp, _vp, _i64, _i, _i, _i, _i, _vp, _i64, _vp]
+        L.avey_static_mix.restype = _i
         L.avey_device_status.argtypes = [_vp]
         L.avey_device_status.restype = _i
         L.avey_status_string.argtypes = [_i]
@@ -160,6 +164,19 @@ def avey_rank(x: torch.Tensor, S: int, k: int, return_scores: bool = False,
     return (idx, w, scores) if return_scores else (idx, w)
 
 
+def avey_topk(scores: torch.Tensor, k: int, causal: bool = False):
+    """Top-k selection and weights from precomputed scores [B, n, n] fp32."""
+    _need(scores, "scores")
+    if scores.dtype != torch.float32 or scores.dim() != 3 or scores.shape[1] != scores.shape[2]:
+        raise TypeError("scores must be fp32 [B, n, n]")
+    B, n, _ = scores.shape
+    idx = torch.empty((B, n, k), dtype=torch.int32, device=scores.device)
+    w = torch.empty((B, n, k), dtype=torch.float32, device=scores.device)
+    flags = AVEY_RANK_UNIDIRECTIONAL if causal else 0
+    _check("avey_topk", lib().avey_topk(_ptr(scores), B, n, k, flags, _ptr(idx), _ptr(w), _stream()))
+    return idx, w
+
+
 # ------------------------------------------------------------- compression --
 
 def avey_compress(x: torch.Tensor, S: int, k: int, idx: torch.Tensor, w: torch.Tensor,
@@ -229,6 +246,26 @@ def avey_dynamic_mix(zt: torch.Tensor, S: int, eps: float, mt: Optional[int] = N
     _need(out, "out")
     _check("avey_dynamic_mix", lib().avey_dynamic_mix(_ptr(zt), ld, dt, rows // S, S, mt, eps,
                                                       _ptr(out), out.shape[-1], _stream()))
+    return out
+
+
+def avey_static_mix(V: torch.Tensor, zt: torch.Tensor, S: int, mt: Optional[int] = None,
+                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Static contextualizer c = V Z_t on split blocks (layouts as avey_dynamic_mix)."""
+    _need(zt, "zt")
+    _need(V, "V")
+    if zt.dtype == torch.float32:
+        dt, rows, ld = AVEY_F32, zt.shape[0], zt.shape[1]
+    elif zt.dtype == torch.bfloat16 and zt.dim() == 3 and zt.shape[0] == 2:
+        dt, rows, ld = AVEY_BF16X2, zt.shape[1], zt.shape[2]
+    else:
+        raise TypeError("zt must be fp32 [rows, ld] or a bf16 pair [2, rows, ld]")
+    mt = ld if mt is None else mt
+    if out is None:
+        out = torch.empty_like(zt)
+    _need(out, "out")
+    _check("avey_static_mix", lib().avey_static_mix(_ptr(V), _ptr(zt), ld, dt, rows // S, S, mt,
+                                                    _ptr(out), out.shape[-1], _stream()))
     return out
 
 

@@ -34,7 +34,7 @@ struct CompressTile {
   static constexpr int XBYTES = S * XLD * 2;
   static constexpr int PBYTES = S * PLD * 2;
   static constexpr int STAGE = XBYTES + PBYTES;
-  static constexpr int NST = S >= 128 ? 2 : 3;  // cp.async pipeline depth over the k+1 blocks
+  static constexpr int NST = S >= 128 ? 2 : (S == 32 ? 3 : 4);  // cp.async depth over the k+1 blocks (2 CTAs / SM at S = 64)
   // output staging (reuses the pipeline buffers): fp32 [S][NS+4], hi/lo [S][NS+8]
   static constexpr int OLD32 = NS + 4;
   static constexpr int OUT_BYTES = S * OLD32 * 4 + 2 * S * XLD * 2;
@@ -122,27 +122,26 @@ __global__ void __launch_bounds__(256) compress_bf16(const bf16 *__restrict__ x,
     const uint8_t *xs = smem + (r % C::NST) * C::STAGE;
     const uint8_t *ps = xs + C::XBYTES;
     const float wr = s_w[r];
-    // Two 8-column subtiles at a time: the fp32 partial product of this block
-    // (tmp) is scaled by its weight and added to acc; A fragments are reloaded
-    // per pair, which keeps tmp at 2 subtiles and the kernel at 3 CTAs / SM.
+    // The fp32 partial product of this block (tmp) is scaled by its weight
+    // and added to acc; each P_r fragment is loaded once per k step.
+    float tmp[C::MI][C::NI][4];
 #pragma unroll
-    for (int j = 0; j < C::NI; j += 2) {
-      float tmp[C::MI][2][4];
+    for (int i = 0; i < C::MI; ++i)
 #pragma unroll
-      for (int i = 0; i < C::MI; ++i)
+      for (int j = 0; j < C::NI; ++j)
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj)
+        for (int q = 0; q < 4; ++q) tmp[i][j][q] = 0.f;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) tmp[i][jj][q] = 0.f;
+    for (int kk = 0; kk < S; kk += 16) {
+      uint32_t af[C::MI][4];
 #pragma unroll
-      for (int kk = 0; kk < S; kk += 16) {
-        uint32_t af[C::MI][4];
+      for (int i = 0; i < C::MI; ++i) {
+        const int row = wm * C::WM + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int col = kk + (lane >> 4) * 8;
+        ldsm_x4(smem_u32(ps + (row * C::PLD + col) * 2), af[i][0], af[i][1], af[i][2], af[i][3]);
+      }
 #pragma unroll
-        for (int i = 0; i < C::MI; ++i) {
-          const int row = wm * C::WM + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const int col = kk + (lane >> 4) * 8;
-          ldsm_x4(smem_u32(ps + (row * C::PLD + col) * 2), af[i][0], af[i][1], af[i][2], af[i][3]);
-        }
+      for (int j = 0; j < C::NI; j += 2) {
         uint32_t b0, b1, b2, b3;
         const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
         const int ncol = wn * C::WN + j * 8 + (lane >> 4) * 8;
@@ -150,17 +149,17 @@ __global__ void __launch_bounds__(256) compress_bf16(const bf16 *__restrict__ x,
         const uint32_t bA[2] = {b0, b1}, bB[2] = {b2, b3};
 #pragma unroll
         for (int i = 0; i < C::MI; ++i) {
-          mma16816(tmp[i][0], af[i], bA);
-          mma16816(tmp[i][1], af[i], bB);
+          mma16816(tmp[i][j], af[i], bA);
+          mma16816(tmp[i][j + 1], af[i], bB);
         }
       }
-#pragma unroll
-      for (int i = 0; i < C::MI; ++i)
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc[i][j + jj][q] = fmaf(wr, tmp[i][jj][q], acc[i][j + jj][q]);
     }
+#pragma unroll
+    for (int i = 0; i < C::MI; ++i)
+#pragma unroll
+      for (int j = 0; j < C::NI; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][j][q] = fmaf(wr, tmp[i][j][q], acc[i][j][q]);
     if (r == 0) {
       // residual: the target split's own tokens (stage 0 holds X_t)
 #pragma unroll

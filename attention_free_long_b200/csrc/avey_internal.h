@@ -47,8 +47,9 @@ avey_status launch_topk(const float *scores, int B, int n, int k, int causal, in
                         float *w, cudaStream_t s);
 
 // ---- mixes (avey_mix.cu) ----
-avey_status launch_static_mix_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int S, int mt,
-                                 int64_t plane, cudaStream_t s);
+avey_status launch_static_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks, int S,
+                                 int mt, int64_t plane, bf16 *out, int64_t ld_out,
+                                 int64_t plane_out, cudaStream_t s);
 avey_status launch_dynamic_mix_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
                                   int64_t ld_out, int64_t plane_out, int blocks, int S, int mt,
                                   float eps, cudaStream_t s);

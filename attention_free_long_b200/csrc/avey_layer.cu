@@ -241,7 +241,8 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
       st = launch_long_dynamic_mix(Zhi + m_h, m, plane, blocks, S, mt, p->eps,
                                    w + avey_layer_workspace_bytes(dt, T, d, m, p->prenorm), s);
   } else if (p->kind == AVEY_STATIC)
-    st = launch_static_mix_x2(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane, s);
+    st = launch_static_mix_x2(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane,
+                              Zhi + m_h, m, plane, s);
   else if (p->kind == AVEY_DYNAMIC)
     st = launch_dynamic_mix_x2(Zhi + m_h, m, plane, Zhi + m_h, m, plane, blocks, S, mt, p->eps, s);
   else

@@ -43,8 +43,10 @@ struct StaticTile {
 };
 
 template <int S>
-__global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V, bf16 *zt,
-                                                     long long ld, int mt, long long plane) {
+__global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V, const bf16 *zt,
+                                                     long long ld, int mt, long long plane,
+                                                     bf16 *out, long long ld_out,
+                                                     long long plane_out) {
   using C = StaticTile<S>;
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t *vs = smem;
@@ -54,7 +56,8 @@ __global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V,
   const int f0 = slab * C::NS;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wm = warp / C::WARPS_N, wn = warp % C::WARPS_N;
-  bf16 *zbase = zt + static_cast<long long>(blk) * S * ld;
+  const bf16 *zbase = zt + static_cast<long long>(blk) * S * ld;
+  bf16 *obase = out + static_cast<long long>(blk) * S * ld_out;
 
   for (int e = tid; e < S * (S / 8); e += 256) {
     const int row = e / (S / 8), cc = e % (S / 8);
@@ -120,9 +123,10 @@ __global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V,
     const int row = e / (C::NS / 8), cc = e % (C::NS / 8);
     const int f = f0 + cc * 8;
     if (f >= mt) continue;
-    bf16 *dst = zbase + row * ld + f;
+    bf16 *dst = obase + row * ld_out + f;
     *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(zh + (row * C::ZLD + cc * 8) * 2);
-    *reinterpret_cast<uint4 *>(dst + plane) = *reinterpret_cast<const uint4 *>(zl + (row * C::ZLD + cc * 8) * 2);
+    *reinterpret_cast<uint4 *>(dst + plane_out) =
+        *reinterpret_cast<const uint4 *>(zl + (row * C::ZLD + cc * 8) * 2);
   }
 }
 
@@ -457,12 +461,13 @@ avey_status set_smem(K kern, int bytes, const char *name) {
 }
 
 template <int S>
-avey_status run_static_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int mt, int64_t plane,
+avey_status run_static_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks, int mt,
+                          int64_t plane, bf16 *out, int64_t ld_out, int64_t plane_out,
                           cudaStream_t s) {
   using C = StaticTile<S>;
   if (avey_status st = set_smem(static_mix_x2<S>, C::SMEM, "static_mix_x2")) return st;
   const dim3 grid((mt + C::NS - 1) / C::NS, blocks);
-  static_mix_x2<S><<<grid, 256, C::SMEM, s>>>(V, zt, ld, mt, plane);
+  static_mix_x2<S><<<grid, 256, C::SMEM, s>>>(V, zt, ld, mt, plane, out, ld_out, plane_out);
   AVEY_CHECK_LAUNCH("static_mix_x2");
   return AVEY_OK;
 }
@@ -481,13 +486,14 @@ avey_status run_dynamic_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16
 
 }  // namespace
 
-avey_status launch_static_mix_x2(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int S, int mt,
-                                 int64_t plane, cudaStream_t s) {
+avey_status launch_static_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks, int S,
+                                 int mt, int64_t plane, bf16 *out, int64_t ld_out,
+                                 int64_t plane_out, cudaStream_t s) {
   switch (S) {
-    case 16: return run_static_x2<16>(V, zt, ld, blocks, mt, plane, s);
-    case 32: return run_static_x2<32>(V, zt, ld, blocks, mt, plane, s);
-    case 64: return run_static_x2<64>(V, zt, ld, blocks, mt, plane, s);
-    case 128: return run_static_x2<128>(V, zt, ld, blocks, mt, plane, s);
+    case 16: return run_static_x2<16>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
+    case 32: return run_static_x2<32>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
+    case 64: return run_static_x2<64>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
+    case 128: return run_static_x2<128>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
   }
   set_detail("static mix: S=%d unsupported", S);
   return AVEY_ERR_UNSUPPORTED;
@@ -562,6 +568,44 @@ avey_status launch_coupled_mix_f32(const float *V, const float *zt, int64_t ld_z
 }  // namespace avey
 
 using namespace avey;
+
+extern "C" avey_status avey_static_mix(const void *V, const void *zt, int64_t ld_zt, avey_dtype dt,
+                                       int blocks, int S, int mt, void *out, int64_t ld_out,
+                                       avey_stream_t stream) {
+  AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16X2, AVEY_ERR_UNSUPPORTED,
+               "avey_static_mix: dtype %d unsupported (F32 or BF16X2)", int(dt));
+  AVEY_REQUIRE(V && zt && out, AVEY_ERR_INVALID_ARG, "avey_static_mix: null pointer");
+  AVEY_REQUIRE(blocks >= 0 && S >= 1 && mt >= 1 && ld_zt >= mt && ld_out >= mt,
+               AVEY_ERR_INVALID_ARG, "avey_static_mix: bad sizes");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (blocks == 0) return AVEY_OK;
+  const char *zb = static_cast<const char *>(zt);
+  const char *obp = static_cast<const char *>(out);
+  const size_t es = dt == AVEY_F32 ? 4 : 2;
+  const size_t planes = dt == AVEY_BF16X2 ? 2 : 1;
+  const size_t zspan = static_cast<size_t>(blocks) * S * ld_zt * es * planes;
+  const size_t ospan = static_cast<size_t>(blocks) * S * ld_out * es * planes;
+  const bool same = zt == out && ld_zt == ld_out;
+  const bool overlap = !same && zb < obp + ospan && obp < zb + zspan;
+  AVEY_REQUIRE(!overlap, AVEY_ERR_INVALID_ARG,
+               "avey_static_mix: out overlaps zt without aliasing it exactly");
+  if (dt == AVEY_BF16X2) {
+    AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
+                 "avey_static_mix(BF16X2): S=%d unsupported (16, 32, 64 or 128)", S);
+    AVEY_REQUIRE(mt % 8 == 0 && ld_zt % 8 == 0 && ld_out % 8 == 0 && aligned16(zt) &&
+                     aligned16(out) && aligned16(V),
+                 AVEY_ERR_INVALID_ARG,
+                 "avey_static_mix(BF16X2): mt and ld must be multiples of 8, pointers 16-byte aligned");
+    const int64_t pz = static_cast<int64_t>(blocks) * S * ld_zt;
+    const int64_t po = static_cast<int64_t>(blocks) * S * ld_out;
+    return launch_static_mix_x2(static_cast<const bf16 *>(V), static_cast<const bf16 *>(zt), ld_zt,
+                                blocks, S, mt, pz, static_cast<bf16 *>(out), ld_out, po, s);
+  }
+  AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
+               "avey_static_mix(F32): S=%d unsupported (power of two <= 64)", S);
+  return launch_static_mix_f32(static_cast<const float *>(V), static_cast<const float *>(zt), ld_zt,
+                               static_cast<float *>(out), ld_out, blocks, S, mt, s);
+}
 
 extern "C" avey_status avey_dynamic_mix(const void *zt, int64_t ld_zt, avey_dtype dt, int blocks,
                                         int S, int mt, float eps, void *out, int64_t ld_out,

@@ -170,55 +170,101 @@ __global__ void __launch_bounds__(256) inv_norms(const bf16 *__restrict__ x, int
   if (lane == 0) inv[row] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
 }
 
-constexpr int kTopkWarps = 4;
+constexpr int kTopkWarps = 8;
+
+// One warp per target split, one pass over its score row.  The warp keeps
+// one sorted list of the k best candidates so far, lane q holding the q-th by
+// the key (score desc, index asc).  Every loaded element is compared with the
+// list's k-th key; the (rare, about k ln(n/k) per row) elements that beat it
+// are inserted one at a time, warp-wide: lanes behind the insertion point take
+// their predecessor's entry.  Self, and c > t for the unidirectional ranker,
+// never enter; -inf and NaN scores never beat the empty list's -inf.
+__device__ __forceinline__ bool key_gt(float a, int ia, float b, int ib) {
+  return a > b || (a == b && ia < ib);
+}
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
-    topk_warp(const float *__restrict__ scores, int B, int n, int k, int causal,
+    topk_warp(const float *__restrict__ scores, int B, int n, int k, int causal, int vec4,
               int32_t *__restrict__ idx, float *__restrict__ w) {
-  extern __shared__ float srow_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long rowid = static_cast<long long>(blockIdx.x) * kTopkWarps + warp;
   if (rowid >= static_cast<long long>(B) * n) return;
   const int t = static_cast<int>(rowid % n);
-  float *srow = srow_all + static_cast<long long>(warp) * n;
   const float *src = scores + rowid * n;
-  // candidates: every other split, or only the preceding ones when causal
-  for (int c = lane; c < n; c += 32) srow[c] = (c == t || (causal && c > t)) ? -INFINITY : src[c];
-  const int avail = causal ? t : n - 1;
-  __syncwarp();
-  float s1 = 1.f;
-  for (int r = 0; r < k; ++r) {
-    float best = -INFINITY;
-    int bi = 0x7fffffff;
-    for (int c = lane; c < n; c += 32) {
-      const float v = srow[c];
-      if (v > best) {  // increasing c per lane: ties keep the lower index
-        best = v;
-        bi = c;
+  const int lim = causal ? t : n;  // candidates c < lim, c != t
+  float lv = -INFINITY;  // this lane's list entry (q = lane)
+  int lc = 0x7fffffff;
+  float tv = -INFINITY;  // the k-th entry: the bar a new candidate must clear
+  int tc = 0x7fffffff;
+  auto consider = [&](float v, int c) {
+    const bool ok = c < lim && c != t && key_gt(v, c, tv, tc);
+    unsigned mask = __ballot_sync(0xffffffffu, ok);
+    while (mask) {
+      const int srcl = __ffs(mask) - 1;
+      mask &= mask - 1;
+      const float nv = __shfl_sync(0xffffffffu, v, srcl);
+      const int nc = __shfl_sync(0xffffffffu, c, srcl);
+      if (!key_gt(nv, nc, tv, tc)) continue;  // the bar rose since the ballot
+      const int pos = __popc(__ballot_sync(0xffffffffu, lane < k && key_gt(lv, lc, nv, nc)));
+      const float pv = __shfl_up_sync(0xffffffffu, lv, 1);
+      const int pc = __shfl_up_sync(0xffffffffu, lc, 1);
+      if (lane == pos) {
+        lv = nv;
+        lc = nc;
+      } else if (lane > pos) {
+        lv = pv;
+        lc = pc;
       }
+      tv = __shfl_sync(0xffffffffu, lv, k - 1);
+      tc = __shfl_sync(0xffffffffu, lc, k - 1);
     }
+  };
+  if (vec4) {
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+    const int n4 = (lim + 3) >> 2;  // float4 groups that hold a candidate
+    for (int g0 = 0; g0 < n4; g0 += 128) {
+      // four loads in flight per lane, then the warp-uniform screening
+      float4 v[4];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (ob > best || (ob == best && oi < bi)) {
-        best = ob;
-        bi = oi;
+      for (int u = 0; u < 4; ++u) {
+        const int g = g0 + 32 * u + lane;
+        v[u] = g < n4 ? __ldg(s4 + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        // one warp vote per group of four: the per-element path runs only when
+        // some lane's group maximum can clear the bar (its lowest index is the
+        // most favourable tie-break)
+        const int c = 4 * (g0 + 32 * u + lane);
+        const float m = fmaxf(fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w));
+        if (!__any_sync(0xffffffffu, key_gt(m, c, tv, tc))) continue;
+        consider(v[u].x, c);
+        consider(v[u].y, c + 1);
+        consider(v[u].z, c + 2);
+        consider(v[u].w, c + 3);
       }
     }
-    const long long o = rowid * k + r;
-    if (r < avail && bi != 0x7fffffff && best != -INFINITY) {
-      if (r == 0) s1 = best > 1e-30f ? best : 1e-30f;
-      if (lane == 0) {
-        idx[o] = bi;
-        w[o] = best / s1;
-        srow[bi] = -INFINITY;
+  } else {
+    for (int c0 = 0; c0 < lim; c0 += 128) {
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u + lane;
+        v[u] = c < lim ? __ldg(src + c) : -INFINITY;
       }
-    } else if (lane == 0) {
-      idx[o] = -1;
-      w[o] = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) consider(v[u], c0 + 32 * u + lane);
     }
-    __syncwarp();
+  }
+  // lane r < k holds the r-th choice; w_r = s_r / max(s_1, 1e-30)
+  const int avail = causal ? t : n - 1;
+  const float b0 = __shfl_sync(0xffffffffu, lv, 0);
+  const float s1 = b0 > 1e-30f ? b0 : 1e-30f;
+  if (lane < k) {
+    const long long o = rowid * k + lane;
+    const bool valid = lane < avail && lc != 0x7fffffff && lv != -INFINITY;
+    idx[o] = valid ? lc : -1;
+    w[o] = valid ? lv / s1 : 0.f;
   }
 }
 
@@ -252,17 +298,9 @@ avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, floa
 avey_status launch_topk(const float *scores, int B, int n, int k, int causal, int32_t *idx,
                         float *w, cudaStream_t s) {
   const long long rows = static_cast<long long>(B) * n;
-  const size_t smem = static_cast<size_t>(kTopkWarps) * n * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(topk_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) {
-      set_detail("topk: %s", cudaGetErrorString(e));
-      return AVEY_ERR_CUDA;
-    }
-  }
   const unsigned grid = static_cast<unsigned>((rows + kTopkWarps - 1) / kTopkWarps);
-  topk_warp<<<grid, kTopkWarps * 32, smem, s>>>(scores, B, n, k, causal, idx, w);
+  const int vec4 = (n % 4 == 0 && aligned16(scores)) ? 1 : 0;
+  topk_warp<<<grid, kTopkWarps * 32, 0, s>>>(scores, B, n, k, causal, vec4, idx, w);
   AVEY_CHECK_LAUNCH("topk_warp");
   return AVEY_OK;
 }
@@ -308,6 +346,20 @@ extern "C" avey_status avey_rank(const void *x, avey_dtype dt, int B, int N, int
   return avey_rank_ex(x, dt, B, N, d, S, k, 0u, idx, w, scores, ws, ws_bytes, stream);
 }
 
+extern "C" avey_status avey_topk(const float *scores, int B, int n, int k, uint32_t flags,
+                                 int32_t *idx, float *w, avey_stream_t stream) {
+  AVEY_REQUIRE(scores && idx && w, AVEY_ERR_INVALID_ARG, "avey_topk: null pointer");
+  AVEY_REQUIRE(B >= 1 && n >= 1 && k >= 1, AVEY_ERR_INVALID_ARG,
+               "avey_topk: sizes must be >= 1 (B=%d n=%d k=%d)", B, n, k);
+  AVEY_REQUIRE(k <= 32, AVEY_ERR_UNSUPPORTED, "avey_topk: k=%d > 32", k);
+  AVEY_REQUIRE((flags & ~static_cast<uint32_t>(AVEY_RANK_UNIDIRECTIONAL)) == 0,
+               AVEY_ERR_INVALID_ARG, "avey_topk: unknown flags 0x%x", flags);
+  AVEY_REQUIRE(static_cast<long long>(B) * n <= (1ll << 31) - 1, AVEY_ERR_UNSUPPORTED,
+               "avey_topk: problem too large");
+  return launch_topk(scores, B, n, k, (flags & AVEY_RANK_UNIDIRECTIONAL) ? 1 : 0, idx, w,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" avey_status avey_rank_ex(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
                                     uint32_t flags, int32_t *idx, float *w, float *scores, void *ws,
                                     size_t ws_bytes, avey_stream_t stream) {
@@ -336,8 +388,6 @@ extern "C" avey_status avey_rank_ex(const void *x, avey_dtype dt, int B, int N, 
   const size_t need = avey_rank_workspace_bytes(dt, B, N, d, S);
   AVEY_REQUIRE(ws_bytes >= need, AVEY_ERR_INVALID_ARG,
                "avey_rank: workspace %zu bytes < %zu required", ws_bytes, need);
-  AVEY_REQUIRE(static_cast<size_t>(n) * 4 * 4 <= 200 * 1024, AVEY_ERR_UNSUPPORTED,
-               "avey_rank: n=%lld too large for the top-k kernel", n);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char *wsb = static_cast<char *>(ws);

@@ -279,7 +279,59 @@ def run_ours(args):
     e1.record()
     torch.cuda.synchronize()
     mix_ms = e0.elapsed_time(e1) / reps
+
+    def time_alone(call, reps_):
+        for _ in range(3):
+            assert call() == 0
+        e0.record()
+        for _ in range(reps_):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps_
+
+    # ---- static mix alone at the layer's shape (V of the first static layer) ----
+    smix_ms = None
+    vstat = next((l_.V for l_ in layers if l_.kind == av.AVEY_STATIC), None)
+    if vstat is not None:
+        smix_ms = time_alone(lambda: L.avey_static_mix(
+            ctypes.c_void_p(vstat.data_ptr()), ctypes.c_void_p(zt.data_ptr()), wl.m, av.AVEY_BF16X2,
+            T // wl.S, wl.S, mt, ctypes.c_void_p(zt.data_ptr()), wl.m, av._stream()), reps)
     del zpair, zt
+
+    # ---- top-k alone: at the workload's shape, and on a larger sweep where
+    # the score matrix (5.4 GB) is far past L2 and launch latency ----
+    def topk_time(B_, n_, reps_):
+        # timed as a captured CUDA graph of reps_ launches, so that host-side
+        # call overhead does not hide the kernel at small sizes
+        sc = torch.rand((B_, n_, n_), device=dev)
+        ti = torch.empty((B_, n_, wl.k), dtype=torch.int32, device=dev)
+        tw = torch.empty((B_, n_, wl.k), dtype=torch.float32, device=dev)
+        call = lambda: L.avey_topk(ctypes.c_void_p(sc.data_ptr()), B_, n_, wl.k, 0,
+                                   ctypes.c_void_p(ti.data_ptr()), ctypes.c_void_p(tw.data_ptr()),
+                                   av._stream())
+        for _ in range(3):
+            assert call() == 0
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps_):
+                call()
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms_ = e0.elapsed_time(e1) / reps_
+        del g, sc, ti, tw
+        by = B_ * n_ * n_ * 4.0 + B_ * n_ * wl.k * 8.0
+        return ms_, by
+
+    topk_ms, topk_bytes = topk_time(wl.B, wl.n, reps)
+    sweep_B, sweep_n = 9, 12288
+    sweep_ms, sweep_bytes = topk_time(sweep_B, sweep_n, 5)
+    torch.cuda.empty_cache()
 
     # ---- end to end through the public API with host buffers ----
     # Every step copies its input embeddings host -> device (pinned) and its
@@ -417,7 +469,17 @@ def run_ours(args):
                                 "peak": hbm, "bytes": mix_bytes},
                 "compress": {"ms": compress_ms, "gbs": comp_bytes / (compress_ms * 1e-3) / 1e9,
                              "frac": comp_bytes / (compress_ms * 1e-3) / 1e9 / hbm,
-                             "bytes": comp_bytes}},
+                             "bytes": comp_bytes},
+                "static_mix": None if smix_ms is None else {
+                    "ms": smix_ms, "gbs": mix_bytes / (smix_ms * 1e-3) / 1e9,
+                    "frac": mix_bytes / (smix_ms * 1e-3) / 1e9 / hbm, "bytes": mix_bytes},
+                "topk": {"ms": topk_ms, "gbs": topk_bytes / (topk_ms * 1e-3) / 1e9,
+                         "frac": topk_bytes / (topk_ms * 1e-3) / 1e9 / hbm, "bytes": topk_bytes,
+                         "note": "9.4 MB of scores: latency-bound at this size"},
+                "topk_sweep": {"B": sweep_B, "n": sweep_n, "k": wl.k, "ms": sweep_ms,
+                               "gbs": sweep_bytes / (sweep_ms * 1e-3) / 1e9,
+                               "frac": sweep_bytes / (sweep_ms * 1e-3) / 1e9 / hbm,
+                               "bytes": sweep_bytes}},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes,

@@ -139,6 +139,16 @@ AVEY_API avey_status avey_rank_static(const void *x, avey_dtype dt, int B, int N
 
 AVEY_API size_t avey_rank_static_max_scratch_bytes(void);
 
+/* avey_topk: the selection and weights of avey_rank from precomputed split
+ * scores ([AB-sum] §3: top-k candidates, weights divided by the largest):
+ * per target t, the k candidates c != t (c < t with AVEY_RANK_UNIDIRECTIONAL)
+ * of highest score, ties to the lower index, w_r = s_r / max(s_1, 1e-30).
+ * scores [B, n, n] fp32 (row t = target t); idx, w [B, n, k] out (idx -1 and
+ * w 0 past the available candidates).  Constraints: k <= 32; B*n < 2^31.
+ */
+AVEY_API avey_status avey_topk(const float *scores, int B, int n, int k, uint32_t flags,
+                               int32_t *idx, float *w, avey_stream_t stream);
+
 /* ---------------------------------------------------------- compression --
  * avey_compress: neural compression of each split with its retrieved splits
  * plus the residual to the split's own tokens ([AB-notes] 关键设计 4, eq. 8):
@@ -182,6 +192,19 @@ AVEY_API avey_status avey_compress(const void *x, avey_dtype dt, int B, int N, i
 AVEY_API avey_status avey_context(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
                                   const int32_t *idx, const float *w, float *out, void *out_lowp,
                                   avey_stream_t stream);
+
+/* ------------------------------------------------------------ static mix --
+ * avey_static_mix: the static contextualizer of one layer on `blocks`
+ * independent split blocks of S tokens ([AB-notes] 关键设计 2):
+ *   c = V Z_t     (V: S x S, shared by all blocks; identity activation, no bias)
+ * V    [S, S] row-major, fp32 for AVEY_F32, bf16 for AVEY_BF16X2.
+ * zt, out: layouts as for avey_dynamic_mix (out may alias zt exactly).
+ * Constraints: S in {16, 32, 64, 128} for AVEY_BF16X2 (a power of two <= 64
+ * for F32); mt % 8 == 0 and ld % 8 == 0 for AVEY_BF16X2.
+ */
+AVEY_API avey_status avey_static_mix(const void *V, const void *zt, int64_t ld_zt, avey_dtype dt,
+                                     int blocks, int S, int mt, void *out, int64_t ld_out,
+                                     avey_stream_t stream);
 
 /* ----------------------------------------------------------- dynamic mix --
  * avey_dynamic_mix: the dynamic contextualizer of one layer on `blocks`
