@@ -34,9 +34,12 @@ avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, con
 
 // Fuser: x_out = x_in + A O, A given as a split pair (ahi, alo) [T, m];
 // Ot [d, m]; writes fp32 x_out and (optionally) its split pair.
+// With chi / clo given, activation columns [k_split, m) are read from the
+// split pair c [T, m - k_split] instead of (ahi, alo); k_split % 64 == 0.
 avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
                            const float *x_in, float *x_out, bf16 *xo_hi, bf16 *xo_lo,
-                           cudaStream_t s);
+                           cudaStream_t s, const bf16 *chi = nullptr, const bf16 *clo = nullptr,
+                           int k_split = 0);
 
 // ---- ranker pieces (avey_rank.cu) ----
 avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, int S, void *xhat,
@@ -68,9 +71,15 @@ avey_status launch_dynamic_mix_f32(const float *zt, int64_t ld_zt, float *out, i
 // In place on the split pair Z_t (hi at zt, lo at zt + plane).  The dynamic
 // mix needs long_dynamic_ws_bytes(blocks, SL) bytes of workspace.
 size_t long_dynamic_ws_bytes(int blocks, int SL);
-avey_status launch_long_static_mix(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int SL, int mt,
-                                   int64_t plane, cudaStream_t s);
-avey_status launch_long_dynamic_mix(bf16 *zt, int64_t ld, int64_t plane, int blocks, int SL, int mt,
-                                    float eps, void *ws, cudaStream_t s);
-
+// Dynamic Gt of every block (bf16 split pair in the workspace, hi at ws, lo
+// at ws + blocks*SL*SL elements) without the apply step.
+avey_status launch_long_dynamic_gt(const bf16 *zt, int64_t ld, int blocks, int SL, int mt, float eps,
+                                   void *ws, cudaStream_t s);
+// c = A Z_t over blocks of SL in {256, 512} tokens on tcgen05 (avey_mix_tc.cu):
+// A = the bf16 [SL, SL] map shared by all blocks (a_lo null, a_batched false)
+// or every block's Gt pair (a_batched true); Z_t a split pair with row stride
+// ldz; c written as a split pair [blocks*SL, mt] (row stride mt) to chi / clo.
+avey_status launch_long_mix_tc(const bf16 *a_hi, const bf16 *a_lo, bool a_batched, const bf16 *zhi,
+                               const bf16 *zlo, int64_t ldz, int blocks, int SL, int mt, bf16 *chi,
+                               bf16 *clo, cudaStream_t s);
 }  // namespace avey

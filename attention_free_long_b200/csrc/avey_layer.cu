@@ -131,8 +131,10 @@ extern "C" size_t avey_layer_workspace_bytes(avey_dtype dt, int T, int d, int m,
 extern "C" size_t avey_layer_workspace_bytes_ex(avey_dtype dt, int T, int d, int m, int prenorm,
                                                 int S, avey_ctx_kind kind) {
   size_t b = avey_layer_workspace_bytes(dt, T, d, m, prenorm);
-  if (b && dt == AVEY_BF16 && kind == AVEY_DYNAMIC && S > 128 && S > 0 && T % S == 0)
-    b += align256(long_dynamic_ws_bytes(T / S, S));
+  if (b && dt == AVEY_BF16 && S > 128 && T % S == 0 && m > 0) {
+    b += align256(static_cast<size_t>(T) * m * 4);  // c split pair (T x m_t, m_t < m)
+    if (kind == AVEY_DYNAMIC) b += align256(long_dynamic_ws_bytes(T / S, S));
+  }
   return b;
 }
 
@@ -166,15 +168,18 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   const size_t need = avey_layer_workspace_bytes_ex(dt, T, d, m, p->prenorm, S, p->kind);
   AVEY_REQUIRE(ws_bytes >= need, AVEY_ERR_INVALID_ARG,
                "avey_layer_forward: workspace %zu bytes < %zu required", ws_bytes, need);
-  if (dt == AVEY_BF16)
+  if (dt == AVEY_BF16) {
     AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128 ||
                      ((S == 256 || S == 512) && p->kind != AVEY_COUPLED_CAUSAL),
                  AVEY_ERR_UNSUPPORTED,
                  "avey_layer_forward(BF16): S=%d unsupported (16, 32, 64 or 128; 256 or 512 for "
                  "static and dynamic layers)", S);
-  else
+    AVEY_REQUIRE(S <= 128 || m_h % 64 == 0, AVEY_ERR_UNSUPPORTED,
+                 "avey_layer_forward(BF16): blocks of %d tokens need m_h %% 64 == 0 (m_h = %d)", S, m_h);
+  } else {
     AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
                  "avey_layer_forward(F32): S=%d unsupported (power of two <= 64)", S);
+  }
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char *w = static_cast<char *>(ws);
@@ -234,12 +239,27 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   if (st != AVEY_OK) return st;
   const int64_t plane = static_cast<int64_t>(T) * m;
   if (S > 128) {
-    // blocks of (k+1)S tokens (the processor without compression)
-    if (p->kind == AVEY_STATIC)
-      st = launch_long_static_mix(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane, s);
-    else
-      st = launch_long_dynamic_mix(Zhi + m_h, m, plane, blocks, S, mt, p->eps,
-                                   w + avey_layer_workspace_bytes(dt, T, d, m, p->prenorm), s);
+    // blocks of (k+1)S tokens (the processor without compression): c goes to
+    // its own split pair, and the fuser reads [Z_h || c] from the two buffers
+    const size_t base = avey_layer_workspace_bytes(dt, T, d, m, p->prenorm);
+    bf16 *Chi = reinterpret_cast<bf16 *>(w + base);
+    bf16 *Clo = Chi + static_cast<long long>(T) * mt;
+    if (p->kind == AVEY_STATIC) {
+      st = launch_long_mix_tc(static_cast<const bf16 *>(p->V), nullptr, false, Zhi + m_h, Zlo + m_h,
+                              m, blocks, S, mt, Chi, Clo, s);
+    } else {
+      void *gws = w + base + align256(static_cast<size_t>(T) * m * 4);
+      st = launch_long_dynamic_gt(Zhi + m_h, m, blocks, S, mt, p->eps, gws, s);
+      if (st != AVEY_OK) return st;
+      const bf16 *gt = static_cast<const bf16 *>(gws);
+      st = launch_long_mix_tc(gt, gt + static_cast<long long>(blocks) * S * S, true, Zhi + m_h,
+                              Zlo + m_h, m, blocks, S, mt, Chi, Clo, s);
+    }
+    if (st != AVEY_OK) return st;
+    bf16 *ohi = static_cast<bf16 *>(x_out_lowp);
+    bf16 *olo = ohi ? ohi + static_cast<long long>(T) * d : nullptr;
+    return launch_fuse_tc(Zhi, Zlo, T, m, static_cast<const bf16 *>(p->Ot), d, x_in, x_out, ohi, olo,
+                          s, Chi, Clo, m_h);
   } else if (p->kind == AVEY_STATIC)
     st = launch_static_mix_x2(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane,
                               Zhi + m_h, m, plane, s);

@@ -7,15 +7,10 @@
 //   dynamic:  Gt_ij = N(z_i).N(z_j) / (sum_j N(z_i).N(z_j) + eps),  c = Gt Z_t
 // Z_t is the activation split pair (hi, lo bf16 planes).
 //
-// At SL = 512 the mix is a real contraction (2 SL FLOP per output element),
-// and its per-block operand (V or Gt, SL x SL) no longer fits next to a Z slab
-// in shared memory.  Kernels:
-//   long_mix_apply   one CTA per (block, 64-feature slab): the A operand (V,
-//                    shared by every block and L2-resident, or the block's Gt
-//                    pair) and the Z slab stream through a cp.async ring in
-//                    chunks of 32 tokens; c = A Z_hi + A Z_lo (+ A_lo Z_hi for
-//                    the Gt pair) with mma.sync; the slab is read only by this
-//                    CTA, so c is written back in place as a split pair.
+// At SL = 512 the mix is a real contraction (2 SL FLOP per output element)
+// whose per-block operand (V or Gt, SL x SL) no longer fits in shared memory
+// next to the activations; c = A Z_t itself runs on tcgen05 (avey_mix_tc.cu).
+// This file builds the dynamic A, Gt, per block:
 //   long_dyn_prep    one CTA per block: 1/|z_j| of the hi rows, the block sum
 //                    s = sum_j u_j of the unit rows, and the row sums of the
 //                    cosine matrix as u_i . s (the same sum, reassociated), so
@@ -30,142 +25,6 @@
 
 namespace avey {
 namespace {
-
-// ----------------------------------------------------------------- apply --
-
-template <int SL, bool PAIR_A>
-struct LongApply {
-  static constexpr int KC = 32;                 // tokens per K chunk
-  static constexpr int FS = 64;                 // features per CTA slab
-  static constexpr int WM = SL / 8;             // rows per warp
-  static constexpr int MI = WM / 16, NI = FS / 8;
-  static constexpr int ALD = KC + 8;            // A chunk row, bf16 (80 B)
-  static constexpr int ZLD = FS + 8;            // Z / output row, bf16 (144 B)
-  static constexpr int APL = PAIR_A ? 2 : 1;
-  static constexpr int ABYTES = SL * ALD * 2;   // one plane of one A chunk
-  static constexpr int ZBYTES = KC * ZLD * 2;   // one plane of one Z chunk
-  static constexpr int STAGE = APL * ABYTES + 2 * ZBYTES;
-  static constexpr int STAGES = (SL == 512 && PAIR_A) ? 2 : 3;
-  static constexpr int OBYTES = 2 * SL * ZLD * 2;
-  static constexpr int SMEM = STAGES * STAGE > OBYTES ? STAGES * STAGE : OBYTES;
-  static_assert(SMEM <= 232448, "shared memory budget");
-};
-
-// c[:, slab] = A Z[:, slab] for one block.  A: [SL, SL] bf16 row-major (hi
-// plane; lo plane at a + a_plane when PAIR_A), a_block = elements between
-// consecutive blocks' A (0: one A for all blocks).  zt: Z_t of block 0 (row
-// stride ld, lo plane at + plane); c overwrites Z_t in place.
-template <int SL, bool PAIR_A>
-__global__ void __launch_bounds__(256, 1)
-    long_mix_apply(const bf16 *__restrict__ a, long long a_block, long long a_plane, bf16 *zt,
-                   long long ld, long long plane, int mt) {
-  using C = LongApply<SL, PAIR_A>;
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int slab = blockIdx.x, blk = blockIdx.y;
-  const int f0 = slab * C::FS;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bf16 *ab = a + static_cast<long long>(blk) * a_block;
-  bf16 *zb = zt + static_cast<long long>(blk) * SL * ld;
-  constexpr int NCH = SL / C::KC;
-
-  auto load = [&](int ch, int stg) {
-    uint8_t *sa = smem + stg * C::STAGE;
-    uint8_t *sz = sa + C::APL * C::ABYTES;
-    const int k0 = ch * C::KC;
-    for (int e = tid; e < SL * (C::KC / 8); e += 256) {
-      const int row = e / (C::KC / 8), cc = e % (C::KC / 8);
-      const bf16 *src = ab + static_cast<long long>(row) * SL + k0 + cc * 8;
-      cp_async16(smem_u32(sa + (row * C::ALD + cc * 8) * 2), src, 16);
-      if (PAIR_A) cp_async16(smem_u32(sa + C::ABYTES + (row * C::ALD + cc * 8) * 2), src + a_plane, 16);
-    }
-    for (int e = tid; e < C::KC * (C::FS / 8); e += 256) {
-      const int row = e / (C::FS / 8), cc = e % (C::FS / 8);
-      const int f = f0 + cc * 8;
-      const bool ok = f < mt;
-      const bf16 *src = ok ? zb + static_cast<long long>(k0 + row) * ld + f : zb;
-      cp_async16(smem_u32(sz + (row * C::ZLD + cc * 8) * 2), src, ok ? 16 : 0);
-      cp_async16(smem_u32(sz + C::ZBYTES + (row * C::ZLD + cc * 8) * 2), ok ? src + plane : zb,
-                 ok ? 16 : 0);
-    }
-    cp_async_commit();
-  };
-
-  float acc[C::MI][C::NI][4] = {};
-#pragma unroll
-  for (int s = 0; s < C::STAGES - 1; ++s) load(s, s);
-#pragma unroll 1
-  for (int ch = 0; ch < NCH; ++ch) {
-    cp_async_wait<C::STAGES - 2>();
-    __syncthreads();  // chunk ch landed; every warp is done with chunk ch-1's stage
-    if (ch + C::STAGES - 1 < NCH)
-      load(ch + C::STAGES - 1, (ch + C::STAGES - 1) % C::STAGES);
-    else
-      cp_async_commit();  // keep the group count uniform
-    const uint8_t *sa = smem + (ch % C::STAGES) * C::STAGE;
-    const uint8_t *szh = sa + C::APL * C::ABYTES;
-    const uint8_t *szl = szh + C::ZBYTES;
-#pragma unroll
-    for (int kk = 0; kk < C::KC; kk += 16) {
-      uint32_t af[C::MI][4], al[C::MI][4];
-#pragma unroll
-      for (int i = 0; i < C::MI; ++i) {
-        const int row = warp * C::WM + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const uint32_t ad = smem_u32(sa + (row * C::ALD + kk + (lane >> 4) * 8) * 2);
-        ldsm_x4(ad, af[i][0], af[i][1], af[i][2], af[i][3]);
-        if (PAIR_A) ldsm_x4(ad + C::ABYTES, al[i][0], al[i][1], al[i][2], al[i][3]);
-      }
-#pragma unroll
-      for (int j = 0; j < C::NI; j += 2) {
-        const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int ncol = j * 8 + (lane >> 4) * 8;
-        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-        ldsm_x4_t(smem_u32(szh + (krow * C::ZLD + ncol) * 2), h0, h1, h2, h3);
-        ldsm_x4_t(smem_u32(szl + (krow * C::ZLD + ncol) * 2), l0, l1, l2, l3);
-        const uint32_t hA[2] = {h0, h1}, hB[2] = {h2, h3}, lA[2] = {l0, l1}, lB[2] = {l2, l3};
-#pragma unroll
-        for (int i = 0; i < C::MI; ++i) {
-          mma16816(acc[i][j], af[i], hA);
-          mma16816(acc[i][j + 1], af[i], hB);
-          mma16816(acc[i][j], af[i], lA);
-          mma16816(acc[i][j + 1], af[i], lB);
-          if (PAIR_A) {
-            mma16816(acc[i][j], al[i], hA);
-            mma16816(acc[i][j + 1], al[i], hB);
-          }
-        }
-      }
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();  // all MMAs done: the stages become the output staging area
-
-  // c as a split pair through shared memory, then 16-byte coalesced stores
-  uint8_t *oh = smem;
-  uint8_t *ol = smem + SL * C::ZLD * 2;
-#pragma unroll
-  for (int i = 0; i < C::MI; ++i)
-#pragma unroll
-    for (int j = 0; j < C::NI; ++j)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = warp * C::WM + i * 16 + (lane >> 2) + h * 8;
-        const int fl = j * 8 + (lane & 3) * 2;
-        uint32_t hi, lo;
-        split_pack(acc[i][j][2 * h], acc[i][j][2 * h + 1], hi, lo);
-        *reinterpret_cast<uint32_t *>(oh + (row * C::ZLD + fl) * 2) = hi;
-        *reinterpret_cast<uint32_t *>(ol + (row * C::ZLD + fl) * 2) = lo;
-      }
-  __syncthreads();
-  for (int e = tid; e < SL * (C::FS / 8); e += 256) {
-    const int row = e / (C::FS / 8), cc = e % (C::FS / 8);
-    const int f = f0 + cc * 8;
-    if (f >= mt) continue;
-    bf16 *dst = zb + static_cast<long long>(row) * ld + f;
-    *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(oh + (row * C::ZLD + cc * 8) * 2);
-    *reinterpret_cast<uint4 *>(dst + plane) =
-        *reinterpret_cast<const uint4 *>(ol + (row * C::ZLD + cc * 8) * 2);
-  }
-}
 
 // --------------------------------------------------------------- dynamic --
 
@@ -358,22 +217,9 @@ avey_status set_smem_long(K kern, int bytes, const char *name) {
   return AVEY_OK;
 }
 
-template <int SL, bool PAIR_A>
-avey_status run_apply(const bf16 *a, long long a_block, long long a_plane, bf16 *zt, int64_t ld,
-                      int64_t plane, int blocks, int mt, cudaStream_t s) {
-  using C = LongApply<SL, PAIR_A>;
-  auto kern = long_mix_apply<SL, PAIR_A>;
-  avey_status st = set_smem_long(kern, C::SMEM, "long_mix_apply");
-  if (st != AVEY_OK) return st;
-  kern<<<dim3((mt + C::FS - 1) / C::FS, blocks), 256, C::SMEM, s>>>(a, a_block, a_plane, zt, ld,
-                                                                     plane, mt);
-  AVEY_CHECK_LAUNCH("long_mix_apply");
-  return AVEY_OK;
-}
-
 template <int SL>
-avey_status run_dynamic(bf16 *zt, int64_t ld, int64_t plane, int blocks, int mt, float eps,
-                        void *ws, cudaStream_t s) {
+avey_status run_dynamic_gt(const bf16 *zt, int64_t ld, int blocks, int mt, float eps, void *ws,
+                           cudaStream_t s) {
   const long long gt_plane = static_cast<long long>(blocks) * SL * SL;
   bf16 *gt = static_cast<bf16 *>(ws);
   float *inv_n = reinterpret_cast<float *>(gt + 2 * gt_plane);
@@ -386,8 +232,7 @@ avey_status run_dynamic(bf16 *zt, int64_t ld, int64_t plane, int blocks, int mt,
   gk<<<dim3(SL / GramTile::TI, SL / GramTile::TI, blocks), 256, GramTile::SMEM, s>>>(
       zt, ld, mt, inv_n, inv_d, gt, gt_plane);
   AVEY_CHECK_LAUNCH("long_gram");
-  return run_apply<SL, true>(gt, static_cast<long long>(SL) * SL, gt_plane, zt, ld, plane, blocks,
-                             mt, s);
+  return AVEY_OK;
 }
 
 }  // namespace
@@ -397,30 +242,17 @@ size_t long_dynamic_ws_bytes(int blocks, int SL) {
   return static_cast<size_t>(blocks) * SL * SL * 4 + static_cast<size_t>(blocks) * SL * 8;
 }
 
-avey_status launch_long_static_mix(const bf16 *V, bf16 *zt, int64_t ld, int blocks, int SL, int mt,
-                                   int64_t plane, cudaStream_t s) {
-  AVEY_REQUIRE(mt % 8 == 0 && ld % 8 == 0 && plane % 8 == 0, AVEY_ERR_INVALID_ARG,
-               "long static mix: mt, ld and plane must be multiples of 8");
-  AVEY_REQUIRE(blocks >= 1 && blocks <= 65535, AVEY_ERR_UNSUPPORTED,
-               "long static mix: %d blocks (1 .. 65535)", blocks);
-  switch (SL) {
-    case 256: return run_apply<256, false>(V, 0, 0, zt, ld, plane, blocks, mt, s);
-    case 512: return run_apply<512, false>(V, 0, 0, zt, ld, plane, blocks, mt, s);
-    default: set_detail("long static mix: block of %d tokens unsupported", SL); return AVEY_ERR_UNSUPPORTED;
-  }
-}
-
-avey_status launch_long_dynamic_mix(bf16 *zt, int64_t ld, int64_t plane, int blocks, int SL, int mt,
-                                    float eps, void *ws, cudaStream_t s) {
-  AVEY_REQUIRE(mt % 8 == 0 && ld % 8 == 0 && plane % 8 == 0 && mt <= kMaxMt, AVEY_ERR_INVALID_ARG,
-               "long dynamic mix: mt (<= %d), ld and plane must be multiples of 8", kMaxMt);
+avey_status launch_long_dynamic_gt(const bf16 *zt, int64_t ld, int blocks, int SL, int mt, float eps,
+                                   void *ws, cudaStream_t s) {
+  AVEY_REQUIRE(mt % 8 == 0 && ld % 8 == 0 && mt <= kMaxMt, AVEY_ERR_INVALID_ARG,
+               "long dynamic mix: mt (<= %d) and ld must be multiples of 8", kMaxMt);
   AVEY_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 15) == 0, AVEY_ERR_INVALID_ARG,
                "long dynamic mix: workspace must be 16-byte aligned");
   AVEY_REQUIRE(blocks >= 1 && blocks <= 65535, AVEY_ERR_UNSUPPORTED,
                "long dynamic mix: %d blocks (1 .. 65535)", blocks);
   switch (SL) {
-    case 256: return run_dynamic<256>(zt, ld, plane, blocks, mt, eps, ws, s);
-    case 512: return run_dynamic<512>(zt, ld, plane, blocks, mt, eps, ws, s);
+    case 256: return run_dynamic_gt<256>(zt, ld, blocks, mt, eps, ws, s);
+    case 512: return run_dynamic_gt<512>(zt, ld, blocks, mt, eps, ws, s);
     default: set_detail("long dynamic mix: block of %d tokens unsupported", SL); return AVEY_ERR_UNSUPPORTED;
   }
 }

@@ -64,6 +64,7 @@ struct TcArgs {
   // fuser
   const float *x_in;
   float *x_out;
+  int k_split;  // > 0: A columns >= k_split come from the second pair of maps
   int *status;
 };
 
@@ -327,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmO0,
               const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2,
+              const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
               const TcArgs a) {
   using L = Layout<A_PLANES>;
   extern __shared__ uint8_t smem_raw[];
@@ -376,6 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmO0);
       prefetch_tmap(&tmO1);
       if (MODE == MODE_FUSE) prefetch_tmap(&tmO2);
+      if (MODE == MODE_FUSE && a.k_split > 0) {
+        prefetch_tmap(&tmC0);
+        prefetch_tmap(&tmC1);
+      }
     }
   }
   tc_fence_before();
@@ -401,8 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t st = sbase + stage * L::STAGE_BYTES;
           mbar_arrive_expect_tx(full_bar(stage), L::STAGE_BYTES);
-          tma_load_3d(st, &tmA0, full_bar(stage), kc * BK, mt * BM, b);
-          if (A_PLANES == 2) tma_load_3d(st + L::A_BYTES, &tmA1, full_bar(stage), kc * BK, mt * BM, b);
+          // fuser with a separate contextualizer output: [Z_h || c] from two
+          // sources, split at a multiple of the K chunk
+          const bool from_c = MODE == MODE_FUSE && a.k_split > 0 && kc * BK >= a.k_split;
+          const CUtensorMap *ma = from_c ? &tmC0 : &tmA0;
+          const CUtensorMap *mal = from_c ? &tmC1 : &tmA1;
+          const int ax = from_c ? kc * BK - a.k_split : kc * BK;
+          tma_load_3d(st, ma, full_bar(stage), ax, mt * BM, b);
+          if (A_PLANES == 2) tma_load_3d(st + L::A_BYTES, mal, full_bar(stage), ax, mt * BM, b);
           tma_load_3d(st + A_PLANES * L::A_BYTES, &tmB, full_bar(stage), kc * BK, nt * BN, b);
           ++issued;
           if (++stage == L::STAGES) {
@@ -534,7 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int MODE, int A_PLANES, int SPLIT_S>
 avey_status run_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                    const CUtensorMap &o0, const CUtensorMap &o1, const CUtensorMap &o2, TcArgs args,
-                   cudaStream_t st, const char *name) {
+                   cudaStream_t st, const char *name, const CUtensorMap *c0 = nullptr,
+                   const CUtensorMap *c1 = nullptr) {
   using L = Layout<A_PLANES>;
   if (args.num_tiles <= 0) return AVEY_OK;
   auto kern = tc_kernel<MODE, A_PLANES, SPLIT_S>;
@@ -545,7 +558,8 @@ avey_status run_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorM
     return AVEY_ERR_CUDA;
   }
   const int grid = std::min(args.num_tiles, sm_count());
-  kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(a0, a1, b, o0, o1, o2, args);
+  kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(a0, a1, b, o0, o1, o2, c0 ? *c0 : a0, c1 ? *c1 : a1,
+                                              args);
   AVEY_CHECK_LAUNCH(name);
   return AVEY_OK;
 }
@@ -611,8 +625,8 @@ avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, con
 
 avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
                            const float *x_in, float *x_out, bf16 *xo_hi, bf16 *xo_lo,
-                           cudaStream_t s) {
-  CUtensorMap a0, a1, mb, o0, o1, o2;
+                           cudaStream_t s, const bf16 *chi, const bf16 *clo, int k_split) {
+  CUtensorMap a0, a1, mb, o0, o1, o2, c0, c1;
   const uint64_t rs = static_cast<uint64_t>(m) * 2;
   const uint64_t fs = static_cast<uint64_t>(d) * 4, hs = static_cast<uint64_t>(d) * 2;
   if (!encode_bf16_map(&a0, ahi, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
@@ -631,6 +645,18 @@ avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const
   a.out_hi = xo_hi;
   a.out_lo = xo_lo;
   a.ld_out = d;
+  if (chi != nullptr) {
+    // columns [k_split, m) of the activation come from c [T, m - k_split]
+    if (k_split <= 0 || k_split % BK != 0 || k_split >= m) {
+      set_detail("fuse_tc: split at %d must be a positive multiple of %d below m = %d", k_split, BK, m);
+      return AVEY_ERR_INVALID_ARG;
+    }
+    const uint64_t cs = static_cast<uint64_t>(m - k_split) * 2;
+    if (!encode_bf16_map(&c0, chi, m - k_split, T, 1, cs, cs * T, BM)) return AVEY_ERR_CUDA;
+    if (!encode_bf16_map(&c1, clo, m - k_split, T, 1, cs, cs * T, BM)) return AVEY_ERR_CUDA;
+    a.k_split = k_split;
+    return run_tc<MODE_FUSE, 2, 0>(a0, a1, mb, o0, o1, o2, a, s, "fuse_tc", &c0, &c1);
+  }
   return run_tc<MODE_FUSE, 2, 0>(a0, a1, mb, o0, o1, o2, a, s, "fuse_tc");
 }
 

@@ -3,8 +3,9 @@
 Each split's (k+1)S-token context goes through every layer as one block
 (Avey-B paperlayer summary §4.3), so the contextualizer mixes blocks of
 (k+1)S tokens: 64 and 128 run on the split-size kernels, 256 and 512 on the
-long-block kernels.  Shapes cover ragged token tails, feature tails (m_t not a
-multiple of 64) and both layer kinds.  As in the compressed parity tests, the
+long-block kernels (tcgen05, Z_t read as an MN-major operand, c into its own
+buffer that the fuser reads beside Z_h).  Shapes cover ragged token tails,
+feature tails (m_t not a multiple of 64) and both layer kinds.  As in the compressed parity tests, the
 oracle never takes the GPU's selection as input: rows whose top-k lists differ
 by a near tie are left out of the layer comparison.
 """
@@ -24,7 +25,7 @@ UNCOMP = [
               dtype="f32", centers=8, sigma=0.3),
     sy.custom("u_bf16_s32_k3", B=2, N=700, S=32, d=96, m=192, m_h=64, k=3,
               pattern=(sy.STATIC, sy.DYNAMIC), centers=12, sigma=0.5),
-    sy.custom("u_bf16_s64_k3_ragged", B=2, N=1000, S=64, d=136, m=272, m_h=136, k=3,
+    sy.custom("u_bf16_s64_k3_ragged", B=2, N=1000, S=64, d=136, m=264, m_h=128, k=3,
               pattern=(sy.STATIC, sy.DYNAMIC), centers=8, sigma=0.5),
     sy.custom("u_bf16_s64_k7_pre", B=1, N=2048, S=64, d=128, m=256, k=7,
               pattern=(sy.DYNAMIC, sy.STATIC, sy.DYNAMIC), centers=12, sigma=0.5, prenorm=True),
@@ -141,3 +142,15 @@ def test_long_block_mix_closed_forms(kind, S, cuda_dev):
     c = z_t * (S / (S + eps)) if kind == sy.DYNAMIC else z_t
     expect = x.double() + c[:d].unsqueeze(0)
     torch.testing.assert_close(y.double(), expect, rtol=2e-4, atol=2e-4)
+
+
+def test_long_blocks_need_head_width_multiple_of_64(cuda_dev):
+    # the fuser reads [Z_h || c] from two buffers split at a K chunk of 64
+    S, blocks, d, m, m_h = 256, 1, 64, 136, 72
+    wl = sy.custom("lm_bad", B=1, N=blocks * S, S=S, d=d, m=m, m_h=m_h, k=1, pattern=(sy.STATIC,))
+    lay = av.device_layers(sy.gen_weights(wl), torch.bfloat16, cuda_dev)[0]
+    x = torch.randn(blocks * S, d, device=cuda_dev)
+    before = av.kernel_launches()
+    with pytest.raises(av.AveyError):
+        av.avey_layer_forward(lay, S, m_h, 1e-8, False, x)
+    assert av.kernel_launches() == before
