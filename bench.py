@@ -475,7 +475,7 @@ def run_ours(args):
                     "frac": mix_bytes / (smix_ms * 1e-3) / 1e9 / hbm, "bytes": mix_bytes},
                 "topk": {"ms": topk_ms, "gbs": topk_bytes / (topk_ms * 1e-3) / 1e9,
                          "frac": topk_bytes / (topk_ms * 1e-3) / 1e9 / hbm, "bytes": topk_bytes,
-                         "note": "9.4 MB of scores: latency-bound at this size"},
+                         "note": f"{topk_bytes / 1e6:.1f} MB of scores: latency-bound at this size"},
                 "topk_sweep": {"B": sweep_B, "n": sweep_n, "k": wl.k, "ms": sweep_ms,
                                "gbs": sweep_bytes / (sweep_ms * 1e-3) / 1e9,
                                "frac": sweep_bytes / (sweep_ms * 1e-3) / 1e9 / hbm,
