@@ -79,6 +79,11 @@ avey_status launch_long_dynamic_gt(const bf16 *zt, int64_t ld, int blocks, int S
 // A = the bf16 [SL, SL] map shared by all blocks (a_lo null, a_batched false)
 // or every block's Gt pair (a_batched true); Z_t a split pair with row stride
 // ldz; c written as a split pair [blocks*SL, mt] (row stride mt) to chi / clo.
+// The hi-plane Gram of every block, scaled to Gt (inv_n, inv_d per token from
+// the dynamic prep) and written as a split pair: gt [blocks][SL][SL], lo plane
+// at gt + blocks*SL*SL (avey_mix_tc.cu).
+avey_status launch_long_gram_tc(const bf16 *zhi, int64_t ldz, int blocks, int SL, int mt,
+                                const float *inv_n, const float *inv_d, bf16 *gt, cudaStream_t s);
 avey_status launch_long_mix_tc(const bf16 *a_hi, const bf16 *a_lo, bool a_batched, const bf16 *zhi,
                                const bf16 *zlo, int64_t ldz, int blocks, int SL, int mt, bf16 *chi,
                                bf16 *clo, cudaStream_t s);

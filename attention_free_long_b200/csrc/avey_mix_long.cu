@@ -14,10 +14,9 @@
 //   long_dyn_prep    one CTA per block: 1/|z_j| of the hi rows, the block sum
 //                    s = sum_j u_j of the unit rows, and the row sums of the
 //                    cosine matrix as u_i . s (the same sum, reassociated), so
-//                    1/(row sum + eps) is known before any Gram tile exists.
-//   long_gram        one CTA per (block, 128 x 128 tile): the hi-plane Gram
-//                    tile with mma.sync, scaled to Gt and written as a split
-//                    pair to the workspace.
+//                    1/(row sum + eps) is known before any Gram tile exists;
+// and the hi-plane Gram itself, scaled to Gt and written as a split pair to
+// the workspace, runs on tcgen05 (gram_tc_kernel in avey_mix_tc.cu).
 #include <algorithm>
 
 #include "avey_common.cuh"
@@ -92,131 +91,6 @@ __global__ void __launch_bounds__(256) long_dyn_prep(const bf16 *__restrict__ zt
   }
 }
 
-struct GramTile {
-  static constexpr int TI = 128, FC = 64;
-  static constexpr int CLD = FC + 8;               // bf16 (144 B)
-  static constexpr int TBYTES = TI * CLD * 2;      // one 128-row chunk
-  static constexpr int STAGES = 3;
-  static constexpr int STAGE = 2 * TBYTES;         // i rows + j rows
-  static constexpr int OLD = TI + 8;               // output staging row, bf16
-  static constexpr int OBYTES = 2 * TI * OLD * 2;  // hi + lo
-  static constexpr int SMEM = STAGES * STAGE > OBYTES ? STAGES * STAGE : OBYTES;
-};
-
-// Gt tile (rows i0.., columns j0..) of one block: the hi-plane Gram R_ij = z_i . z_j
-// (mma.sync, fp32 accumulation) times inv_n[i] inv_n[j] inv_d[i], written as a
-// split pair: gt[blk][i][j] (row-major SL x SL), lo plane at + gt_plane.
-template <int SL>
-__global__ void __launch_bounds__(256) long_gram(const bf16 *__restrict__ zt, long long ld, int mt,
-                                                 const float *__restrict__ inv_n,
-                                                 const float *__restrict__ inv_d, bf16 *gt,
-                                                 long long gt_plane) {
-  using C = GramTile;
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int j0 = blockIdx.x * C::TI, i0 = blockIdx.y * C::TI, blk = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wm = warp / 4, wn = warp % 4;  // warp tile: 64 rows x 32 columns
-  const bf16 *zb = zt + static_cast<long long>(blk) * SL * ld;
-  const int nch = (mt + C::FC - 1) / C::FC;
-
-  auto load = [&](int ch, int stg) {
-    uint8_t *si = smem + stg * C::STAGE;
-    uint8_t *sj = si + C::TBYTES;
-    for (int e = tid; e < 2 * C::TI * (C::FC / 8); e += 256) {
-      const int side = e / (C::TI * (C::FC / 8));
-      const int r = e % (C::TI * (C::FC / 8));
-      const int row = r / (C::FC / 8), cc = r % (C::FC / 8);
-      const int f = ch * C::FC + cc * 8;
-      const bool ok = f < mt;
-      const bf16 *src = ok ? zb + static_cast<long long>((side ? j0 : i0) + row) * ld + f : zb;
-      cp_async16(smem_u32((side ? sj : si) + (row * C::CLD + cc * 8) * 2), src, ok ? 16 : 0);
-    }
-    cp_async_commit();
-  };
-
-  float g[4][4][4] = {};
-#pragma unroll
-  for (int s = 0; s < C::STAGES - 1; ++s) {
-    if (s < nch)
-      load(s, s);
-    else
-      cp_async_commit();
-  }
-#pragma unroll 1
-  for (int ch = 0; ch < nch; ++ch) {
-    cp_async_wait<C::STAGES - 2>();
-    __syncthreads();
-    if (ch + C::STAGES - 1 < nch)
-      load(ch + C::STAGES - 1, (ch + C::STAGES - 1) % C::STAGES);
-    else
-      cp_async_commit();
-    const uint8_t *si = smem + (ch % C::STAGES) * C::STAGE;
-    const uint8_t *sj = si + C::TBYTES;
-#pragma unroll
-    for (int kk = 0; kk < C::FC; kk += 16) {
-      uint32_t af[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int row = wm * 64 + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        ldsm_x4(smem_u32(si + (row * C::CLD + kk + (lane >> 4) * 8) * 2), af[i][0], af[i][1],
-                af[i][2], af[i][3]);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t b0, b1;
-        const int jrow = wn * 32 + j * 8 + (lane & 7);
-        ldsm_x2(smem_u32(sj + (jrow * C::CLD + kk + ((lane >> 3) & 1) * 8) * 2), b0, b1);
-        const uint32_t bb[2] = {b0, b1};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) mma16816(g[i][j], af[i], bb);
-      }
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-
-  const float *nb = inv_n + static_cast<long long>(blk) * SL;
-  const float *db = inv_d + static_cast<long long>(blk) * SL;
-  uint8_t *oh = smem;
-  uint8_t *ol = smem + C::TI * C::OLD * 2;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int row = wm * 64 + i * 16 + (lane >> 2) + hh * 8;
-      const float ri = nb[i0 + row] * db[i0 + row];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int col = wn * 32 + j * 8 + (lane & 3) * 2;
-        const float v0 = g[i][j][2 * hh] * ri * nb[j0 + col];
-        const float v1 = g[i][j][2 * hh + 1] * ri * nb[j0 + col + 1];
-        uint32_t hi, lo;
-        split_pack(v0, v1, hi, lo);
-        *reinterpret_cast<uint32_t *>(oh + (row * C::OLD + col) * 2) = hi;
-        *reinterpret_cast<uint32_t *>(ol + (row * C::OLD + col) * 2) = lo;
-      }
-    }
-  __syncthreads();
-  bf16 *gb = gt + static_cast<long long>(blk) * SL * SL;
-  for (int e = tid; e < C::TI * (C::TI / 8); e += 256) {
-    const int row = e / (C::TI / 8), cc = e % (C::TI / 8);
-    bf16 *dst = gb + static_cast<long long>(i0 + row) * SL + j0 + cc * 8;
-    *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(oh + (row * C::OLD + cc * 8) * 2);
-    *reinterpret_cast<uint4 *>(dst + gt_plane) =
-        *reinterpret_cast<const uint4 *>(ol + (row * C::OLD + cc * 8) * 2);
-  }
-}
-
-template <typename K>
-avey_status set_smem_long(K kern, int bytes, const char *name) {
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e != cudaSuccess) {
-    set_detail("%s: cudaFuncSetAttribute: %s", name, cudaGetErrorString(e));
-    return AVEY_ERR_CUDA;
-  }
-  return AVEY_OK;
-}
-
 template <int SL>
 avey_status run_dynamic_gt(const bf16 *zt, int64_t ld, int blocks, int mt, float eps, void *ws,
                            cudaStream_t s) {
@@ -226,13 +100,7 @@ avey_status run_dynamic_gt(const bf16 *zt, int64_t ld, int blocks, int mt, float
   float *inv_d = inv_n + static_cast<long long>(blocks) * SL;
   long_dyn_prep<SL><<<blocks, 256, 0, s>>>(zt, ld, mt, eps, inv_n, inv_d);
   AVEY_CHECK_LAUNCH("long_dyn_prep");
-  auto gk = long_gram<SL>;
-  avey_status st = set_smem_long(gk, GramTile::SMEM, "long_gram");
-  if (st != AVEY_OK) return st;
-  gk<<<dim3(SL / GramTile::TI, SL / GramTile::TI, blocks), 256, GramTile::SMEM, s>>>(
-      zt, ld, mt, inv_n, inv_d, gt, gt_plane);
-  AVEY_CHECK_LAUNCH("long_gram");
-  return AVEY_OK;
+  return launch_long_gram_tc(zt, ld, blocks, SL, mt, inv_n, inv_d, gt, s);
 }
 
 }  // namespace

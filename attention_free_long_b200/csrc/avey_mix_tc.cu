@@ -290,6 +290,215 @@ __global__ void __launch_bounds__(kThr, 1)
   }
 }
 
+// ---- Gt of the dynamic mix over long blocks: the hi-plane Gram on tcgen05 ----
+//   Gt_ij = (z_i . z_j) inv_n[i] inv_n[j] inv_d[i]
+// (inv_n = 1/|z| of the hi rows, inv_d = 1/(row sum + eps), both from
+// long_dyn_prep).  A tile is (block, 128 rows i, 256 columns j); both operands
+// are the block's hi rows, K-major (features contiguous), in 64-feature
+// chunks: A boxes of 128 rows, B boxes of 256 rows.
+constexpr uint32_t G_A = 128 * 64 * 2, G_B = 256 * 64 * 2;  // 16 KB, 32 KB
+constexpr uint32_t G_STAGE = G_A + G_B;
+constexpr int G_STAGES = 4;
+constexpr uint32_t G_SMEM = G_STAGES * G_STAGE + 1024 + 1024;
+static_assert(G_SMEM <= 232448, "shared memory budget");
+
+struct GramArgs {
+  int SL, mt, blocks, iblocks, jblocks, num_tiles;
+  const float *inv_n, *inv_d;
+  bf16 *gt;
+  long long gt_plane;
+  int *status;
+};
+
+__global__ void __launch_bounds__(kThr, 1)
+    gram_tc_kernel(const __grid_constant__ CUtensorMap tmZa, const __grid_constant__ CUtensorMap tmZb,
+                   const GramArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t *ctrl = smem_raw + pad + G_STAGES * G_STAGE;
+  const uint32_t sbase = raw_s + pad;
+  const uint32_t cbase = sbase + G_STAGES * G_STAGE;
+  // control block: full[4] @0, empty[4] @32, tfull[2] @64, tempty[2] @80,
+  // drain @96, tmem base @104, abort flag @108
+  auto full_bar = [&](int s) { return cbase + 8u * s; };
+  auto empty_bar = [&](int s) { return cbase + 32u + 8u * s; };
+  auto tfull_bar = [&](int i) { return cbase + 64u + 8u * i; };
+  auto tempty_bar = [&](int i) { return cbase + 80u + 8u * i; };
+  const uint32_t drain_bar = cbase + 96u;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 104);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 108);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G_STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), kEpiW);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(ctrl + 104), kCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmZa);
+    prefetch_tmap(&tmZb);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int kchunks = (a.mt + 63) / 64;
+  auto decode = [&](int tile, int &b, int &ib, int &jb) {
+    jb = tile % a.jblocks;
+    const int r = tile / a.jblocks;
+    ib = r % a.iblocks;
+    b = r / a.iblocks;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        int b, ib, jb;
+        decode(tile, b, ib, jb);
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = sbase + stage * G_STAGE;
+          mbar_arrive_expect_tx(full_bar(stage), G_STAGE);
+          tma_load_3d(st, &tmZa, full_bar(stage), kc * 64, b * a.SL + ib * 128, 0);
+          tma_load_3d(st + G_A, &tmZb, full_bar(stage), kc * 64, b * a.SL + jb * 256, 0);
+          ++issued;
+          if (++stage == G_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      for (int s = 0; s < G_STAGES; ++s) {
+        if (issued > s) {
+          const long long last = ((issued - 1 - s) / G_STAGES) * G_STAGES + s;
+          wait_drain_mix(full_bar(s), static_cast<uint32_t>((last / G_STAGES) & 1));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 256);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + stage * G_STAGE;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_bf16(d_tmem, desc_k(st + 32u * kk), desc_k(st + G_A + 32u * kk), idesc,
+                        (kc | kk) != 0);
+          tc_commit(empty_bar(stage));
+          if (++stage == G_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      tc_commit(drain_bar);
+      wait_drain_mix(drain_bar, 0);
+    }
+  } else {
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+      int b, ib, jb;
+      decode(tile, b, ib, jb);
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr =
+          tmem_base + static_cast<uint32_t>(acc * 256) + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int i = ib * 128 + quarter * 32 + lane;
+      const long long rb = static_cast<long long>(b) * a.SL;
+      const float ri = __ldg(a.inv_n + rb + i) * __ldg(a.inv_d + rb + i);
+      const float *nj = a.inv_n + rb + jb * 256;
+      bf16 *gh = a.gt + (rb + i) * a.SL + jb * 256;
+      bf16 *gl = gh + a.gt_plane;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 64) {
+        float v[64];
+        tmem_ld64(taddr + c0, v);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const float4 n0 = __ldg(reinterpret_cast<const float4 *>(nj + c0 + 8 * g));
+          const float4 n1 = __ldg(reinterpret_cast<const float4 *>(nj + c0 + 8 * g + 4));
+          uint4 h, l;
+          split_pack(v[8 * g] * ri * n0.x, v[8 * g + 1] * ri * n0.y, h.x, l.x);
+          split_pack(v[8 * g + 2] * ri * n0.z, v[8 * g + 3] * ri * n0.w, h.y, l.y);
+          split_pack(v[8 * g + 4] * ri * n1.x, v[8 * g + 5] * ri * n1.y, h.z, l.z);
+          split_pack(v[8 * g + 6] * ri * n1.z, v[8 * g + 7] * ri * n1.w, h.w, l.w);
+          *reinterpret_cast<uint4 *>(gh + c0 + 8 * g) = h;
+          *reinterpret_cast<uint4 *>(gl + c0 + 8 * g) = l;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kCols);
+  }
+}
+
 template <int A_PLANES>
 avey_status run_mix_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &z0,
                        const CUtensorMap &z1, const MixArgs &args, cudaStream_t s) {
@@ -344,6 +553,43 @@ avey_status launch_long_mix_tc(const bf16 *a_hi, const bf16 *a_lo, bool a_batche
   args.status = device_status_word();
   if (a_lo) return run_mix_tc<2>(ma0, ma1, mz0, mz1, args, s);
   return run_mix_tc<1>(ma0, ma0, mz0, mz1, args, s);
+}
+
+avey_status launch_long_gram_tc(const bf16 *zhi, int64_t ldz, int blocks, int SL, int mt,
+                                const float *inv_n, const float *inv_d, bf16 *gt, cudaStream_t s) {
+  AVEY_REQUIRE(SL == 256 || SL == 512, AVEY_ERR_UNSUPPORTED,
+               "long Gram: block of %d tokens unsupported (256 or 512)", SL);
+  AVEY_REQUIRE(mt >= 8 && mt % 8 == 0 && ldz % 8 == 0 && aligned16(zhi) && aligned16(gt),
+               AVEY_ERR_INVALID_ARG, "long Gram: mt, ld multiples of 8; 16-byte aligned pointers");
+  const long long T = static_cast<long long>(blocks) * SL;
+  const uint64_t zrow = static_cast<uint64_t>(ldz) * 2;
+  CUtensorMap za, zb;
+  if (!encode_bf16_map(&za, zhi, mt, T, 1, zrow, zrow * T, 128)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&zb, zhi, mt, T, 1, zrow, zrow * T, 256)) return AVEY_ERR_CUDA;
+  GramArgs g{};
+  g.SL = SL;
+  g.mt = mt;
+  g.blocks = blocks;
+  g.iblocks = SL / 128;
+  g.jblocks = SL / 256;
+  const long long tiles = static_cast<long long>(blocks) * g.iblocks * g.jblocks;
+  AVEY_REQUIRE(tiles <= 0x7fffffffll, AVEY_ERR_UNSUPPORTED, "long Gram: too many tiles");
+  g.num_tiles = static_cast<int>(tiles);
+  g.inv_n = inv_n;
+  g.inv_d = inv_d;
+  g.gt = gt;
+  g.gt_plane = static_cast<long long>(blocks) * SL * SL;
+  g.status = device_status_word();
+  cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(G_SMEM));
+  if (e != cudaSuccess) {
+    set_detail("gram_tc: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return AVEY_ERR_CUDA;
+  }
+  const int grid = std::min(g.num_tiles, sm_count());
+  gram_tc_kernel<<<grid, kThr, G_SMEM, s>>>(za, zb, g);
+  AVEY_CHECK_LAUNCH("gram_tc");
+  return AVEY_OK;
 }
 
 }  // namespace avey
