@@ -84,6 +84,13 @@ def lib() -> ctypes.CDLL:
         L.avey_topk.restype = _i
         L.avey_static_mix.argtypes = [_vp, _vp, _i64, _i, _i, _i, _i, _vp, _i64, _vp]
         L.avey_static_mix.restype = _i
+        L.avey_topk_rows.argtypes = [_vp, _i, _i, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _vp]
+        L.avey_topk_rows.restype = _i
+        L.avey_maxsim_part.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]
+        L.avey_maxsim_part.restype = _i
+        L.avey_compress_rows.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
+                                         _vp, _vp]
+        L.avey_compress_rows.restype = _i
         L.avey_device_status.argtypes = [_vp]
         L.avey_device_status.restype = _i
         L.avey_status_string.argtypes = [_i]
@@ -459,3 +466,126 @@ def encoder_forward_uncompressed(x: torch.Tensor, layers: Sequence[DeviceLayer],
             marks[3 + li].record()
         cur, nxt = nxt, cur
     return cur[0].view(B, n, L_, d)[:, :, :S, :]
+
+
+# ------------------------------------------- one sequence across several GPUs --
+
+def shard_targets(n: int, world: int, rank: int):
+    """Contiguous, balanced target-split range [t0, t1) of ``rank``."""
+    base, extra = divmod(n, world)
+    t0 = rank * base + min(rank, extra)
+    return t0, t0 + base + (1 if rank < extra else 0)
+
+
+def avey_maxsim_part(x: torch.Tensor, S: int, part: int, nparts: int, scores: torch.Tensor,
+                     ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Adds part ``part`` of ``nparts`` of the split scores into the zeroed
+    ``scores`` [B, n, n] (its entries only; see include/avey.h)."""
+    _need(x, "x")
+    _need(scores, "scores")
+    B, N, d = x.shape
+    dt = _dt(x)
+    need = rank_workspace_bytes(dt, B, N, d, S)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, x.device)
+    _check("avey_maxsim_part", lib().avey_maxsim_part(_ptr(x), dt, B, N, d, S, part, nparts,
+                                                      _ptr(scores), _ptr(ws), ws.numel(), _stream()))
+    return scores
+
+
+@dataclass
+class ShardWorkspace:
+    """Buffers of encoder_forward_sharded for one rank at one shape."""
+    t0: int
+    t1: int
+    rank_ws: torch.Tensor
+    scores: torch.Tensor
+    layer_ws: torch.Tensor
+    idx: torch.Tensor
+    w: torch.Tensor
+    x0: torch.Tensor
+    x1: torch.Tensor
+    pair0: Optional[torch.Tensor]
+    pair1: Optional[torch.Tensor]
+
+
+def make_shard_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: torch.dtype,
+                         prenorm: bool, rank: int, world: int, device) -> ShardWorkspace:
+    n = -(-N // S)
+    t0, t1 = shard_targets(n, world, rank)
+    T = B * (t1 - t0) * S
+    dt = AVEY_BF16 if dtype == torch.bfloat16 else AVEY_F32
+    pair = lambda: (torch.empty((2, T, d), dtype=torch.bfloat16, device=device)
+                    if dt == AVEY_BF16 else None)
+    return ShardWorkspace(
+        t0, t1, _ws(rank_workspace_bytes(dt, B, N, d, S), device),
+        torch.empty((B, n, n), dtype=torch.float32, device=device),
+        _ws(layer_workspace_bytes(dt, max(T, S), d, m, prenorm), device),
+        torch.empty((B, t1 - t0, k), dtype=torch.int32, device=device),
+        torch.empty((B, t1 - t0, k), dtype=torch.float32, device=device),
+        torch.empty((max(T, 1), d), dtype=torch.float32, device=device),
+        torch.empty((max(T, 1), d), dtype=torch.float32, device=device), pair(), pair())
+
+
+def encoder_forward_sharded(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLayer], S: int,
+                            k: int, m_h: int, eps: float, prenorm: bool, rank: int, world: int,
+                            allreduce, ws: Optional[ShardWorkspace] = None, marks=None,
+                            causal: bool = False) -> torch.Tensor:
+    """One long sequence (or batch) split across ``world`` GPUs; this is rank
+    ``rank``'s share.  Every rank holds the whole input x.
+
+    1. MaxSim: the triangular tiles are dealt round-robin; this rank writes its
+       tiles' entries into zeroed scores, and ``allreduce(scores)`` (an
+       in-place sum over the ranks, e.g. torch.distributed.all_reduce) makes
+       every rank's scores the full matrix: the one exchange step.
+    2. Top-k, compression and every layer for this rank's target splits
+       [t0, t1) only (each split's processing is independent).
+    Returns fp32 [B, (t1-t0)*S, d], the rows of targets t0 .. t1-1.
+
+    ``marks``: optional list of 3 + len(layers) torch.cuda.Event, recorded
+    before MaxSim, after the all-reduce, after compression and after every layer.
+    """
+    B, N, d = x.shape
+    dt = _dt(x)
+    if dt != AVEY_BF16:
+        raise TypeError("the sharded forward takes bf16 embeddings")
+    n = -(-N // S)
+    m = layers[0].Ut.shape[0] if layers else d
+    if ws is None:
+        ws = make_shard_workspace(B, N, d, S, k, m, x.dtype, prenorm, rank, world, x.device)
+    L = lib()
+    st = _stream()
+    if marks is not None:
+        marks[0].record()
+    ws.scores.zero_()
+    _check("avey_maxsim_part", L.avey_maxsim_part(_ptr(x), dt, B, N, d, S, rank, world,
+                                                  _ptr(ws.scores), _ptr(ws.rank_ws),
+                                                  ws.rank_ws.numel(), st))
+    allreduce(ws.scores)
+    if marks is not None:
+        marks[1].record()
+    t0, t1 = ws.t0, ws.t1
+    T = B * (t1 - t0) * S
+    if T == 0:
+        return ws.x0[:0].view(B, 0, d)
+    flags = AVEY_RANK_UNIDIRECTIONAL if causal else 0
+    _check("avey_topk_rows", L.avey_topk_rows(_ptr(ws.scores), B, n, t0, t1, k, flags, _ptr(ws.idx),
+                                              _ptr(ws.w), st))
+    _check("avey_compress_rows", L.avey_compress_rows(_ptr(x), dt, B, N, d, S, k, t0, t1,
+                                                      _ptr(ws.idx), _ptr(ws.w), _ptr(P),
+                                                      _ptr(ws.x0), _ptr(ws.pair0), st))
+    if marks is not None:
+        marks[2].record()
+    cur, nxt = (ws.x0, ws.pair0), (ws.x1, ws.pair1)
+    for li, lay in enumerate(layers):
+        p = LayerParams(lay.kind, d, m, m_h, S, eps, int(bool(prenorm)), lay.Ut.data_ptr(),
+                        lay.bU.data_ptr(), None if lay.V is None else lay.V.data_ptr(),
+                        lay.Ot.data_ptr())
+        _check("avey_layer_forward",
+               L.avey_layer_forward(ctypes.byref(p), dt, T, _ptr(cur[0]), _ptr(cur[1]),
+                                    _ptr(nxt[0]), _ptr(nxt[1]), _ptr(ws.layer_ws),
+                                    ws.layer_ws.numel(), st))
+        if marks is not None:
+            marks[3 + li].record()
+        cur, nxt = nxt, cur
+    return cur[0][:T].view(B, (t1 - t0) * S, d)

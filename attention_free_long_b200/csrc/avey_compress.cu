@@ -49,22 +49,22 @@ __global__ void __launch_bounds__(256) compress_bf16(const bf16 *__restrict__ x,
                                                      float *__restrict__ out,
                                                      bf16 *__restrict__ out_hi,
                                                      bf16 *__restrict__ out_lo, long long plane,
-                                                     int *status) {
+                                                     int t0, int nr, int *status) {
   using C = CompressTile<S>;
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int s_c[33];
   __shared__ float s_w[33];
-  const int slab = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
+  // target split t = t0 + blockIdx.y; its idx / w row and its output rows
+  // are the blockIdx.y-th of the nr targets handled by this launch
+  const int slab = blockIdx.x, tl = blockIdx.y, t = t0 + tl, b = blockIdx.z;
   const int q0 = slab * C::NS;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wm = warp / C::WARPS_N, wn = warp % C::WARPS_N;
-  const long long R = static_cast<long long>(n) * S;
-
   if (tid <= k) {
     int c = t;
     float wr = 1.f;
     if (tid > 0) {
-      const long long o = (static_cast<long long>(b) * n + t) * k + (tid - 1);
+      const long long o = (static_cast<long long>(b) * nr + tl) * k + (tid - 1);
       c = idx[o];
       wr = w[o];
       if (c < -1 || c >= n) {
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(256) compress_bf16(const bf16 *__restrict__ x,
         }
       }
   __syncthreads();
-  const long long row0 = static_cast<long long>(b) * R + static_cast<long long>(t) * S;
+  const long long row0 = (static_cast<long long>(b) * nr + tl) * S;
   for (int e = tid; e < S * (C::NS / 4); e += 256) {
     const int row = e / (C::NS / 4), cc = e % (C::NS / 4);
     const int col = q0 + cc * 4;
@@ -230,20 +230,21 @@ __global__ void __launch_bounds__(256) compress_f32(const float *__restrict__ x,
                                                     int n, int k, const int32_t *__restrict__ idx,
                                                     const float *__restrict__ w,
                                                     const float *__restrict__ P,
-                                                    float *__restrict__ out, int *status) {
+                                                    float *__restrict__ out, int t0, int nr,
+                                                    int *status) {
   constexpr int NSL = 64;
   constexpr int PER = (S * NSL + 255) / 256;  // outputs per thread
   __shared__ float xs[S][NSL];
   __shared__ float ps[S][S];
   __shared__ int s_c[33];
   __shared__ float s_w[33];
-  const int slab = blockIdx.x, t = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int slab = blockIdx.x, tl = blockIdx.y, t = t0 + tl, b = blockIdx.z, tid = threadIdx.x;
   const int q0 = slab * NSL;
   if (tid <= k) {
     int c = t;
     float wr = 1.f;
     if (tid > 0) {
-      const long long o = (static_cast<long long>(b) * n + t) * k + (tid - 1);
+      const long long o = (static_cast<long long>(b) * nr + tl) * k + (tid - 1);
       c = idx[o];
       wr = w[o];
       if (c < -1 || c >= n) {
@@ -286,23 +287,22 @@ __global__ void __launch_bounds__(256) compress_f32(const float *__restrict__ x,
     }
     __syncthreads();
   }
-  const long long R = static_cast<long long>(n) * S;
 #pragma unroll
   for (int p = 0; p < PER; ++p) {
     const int e = tid + p * 256;
     if (e < S * NSL) {
       const int i = e / NSL, col = e % NSL;
       if (q0 + col < d)
-        out[(static_cast<long long>(b) * R + static_cast<long long>(t) * S + i) * d + q0 + col] =
+        out[((static_cast<long long>(b) * nr + tl) * S + i) * d + q0 + col] =
             acc[p] + res[p];
     }
   }
 }
 
 template <int S>
-avey_status run_compress_bf16(const bf16 *x, int B, int N, int d, int n, int k, const int32_t *idx,
-                              const float *w, const bf16 *P, float *out, bf16 *hi, bf16 *lo,
-                              cudaStream_t s) {
+avey_status run_compress_bf16(const bf16 *x, int B, int N, int d, int n, int k, int t0, int nr,
+                              const int32_t *idx, const float *w, const bf16 *P, float *out,
+                              bf16 *hi, bf16 *lo, cudaStream_t s) {
   using C = CompressTile<S>;
   auto kern = compress_bf16<S>;
   if (C::SMEM > 48 * 1024) {
@@ -312,9 +312,9 @@ avey_status run_compress_bf16(const bf16 *x, int B, int N, int d, int n, int k, 
       return AVEY_ERR_CUDA;
     }
   }
-  const dim3 grid((d + C::NS - 1) / C::NS, n, B);
-  const long long plane = static_cast<long long>(B) * n * S * d;
-  kern<<<grid, 256, C::SMEM, s>>>(x, N, d, n, k, idx, w, P, out, hi, lo, plane,
+  const dim3 grid((d + C::NS - 1) / C::NS, nr, B);
+  const long long plane = static_cast<long long>(B) * nr * S * d;
+  kern<<<grid, 256, C::SMEM, s>>>(x, N, d, n, k, idx, w, P, out, hi, lo, plane, t0, nr,
                                   device_status_word());
   AVEY_CHECK_LAUNCH("compress_bf16");
   return AVEY_OK;
@@ -325,47 +325,67 @@ avey_status run_compress_bf16(const bf16 *x, int B, int N, int d, int n, int k, 
 
 using namespace avey;
 
-extern "C" avey_status avey_compress(const void *x, avey_dtype dt, int B, int N, int d, int S,
-                                     int k, const int32_t *idx, const float *w, const void *P,
-                                     float *out, void *out_lowp, avey_stream_t stream) {
+static avey_status compress_range(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
+                                  int t0, int t1, const int32_t *idx, const float *w,
+                                  const void *P, float *out, void *out_lowp, cudaStream_t s,
+                                  const char *fn) {
   AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
-               "avey_compress: dtype %d unsupported (F32 or BF16)", int(dt));
-  AVEY_REQUIRE(x && idx && w && P && out, AVEY_ERR_INVALID_ARG, "avey_compress: null pointer");
+               "%s: dtype %d unsupported (F32 or BF16)", fn, int(dt));
+  AVEY_REQUIRE(x && idx && w && P && out, AVEY_ERR_INVALID_ARG, "%s: null pointer", fn);
   AVEY_REQUIRE(B >= 1 && N >= 1 && d >= 1 && S >= 1 && k >= 1, AVEY_ERR_INVALID_ARG,
-               "avey_compress: sizes must be >= 1");
-  AVEY_REQUIRE(d % 8 == 0, AVEY_ERR_INVALID_ARG, "avey_compress: d=%d must be a multiple of 8", d);
-  AVEY_REQUIRE(k <= 32, AVEY_ERR_UNSUPPORTED, "avey_compress: k=%d > 32", k);
+               "%s: sizes must be >= 1", fn);
+  AVEY_REQUIRE(d % 8 == 0, AVEY_ERR_INVALID_ARG, "%s: d=%d must be a multiple of 8", fn, d);
+  AVEY_REQUIRE(k <= 32, AVEY_ERR_UNSUPPORTED, "%s: k=%d > 32", fn, k);
   AVEY_REQUIRE(aligned16(x) && aligned16(P) && aligned16(out) && (!out_lowp || aligned16(out_lowp)),
-               AVEY_ERR_INVALID_ARG, "avey_compress: pointers must be 16-byte aligned");
+               AVEY_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
   const int n = (N + S - 1) / S;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  AVEY_REQUIRE(0 <= t0 && t0 <= t1 && t1 <= n && t1 - t0 <= 65535, AVEY_ERR_INVALID_ARG,
+               "%s: target range [%d, %d) outside [0, %d) or wider than 65535", fn, t0, t1, n);
+  const int nr = t1 - t0;
+  if (nr == 0) return AVEY_OK;
   if (dt == AVEY_BF16) {
     AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
-                 "avey_compress(BF16): S=%d unsupported (16, 32, 64 or 128)", S);
+                 "%s(BF16): S=%d unsupported (16, 32, 64 or 128)", fn, S);
     const bf16 *xb = static_cast<const bf16 *>(x);
     const bf16 *Pb = static_cast<const bf16 *>(P);
     bf16 *hi = static_cast<bf16 *>(out_lowp);
-    bf16 *lo = hi ? hi + static_cast<long long>(B) * n * S * d : nullptr;
+    bf16 *lo = hi ? hi + static_cast<long long>(B) * nr * S * d : nullptr;
     switch (S) {
-      case 16: return run_compress_bf16<16>(xb, B, N, d, n, k, idx, w, Pb, out, hi, lo, s);
-      case 32: return run_compress_bf16<32>(xb, B, N, d, n, k, idx, w, Pb, out, hi, lo, s);
-      case 64: return run_compress_bf16<64>(xb, B, N, d, n, k, idx, w, Pb, out, hi, lo, s);
-      default: return run_compress_bf16<128>(xb, B, N, d, n, k, idx, w, Pb, out, hi, lo, s);
+      case 16: return run_compress_bf16<16>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
+      case 32: return run_compress_bf16<32>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
+      case 64: return run_compress_bf16<64>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
+      default: return run_compress_bf16<128>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
     }
   }
   AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
-               "avey_compress(F32): S=%d unsupported (power of two <= 64)", S);
-  const dim3 grid((d + 63) / 64, n, B);
+               "%s(F32): S=%d unsupported (power of two <= 64)", fn, S);
+  const dim3 grid((d + 63) / 64, nr, B);
   const float *xf = static_cast<const float *>(x);
   const float *Pf = static_cast<const float *>(P);
   int *st = device_status_word();
   switch (S) {
 #define AVEY_CF_CASE(SS) \
-  case SS: compress_f32<SS><<<grid, 256, 0, s>>>(xf, N, d, n, k, idx, w, Pf, out, st); break;
+  case SS: compress_f32<SS><<<grid, 256, 0, s>>>(xf, N, d, n, k, idx, w, Pf, out, t0, nr, st); break;
     AVEY_CF_CASE(1) AVEY_CF_CASE(2) AVEY_CF_CASE(4) AVEY_CF_CASE(8) AVEY_CF_CASE(16)
     AVEY_CF_CASE(32) AVEY_CF_CASE(64)
 #undef AVEY_CF_CASE
   }
   AVEY_CHECK_LAUNCH("compress_f32");
   return AVEY_OK;
+}
+
+extern "C" avey_status avey_compress(const void *x, avey_dtype dt, int B, int N, int d, int S,
+                                     int k, const int32_t *idx, const float *w, const void *P,
+                                     float *out, void *out_lowp, avey_stream_t stream) {
+  const int n = S >= 1 ? (N + S - 1) / S : 0;
+  return compress_range(x, dt, B, N, d, S, k, 0, n, idx, w, P, out, out_lowp,
+                        reinterpret_cast<cudaStream_t>(stream), "avey_compress");
+}
+
+extern "C" avey_status avey_compress_rows(const void *x, avey_dtype dt, int B, int N, int d, int S,
+                                          int k, int t0, int t1, const int32_t *idx,
+                                          const float *w, const void *P, float *out,
+                                          void *out_lowp, avey_stream_t stream) {
+  return compress_range(x, dt, B, N, d, S, k, t0, t1, idx, w, P, out, out_lowp,
+                        reinterpret_cast<cudaStream_t>(stream), "avey_compress_rows");
 }

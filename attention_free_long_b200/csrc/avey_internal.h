@@ -22,8 +22,11 @@ avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N,
 
 // The same scores from 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2),
 // avey_maxsim2.cu; S in {32, 64, 128}, rs_ld >= R rounded up to 256.
+// part / nparts: compute only the tiles t with t % nparts == part (the others'
+// score entries are left untouched); every entry comes from exactly one tile.
 avey_status launch_maxsim_pair(const bf16 *x, const float *inv_norm, int B, int N, int R, int rs_ld,
-                               int d, int S, int n, float *scores, cudaStream_t s);
+                               int d, int S, int n, float *scores, cudaStream_t s, int part = 0,
+                               int nparts = 1);
 
 // Enricher: Z = relu(scale_row * (X U) + b)^2, X given as a split pair
 // (xhi, xlo) [T, d]; Ut [m, d]; writes the split pair of Z (zhi, zlo) [T, m].
@@ -48,6 +51,9 @@ avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, floa
                              cudaStream_t s);
 avey_status launch_topk(const float *scores, int B, int n, int k, int causal, int32_t *idx,
                         float *w, cudaStream_t s);
+// Targets t0 .. t0+nr-1 of every sequence; idx, w are [B, nr, k].
+avey_status launch_topk_rows(const float *scores, int B, int n, int t0, int nr, int k, int causal,
+                             int32_t *idx, float *w, cudaStream_t s);
 
 // ---- mixes (avey_mix.cu) ----
 avey_status launch_static_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks, int S,

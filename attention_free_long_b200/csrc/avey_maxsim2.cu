@@ -50,6 +50,7 @@ struct PairArgs {
   int tiles;          // 256-blocks per sequence (rows = columns)
   long long slots;    // triangular-order slots per sequence
   int num_tiles;      // B * slots
+  int part, nparts;   // this launch computes the tiles t with t % nparts == part
   int kchunks;
   float *scores;      // [B, n, n]
   const float *inv_norm;
@@ -210,6 +211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int first = pair * a.nparts + a.part, step = npairs * a.nparts;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -246,7 +248,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int tile = pair; tile < a.num_tiles && ok; tile += npairs) {
+      for (int tile = first; tile < a.num_tiles && ok; tile += step) {
         int b, mt, nt;
         if (!decode_pair(a, tile, b, mt, nt)) continue;
         for (int kc = 0; kc < a.kchunks; ++kc) {
@@ -286,7 +288,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = pair; tile < a.num_tiles && ok; tile += npairs) {
+      for (int tile = first; tile < a.num_tiles && ok; tile += step) {
         int b, mt, nt;
         if (!decode_pair(a, tile, b, mt, nt)) continue;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
@@ -333,7 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = pair; tile < a.num_tiles; tile += npairs) {
+    for (int tile = first; tile < a.num_tiles; tile += step) {
       int b, mt, nt;
       if (!decode_pair(a, tile, b, mt, nt)) continue;
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
@@ -421,7 +423,8 @@ avey_status run_pair(const CUtensorMap &mx, PairArgs a, cudaStream_t st) {
     }
     cap = std::min(clusters, sm_count() / 2);
   }
-  const int pairs = std::max(1, std::min(a.num_tiles, cap));
+  const int mine = (a.num_tiles - a.part + a.nparts - 1) / a.nparts;  // tiles of this part
+  const int pairs = std::max(1, std::min(mine, cap));
   kern<<<2 * pairs, kThreads, SMEM_BYTES, st>>>(mx, a);
   AVEY_CHECK_LAUNCH("maxsim_pair");
   return AVEY_OK;
@@ -430,7 +433,8 @@ avey_status run_pair(const CUtensorMap &mx, PairArgs a, cudaStream_t st) {
 }  // namespace
 
 avey_status launch_maxsim_pair(const bf16 *x, const float *inv_norm, int B, int N, int R, int rs_ld,
-                               int d, int S, int n, float *scores, cudaStream_t s) {
+                               int d, int S, int n, float *scores, cudaStream_t s, int part,
+                               int nparts) {
   CUtensorMap mx;
   const uint64_t rs = static_cast<uint64_t>(d) * 2, bs = rs * static_cast<uint64_t>(N);
   if (!encode_bf16_map(&mx, x, d, N, B, rs, bs, 128)) return AVEY_ERR_CUDA;
@@ -446,6 +450,8 @@ avey_status launch_maxsim_pair(const bf16 *x, const float *inv_norm, int B, int 
     return AVEY_ERR_UNSUPPORTED;
   }
   a.num_tiles = static_cast<int>(slots * B);
+  a.part = part;
+  a.nparts = nparts;
   a.kchunks = (d + BK - 1) / BK;
   a.scores = scores;
   a.inv_norm = inv_norm;

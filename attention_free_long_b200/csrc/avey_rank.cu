@@ -184,13 +184,16 @@ __device__ __forceinline__ bool key_gt(float a, int ia, float b, int ib) {
 }
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
-    topk_warp(const float *__restrict__ scores, int B, int n, int k, int causal, int vec4,
-              int32_t *__restrict__ idx, float *__restrict__ w) {
+    topk_warp(const float *__restrict__ scores, int B, int n, int t0, int nr, int k, int causal,
+              int vec4, int32_t *__restrict__ idx, float *__restrict__ w) {
+  // rows of this launch: targets t0 .. t0+nr-1 of every sequence; outputs are
+  // [B, nr, k]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long rowid = static_cast<long long>(blockIdx.x) * kTopkWarps + warp;
-  if (rowid >= static_cast<long long>(B) * n) return;
-  const int t = static_cast<int>(rowid % n);
-  const float *src = scores + rowid * n;
+  if (rowid >= static_cast<long long>(B) * nr) return;
+  const long long bq = rowid / nr;
+  const int t = t0 + static_cast<int>(rowid - bq * nr);
+  const float *src = scores + (bq * n + t) * n;
   const int lim = causal ? t : n;  // candidates c < lim, c != t
   float lv = -INFINITY;  // this lane's list entry (q = lane)
   int lc = 0x7fffffff;
@@ -295,14 +298,20 @@ avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, floa
   return AVEY_OK;
 }
 
-avey_status launch_topk(const float *scores, int B, int n, int k, int causal, int32_t *idx,
-                        float *w, cudaStream_t s) {
-  const long long rows = static_cast<long long>(B) * n;
+avey_status launch_topk_rows(const float *scores, int B, int n, int t0, int nr, int k, int causal,
+                             int32_t *idx, float *w, cudaStream_t s) {
+  const long long rows = static_cast<long long>(B) * nr;
+  if (rows == 0) return AVEY_OK;
   const unsigned grid = static_cast<unsigned>((rows + kTopkWarps - 1) / kTopkWarps);
   const int vec4 = (n % 4 == 0 && aligned16(scores)) ? 1 : 0;
-  topk_warp<<<grid, kTopkWarps * 32, 0, s>>>(scores, B, n, k, causal, vec4, idx, w);
+  topk_warp<<<grid, kTopkWarps * 32, 0, s>>>(scores, B, n, t0, nr, k, causal, vec4, idx, w);
   AVEY_CHECK_LAUNCH("topk_warp");
   return AVEY_OK;
+}
+
+avey_status launch_topk(const float *scores, int B, int n, int k, int causal, int32_t *idx,
+                        float *w, cudaStream_t s) {
+  return launch_topk_rows(scores, B, n, 0, n, k, causal, idx, w, s);
 }
 
 static avey_status launch_maxsim_f32(const float *xhat, int B, int R, int d, int S, int n,
@@ -358,6 +367,51 @@ extern "C" avey_status avey_topk(const float *scores, int B, int n, int k, uint3
                "avey_topk: problem too large");
   return launch_topk(scores, B, n, k, (flags & AVEY_RANK_UNIDIRECTIONAL) ? 1 : 0, idx, w,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" avey_status avey_topk_rows(const float *scores, int B, int n, int t0, int t1, int k,
+                                      uint32_t flags, int32_t *idx, float *w,
+                                      avey_stream_t stream) {
+  AVEY_REQUIRE(scores && idx && w, AVEY_ERR_INVALID_ARG, "avey_topk_rows: null pointer");
+  AVEY_REQUIRE(B >= 1 && n >= 1 && k >= 1 && k <= 32, AVEY_ERR_INVALID_ARG,
+               "avey_topk_rows: sizes (B=%d n=%d, 1 <= k=%d <= 32)", B, n, k);
+  AVEY_REQUIRE(0 <= t0 && t0 <= t1 && t1 <= n, AVEY_ERR_INVALID_ARG,
+               "avey_topk_rows: target range [%d, %d) outside [0, %d)", t0, t1, n);
+  AVEY_REQUIRE((flags & ~static_cast<uint32_t>(AVEY_RANK_UNIDIRECTIONAL)) == 0,
+               AVEY_ERR_INVALID_ARG, "avey_topk_rows: unknown flags 0x%x", flags);
+  return launch_topk_rows(scores, B, n, t0, t1 - t0, k, (flags & AVEY_RANK_UNIDIRECTIONAL) ? 1 : 0,
+                          idx, w, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" avey_status avey_maxsim_part(const void *x, avey_dtype dt, int B, int N, int d, int S,
+                                        int part, int nparts, float *scores, void *ws,
+                                        size_t ws_bytes, avey_stream_t stream) {
+  AVEY_REQUIRE(dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
+               "avey_maxsim_part: dtype %d unsupported (BF16)", int(dt));
+  AVEY_REQUIRE(x && scores && ws, AVEY_ERR_INVALID_ARG, "avey_maxsim_part: null pointer");
+  AVEY_REQUIRE(B >= 1 && N >= 1 && d >= 1, AVEY_ERR_INVALID_ARG,
+               "avey_maxsim_part: sizes must be >= 1 (B=%d N=%d d=%d)", B, N, d);
+  AVEY_REQUIRE(S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
+               "avey_maxsim_part: S=%d unsupported (32, 64 or 128)", S);
+  AVEY_REQUIRE(nparts >= 1 && part >= 0 && part < nparts, AVEY_ERR_INVALID_ARG,
+               "avey_maxsim_part: part %d of %d", part, nparts);
+  AVEY_REQUIRE(d % 8 == 0, AVEY_ERR_INVALID_ARG, "avey_maxsim_part: d=%d must be a multiple of 8", d);
+  AVEY_REQUIRE(aligned16(x) && aligned16(scores) && (reinterpret_cast<uintptr_t>(ws) & 255) == 0,
+               AVEY_ERR_INVALID_ARG,
+               "avey_maxsim_part: x, scores 16-byte and the workspace 256-byte aligned");
+  const long long n = (N + S - 1) / S, R = n * S;
+  AVEY_REQUIRE(n <= 46340 && static_cast<long long>(B) * R <= (1ll << 31) - 1,
+               AVEY_ERR_UNSUPPORTED, "avey_maxsim_part: problem too large");
+  const size_t need = avey_rank_workspace_bytes(dt, B, N, d, S);
+  AVEY_REQUIRE(ws_bytes >= need, AVEY_ERR_INVALID_ARG,
+               "avey_maxsim_part: workspace %zu bytes < %zu required", ws_bytes, need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float *inv = static_cast<float *>(ws);
+  const int ld = static_cast<int>(scale_ld(R));
+  avey_status st = launch_inv_norms(static_cast<const bf16 *>(x), B, N, d, ld, inv, s);
+  if (st != AVEY_OK) return st;
+  return launch_maxsim_pair(static_cast<const bf16 *>(x), inv, B, N, static_cast<int>(R), ld, d, S,
+                            static_cast<int>(n), scores, s, part, nparts);
 }
 
 extern "C" avey_status avey_rank_ex(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,

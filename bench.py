@@ -498,6 +498,122 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
+# ----------------------------------------------- one sequence, N GPUs ---
+
+def run_sharded(args):
+    """--shard sequence: the workload's sequence split across the ranks (strong
+    scaling).  Every rank holds the whole input; MaxSim tiles are dealt
+    round-robin, the score partials are summed by one NCCL all-reduce, and
+    top-k, compression and the layers run on each rank's target splits."""
+    import torch
+    import attention_free_long_b200 as av
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl", world)
+    barrier = (lambda: dist.barrier(device_ids=[local])) if world > 1 else (lambda: None)
+    allreduce = (lambda buf: dist.all_reduce(buf)) if world > 1 else (lambda buf: None)
+
+    wl = sy.WORKLOADS[args.workload]
+    E = sy.gen_embeddings(wl, seed=rank_seed(0))  # the same sequence on every rank
+    W = sy.gen_weights(wl)
+    x = torch.from_numpy(E.X).to(dev, torch.bfloat16)
+    P = torch.from_numpy(W.P).to(dev, torch.bfloat16)
+    layers = av.device_layers(W, torch.bfloat16, dev)
+    ws = av.make_shard_workspace(wl.B, wl.N, wl.d, wl.S, wl.k, wl.m, torch.bfloat16, wl.prenorm,
+                                 rank, world, dev)
+
+    def step(marks=None):
+        return av.encoder_forward_sharded(x, P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm,
+                                          rank, world, allreduce, ws, marks)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = av.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after warm-up")
+    n_marks = 2 + wl.layers
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks + 1)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    l0 = av.kernel_launches()
+    with ClockSampler(local) as clk:
+        start.record()
+        for s_ in range(args.steps):
+            step(marks[s_])
+        end.record()
+        torch.cuda.synchronize()
+    launches = av.kernel_launches() - l0
+    barrier()
+    torch.cuda.synchronize()
+    ms_max = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
+    stage = np.array([[marks[s_][i].elapsed_time(marks[s_][i + 1]) for i in range(n_marks)]
+                      for s_ in range(args.steps)]).mean(axis=0)
+    st = av.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after the timed region")
+
+    # end to end: every step copies the whole input in and this rank's rows out
+    xh = torch.from_numpy(E.X).to(torch.bfloat16).pin_memory()
+    T_r = wl.B * (ws.t1 - ws.t0) * wl.S
+    outh = torch.empty((max(T_r, 1), wl.d), dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(x)
+    for _ in range(2):
+        xd.copy_(xh, non_blocking=True)
+        o = step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        o = av.encoder_forward_sharded(xd, P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm, rank,
+                                       world, allreduce, ws)
+        outh[:T_r].copy_(o.reshape(T_r, wl.d), non_blocking=True)
+    end.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
+
+    tokens = wl.B * wl.N
+    peaks, peak_kind = load_peaks()
+    sustained = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    part_ms = float(stage[0])
+    result = {
+        "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian mixture, random N(0,1/fan_in) weights)",
+        "config": {"workload": workload_desc(wl), "global_batch": wl.B, "seq_len": wl.N,
+                   "parallelism": (f"sp{world}: one sequence across {world} GPU(s); MaxSim tiles "
+                                   "round-robin, score partials summed by one all-reduce of "
+                                   f"{wl.B * wl.n * wl.n * 4 / 1e6:.1f} MB, then each rank's "
+                                   "target splits"),
+                   "l2": "inputs larger than L2 (X is 151 MB bf16, 126 MB L2); no flush"},
+        "roofline": {"bound": "tensor", "kernel": "maxsim part + all-reduce (rank 0)",
+                     "achieved": maxsim_executed_flops(wl) / world / (part_ms * 1e-3) / 1e12,
+                     "peak": sustained, "unit": "TFLOP/s",
+                     "frac": maxsim_executed_flops(wl) / world / (part_ms * 1e-3) / 1e12 / sustained,
+                     "peak_kind": f"{peak_kind} bf16 sustained", "traffic": None,
+                     "note": "executed MMA work of this rank's 1/N of the triangular tiles over "
+                             "the duration of its MaxSim part plus the all-reduce"},
+        "kernels_ms": {"maxsim_part_and_allreduce": part_ms, "topk_and_compress": float(stage[1]),
+                       "layers": stage[2:].tolist()},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
+                "d2h_bytes_per_step": int(T_r * wl.d * 4),
+                "note": "every rank copies the whole input in and its own rows out"},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 # -------------------------------------------------------- reference arm ---
 
 def run_reference(args):
@@ -548,6 +664,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-uncompressed", action="store_true",
                     help="skip the measurement of the processor without compression")
+    ap.add_argument("--shard", choices=["replicas", "sequence"], default="replicas",
+                    help="replicas: one sequence per GPU (weak scaling, no collective); "
+                         "sequence: the workload's sequence split across the GPUs (strong scaling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -557,6 +676,8 @@ def main(argv=None):
             ap.error(f"--gpus {args.gpus} needs torchrun with {args.gpus} ranks (WORLD_SIZE={world})")
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard == "sequence":
+        run_sharded(args)
     else:
         run_ours(args)
 

@@ -149,6 +149,27 @@ AVEY_API size_t avey_rank_static_max_scratch_bytes(void);
 AVEY_API avey_status avey_topk(const float *scores, int B, int n, int k, uint32_t flags,
                                int32_t *idx, float *w, avey_stream_t stream);
 
+/* avey_topk_rows: avey_topk for the targets t0 .. t1-1 of every sequence
+ * (scores [B, n, n] as above; idx, w [B, t1-t0, k]).  With one long sequence
+ * sharded across GPUs, each rank selects for its own targets. */
+AVEY_API avey_status avey_topk_rows(const float *scores, int B, int n, int t0, int t1, int k,
+                                    uint32_t flags, int32_t *idx, float *w, avey_stream_t stream);
+
+/* avey_maxsim_part: the split scores of avey_rank from one part of the work,
+ * for one long sequence sharded across GPUs.  The triangular tile order of
+ * the MaxSim kernel (each 256x256 tile on or right of the diagonal gives the
+ * scores of its split pairs in both directions) is dealt round-robin into
+ * nparts parts; part `part` writes the entries of its tiles and leaves the
+ * others untouched.  Every entry belongs to exactly one part, so zeroed score
+ * buffers summed over all parts (an all-reduce) give avey_rank's scores bit
+ * for bit.  x, ws as for avey_rank (ws >= avey_rank_workspace_bytes);
+ * scores [B, n, n] fp32, zeroed by the caller.
+ * Constraints: AVEY_BF16, S in {32, 64, 128}; 0 <= part < nparts.
+ */
+AVEY_API avey_status avey_maxsim_part(const void *x, avey_dtype dt, int B, int N, int d, int S,
+                                      int part, int nparts, float *scores, void *ws,
+                                      size_t ws_bytes, avey_stream_t stream);
+
 /* ---------------------------------------------------------- compression --
  * avey_compress: neural compression of each split with its retrieved splits
  * plus the residual to the split's own tokens ([AB-notes] 关键设计 4, eq. 8):
@@ -170,6 +191,15 @@ AVEY_API avey_status avey_topk(const float *scores, int B, int n, int k, uint32_
 AVEY_API avey_status avey_compress(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
                           const int32_t *idx, const float *w, const void *P, float *out,
                           void *out_lowp, avey_stream_t stream);
+
+/* avey_compress_rows: avey_compress for the target splits t0 .. t1-1 of every
+ * sequence: idx, w are [B, t1-t0, k] (as from avey_topk_rows; candidate
+ * indices still refer to the whole sequence), out [B, (t1-t0)*S, d] fp32,
+ * out_lowp the pair [2][B*(t1-t0)*S][d] or NULL. */
+AVEY_API avey_status avey_compress_rows(const void *x, avey_dtype dt, int B, int N, int d, int S,
+                                        int k, int t0, int t1, const int32_t *idx, const float *w,
+                                        const void *P, float *out, void *out_lowp,
+                                        avey_stream_t stream);
 
 /* --------------------------------------------------- uncompressed context --
  * avey_context: the context of every split without neural compression, for

@@ -74,3 +74,29 @@ def test_pair_long_workload_tiles():
     bad, tiles, full = _coverage_pair(98304, 64)
     assert not bad
     assert full == 384 * 384 and tiles == 384 * 385 // 2
+
+
+@pytest.mark.parametrize("nparts", [2, 3, 8])
+@pytest.mark.parametrize("N,S", [(4096, 64), (5000, 32), (2500, 128)])
+def test_pair_parts_partition_the_entries(N, S, nparts):
+    # avey_maxsim_part: part p takes the tiles t with t % nparts == p of the
+    # same slot order; every ordered split pair is written by exactly one part
+    n = -(-N // S)
+    tn = -(-(n * S) // 256)
+    slots = sum(min(GP, tn - g * GP) * (tn - g * GP) for g in range(-(-tn // GP)))
+    TS = CB = 128 // S
+    owner = {}
+    for x in range(slots):
+        mt, nt, ok = _decode_pair(x, tn)
+        if not ok:
+            continue
+        part = x % nparts
+        for rank, half in itertools.product(range(2), range(2)):
+            t0, c0 = (mt * 256 + rank * 128) // S, (nt * 256 + half * 128) // S
+            for ts, cl in itertools.product(range(TS), range(CB)):
+                t, c = t0 + ts, c0 + cl
+                if t < n and c < n:
+                    for key in ((t, c), (c, t)) if nt > mt else ((t, c),):
+                        assert key not in owner
+                        owner[key] = part
+    assert len(owner) == n * n
