@@ -350,6 +350,8 @@ static avey_status compress_range(const void *x, avey_dtype dt, int B, int N, in
     const bf16 *Pb = static_cast<const bf16 *>(P);
     bf16 *hi = static_cast<bf16 *>(out_lowp);
     bf16 *lo = hi ? hi + static_cast<long long>(B) * nr * S * d : nullptr;
+    if (compress_tc_supported(S, d))
+      return launch_compress_tc(xb, B, N, d, k, t0, nr, idx, w, Pb, out, hi, lo, s);
     switch (S) {
       case 16: return run_compress_bf16<16>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
       case 32: return run_compress_bf16<32>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);

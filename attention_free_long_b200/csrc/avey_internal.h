@@ -44,6 +44,14 @@ avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const
                            cudaStream_t s, const bf16 *chi = nullptr, const bf16 *clo = nullptr,
                            int k_split = 0);
 
+// Compression on tcgen05 (avey_compress_tc.cu) for S = 64, targets t0 ..
+// t0+nr-1 (idx, w, out as for avey_compress_rows); the split-size mma.sync
+// kernel covers the other S.
+bool compress_tc_supported(int S, int d);
+avey_status launch_compress_tc(const bf16 *x, int B, int N, int d, int k, int t0, int nr,
+                               const int32_t *idx, const float *w, const bf16 *P, float *out,
+                               bf16 *hi, bf16 *lo, cudaStream_t s);
+
 // ---- ranker pieces (avey_rank.cu) ----
 avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, int S, void *xhat,
                              cudaStream_t s);
