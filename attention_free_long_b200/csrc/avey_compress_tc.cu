@@ -31,10 +31,13 @@ constexpr int C_EPI = 4, C_THR = 64 + 32 * C_EPI;
 constexpr uint32_t C_XBOX = 64 * CS * 2;      // 8 KB: 64 features x 64 tokens
 constexpr uint32_t C_PBOX = CS * CS * 2;      // 8 KB: P_r, 64 i x 64 j
 constexpr uint32_t C_STAGE = 2 * C_XBOX + C_PBOX;
-constexpr int C_STAGES = 8;
+constexpr int C_STAGES = 6;
 constexpr int C_NACC = 8;                     // TMEM buffers of 64 columns
 constexpr uint32_t C_IDENT = CS * CS * 2;     // 8 KB: the 64 x 64 identity (B operand)
-constexpr uint32_t C_SMEM = C_STAGES * C_STAGE + C_IDENT + 1024 + 1024;
+constexpr uint32_t C_W32 = CS * 32 * 4;       // 8 KB: one warp's fp32 output [64 i][32 f]
+constexpr uint32_t C_W16 = CS * 32 * 2;       // 4 KB: one bf16 plane of it
+constexpr uint32_t C_WSTG = C_W32 + 2 * C_W16;
+constexpr uint32_t C_SMEM = C_STAGES * C_STAGE + C_IDENT + C_EPI * C_WSTG + 1024 + 1024;
 static_assert(C_SMEM <= 232448, "shared memory budget");
 
 struct CompArgs {
@@ -98,15 +101,18 @@ __device__ __forceinline__ void block_list(const CompArgs &a, long long seg, int
 template <int KM>
 __global__ void __launch_bounds__(C_THR, 1)
     compress_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
-                       const CompArgs a) {
+                       const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmOh,
+                       const __grid_constant__ CUtensorMap tmOl, const CompArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
   uint8_t *ident = smem_raw + pad + C_STAGES * C_STAGE;
-  uint8_t *ctrl = ident + C_IDENT;
+  uint8_t *ostage = ident + C_IDENT;  // per epilogue warp: fp32 [64][32], hi, lo
+  uint8_t *ctrl = ostage + C_EPI * C_WSTG;
   const uint32_t sbase = raw_s + pad;
   const uint32_t ibase = sbase + C_STAGES * C_STAGE;
-  const uint32_t cbase = ibase + C_IDENT;
+  const uint32_t obase = ibase + C_IDENT;
+  const uint32_t cbase = obase + C_EPI * C_WSTG;
   // control block: full[8] @0, empty[8] @64, tfull[8] @128, tempty[8] @192,
   // drain @256, tmem base @264, abort flag @268
   auto full_bar = [&](int s) { return cbase + 8u * s; };
@@ -138,6 +144,7 @@ __global__ void __launch_bounds__(C_THR, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmP);
+    prefetch_tmap(&tmO);
   }
   // The residual X_t enters block 0's accumulator through the tensor cores:
   // D_0 += X_t^T I with I the 64 x 64 identity, a K-major B operand in the
@@ -267,7 +274,6 @@ __global__ void __launch_bounds__(C_THR, 1)
       const int slab = static_cast<int>(tile - seg * a.nslab);
       const int b = static_cast<int>(seg / a.nr);
       const int t = a.t0 + static_cast<int>(seg - static_cast<long long>(b) * a.nr);
-      const int f = slab * CF + quarter * 32 + lane;
       float o[CS];
 #pragma unroll
       for (int i = 0; i < CS; ++i) o[i] = 0.f;
@@ -296,25 +302,39 @@ __global__ void __launch_bounds__(C_THR, 1)
         }
       }
       if (!ok) break;
-      if (f < a.d) {
-        // fp32 out and the split pair; per token i the warp's 32 lanes store
-        // 32 consecutive features
-        const long long orow = seg * CS;
-        float *__restrict__ op = a.out + orow * a.d + f;
-        bf16 *__restrict__ oh = a.out_hi ? a.out_hi + orow * a.d + f : nullptr;
-        bf16 *__restrict__ ol = a.out_lo ? a.out_lo + orow * a.d + f : nullptr;
+      // fp32 out and the split pair: each warp stages its 32 features x 64
+      // tokens and writes them with its own three TMA stores (the tensor's
+      // bounds clip the feature tail)
+      uint8_t *wst = ostage + (warp - 2) * C_WSTG;
+      const uint32_t wsa = obase + (warp - 2) * C_WSTG;
+      if (lane == 0) bulk_wait_read<0>();  // this warp's previous stores have read it
+      __syncwarp();
+      {
+        float *o32 = reinterpret_cast<float *>(wst);
+        bf16 *oh = reinterpret_cast<bf16 *>(wst + C_W32);
+        bf16 *ol = reinterpret_cast<bf16 *>(wst + C_W32 + C_W16);
 #pragma unroll
         for (int i = 0; i < CS; ++i) {
           const float y = o[i];
-          op[static_cast<long long>(i) * a.d] = y;
-          if (oh) {
-            const bf16 h = __float2bfloat16_rn(y);
-            oh[static_cast<long long>(i) * a.d] = h;
-            ol[static_cast<long long>(i) * a.d] = __float2bfloat16_rn(y - __bfloat162float(h));
-          }
+          const bf16 h = __float2bfloat16_rn(y);
+          o32[i * 32 + lane] = y;
+          oh[i * 32 + lane] = h;
+          ol[i * 32 + lane] = __float2bfloat16_rn(y - __bfloat162float(h));
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int orow = static_cast<int>(seg * CS), ox = slab * CF + quarter * 32;
+        tma_store_3d(&tmO, wsa, ox, orow, 0);
+        if (a.out_hi) {
+          tma_store_3d(&tmOh, wsa + C_W32, ox, orow, 0);
+          tma_store_3d(&tmOl, wsa + C_W32 + C_W16, ox, orow, 0);
+        }
+        bulk_commit();
+      }
     }
+    if (lane == 0) bulk_wait_all();  // this warp's outputs written before exit
     if (!ok) {
       *abort_flag = 1;
       record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
@@ -330,8 +350,9 @@ __global__ void __launch_bounds__(C_THR, 1)
 }
 
 template <int KM>
-avey_status run_compress_tc(const CUtensorMap &mx, const CUtensorMap &mp, const CompArgs &a, int grid,
-                            cudaStream_t s) {
+avey_status run_compress_tc(const CUtensorMap &mx, const CUtensorMap &mp, const CUtensorMap &mo,
+                            const CUtensorMap &moh, const CUtensorMap &mol, const CompArgs &a,
+                            int grid, cudaStream_t s) {
   auto kern = compress_tc_kernel<KM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C_SMEM));
@@ -339,7 +360,7 @@ avey_status run_compress_tc(const CUtensorMap &mx, const CUtensorMap &mp, const 
     set_detail("compress_tc: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     return AVEY_ERR_CUDA;
   }
-  kern<<<grid, C_THR, C_SMEM, s>>>(mx, mp, a);
+  kern<<<grid, C_THR, C_SMEM, s>>>(mx, mp, mo, moh, mol, a);
   AVEY_CHECK_LAUNCH("compress_tc");
   return AVEY_OK;
 }
@@ -377,9 +398,20 @@ avey_status launch_compress_tc(const bf16 *x, int B, int N, int d, int k, int t0
   a.out_lo = lo;
   a.status = device_status_word();
   const int grid = std::max(1, std::min(a.num_tiles, sm_count()));
-  if (k + 1 <= 8) return run_compress_tc<8>(mx, mp, a, grid, s);
-  if (k + 1 <= 16) return run_compress_tc<16>(mx, mp, a, grid, s);
-  return run_compress_tc<32>(mx, mp, a, grid, s);
+  // outputs [B*nr*64 rows, d]: fp32 and the bf16 planes, dense boxes of 32 x 64
+  CUtensorMap mo, moh, mol;
+  const uint64_t orows = static_cast<uint64_t>(B) * nr * CS;
+  const uint64_t o4 = static_cast<uint64_t>(d) * 4, o2 = static_cast<uint64_t>(d) * 2;
+  if (!encode_map(&mo, true, out, d, orows, 1, o4, o4 * orows, 32, CS, 0)) return AVEY_ERR_CUDA;
+  moh = mo;
+  mol = mo;
+  if (hi) {
+    if (!encode_map(&moh, false, hi, d, orows, 1, o2, o2 * orows, 32, CS, 0)) return AVEY_ERR_CUDA;
+    if (!encode_map(&mol, false, lo, d, orows, 1, o2, o2 * orows, 32, CS, 0)) return AVEY_ERR_CUDA;
+  }
+  if (k + 1 <= 8) return run_compress_tc<8>(mx, mp, mo, moh, mol, a, grid, s);
+  if (k + 1 <= 16) return run_compress_tc<16>(mx, mp, mo, moh, mol, a, grid, s);
+  return run_compress_tc<32>(mx, mp, mo, moh, mol, a, grid, s);
 }
 
 }  // namespace avey
