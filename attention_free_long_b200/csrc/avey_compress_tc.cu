@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(C_THR, 1)
   const uint32_t ibase = sbase + C_STAGES * C_STAGE;
   const uint32_t obase = ibase + C_IDENT;
   const uint32_t cbase = obase + C_EPI * C_WSTG;
+  static_assert(C_STAGES <= 8 && C_NACC <= 8, "the control block holds at most 8 of each");
   // control block: full[8] @0, empty[8] @64, tfull[8] @128, tempty[8] @192,
   // drain @256, tmem base @264, abort flag @268
   auto full_bar = [&](int s) { return cbase + 8u * s; };

@@ -193,6 +193,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t *ctrl = smem_raw + pad + TILES_BYTES;
   const uint32_t sbase = raw_s + pad;
   const uint32_t cbase = sbase + TILES_BYTES;
+  static_assert(kStages <= 8, "the control block holds at most 8 stages");
   // control block: full[6] @0, empty[6] @64, tfull[2] @128, tempty[2] @144,
   // redbar[4] @160, redfree[4] @192, drain @224, tmem base @232, abort @236,
   // red @256, column maxima @2048

@@ -8,6 +8,8 @@
 //
 // One persistent, warp-specialised kernel; a tile is (block, 128 rows i,
 // 256 features f), accumulated in TMEM over the SL tokens j:
+//   * two stages of 64 tokens (stages of 32 tokens with 64-byte-swizzled A
+//     boxes allowed four or five stages but measured slower);
 //   * A (rows i, K = j) is K-major: a TMA box of 64 tokens x 128 rows, 128-byte
 //     swizzle, as in the other tcgen05 kernels;
 //   * B = Z_b (N = f, K = j) is read straight from the token-major activation:
@@ -98,15 +100,16 @@ __global__ void __launch_bounds__(kThr, 1)
   uint8_t *ctrl = smem_raw + pad + L::TILES;
   const uint32_t sbase = raw_s + pad;
   const uint32_t cbase = sbase + L::TILES;
-  // control block: full[2] @0, empty[2] @16, tfull[2] @32, tempty[2] @48,
-  // drain @64, tmem base @72, abort flag @76
+  // control block (room for up to 8 stages): full[s] @8s, empty[s] @64+8s,
+  // tfull[2] @128, tempty[2] @144, drain @160, tmem base @168, abort flag @172
+  static_assert(L::STAGES <= 8, "control block holds at most 8 stages");
   auto full_bar = [&](int s) { return cbase + 8u * s; };
-  auto empty_bar = [&](int s) { return cbase + 16u + 8u * s; };
-  auto tfull_bar = [&](int i) { return cbase + 32u + 8u * i; };
-  auto tempty_bar = [&](int i) { return cbase + 48u + 8u * i; };
-  const uint32_t drain_bar = cbase + 64u;
-  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 72);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 76);
+  auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
+  auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
+  auto tempty_bar = [&](int i) { return cbase + 144u + 8u * i; };
+  const uint32_t drain_bar = cbase + 160u;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 168);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 172);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(kThr, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(ctrl + 72), kCols);
+    tmem_alloc(smem_u32(ctrl + 168), kCols);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -319,6 +322,7 @@ __global__ void __launch_bounds__(kThr, 1)
   uint8_t *ctrl = smem_raw + pad + G_STAGES * G_STAGE;
   const uint32_t sbase = raw_s + pad;
   const uint32_t cbase = sbase + G_STAGES * G_STAGE;
+  static_assert(G_STAGES <= 4, "the Gram control block holds at most 4 stages");
   // control block: full[4] @0, empty[4] @32, tfull[2] @64, tempty[2] @80,
   // drain @96, tmem base @104, abort flag @108
   auto full_bar = [&](int s) { return cbase + 8u * s; };

@@ -337,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *ctrl = smem_raw + pad + L::TILES_BYTES;
   const uint32_t sbase = raw_s + pad;
   const uint32_t cbase = sbase + L::TILES_BYTES;
+  static_assert(L::STAGES <= 8, "the control block holds at most 8 stages");
   // control block: full[4] @0, empty[4] @64, tfull[2] @128, tempty[2] @144,
   // redbar[2 acc] @160, drain @192, tmem base @200, abort flag @204,
   // MaxSim partial sums [2 acc][8 groups][16 candidates] @256
