@@ -154,3 +154,29 @@ def test_long_blocks_need_head_width_multiple_of_64(cuda_dev):
     with pytest.raises(av.AveyError):
         av.avey_layer_forward(lay, S, m_h, 1e-8, False, x)
     assert av.kernel_launches() == before
+
+
+def test_uncompressed_long_workload_sampled(cuda_dev):
+    # the bench's workload at full size (1536 blocks of 512 tokens), in the
+    # launch configuration the bench times; the oracle computes seeded target
+    # splits one by one (each needs only its own score row and context)
+    wl = sy.WORKLOADS["long_bf16"]
+    E = sy.gen_embeddings(wl)
+    W = sy.gen_weights(wl, block=(wl.k + 1) * wl.S)
+    x = torch.from_numpy(E.X).to(cuda_dev, torch.bfloat16)
+    layers = av.device_layers(W, torch.bfloat16, cuda_dev)
+    out = av.encoder_forward_uncompressed(x, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm)
+    torch.cuda.synchronize()
+    assert av.device_status() == 0
+    sel = sy.sample_targets(wl, per_seq=4, seed=7)
+    sb, st = torch.from_numpy(sel[:, 0]).long(), torch.from_numpy(sel[:, 1]).long()
+    g_out = out.cpu()[sb, st].numpy()
+    g_idx, g_w = av.avey_rank(x, wl.S, wl.k)
+    o = orc.forward_uncompressed(E.X, W, wl, sel=sel)
+    exact = check_topk(g_idx.cpu()[sb, st].numpy(), g_w.cpu()[sb, st].numpy(), o["idx"], o["scores"],
+                       sel[:, 1], TOL["bf16"])
+    assert exact.any(), "no sampled row has an identical top-k list"
+    err = rel_err(g_out[exact], o["out"][exact])
+    assert err <= TOL["bf16"], f"uncompressed output err {err:.3g}"
+    del out, layers
+    torch.cuda.empty_cache()
