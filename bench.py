@@ -200,9 +200,31 @@ def cpu_baseline(wl, E, W, budget_s: float = 15.0, max_splits: int = 64):
     orc.forward(X64, W, wl, sel=sel)
     el = time.perf_counter() - t0
     toks = sel.shape[0] * wl.S
-    return {"value": toks / el, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+    # the same oracle on one core, on the one-split sample
+    cores = orc.threads()
+    orc.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        orc.forward(X64, W, wl, sel=one)
+        el1 = time.perf_counter() - t0
+    finally:
+        orc.set_threads(cores)
+    return {"value": toks / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "value_1core": wl.S / el1,
             "sample": f"{sel.shape[0]} seeded target splits x {wl.S} tokens of {wl.name} "
-                      f"(full rank row, compression, {wl.layers} layers each), {el:.1f} s"}
+                      f"(full rank row, compression, {wl.layers} layers each), {el:.1f} s; "
+                      f"1 core: 1 split, {el1:.1f} s"}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 # -------------------------------------------------------------- our arm ---
@@ -649,7 +671,7 @@ def run_reference(args):
         "config": {"workload": workload_desc(wl), "global_batch": wl.B, "seq_len": wl.N,
                    "parallelism": "host cores (OpenMP)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
-                         "sample": sample},
+                         "cpu_model": cpu_model(), "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
