@@ -176,6 +176,8 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
                  "static and dynamic layers)", S);
     AVEY_REQUIRE(S <= 128 || m_h % 64 == 0, AVEY_ERR_UNSUPPORTED,
                  "avey_layer_forward(BF16): blocks of %d tokens need m_h %% 64 == 0 (m_h = %d)", S, m_h);
+    AVEY_REQUIRE(S <= 128 || p->kind != AVEY_DYNAMIC || m - m_h <= 1024, AVEY_ERR_UNSUPPORTED,
+                 "avey_layer_forward(BF16): dynamic blocks of %d tokens need m - m_h <= 1024", S);
   } else {
     AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
                  "avey_layer_forward(F32): S=%d unsupported (power of two <= 64)", S);

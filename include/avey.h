@@ -285,7 +285,8 @@ AVEY_API avey_status avey_dynamic_mix(const void *zt, int64_t ld_zt, avey_dtype 
  * Constraints: T % S == 0; d, m, m_h multiples of 8 with 0 < m_h < m;
  * S in {16, 32, 64, 128} for AVEY_BF16, and also 256 or 512 for static and
  * dynamic layers (the blocks of (k+1)S tokens of the uncompressed processor,
- * see avey_context); a power of two <= 64 for F32; eps >= 0.
+ * see avey_context; these need m_h % 64 == 0, and m - m_h <= 1024 for a
+ * dynamic layer); a power of two <= 64 for F32; eps >= 0.
  */
 typedef struct {
   avey_ctx_kind kind;
