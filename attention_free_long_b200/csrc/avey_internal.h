@@ -16,7 +16,7 @@ using bf16 = __nv_bfloat16;
 
 // MaxSim split scores from the raw embeddings x [B, N, d] bf16 and the
 // inverse row norms inv_norm [B, rs_ld] (rs_ld >= R rounded up to 256, zero
-// past N); R = n*S.
+// past N); R = n*S.  Full tile grid on one CTA per SM, for S = 16.
 avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N, int R, int rs_ld,
                              int d, int S, int n, float *scores, cudaStream_t s);
 

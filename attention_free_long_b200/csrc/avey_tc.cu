@@ -598,10 +598,9 @@ avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N,
   a.rs_ld = rs_ld;
   switch (S) {
     case 16: return run_tc<MODE_MAXSIM, 1, 16>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
-    case 32: return run_tc<MODE_MAXSIM, 1, 32>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
-    case 64: return run_tc<MODE_MAXSIM, 1, 64>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
-    case 128: return run_tc<MODE_MAXSIM, 1, 128>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
-    default: set_detail("maxsim_tc: S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
+    default:
+      set_detail("maxsim_tc: S=%d unsupported (16; larger splits use the CTA-pair kernel)", S);
+      return AVEY_ERR_UNSUPPORTED;
   }
 }
 
