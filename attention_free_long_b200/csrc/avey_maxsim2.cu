@@ -1,8 +1,9 @@
-// avey_maxsim2.cu -- MaxSim split scores on CTA pairs (tcgen05 cta_group::2).
-//
-// Same computation as the triangular MaxSim of avey_tc.cu (Avey-B paperlayer
-// summary §3 and papernotes 整体框架: score(t, c) = sum over the rows of split t
-// of the max cosine to a row of split c), laid out for two SMs per tile:
+// avey_maxsim2.cu -- MaxSim split scores on CTA pairs (tcgen05 cta_group::2),
+// the ranker's dominant step for S in {32, 64, 128} (Avey-B paperlayer summary
+// §3 and papernotes 整体框架: score(t, c) = sum over the rows of split t of the
+// max cosine to a row of split c).  The cosines are formed from the raw bf16
+// dot products and the scales 1/|x_i|, 1/|x_j|; only the [B, n, n] split
+// scores reach HBM.  Laid out for two SMs per tile:
 //
 //   * A cluster of two CTAs owns a 256 x 256 tile of G = X X^T: each CTA
 //     holds 128 of its rows in TMEM (fp32), loads those 128 rows of X (A) and
@@ -22,6 +23,9 @@
 //     commit frees the stage in both CTAs and publishes the accumulator to
 //     both; both CTAs' epilogue warps release the accumulator to CTA 0.
 //     Every wait is bounded (avey_common.cuh); no load uses multicast.
+//   * Tiles are visited in groups of 32 row blocks (the group's rows stay in
+//     L2 while its column blocks stream past); a launch may compute only the
+//     tiles t with t % nparts == part (one long sequence across GPUs).
 #include <algorithm>
 
 #include "avey_common.cuh"
