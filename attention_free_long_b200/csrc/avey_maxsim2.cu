@@ -66,12 +66,31 @@ __device__ __forceinline__ long long pair_prefix(long long g, long long tn) {
   return kGroup * g * tn - static_cast<long long>(kGroup) * kGroup * g * (g - 1) / 2;
 }
 
-// Slot -> (sequence, row block, column block).  Group g holds row blocks
-// 32g .. 32g+31 and column blocks 32g .. tiles-1; slots left of the diagonal
-// (nt < mt) hold no work and every role skips them alike.
-__device__ __forceinline__ bool decode_pair(const PairArgs &a, int tile, int &b, int &mt, int &nt) {
-  b = static_cast<int>(tile / a.slots);
-  const long long x = tile - static_cast<long long>(b) * a.slots;
+// Slots of group g: its row blocks (32, fewer in the last group) times the
+// column blocks 32g .. tiles-1.
+__device__ __forceinline__ int group_slots(int tiles, int g, int &rows) {
+  rows = min(kGroup, tiles - g * kGroup);
+  return rows * (tiles - g * kGroup);
+}
+
+// One pair's walk over the slots first, first + step, ... of the triangular
+// order.  Group g holds row blocks 32g .. 32g+31 and column blocks
+// 32g .. tiles-1, row block fastest; slots left of the diagonal (nt < mt)
+// hold no work and every role skips them alike.  Only the first slot is
+// located from scratch (a square root); each step then moves the in-group
+// offset on and crosses whole groups and sequences, a few integer operations
+// per tile on the MMA issuer's critical path.
+struct PairCursor {
+  long long tile;  // global slot (sequence-major)
+  int b, g;        // sequence, group
+  int x;           // slot inside group g
+  int size, rows;  // slots and row blocks of group g
+};
+
+__device__ __forceinline__ void cursor_init(const PairArgs &a, PairCursor &c, long long first) {
+  c.tile = first;
+  c.b = static_cast<int>(first / a.slots);
+  const long long x = first - static_cast<long long>(c.b) * a.slots;
   const long long tn = a.tiles;
   const double A = static_cast<double>(kGroup) * tn + kGroup * kGroup / 2.0;
   const double disc = A * A - 2.0 * kGroup * kGroup * static_cast<double>(x);
@@ -79,10 +98,30 @@ __device__ __forceinline__ bool decode_pair(const PairArgs &a, int tile, int &b,
   if (g < 0) g = 0;
   while (g > 0 && pair_prefix(g, tn) > x) --g;
   while (pair_prefix(g + 1, tn) <= x && (g + 1) * kGroup < a.tiles) ++g;
-  const long long rem = x - pair_prefix(g, tn);
-  const int rows_g = min(kGroup, a.tiles - static_cast<int>(g) * kGroup);
-  nt = static_cast<int>(g * kGroup + rem / rows_g);
-  mt = static_cast<int>(g * kGroup + rem % rows_g);
+  c.g = static_cast<int>(g);
+  c.x = static_cast<int>(x - pair_prefix(g, tn));
+  c.size = group_slots(a.tiles, c.g, c.rows);
+}
+
+__device__ __forceinline__ void cursor_next(const PairArgs &a, PairCursor &c, int step) {
+  c.tile += step;
+  if (c.tile >= a.num_tiles) return;
+  c.x += step;
+  while (c.x >= c.size) {
+    c.x -= c.size;
+    if (++c.g * kGroup >= a.tiles) {
+      c.g = 0;
+      ++c.b;
+    }
+    c.size = group_slots(a.tiles, c.g, c.rows);
+  }
+}
+
+// (row block, column block) of the cursor's slot; false left of the diagonal.
+__device__ __forceinline__ bool cursor_tile(const PairCursor &c, int &mt, int &nt) {
+  const int q = c.rows == kGroup ? (c.x >> 5) : c.x / c.rows;
+  nt = c.g * kGroup + q;
+  mt = c.g * kGroup + (c.x - q * c.rows);
   return nt >= mt;
 }
 
@@ -253,9 +292,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int tile = first; tile < a.num_tiles && ok; tile += step) {
-        int b, mt, nt;
-        if (!decode_pair(a, tile, b, mt, nt)) continue;
+      PairCursor cur;
+      cursor_init(a, cur, first);
+      for (; cur.tile < a.num_tiles && ok; cursor_next(a, cur, step)) {
+        int mt, nt;
+        if (!cursor_tile(cur, mt, nt)) continue;
+        const int b = cur.b;
         for (int kc = 0; kc < a.kchunks; ++kc) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
             ok = false;
@@ -293,9 +335,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = first; tile < a.num_tiles && ok; tile += step) {
-        int b, mt, nt;
-        if (!decode_pair(a, tile, b, mt, nt)) continue;
+      PairCursor cur;
+      cursor_init(a, cur, first);
+      for (; cur.tile < a.num_tiles && ok; cursor_next(a, cur, step)) {
+        int mt, nt;
+        if (!cursor_tile(cur, mt, nt)) continue;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -340,9 +384,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = first; tile < a.num_tiles; tile += step) {
-      int b, mt, nt;
-      if (!decode_pair(a, tile, b, mt, nt)) continue;
+    PairCursor cur;
+    cursor_init(a, cur, first);
+    for (; cur.tile < a.num_tiles; cursor_next(a, cur, step)) {
+      int mt, nt;
+      if (!cursor_tile(cur, mt, nt)) continue;
+      const int b = cur.b;
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
         ok = false;
         break;

@@ -7,7 +7,9 @@ writes row-direction scores for its candidate splits and, right of the
 diagonal, the mirrored column-direction scores.  This transcribes the
 kernel's slot decode and write rules (decode_pair, pair_write) and checks
 that every ordered split pair (t, c) is written exactly once, for many
-sequence lengths and split sizes, and that every index stays in range.
+sequence lengths and split sizes, and that every index stays in range.  The
+kernel's roles walk their slots incrementally (PairCursor); a mirror of that
+walk is checked against the closed-form decode.
 """
 import itertools
 import math
@@ -100,3 +102,65 @@ def test_pair_parts_partition_the_entries(N, S, nparts):
                         assert key not in owner
                         owner[key] = part
     assert len(owner) == n * n
+
+
+class _Cursor:
+    """The kernel's incremental walk (PairCursor): the first slot is located
+    with the closed-form decode, then each step moves the in-group offset on
+    and crosses whole groups and sequences."""
+
+    def __init__(self, first, tn, slots, num_tiles):
+        self.tn, self.num_tiles = tn, num_tiles
+        self.tile = first
+        self.b = first // slots
+        x = first - self.b * slots
+        A = GP * tn + GP * GP / 2.0
+        disc = A * A - 2.0 * GP * GP * x
+        g = max(int((A - math.sqrt(max(disc, 0.0))) / (GP * GP)), 0)
+        while g > 0 and _prefix_pair(g, tn) > x:
+            g -= 1
+        while _prefix_pair(g + 1, tn) <= x and (g + 1) * GP < tn:
+            g += 1
+        self.g, self.x = g, x - _prefix_pair(g, tn)
+        self._size()
+
+    def _size(self):
+        self.rows = min(GP, self.tn - self.g * GP)
+        self.size = self.rows * (self.tn - self.g * GP)
+
+    def next(self, step):
+        self.tile += step
+        if self.tile >= self.num_tiles:
+            return
+        self.x += step
+        while self.x >= self.size:
+            self.x -= self.size
+            self.g += 1
+            if self.g * GP >= self.tn:
+                self.g, self.b = 0, self.b + 1
+            self._size()
+
+    def tile_of(self):
+        q = self.x // self.rows
+        return self.g * GP + (self.x - q * self.rows), self.g * GP + q
+
+
+@pytest.mark.parametrize("tn", [1, 2, 31, 32, 33, 64, 100, 384, 513])
+@pytest.mark.parametrize("B", [1, 3])
+@pytest.mark.parametrize("step", [1, 7, 74, 148, 592])
+def test_cursor_walks_the_decoded_order(tn, B, step):
+    # every pair's incremental walk visits exactly the slots the closed-form
+    # decode gives, sequence by sequence, and the pairs together visit each
+    # slot once
+    slots = sum(min(GP, tn - g * GP) * (tn - g * GP) for g in range(-(-tn // GP)))
+    num = B * slots
+    seen = 0
+    for first in range(min(step, num)):
+        c = _Cursor(first, tn, slots, num)
+        while c.tile < num:
+            x = c.tile % slots
+            mt, nt, _ = _decode_pair(x, tn)
+            assert (c.b, c.tile_of()) == (c.tile // slots, (mt, nt)), (first, c.tile)
+            seen += 1
+            c.next(step)
+    assert seen == num
