@@ -1,31 +1,34 @@
 // avey_tc.cu -- tcgen05 / TMEM / TMA contractions of the Avey-B hot path.
 //
-// One persistent, warp-specialised kernel template serves three contractions:
+// Two persistent, warp-specialised kernels:
 //
-//   MaxSim  (ranker, Avey-B paperlayer summary §3 and papernotes 整体框架):
-//           D = X_tile(128 rows) . X_tile(256 rows)^T per sequence on the raw
-//           bf16 embeddings (exact products, fp32 accumulation); the epilogue
-//           scales each column by 1/||x_j||, takes per row the max over each
-//           candidate split's S columns, scales it by 1/||x_i|| (a positive
-//           factor commutes with the max), then sums the maxima over the S
-//           rows of each target split.  Only the [B, n, n] split scores reach
-//           HBM; neither the N x N cosines nor a normalised copy of X exist.
-//           Full grid of tiles; serves S = 16 (for S >= 32 the triangular
-//           CTA-pair kernel of avey_maxsim2.cu computes half the tiles).
-//   Enricher (papernotes 整体框架, Z = sigma(XU+b); ReLU^2 per the paperlayer
+//   maxsim_tc_kernel (ranker, Avey-B paperlayer summary §3 and papernotes
+//           整体框架), one CTA per SM: D = X_tile(128 rows) . X_tile(256 rows)^T
+//           per sequence on the raw bf16 embeddings (exact products, fp32
+//           accumulation); the epilogue scales each column by 1/||x_j||, takes
+//           per row the max over each candidate split's S columns, scales it
+//           by 1/||x_i|| (a positive factor commutes with the max), then sums
+//           the maxima over the S rows of each target split.  Only the
+//           [B, n, n] split scores reach HBM; neither the N x N cosines nor a
+//           normalised copy of X exist.  Full grid of tiles; serves S = 16 (for
+//           S >= 32 the triangular CTA-pair kernel of avey_maxsim2.cu computes
+//           half the tiles).
+//   layer_pair_kernel, on CTA pairs (256 x 256 tiles, cta_group::2):
+//     Enricher (papernotes 整体框架, Z = sigma(XU+b); ReLU^2 per the paperlayer
 //           summary App. A): D = X U with X as a bf16 split pair (two MMAs per
 //           K step); epilogue scale (optional prenorm) + bias + ReLU^2, Z
 //           written as a bf16 split pair.
-//   Fuser   (papernotes 整体框架, f = [Z_h || c] O plus residual):
+//     Fuser (papernotes 整体框架, f = [Z_h || c] O plus residual):
 //           D = [Z_h || c] O with the activation as a split pair; epilogue adds
 //           the fp32 residual and writes fp32 plus the next layer's split pair.
 //
-// Roles (192 threads, one CTA per SM, persistent over output tiles):
+// Roles (192 threads per CTA, persistent over output tiles):
 //   warp 0      TMA producer: K-chunks of 64 bf16 (128-byte swizzle) of the A
 //               plane(s) and B into a ring of shared-memory stages.
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
-//               and, from one thread, issues tcgen05.mma (M=128, N=256, K=16)
-//               and tcgen05.commit to release stages / publish accumulators.
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators per
+//               CTA) and, from one thread (of CTA 0 of a pair), issues
+//               tcgen05.mma and tcgen05.commit to release stages and publish
+//               accumulators.
 //   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes (rows), fused
 //               reduction / activation / residual, stores to HBM.
 // The two TMEM accumulators let the epilogue of tile i overlap the MMAs of
@@ -68,42 +71,31 @@ struct TcArgs {
   int *status;
 };
 
-template <int A_PLANES>
-struct Layout {
+// Single-CTA MaxSim: 128-row A tiles and 256-row B tiles of X.
+struct MaxSimLayout {
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
-  static constexpr uint32_t STAGE_BYTES = A_PLANES * A_BYTES + B_BYTES;
-  static constexpr int STAGES = A_PLANES == 1 ? 4 : 3;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 4;
   static constexpr uint32_t TILES_BYTES = STAGES * STAGE_BYTES;
-  // barriers etc. (+ the MaxSim partial sums), 1 KB units
-  static constexpr uint32_t CTRL_BYTES = A_PLANES == 1 ? 2048 : 1024;
-  // layer GEMMs: per epilogue warp 8 KB of swizzled output staging for TMA stores
-  static constexpr uint32_t STAGING_BYTES = A_PLANES == 1 ? 0 : 4 * 8192;
-  static constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + STAGING_BYTES + 1024;
+  static constexpr uint32_t CTRL_BYTES = 2048;  // barriers and the partial sums
+  static constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// Decodes a tile index into (sequence, row tile, column tile).
-template <int MODE>
-__device__ __forceinline__ bool decode_tile(const TcArgs &a, int tile, int &b, int &mt, int &nt) {
-  if (MODE == MODE_MAXSIM) {
-    // Groups of group_m row tiles walk the column tiles together so that the
-    // group's rows stay in L2 while every column tile streams past once.
-    const int per_b = a.tiles_m * a.tiles_n;
-    b = tile / per_b;
-    const int local = tile - b * per_b;
-    const int gsz = a.group_m * a.tiles_n;
-    const int g = local / gsz;
-    const int rem = local - g * gsz;
-    const int rows_g = min(a.group_m, a.tiles_m - g * a.group_m);
-    nt = rem / rows_g;
-    mt = g * a.group_m + (rem - nt * rows_g);
-  } else {
-    b = 0;
-    mt = tile / a.tiles_n;
-    nt = tile - mt * a.tiles_n;
-  }
-  return true;
+// Decodes a MaxSim tile index into (sequence, row tile, column tile).  Groups
+// of group_m row tiles walk the column tiles together so that the group's
+// rows stay in L2 while every column tile streams past once.
+__device__ __forceinline__ void decode_maxsim_tile(const TcArgs &a, int tile, int &b, int &mt, int &nt) {
+  const int per_b = a.tiles_m * a.tiles_n;
+  b = tile / per_b;
+  const int local = tile - b * per_b;
+  const int gsz = a.group_m * a.tiles_n;
+  const int g = local / gsz;
+  const int rem = local - g * gsz;
+  const int rows_g = min(a.group_m, a.tiles_m - g * a.group_m);
+  nt = rem / rows_g;
+  mt = g * a.group_m + (rem - nt * rows_g);
 }
 
 // Time-bounded wait that ignores the abort flag (used to drain in-flight work).
@@ -260,25 +252,31 @@ __device__ __forceinline__ void epi_enrich(const TcArgs &a, const CUtensorMap *m
   }
 }
 
+// The fp32 residual of one row's 32-column chunk (zeros outside the matrix).
+__device__ __forceinline__ void fuse_load_residual(const TcArgs &a, int row, int col0, float4 (&xi)[8]) {
+  const bool valid = row < a.rows;
+  const float4 *src = reinterpret_cast<const float4 *>(a.x_in + static_cast<long long>(row) * a.cols + col0);
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    xi[q] = (valid && col0 + 4 * q < a.cols) ? src[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 // Fuser epilogue: x_out = x_in + acc (fp32) and its split pair; one 8 KB
-// staging buffer (fp32 4 KB, hi 2 KB, lo 2 KB).  The residual loads are
-// issued before the TMEM load so that their latency overlaps it.
+// staging buffer (fp32 4 KB, hi 2 KB, lo 2 KB).  The residual of chunk 0
+// arrives loaded (xi, issued before the accumulator wait); each chunk issues
+// the next chunk's loads before its own math, so their latency overlaps it.
 __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mout,
                                          const CUtensorMap *mhi, const CUtensorMap *mlo,
                                          uint32_t taddr, int row0, int lane, int nt, uint32_t stg,
-                                         int &it) {
+                                         int &it, float4 (&xi)[8]) {
   const int row = row0 + lane;
-  const bool valid = row < a.rows;
   const bool pair = a.out_hi != nullptr;
 #pragma unroll 1
   for (int ch = 0; ch < BN / 32; ++ch) {
     const int col0 = nt * BN + ch * 32;
     if (col0 >= a.cols) break;  // warp-uniform
-    const float4 *src = reinterpret_cast<const float4 *>(a.x_in + static_cast<long long>(row) * a.cols + col0);
-    float4 xi[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      xi[q] = (valid && col0 + 4 * q < a.cols) ? src[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 xn[8];
+    if (ch + 1 < BN / 32) fuse_load_residual(a, row, col0 + 32, xn);
     float v[32];
     tmem_ld32(taddr + ch * 32, v);
     if (it >= 1) {  // the previous chunk's stores must have read the buffer
@@ -318,19 +316,18 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mou
       bulk_commit();
     }
     ++it;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) xi[q] = xn[q];
   }
 }
 
-// ---- the kernel ------------------------------------------------------------
+// ---- single-CTA MaxSim ------------------------------------------------------
 
-template <int MODE, int A_PLANES, int SPLIT_S>
+template <int SPLIT_S>
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-              const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmO0,
-              const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2,
-              const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
-              const TcArgs a) {
-  using L = Layout<A_PLANES>;
+    maxsim_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const TcArgs a) {
+  using L = MaxSimLayout;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
@@ -338,9 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = raw_s + pad;
   const uint32_t cbase = sbase + L::TILES_BYTES;
   static_assert(L::STAGES <= 8, "the control block holds at most 8 stages");
-  // control block: full[4] @0, empty[4] @64, tfull[2] @128, tempty[2] @144,
+  // control block: full[8] @0, empty[8] @64, tfull[2] @128, tempty[2] @144,
   // redbar[2 acc] @160, drain @192, tmem base @200, abort flag @204,
-  // MaxSim partial sums [2 acc][8 groups][16 candidates] @256
+  // partial sums [2 acc][8 groups][16 candidates] @256
   auto full_bar = [&](int s) { return cbase + 8u * s; };
   auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
   auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
@@ -372,18 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA0);
-    if (A_PLANES == 2) prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (MODE == MODE_ENRICH || MODE == MODE_FUSE) {
-      prefetch_tmap(&tmO0);
-      prefetch_tmap(&tmO1);
-      if (MODE == MODE_FUSE) prefetch_tmap(&tmO2);
-      if (MODE == MODE_FUSE && a.k_split > 0) {
-        prefetch_tmap(&tmC0);
-        prefetch_tmap(&tmC1);
-      }
-    }
   }
   tc_fence_before();
   __syncthreads();
@@ -400,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
         int b, mt, nt;
-        if (!decode_tile<MODE>(a, tile, b, mt, nt)) continue;
+        decode_maxsim_tile(a, tile, b, mt, nt);
         for (int kc = 0; kc < kchunks; ++kc) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
             ok = false;
@@ -408,15 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t st = sbase + stage * L::STAGE_BYTES;
           mbar_arrive_expect_tx(full_bar(stage), L::STAGE_BYTES);
-          // fuser with a separate contextualizer output: [Z_h || c] from two
-          // sources, split at a multiple of the K chunk
-          const bool from_c = MODE == MODE_FUSE && a.k_split > 0 && kc * BK >= a.k_split;
-          const CUtensorMap *ma = from_c ? &tmC0 : &tmA0;
-          const CUtensorMap *mal = from_c ? &tmC1 : &tmA1;
-          const int ax = from_c ? kc * BK - a.k_split : kc * BK;
-          tma_load_3d(st, ma, full_bar(stage), ax, mt * BM, b);
-          if (A_PLANES == 2) tma_load_3d(st + L::A_BYTES, mal, full_bar(stage), ax, mt * BM, b);
-          tma_load_3d(st + A_PLANES * L::A_BYTES, &tmB, full_bar(stage), kc * BK, nt * BN, b);
+          tma_load_3d(st, &tmA, full_bar(stage), kc * BK, mt * BM, b);
+          tma_load_3d(st + L::A_BYTES, &tmB, full_bar(stage), kc * BK, nt * BN, b);
           ++issued;
           if (++stage == L::STAGES) {
             stage = 0;
@@ -457,15 +437,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t st = sbase + stage * L::STAGE_BYTES;
-          const uint64_t da0 = sdesc_k_sw128(st);
-          const uint64_t da1 = sdesc_k_sw128(st + L::A_BYTES);
-          const uint64_t db = sdesc_k_sw128(st + A_PLANES * L::A_BYTES);
+          const uint64_t da = sdesc_k_sw128(st);
+          const uint64_t db = sdesc_k_sw128(st + L::A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             // +32 bytes along K inside the 128-byte swizzled row = +2 in the
             // descriptor's 16-byte address units.
-            tc_mma_bf16(d_tmem, da0 + 2u * kk, db + 2u * kk, idesc, (kc | kk) != 0);
-            if (A_PLANES == 2) tc_mma_bf16(d_tmem, da1 + 2u * kk, db + 2u * kk, idesc, 1u);
+            tc_mma_bf16(d_tmem, da + 2u * kk, db + 2u * kk, idesc, (kc | kk) != 0);
           }
           tc_commit(empty_bar(stage));
           if (++stage == L::STAGES) {
@@ -488,13 +466,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-    const uint32_t stg = cbase + L::CTRL_BYTES + static_cast<uint32_t>(warp - 2) * 8192u;
-    int acc = 0, it = 0;
+    int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
       int b, mt, nt;
-      if (!decode_tile<MODE>(a, tile, b, mt, nt)) continue;
+      decode_maxsim_tile(a, tile, b, mt, nt);
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
         ok = false;
         break;
@@ -503,24 +480,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr =
           tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
       const int row = mt * BM + quarter * 32 + lane;
-      if constexpr (MODE == MODE_MAXSIM) {
-        float *red_acc = red + acc * kRedGroups * kRedCands;
-        const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
-        epi_maxsim_rows<SPLIT_S>(taddr, lane, quarter, red_acc, rs + nt * BN, rs[row]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(red_bar(acc));
-        if (warp == 2) {
-          // leader warp: combine the four warps' partial sums
-          if (!mbar_wait(red_bar(acc), acc_phase, abort_flag)) {
-            ok = false;
-          } else {
-            epi_maxsim_write<SPLIT_S>(a, red_acc, lane, b, mt, nt);
-          }
+      float *red_acc = red + acc * kRedGroups * kRedCands;
+      const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
+      epi_maxsim_rows<SPLIT_S>(taddr, lane, quarter, red_acc, rs + nt * BN, rs[row]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(red_bar(acc));
+      if (warp == 2) {
+        // leader warp: combine the four warps' partial sums
+        if (!mbar_wait(red_bar(acc), acc_phase, abort_flag)) {
+          ok = false;
+        } else {
+          epi_maxsim_write<SPLIT_S>(a, red_acc, lane, b, mt, nt);
         }
-      } else if constexpr (MODE == MODE_ENRICH) {
-        epi_enrich(a, &tmO0, &tmO1, taddr, row - lane, lane, nt, stg, it);
-      } else {
-        epi_fuse(a, &tmO0, &tmO1, &tmO2, taddr, row - lane, lane, nt, stg, it);
       }
       tc_fence_before();
       __syncwarp();
@@ -533,7 +504,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       *abort_flag = 1;
       record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
     }
-    if ((MODE == MODE_ENRICH || MODE == MODE_FUSE) && lane == 0) bulk_wait_all();  // outputs written
   }
 
   tc_fence_before();
@@ -544,24 +514,306 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int MODE, int A_PLANES, int SPLIT_S>
-avey_status run_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
-                   const CUtensorMap &o0, const CUtensorMap &o1, const CUtensorMap &o2, TcArgs args,
-                   cudaStream_t st, const char *name, const CUtensorMap *c0 = nullptr,
-                   const CUtensorMap *c1 = nullptr) {
-  using L = Layout<A_PLANES>;
+// ---- layer GEMMs on CTA pairs ------------------------------------------------
+//
+// The enricher and the fuser on clusters of two CTAs (tcgen05 cta_group::2):
+// a pair owns a 256 x 256 output tile.  Each CTA keeps 128 of its rows in
+// TMEM, loads those rows of both activation planes and one 128-row half of
+// the weight tile, and CTA 0 issues M = 256, N = 256, K = 16 MMAs that read
+// the activation rows and both weight halves across the pair.  Per FLOP each
+// SM moves a quarter fewer operand bytes from L2 than with 128 x 256 tiles on
+// one SM, and four 48 KB stages cover a third more load latency than three
+// of 64 KB.  The epilogues are the single-CTA ones, each CTA on its own rows.
+//
+// Barriers: both CTAs' loads complete on CTA 0's "full" barrier; the MMA
+// commit frees the stage in both CTAs and publishes the accumulator to both;
+// both CTAs' epilogue warps release the accumulator to CTA 0.  No load uses
+// multicast.
+
+struct PairLayout {
+  static constexpr int PM = 256;                        // rows per pair tile
+  static constexpr uint32_t A_BYTES = 128 * BK * 2;     // one plane, this CTA's rows
+  static constexpr uint32_t B_BYTES = 128 * BK * 2;     // this CTA's half of the weight tile
+  static constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + B_BYTES;
+  static constexpr int STAGES = 4;
+  static constexpr uint32_t TILES_BYTES = STAGES * STAGE_BYTES;
+  static constexpr uint32_t CTRL_BYTES = 1024;
+  static constexpr uint32_t STAGING_BYTES = kEpi * 8192;
+  static constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + STAGING_BYTES + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(STAGES <= 8, "the control block holds at most 8 stages");
+};
+
+__device__ __forceinline__ void wait_drain_pair(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    layer_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmO0,
+                      const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2,
+                      const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
+                      const TcArgs a) {
+  static_assert(MODE == MODE_ENRICH || MODE == MODE_FUSE, "layer GEMMs only");
+  using P = PairLayout;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t *ctrl = smem_raw + pad + P::TILES_BYTES;
+  const uint32_t sbase = raw_s + pad;
+  const uint32_t cbase = sbase + P::TILES_BYTES;
+  // control block: full[8] @0, empty[8] @64, tfull[2] @128, tempty[2] @144,
+  // drain @160, tmem base @168, abort flag @172
+  auto full_bar = [&](int s) { return cbase + 8u * s; };
+  auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
+  auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
+  auto tempty_bar = [&](int i) { return cbase + 144u + 8u * i; };
+  const uint32_t drain_bar = cbase + 160u;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 168);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 172);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), 2 * kEpi);  // both CTAs' epilogue warps (used in CTA 0)
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA0);
+    prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmO0);
+    prefetch_tmap(&tmO1);
+    if (MODE == MODE_FUSE) prefetch_tmap(&tmO2);
+    if (MODE == MODE_FUSE && a.k_split > 0) {
+      prefetch_tmap(&tmC0);
+      prefetch_tmap(&tmC1);
+    }
+  }
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote use
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(ctrl + 168), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int kchunks = (a.kdim + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < a.num_tiles && ok; tile += npairs) {
+        const int mt = tile / a.tiles_n, nt = tile - (tile / a.tiles_n) * a.tiles_n;
+        const int arow = mt * P::PM + static_cast<int>(rank) * 128;
+        const int brow = nt * BN + static_cast<int>(rank) * 128;
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * P::STAGE_BYTES);
+          const uint32_t full0 = mapa_shared(full_bar(stage), 0);
+          const uint32_t st = sbase + stage * P::STAGE_BYTES;
+          // fuser with a separate contextualizer output: [Z_h || c] from two
+          // sources, split at a multiple of the K chunk
+          const bool from_c = MODE == MODE_FUSE && a.k_split > 0 && kc * BK >= a.k_split;
+          const CUtensorMap *ma = from_c ? &tmC0 : &tmA0;
+          const CUtensorMap *mal = from_c ? &tmC1 : &tmA1;
+          const int ax = from_c ? kc * BK - a.k_split : kc * BK;
+          tma_load_3d_pair(st, ma, full0, ax, arow, 0);
+          tma_load_3d_pair(st + P::A_BYTES, mal, full0, ax, arow, 0);
+          tma_load_3d_pair(st + 2 * P::A_BYTES, &tmB, full0, kc * BK, brow, 0);
+          ++issued;
+          if (++stage == P::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      // Drain: the pair's MMA has consumed (so the loads have landed in) every
+      // stage this CTA filled once its last use is released.
+      for (int s = 0; s < P::STAGES; ++s) {
+        if (issued > s) {
+          const long long last = ((issued - 1 - s) / P::STAGES) * P::STAGES + s;
+          wait_drain_pair(empty_bar(s), static_cast<uint32_t>((last / P::STAGES) & 1));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------- MMA issue (CTA 0)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(P::PM, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < a.num_tiles && ok; tile += npairs) {
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + stage * P::STAGE_BYTES;
+          const uint64_t da0 = sdesc_k_sw128(st);
+          const uint64_t da1 = sdesc_k_sw128(st + P::A_BYTES);
+          const uint64_t db = sdesc_k_sw128(st + 2 * P::A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            tc_mma_bf16_pair(d_tmem, da0 + 2u * kk, db + 2u * kk, idesc, (kc | kk) != 0);
+            tc_mma_bf16_pair(d_tmem, da1 + 2u * kk, db + 2u * kk, idesc, 1u);
+          }
+          tc_commit_pair_both(empty_bar(stage));
+          if (++stage == P::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(tfull_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      tc_commit_pair_both(drain_bar);
+      wait_drain_pair(drain_bar, 0);
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const uint32_t stg = cbase + P::CTRL_BYTES + static_cast<uint32_t>(warp - 2) * 8192u;
+    const uint32_t tempty_r0 = mapa_shared(tempty_bar(0), 0), tempty_r1 = mapa_shared(tempty_bar(1), 0);
+    int acc = 0, it = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < a.num_tiles; tile += npairs) {
+      const int mt = tile / a.tiles_n, nt = tile - (tile / a.tiles_n) * a.tiles_n;
+      const int row0 = mt * P::PM + static_cast<int>(rank) * 128 + quarter * 32;
+      float4 xi[8];
+      if constexpr (MODE == MODE_FUSE) fuse_load_residual(a, row0 + lane, nt * BN, xi);
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr =
+          tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
+      if constexpr (MODE == MODE_ENRICH) {
+        epi_enrich(a, &tmO0, &tmO1, taddr, row0, lane, nt, stg, it);
+      } else {
+        epi_fuse(a, &tmO0, &tmO1, &tmO2, taddr, row0, lane, nt, stg, it, xi);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_r1 : tempty_r0);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+    }
+    if (lane == 0) bulk_wait_all();  // outputs written
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // Both CTAs past their loops: the pair's MMAs have drained (CTA 0 waited on
+  // the drain commit) and no remote arrival is still on its way.
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+  cluster_sync_all();
+}
+
+template <int MODE>
+avey_status run_layer_pair(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+                           const CUtensorMap &o0, const CUtensorMap &o1, const CUtensorMap &o2,
+                           const CUtensorMap &c0, const CUtensorMap &c1, TcArgs args, cudaStream_t st,
+                           const char *name) {
+  using P = PairLayout;
   if (args.num_tiles <= 0) return AVEY_OK;
-  auto kern = tc_kernel<MODE, A_PLANES, SPLIT_S>;
+  auto kern = layer_pair_kernel<MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(L::SMEM_BYTES));
+                                       static_cast<int>(P::SMEM_BYTES));
   if (e != cudaSuccess) {
     set_detail("%s: cudaFuncSetAttribute: %s", name, cudaGetErrorString(e));
     return AVEY_ERR_CUDA;
   }
-  const int grid = std::min(args.num_tiles, sm_count());
-  kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(a0, a1, b, o0, o1, o2, c0 ? *c0 : a0, c1 ? *c1 : a1,
-                                              args);
+  // Persistent grid: as many pairs as can be resident at once (a pair needs
+  // two SMs of one GPC, so this can be below half the SM count).
+  static int resident[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &cap = resident[dev & 63];
+  if (cap == 0) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * (sm_count() / 2));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = P::SMEM_BYTES;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    if (e != cudaSuccess || clusters < 1) {
+      set_detail("%s: no resident CTA pair (%s)", name, cudaGetErrorString(e));
+      return AVEY_ERR_CUDA;
+    }
+    cap = std::min(clusters, sm_count() / 2);
+  }
+  const int pairs = std::max(1, std::min(args.num_tiles, cap));
+  kern<<<2 * pairs, kThreads, P::SMEM_BYTES, st>>>(a0, a1, b, o0, o1, o2, c0, c1, args);
   AVEY_CHECK_LAUNCH(name);
+  return AVEY_OK;
+}
+
+template <int SPLIT_S>
+avey_status run_maxsim_tc(const CUtensorMap &ma, const CUtensorMap &mb, TcArgs args, cudaStream_t st) {
+  using L = MaxSimLayout;
+  if (args.num_tiles <= 0) return AVEY_OK;
+  auto kern = maxsim_tc_kernel<SPLIT_S>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::SMEM_BYTES));
+  if (e != cudaSuccess) {
+    set_detail("maxsim_tc: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return AVEY_ERR_CUDA;
+  }
+  const int grid = std::min(args.num_tiles, sm_count());
+  kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(ma, mb, args);
+  AVEY_CHECK_LAUNCH("maxsim_tc");
   return AVEY_OK;
 }
 
@@ -575,6 +827,14 @@ TcArgs base_args(int rows, int cols, int kdim) {
   a.num_tiles = a.tiles_m * a.tiles_n;
   a.group_m = 1;
   a.status = device_status_word();
+  return a;
+}
+
+// Pair tiles: 256 rows (two CTAs of 128) x 256 output columns.
+TcArgs pair_args(int rows, int cols, int kdim) {
+  TcArgs a = base_args(rows, cols, kdim);
+  a.tiles_m = (rows + PairLayout::PM - 1) / PairLayout::PM;
+  a.num_tiles = a.tiles_m * a.tiles_n;
   return a;
 }
 
@@ -597,7 +857,7 @@ avey_status launch_maxsim_tc(const bf16 *x, const float *inv_norm, int B, int N,
   a.inv_norm = inv_norm;
   a.rs_ld = rs_ld;
   switch (S) {
-    case 16: return run_tc<MODE_MAXSIM, 1, 16>(ma, ma, mb, ma, ma, ma, a, s, "maxsim_tc");
+    case 16: return run_maxsim_tc<16>(ma, mb, a, s);
     default:
       set_detail("maxsim_tc: S=%d unsupported (16; larger splits use the CTA-pair kernel)", S);
       return AVEY_ERR_UNSUPPORTED;
@@ -611,16 +871,16 @@ avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, con
   const uint64_t rs = static_cast<uint64_t>(d) * 2, zs = static_cast<uint64_t>(m) * 2;
   if (!encode_bf16_map(&a0, xhi, d, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&a1, xlo, d, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
-  if (!encode_bf16_map(&mb, Ut, d, m, 1, rs, rs * m, BN)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&mb, Ut, d, m, 1, rs, rs * m, 128)) return AVEY_ERR_CUDA;
   if (!encode_map(&o0, false, zhi, m, T, 1, zs, zs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
   if (!encode_map(&o1, false, zlo, m, T, 1, zs, zs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
-  TcArgs a = base_args(T, m, d);
+  TcArgs a = pair_args(T, m, d);
   a.bias = bias;
   a.inv_rms = inv_rms;
   a.out_hi = zhi;
   a.out_lo = zlo;
   a.ld_out = m;
-  return run_tc<MODE_ENRICH, 2, 0>(a0, a1, mb, o0, o1, o1, a, s, "enrich_tc");
+  return run_layer_pair<MODE_ENRICH>(a0, a1, mb, o0, o1, o1, a0, a1, a, s, "enrich_tc");
 }
 
 avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
@@ -631,7 +891,7 @@ avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const
   const uint64_t fs = static_cast<uint64_t>(d) * 4, hs = static_cast<uint64_t>(d) * 2;
   if (!encode_bf16_map(&a0, ahi, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&a1, alo, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
-  if (!encode_bf16_map(&mb, Ot, m, d, 1, rs, rs * d, BN)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&mb, Ot, m, d, 1, rs, rs * d, 128)) return AVEY_ERR_CUDA;
   if (!encode_map(&o0, true, x_out, d, T, 1, fs, fs * T, 32, 32, 128)) return AVEY_ERR_CUDA;
   o1 = o0;
   o2 = o0;
@@ -639,7 +899,7 @@ avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const
     if (!encode_map(&o1, false, xo_hi, d, T, 1, hs, hs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
     if (!encode_map(&o2, false, xo_lo, d, T, 1, hs, hs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
   }
-  TcArgs a = base_args(T, d, m);
+  TcArgs a = pair_args(T, d, m);
   a.x_in = x_in;
   a.x_out = x_out;
   a.out_hi = xo_hi;
@@ -655,9 +915,9 @@ avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const
     if (!encode_bf16_map(&c0, chi, m - k_split, T, 1, cs, cs * T, BM)) return AVEY_ERR_CUDA;
     if (!encode_bf16_map(&c1, clo, m - k_split, T, 1, cs, cs * T, BM)) return AVEY_ERR_CUDA;
     a.k_split = k_split;
-    return run_tc<MODE_FUSE, 2, 0>(a0, a1, mb, o0, o1, o2, a, s, "fuse_tc", &c0, &c1);
+    return run_layer_pair<MODE_FUSE>(a0, a1, mb, o0, o1, o2, c0, c1, a, s, "fuse_tc");
   }
-  return run_tc<MODE_FUSE, 2, 0>(a0, a1, mb, o0, o1, o2, a, s, "fuse_tc");
+  return run_layer_pair<MODE_FUSE>(a0, a1, mb, o0, o1, o2, a0, a1, a, s, "fuse_tc");
 }
 
 }  // namespace avey
