@@ -15,8 +15,9 @@
 // store 32 consecutive features).
 // The kernel is bound by HBM: (k+1) gathered 64 x d bf16 blocks in, 64 x d x 8
 // bytes out per split; eight stages of 24 KB keep 192 KB of loads in flight.
-// Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue, warps 2-5
-// epilogue (one per TMEM lane quarter = 32 features).  Every wait is bounded.
+// Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue, warps 2-9
+// epilogue (two per TMEM lane quarter = 32 features, each on 32 of the
+// split's 64 tokens).  Every wait is bounded.
 #include <algorithm>
 
 #include "avey_common.cuh"
@@ -27,15 +28,16 @@ namespace {
 
 constexpr int CS = 64;                        // split size handled here
 constexpr int CF = 128;                       // features per tile (M)
-constexpr int C_EPI = 4, C_THR = 64 + 32 * C_EPI;
+constexpr int C_EPI = 8, C_THR = 64 + 32 * C_EPI;
+constexpr int C_TOK = CS / 2;                 // tokens per epilogue warp
 constexpr uint32_t C_XBOX = 64 * CS * 2;      // 8 KB: 64 features x 64 tokens
 constexpr uint32_t C_PBOX = CS * CS * 2;      // 8 KB: P_r, 64 i x 64 j
 constexpr uint32_t C_STAGE = 2 * C_XBOX + C_PBOX;
 constexpr int C_STAGES = 6;
 constexpr int C_NACC = 8;                     // TMEM buffers of 64 columns
 constexpr uint32_t C_IDENT = CS * CS * 2;     // 8 KB: the 64 x 64 identity (B operand)
-constexpr uint32_t C_W32 = CS * 32 * 4;       // 8 KB: one warp's fp32 output [64 i][32 f]
-constexpr uint32_t C_W16 = CS * 32 * 2;       // 4 KB: one bf16 plane of it
+constexpr uint32_t C_W32 = C_TOK * 32 * 4;    // 4 KB: one warp's fp32 output [32 i][32 f]
+constexpr uint32_t C_W16 = C_TOK * 32 * 2;    // 2 KB: one bf16 plane of it
 constexpr uint32_t C_WSTG = C_W32 + 2 * C_W16;
 constexpr uint32_t C_SMEM = C_STAGES * C_STAGE + C_IDENT + C_EPI * C_WSTG + 1024 + 1024;
 static_assert(C_SMEM <= 232448, "shared memory budget");
@@ -266,7 +268,8 @@ __global__ void __launch_bounds__(C_THR, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int quarter = warp & 3;  // TMEM lanes = features 32*quarter .. +31 of the slab
+    const int quarter = warp & 3;      // TMEM lanes = features 32*quarter .. +31 of the slab
+    const int half = (warp - 2) >> 2;  // TMEM columns = tokens 32*half .. +31 of the split
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -275,9 +278,9 @@ __global__ void __launch_bounds__(C_THR, 1)
       const int slab = static_cast<int>(tile - seg * a.nslab);
       const int b = static_cast<int>(seg / a.nr);
       const int t = a.t0 + static_cast<int>(seg - static_cast<long long>(b) * a.nr);
-      float o[CS];
+      float o[C_TOK];
 #pragma unroll
-      for (int i = 0; i < CS; ++i) o[i] = 0.f;
+      for (int i = 0; i < C_TOK; ++i) o[i] = 0.f;
       int cl[KM];
       float wl[KM];
       block_list<KM>(a, seg, t, false, cl, wl);
@@ -290,20 +293,22 @@ __global__ void __launch_bounds__(C_THR, 1)
           continue;
         }
         tc_fence_after();
-        float v[64];
-        tmem_ld64(tmem_base + static_cast<uint32_t>(acc * 64) + (static_cast<uint32_t>(quarter * 32) << 16), v);
+        float v[C_TOK];
+        tmem_ld32(tmem_base + static_cast<uint32_t>(acc * 64 + half * C_TOK) +
+                      (static_cast<uint32_t>(quarter * 32) << 16),
+                  v);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty_bar(acc));
 #pragma unroll
-        for (int i = 0; i < CS; ++i) o[i] = fmaf(wr, v[i], o[i]);
+        for (int i = 0; i < C_TOK; ++i) o[i] = fmaf(wr, v[i], o[i]);
         if (++acc == C_NACC) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       if (!ok) break;
-      // fp32 out and the split pair: each warp stages its 32 features x 64
+      // fp32 out and the split pair: each warp stages its 32 features x 32
       // tokens and writes them with its own three TMA stores (the tensor's
       // bounds clip the feature tail)
       uint8_t *wst = ostage + (warp - 2) * C_WSTG;
@@ -315,7 +320,7 @@ __global__ void __launch_bounds__(C_THR, 1)
         bf16 *oh = reinterpret_cast<bf16 *>(wst + C_W32);
         bf16 *ol = reinterpret_cast<bf16 *>(wst + C_W32 + C_W16);
 #pragma unroll
-        for (int i = 0; i < CS; ++i) {
+        for (int i = 0; i < C_TOK; ++i) {
           const float y = o[i];
           const bf16 h = __float2bfloat16_rn(y);
           o32[i * 32 + lane] = y;
@@ -326,7 +331,7 @@ __global__ void __launch_bounds__(C_THR, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        const int orow = static_cast<int>(seg * CS), ox = slab * CF + quarter * 32;
+        const int orow = static_cast<int>(seg * CS) + half * C_TOK, ox = slab * CF + quarter * 32;
         tma_store_3d(&tmO, wsa, ox, orow, 0);
         if (a.out_hi) {
           tma_store_3d(&tmOh, wsa + C_W32, ox, orow, 0);
@@ -399,16 +404,16 @@ avey_status launch_compress_tc(const bf16 *x, int B, int N, int d, int k, int t0
   a.out_lo = lo;
   a.status = device_status_word();
   const int grid = std::max(1, std::min(a.num_tiles, sm_count()));
-  // outputs [B*nr*64 rows, d]: fp32 and the bf16 planes, dense boxes of 32 x 64
+  // outputs [B*nr*64 rows, d]: fp32 and the bf16 planes, dense boxes of 32 x 32
   CUtensorMap mo, moh, mol;
   const uint64_t orows = static_cast<uint64_t>(B) * nr * CS;
   const uint64_t o4 = static_cast<uint64_t>(d) * 4, o2 = static_cast<uint64_t>(d) * 2;
-  if (!encode_map(&mo, true, out, d, orows, 1, o4, o4 * orows, 32, CS, 0)) return AVEY_ERR_CUDA;
+  if (!encode_map(&mo, true, out, d, orows, 1, o4, o4 * orows, 32, C_TOK, 0)) return AVEY_ERR_CUDA;
   moh = mo;
   mol = mo;
   if (hi) {
-    if (!encode_map(&moh, false, hi, d, orows, 1, o2, o2 * orows, 32, CS, 0)) return AVEY_ERR_CUDA;
-    if (!encode_map(&mol, false, lo, d, orows, 1, o2, o2 * orows, 32, CS, 0)) return AVEY_ERR_CUDA;
+    if (!encode_map(&moh, false, hi, d, orows, 1, o2, o2 * orows, 32, C_TOK, 0)) return AVEY_ERR_CUDA;
+    if (!encode_map(&mol, false, lo, d, orows, 1, o2, o2 * orows, 32, C_TOK, 0)) return AVEY_ERR_CUDA;
   }
   if (k + 1 <= 8) return run_compress_tc<8>(mx, mp, mo, moh, mol, a, grid, s);
   if (k + 1 <= 16) return run_compress_tc<16>(mx, mp, mo, moh, mol, a, grid, s);
