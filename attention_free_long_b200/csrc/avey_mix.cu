@@ -16,7 +16,7 @@
 //                      and fp32 row sums of squares, so G is the cosine matrix
 //                      of the hi vectors (within about 1e-4 of the exact one);
 //                   2. G = R / (n_i n_j), row sums, Gt in fp32, split to bf16
-//                      hi/lo in shared memory;
+//                      hi/lo in shared memory (all threads, 256 / S per row);
 //                   3. c = Gt_hi Z_hi + Gt_lo Z_hi + Gt_hi Z_lo, split pair out.
 // fp32 path: plain SIMT kernels.
 #include <algorithm>
@@ -149,7 +149,7 @@ struct DynTile {
   static constexpr int GLD = S + 8;             // bf16 Gt row
   static constexpr int GBYTES = S * GLD * 2;
   static constexpr int FLD = S + 4;             // fp32 G row
-  static constexpr int TR = 256 / S;            // threads per row for sums of squares
+  static constexpr int TR = 256 / S;            // threads per row (sums of squares, eq. 6)
   static constexpr int SMEM = 2 * BUF + 2 * GBYTES;
   static_assert(S * FLD * 4 <= 2 * BUF, "fp32 G must fit in the chunk buffers");
 };
@@ -170,7 +170,6 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
   uint8_t *gtl = gth + C::GBYTES;             // Gt lo
   __shared__ float s_ss[S * C::TR];
   __shared__ float s_nf[S];
-  __shared__ float s_den[S];
   const int blk = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bf16 *zb = zt + static_cast<long long>(blk) * S * ld_zt;
@@ -265,28 +264,37 @@ __global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long 
     s_nf[tid] = fmaxf(sqrtf(t2), 1e-12f);
   }
   __syncthreads();
-  if (tid < S) {
-    const float ni = s_nf[tid];
+  {
+    // All 256 threads: TR consecutive threads per row i, S / TR columns each.
+    // The cosines, the row sum (a shuffle reduction among the row's threads)
+    // and Gt = G / (row sum + eps) as a split pair, in one step.
+    constexpr int CPT = S / C::TR;
+    const int i = tid / C::TR, part = tid % C::TR;
+    const float ni = s_nf[i];
+    float v[CPT];
     float rs = 0.f;
-    for (int j = 0; j < S; ++j) {
-      const float v = G[tid * C::FLD + j] / (ni * s_nf[j]);
-      G[tid * C::FLD + j] = v;
-      rs += v;
+#pragma unroll
+    for (int q = 0; q < CPT; ++q) {
+      const int j = part * CPT + q;
+      v[q] = G[i * C::FLD + j] / (ni * s_nf[j]);
+      rs += v[q];
     }
-    s_den[tid] = rs + eps;
-  }
-  __syncthreads();
-  for (int e = tid; e < S * S; e += 256) {
-    const int i = e / S, j = e % S;
-    float v;
-    if constexpr (COUPLED)
-      v = j <= i ? __bfloat162float(V[i * S + j]) * G[i * C::FLD + j] : 0.f;
-    else
-      v = G[i * C::FLD + j] / s_den[i];
-    float hi, lo;
-    split_bf16(v, hi, lo);
-    reinterpret_cast<bf16 *>(gth)[i * C::GLD + j] = __float2bfloat16_rn(hi);
-    reinterpret_cast<bf16 *>(gtl)[i * C::GLD + j] = __float2bfloat16_rn(lo);
+#pragma unroll
+    for (int off = 1; off < C::TR; off <<= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
+    const float den = rs + eps;
+#pragma unroll
+    for (int q = 0; q < CPT; ++q) {
+      const int j = part * CPT + q;
+      float out;
+      if constexpr (COUPLED)
+        out = j <= i ? __bfloat162float(V[i * S + j]) * v[q] : 0.f;
+      else
+        out = v[q] / den;
+      float hi, lo;
+      split_bf16(out, hi, lo);
+      reinterpret_cast<bf16 *>(gth)[i * C::GLD + j] = __float2bfloat16_rn(hi);
+      reinterpret_cast<bf16 *>(gtl)[i * C::GLD + j] = __float2bfloat16_rn(lo);
+    }
   }
   __syncthreads();
 
