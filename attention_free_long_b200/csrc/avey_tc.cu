@@ -544,13 +544,6 @@ struct PairLayout {
   static_assert(STAGES <= 8, "the control block holds at most 8 stages");
 };
 
-__device__ __forceinline__ void wait_drain_pair(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-  }
-}
-
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     layer_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -660,7 +653,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int s = 0; s < P::STAGES; ++s) {
         if (issued > s) {
           const long long last = ((issued - 1 - s) / P::STAGES) * P::STAGES + s;
-          wait_drain_pair(empty_bar(s), static_cast<uint32_t>((last / P::STAGES) & 1));
+          mbar_wait_drain(empty_bar(s), static_cast<uint32_t>((last / P::STAGES) & 1));
         }
       }
     }
@@ -709,7 +702,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
       }
       tc_commit_pair_both(drain_bar);
-      wait_drain_pair(drain_bar, 0);
+      mbar_wait_drain(drain_bar, 0);
     }
   } else {
     // ------------------------------------------------------------- epilogue

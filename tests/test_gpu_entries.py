@@ -69,3 +69,10 @@ def test_topk_entry_point(n, k, causal, cuda_dev):
     o_idx, o_w = orc.topk(rows, targets, k, causal)
     np.testing.assert_array_equal(g_idx.reshape(B * n, k), o_idx)
     np.testing.assert_allclose(g_w.reshape(B * n, k), o_w, rtol=2e-7, atol=0)
+
+
+def test_smoke_entry_passes(cuda_dev):
+    # the build's one-call smoke check: rank, compression and two layers on
+    # cuda:0 against the oracle
+    import __graft_entry__ as ge
+    ge.smoke()
