@@ -298,26 +298,35 @@ def layer_workspace_bytes(dtype: int, T: int, d: int, m: int, prenorm: bool, S: 
 
 
 def avey_layer_forward(layer: DeviceLayer, S: int, m_h: int, eps: float, prenorm: bool,
-                       x_in: torch.Tensor, x_in_lowp: Optional[torch.Tensor] = None,
+                       x_in: Optional[torch.Tensor], x_in_lowp: Optional[torch.Tensor] = None,
                        x_out: Optional[torch.Tensor] = None, lowp_out: bool = True,
                        x_out_lowp: Optional[torch.Tensor] = None,
-                       ws: Optional[torch.Tensor] = None):
+                       ws: Optional[torch.Tensor] = None, fp32_out: bool = True):
     """One layer on x_in fp32 [T, d] (any leading shape that flattens to T rows).
 
-    Returns (x_out fp32, x_out_lowp pair or None).
+    For a bf16 layer, x_in may be None when x_in_lowp (the split pair
+    [2, T, d]) is given: the residual is then hi + lo.  fp32_out=False writes
+    only the pair.  Returns (x_out fp32 or None, x_out_lowp pair or None).
     """
-    _need(x_in, "x_in")
-    d = x_in.shape[-1]
-    T = x_in.numel() // d
     m = layer.Ut.shape[0]
     dt = _dt(layer.Ut)
-    if x_out is None:
-        x_out = torch.empty_like(x_in)
+    if x_in is None:
+        _need(x_in_lowp, "x_in_lowp")
+        d = x_in_lowp.shape[-1]
+        T = x_in_lowp.numel() // (2 * d)
+        dev = x_in_lowp.device
+    else:
+        _need(x_in, "x_in")
+        d = x_in.shape[-1]
+        T = x_in.numel() // d
+        dev = x_in.device
+    if x_out is None and fp32_out:
+        x_out = torch.empty_like(x_in) if x_in is not None else torch.empty((T, d), device=dev)
     if dt == AVEY_BF16 and lowp_out and x_out_lowp is None:
-        x_out_lowp = torch.empty((2, T, d), dtype=torch.bfloat16, device=x_in.device)
+        x_out_lowp = torch.empty((2, T, d), dtype=torch.bfloat16, device=dev)
     need = layer_workspace_bytes(dt, T, d, m, prenorm, S, layer.kind)
     if ws is None or ws.numel() < need:
-        ws = _ws(need, x_in.device)
+        ws = _ws(need, dev)
     p = LayerParams(layer.kind, d, m, m_h, S, eps, int(bool(prenorm)), layer.Ut.data_ptr(),
                     layer.bU.data_ptr(), None if layer.V is None else layer.V.data_ptr(),
                     layer.Ot.data_ptr())
@@ -374,6 +383,34 @@ def make_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: torch.
     return EncoderWorkspace(rank_ws, layer_ws, idx, w, x0, x1, pair0, pair1)
 
 
+def _pair_stream(dt: int, layers) -> bool:
+    """bf16 stacks pass the residual stream between the calls as its split pair
+    alone; fp32 is written once, by the last layer."""
+    return dt == AVEY_BF16 and len(layers) > 0
+
+
+def _run_layers(L, layers, dt, T, d, m, m_h, S, eps, prenorm, ws, st, marks):
+    """Every layer over the stream in (ws.x0, ws.pair0); returns the fp32 output
+    buffer.  ``marks[3 + li]`` is recorded after layer li."""
+    pair_only = _pair_stream(dt, layers)
+    cur, nxt = (ws.x0, ws.pair0), (ws.x1, ws.pair1)
+    for li, lay in enumerate(layers):
+        last = li == len(layers) - 1
+        p = LayerParams(lay.kind, d, m, m_h, S, eps, int(bool(prenorm)), lay.Ut.data_ptr(),
+                        lay.bU.data_ptr(), None if lay.V is None else lay.V.data_ptr(),
+                        lay.Ot.data_ptr())
+        x_in = None if pair_only else _ptr(cur[0])
+        x_out = _ptr(nxt[0]) if (last or not pair_only) else None
+        x_out_lowp = None if (last and pair_only) else _ptr(nxt[1])
+        _check("avey_layer_forward",
+               L.avey_layer_forward(ctypes.byref(p), dt, T, x_in, _ptr(cur[1]), x_out, x_out_lowp,
+                                    _ptr(ws.layer_ws), ws.layer_ws.numel(), st))
+        if marks is not None:
+            marks[3 + li].record()
+        cur, nxt = nxt, cur
+    return cur[0]
+
+
 def encoder_forward(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLayer], S: int, k: int,
                     m_h: int, eps: float, prenorm: bool,
                     ws: Optional[EncoderWorkspace] = None, marks=None,
@@ -401,22 +438,12 @@ def encoder_forward(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLay
     if marks is not None:
         marks[1].record()
     _check("avey_compress", L.avey_compress(_ptr(x), dt, B, N, d, S, k, _ptr(ws.idx), _ptr(ws.w),
-                                            _ptr(P), _ptr(ws.x0), _ptr(ws.pair0), st))
+                                            _ptr(P), None if _pair_stream(dt, layers) else _ptr(ws.x0),
+                                            _ptr(ws.pair0), st))
     if marks is not None:
         marks[2].record()
-    cur, nxt = (ws.x0, ws.pair0), (ws.x1, ws.pair1)
-    for li, lay in enumerate(layers):
-        p = LayerParams(lay.kind, d, m, m_h, S, eps, int(bool(prenorm)), lay.Ut.data_ptr(),
-                        lay.bU.data_ptr(), None if lay.V is None else lay.V.data_ptr(),
-                        lay.Ot.data_ptr())
-        _check("avey_layer_forward",
-               L.avey_layer_forward(ctypes.byref(p), dt, T, _ptr(cur[0]), _ptr(cur[1]),
-                                    _ptr(nxt[0]), _ptr(nxt[1]), _ptr(ws.layer_ws),
-                                    ws.layer_ws.numel(), st))
-        if marks is not None:
-            marks[3 + li].record()
-        cur, nxt = nxt, cur
-    return cur[0].view(B, n * S, d)
+    out = _run_layers(L, layers, dt, T, d, m, m_h, S, eps, prenorm, ws, st, marks)
+    return out.view(B, n * S, d)
 
 
 def encoder_forward_uncompressed(x: torch.Tensor, layers: Sequence[DeviceLayer], S: int, k: int,
@@ -571,21 +598,10 @@ def encoder_forward_sharded(x: torch.Tensor, P: torch.Tensor, layers: Sequence[D
     flags = AVEY_RANK_UNIDIRECTIONAL if causal else 0
     _check("avey_topk_rows", L.avey_topk_rows(_ptr(ws.scores), B, n, t0, t1, k, flags, _ptr(ws.idx),
                                               _ptr(ws.w), st))
-    _check("avey_compress_rows", L.avey_compress_rows(_ptr(x), dt, B, N, d, S, k, t0, t1,
-                                                      _ptr(ws.idx), _ptr(ws.w), _ptr(P),
-                                                      _ptr(ws.x0), _ptr(ws.pair0), st))
+    _check("avey_compress_rows", L.avey_compress_rows(
+        _ptr(x), dt, B, N, d, S, k, t0, t1, _ptr(ws.idx), _ptr(ws.w), _ptr(P),
+        None if _pair_stream(dt, layers) else _ptr(ws.x0), _ptr(ws.pair0), st))
     if marks is not None:
         marks[2].record()
-    cur, nxt = (ws.x0, ws.pair0), (ws.x1, ws.pair1)
-    for li, lay in enumerate(layers):
-        p = LayerParams(lay.kind, d, m, m_h, S, eps, int(bool(prenorm)), lay.Ut.data_ptr(),
-                        lay.bU.data_ptr(), None if lay.V is None else lay.V.data_ptr(),
-                        lay.Ot.data_ptr())
-        _check("avey_layer_forward",
-               L.avey_layer_forward(ctypes.byref(p), dt, T, _ptr(cur[0]), _ptr(cur[1]),
-                                    _ptr(nxt[0]), _ptr(nxt[1]), _ptr(ws.layer_ws),
-                                    ws.layer_ws.numel(), st))
-        if marks is not None:
-            marks[3 + li].record()
-        cur, nxt = nxt, cur
-    return cur[0][:T].view(B, (t1 - t0) * S, d)
+    out = _run_layers(L, layers, dt, T, d, m, m_h, S, eps, prenorm, ws, st, marks)
+    return out[:T].view(B, (t1 - t0) * S, d)

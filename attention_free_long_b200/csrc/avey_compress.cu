@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(256) compress_bf16(const bf16 *__restrict__ x,
       }
   __syncthreads();
   const long long row0 = (static_cast<long long>(b) * nr + tl) * S;
-  for (int e = tid; e < S * (C::NS / 4); e += 256) {
+  for (int e = tid; out != nullptr && e < S * (C::NS / 4); e += 256) {
     const int row = e / (C::NS / 4), cc = e % (C::NS / 4);
     const int col = q0 + cc * 4;
     if (col >= d) continue;
@@ -331,12 +331,14 @@ static avey_status compress_range(const void *x, avey_dtype dt, int B, int N, in
                                   const char *fn) {
   AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
                "%s: dtype %d unsupported (F32 or BF16)", fn, int(dt));
-  AVEY_REQUIRE(x && idx && w && P && out, AVEY_ERR_INVALID_ARG, "%s: null pointer", fn);
+  AVEY_REQUIRE(x && idx && w && P, AVEY_ERR_INVALID_ARG, "%s: null pointer", fn);
+  AVEY_REQUIRE(out || (dt == AVEY_BF16 && out_lowp), AVEY_ERR_INVALID_ARG,
+               "%s: out may be NULL only for AVEY_BF16 with out_lowp", fn);
   AVEY_REQUIRE(B >= 1 && N >= 1 && d >= 1 && S >= 1 && k >= 1, AVEY_ERR_INVALID_ARG,
                "%s: sizes must be >= 1", fn);
   AVEY_REQUIRE(d % 8 == 0, AVEY_ERR_INVALID_ARG, "%s: d=%d must be a multiple of 8", fn, d);
   AVEY_REQUIRE(k <= 32, AVEY_ERR_UNSUPPORTED, "%s: k=%d > 32", fn, k);
-  AVEY_REQUIRE(aligned16(x) && aligned16(P) && aligned16(out) && (!out_lowp || aligned16(out_lowp)),
+  AVEY_REQUIRE(aligned16(x) && aligned16(P) && (!out || aligned16(out)) && (!out_lowp || aligned16(out_lowp)),
                AVEY_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
   const int n = (N + S - 1) / S;
   AVEY_REQUIRE(0 <= t0 && t0 <= t1 && t1 <= n && t1 - t0 <= 65535, AVEY_ERR_INVALID_ARG,

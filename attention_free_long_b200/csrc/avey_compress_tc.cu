@@ -319,11 +319,12 @@ __global__ void __launch_bounds__(C_THR, 1)
         float *o32 = reinterpret_cast<float *>(wst);
         bf16 *oh = reinterpret_cast<bf16 *>(wst + C_W32);
         bf16 *ol = reinterpret_cast<bf16 *>(wst + C_W32 + C_W16);
+        const bool f32out = a.out != nullptr;
 #pragma unroll
         for (int i = 0; i < C_TOK; ++i) {
           const float y = o[i];
           const bf16 h = __float2bfloat16_rn(y);
-          o32[i * 32 + lane] = y;
+          if (f32out) o32[i * 32 + lane] = y;
           oh[i * 32 + lane] = h;
           ol[i * 32 + lane] = __float2bfloat16_rn(y - __bfloat162float(h));
         }
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(C_THR, 1)
       __syncwarp();
       if (lane == 0) {
         const int orow = static_cast<int>(seg * CS) + half * C_TOK, ox = slab * CF + quarter * 32;
-        tma_store_3d(&tmO, wsa, ox, orow, 0);
+        if (a.out) tma_store_3d(&tmO, wsa, ox, orow, 0);
         if (a.out_hi) {
           tma_store_3d(&tmOh, wsa + C_W32, ox, orow, 0);
           tma_store_3d(&tmOl, wsa + C_W32 + C_W16, ox, orow, 0);
@@ -408,13 +409,14 @@ avey_status launch_compress_tc(const bf16 *x, int B, int N, int d, int k, int t0
   CUtensorMap mo, moh, mol;
   const uint64_t orows = static_cast<uint64_t>(B) * nr * CS;
   const uint64_t o4 = static_cast<uint64_t>(d) * 4, o2 = static_cast<uint64_t>(d) * 2;
-  if (!encode_map(&mo, true, out, d, orows, 1, o4, o4 * orows, 32, C_TOK, 0)) return AVEY_ERR_CUDA;
-  moh = mo;
-  mol = mo;
+  if (out && !encode_map(&mo, true, out, d, orows, 1, o4, o4 * orows, 32, C_TOK, 0)) return AVEY_ERR_CUDA;
   if (hi) {
     if (!encode_map(&moh, false, hi, d, orows, 1, o2, o2 * orows, 32, C_TOK, 0)) return AVEY_ERR_CUDA;
     if (!encode_map(&mol, false, lo, d, orows, 1, o2, o2 * orows, 32, C_TOK, 0)) return AVEY_ERR_CUDA;
   }
+  // the kernel never uses the map of an output it does not write
+  if (!out) mo = moh;
+  if (!hi) moh = mol = mo;
   if (k + 1 <= 8) return run_compress_tc<8>(mx, mp, mo, moh, mol, a, grid, s);
   if (k + 1 <= 16) return run_compress_tc<16>(mx, mp, mo, moh, mol, a, grid, s);
   return run_compress_tc<32>(mx, mp, mo, moh, mol, a, grid, s);

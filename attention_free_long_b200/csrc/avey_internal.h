@@ -39,10 +39,12 @@ avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, con
 // Ot [d, m]; writes fp32 x_out and (optionally) its split pair.
 // With chi / clo given, activation columns [k_split, m) are read from the
 // split pair c [T, m - k_split] instead of (ahi, alo); k_split % 64 == 0.
+// Residual: x_in (fp32) or, when x_in is null, the pair (xin_hi, xin_lo).
+// Output: x_out (fp32) and/or the pair (xo_hi, xo_lo); either may be null.
 avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
-                           const float *x_in, float *x_out, bf16 *xo_hi, bf16 *xo_lo,
-                           cudaStream_t s, const bf16 *chi = nullptr, const bf16 *clo = nullptr,
-                           int k_split = 0);
+                           const float *x_in, const bf16 *xin_hi, const bf16 *xin_lo, float *x_out,
+                           bf16 *xo_hi, bf16 *xo_lo, cudaStream_t s, const bf16 *chi = nullptr,
+                           const bf16 *clo = nullptr, int k_split = 0);
 
 // Compression on tcgen05 (avey_compress_tc.cu) for S = 64, targets t0 ..
 // t0+nr-1 (idx, w, out as for avey_compress_rows); the split-size mma.sync

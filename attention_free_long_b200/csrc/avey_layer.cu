@@ -36,6 +36,32 @@ __global__ void __launch_bounds__(256) row_inv_rms(const float *__restrict__ x, 
   if (lane == 0) inv[row] = 1.0f / sqrtf(ss / static_cast<float>(d) + 1e-6f);
 }
 
+// The same scale from the split pair of x.  hi + lo is the value exactly, and
+// every lane visits the same four columns in the same order as row_inv_rms,
+// so both give bit-identical scales for the same values.
+__global__ void __launch_bounds__(256) row_inv_rms_pair(const bf16 *__restrict__ hi,
+                                                        const bf16 *__restrict__ lo, int T, int d,
+                                                        float *__restrict__ inv) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= T) return;
+  float ss = 0.f;
+  for (int j = lane * 4; j < d; j += 128) {
+    const uint2 h = *reinterpret_cast<const uint2 *>(hi + row * d + j);
+    const uint2 l = *reinterpret_cast<const uint2 *>(lo + row * d + j);
+    const float2 h0 = unpack_bf16(h.x), h1 = unpack_bf16(h.y);
+    const float2 l0 = unpack_bf16(l.x), l1 = unpack_bf16(l.y);
+    const float v0 = h0.x + l0.x, v1 = h0.y + l0.y, v2 = h1.x + l1.x, v3 = h1.y + l1.y;
+    ss = fmaf(v0, v0, ss);
+    ss = fmaf(v1, v1, ss);
+    ss = fmaf(v2, v2, ss);
+    ss = fmaf(v3, v3, ss);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if (lane == 0) inv[row] = 1.0f / sqrtf(ss / static_cast<float>(d) + 1e-6f);
+}
+
 __global__ void __launch_bounds__(256) split_rows(const float *__restrict__ x, long long count,
                                                   bf16 *__restrict__ hi, bf16 *__restrict__ lo) {
   const long long i = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) * 8;
@@ -147,8 +173,12 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
                "avey_layer_forward: dtype %d unsupported (F32 or BF16)", int(dt));
   const int d = p->d, m = p->m, m_h = p->m_h, S = p->S;
   const int mt = m - m_h;
-  AVEY_REQUIRE(x_in && x_out && ws && p->Ut && p->bU && p->Ot, AVEY_ERR_INVALID_ARG,
+  AVEY_REQUIRE(ws && p->Ut && p->bU && p->Ot, AVEY_ERR_INVALID_ARG,
                "avey_layer_forward: null pointer");
+  AVEY_REQUIRE(x_in || (dt == AVEY_BF16 && x_in_lowp), AVEY_ERR_INVALID_ARG,
+               "avey_layer_forward: x_in may be NULL only for AVEY_BF16 with x_in_lowp");
+  AVEY_REQUIRE(x_out || (dt == AVEY_BF16 && x_out_lowp), AVEY_ERR_INVALID_ARG,
+               "avey_layer_forward: x_out may be NULL only for AVEY_BF16 with x_out_lowp");
   AVEY_REQUIRE(p->kind == AVEY_STATIC || p->kind == AVEY_DYNAMIC ||
                    p->kind == AVEY_COUPLED_CAUSAL,
                AVEY_ERR_INVALID_ARG, "avey_layer_forward: bad kind %d", int(p->kind));
@@ -159,7 +189,8 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   AVEY_REQUIRE(d >= 8 && d % 8 == 0 && m % 8 == 0 && m_h % 8 == 0 && m_h > 0 && m_h < m,
                AVEY_ERR_INVALID_ARG, "avey_layer_forward: need d, m, m_h multiples of 8, 0 < m_h < m");
   AVEY_REQUIRE(p->eps >= 0.f, AVEY_ERR_INVALID_ARG, "avey_layer_forward: eps < 0");
-  AVEY_REQUIRE(aligned16(x_in) && aligned16(x_out) && aligned16(p->Ut) && aligned16(p->Ot) &&
+  AVEY_REQUIRE((!x_in || aligned16(x_in)) && (!x_out || aligned16(x_out)) && aligned16(p->Ut) &&
+                   aligned16(p->Ot) &&
                    aligned16(p->bU) && (!p->V || aligned16(p->V)) &&
                    (!x_in_lowp || aligned16(x_in_lowp)) && (!x_out_lowp || aligned16(x_out_lowp)),
                AVEY_ERR_INVALID_ARG, "avey_layer_forward: pointers must be 16-byte aligned");
@@ -234,7 +265,10 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   float *inv = nullptr;
   if (p->prenorm) {
     inv = reinterpret_cast<float *>(w + zbytes + xbytes);
-    row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_in, T, d, inv);
+    if (x_in)
+      row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_in, T, d, inv);
+    else
+      row_inv_rms_pair<<<(T + 7) / 8, 256, 0, s>>>(xhi, xlo, T, d, inv);
     AVEY_CHECK_LAUNCH("row_inv_rms");
   }
   st = launch_enrich_tc(xhi, xlo, T, d, static_cast<const bf16 *>(p->Ut), m, p->bU, inv, Zhi, Zlo, s);
@@ -260,8 +294,8 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
     if (st != AVEY_OK) return st;
     bf16 *ohi = static_cast<bf16 *>(x_out_lowp);
     bf16 *olo = ohi ? ohi + static_cast<long long>(T) * d : nullptr;
-    return launch_fuse_tc(Zhi, Zlo, T, m, static_cast<const bf16 *>(p->Ot), d, x_in, x_out, ohi, olo,
-                          s, Chi, Clo, m_h);
+    return launch_fuse_tc(Zhi, Zlo, T, m, static_cast<const bf16 *>(p->Ot), d, x_in, xhi, xlo, x_out,
+                          ohi, olo, s, Chi, Clo, m_h);
   } else if (p->kind == AVEY_STATIC)
     st = launch_static_mix_x2(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane,
                               Zhi + m_h, m, plane, s);
@@ -273,5 +307,6 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   if (st != AVEY_OK) return st;
   bf16 *ohi = static_cast<bf16 *>(x_out_lowp);
   bf16 *olo = ohi ? ohi + static_cast<long long>(T) * d : nullptr;
-  return launch_fuse_tc(Zhi, Zlo, T, m, static_cast<const bf16 *>(p->Ot), d, x_in, x_out, ohi, olo, s);
+  return launch_fuse_tc(Zhi, Zlo, T, m, static_cast<const bf16 *>(p->Ot), d, x_in, xhi, xlo, x_out, ohi,
+                        olo, s);
 }

@@ -64,8 +64,11 @@ struct TcArgs {
   bf16 *out_hi;
   bf16 *out_lo;
   long long ld_out;
-  // fuser
+  // fuser: the residual is x_in (fp32) or, when x_in is null, the split pair
+  // (xin_hi, xin_lo); a null x_out skips the fp32 output
   const float *x_in;
+  const bf16 *xin_hi;
+  const bf16 *xin_lo;
   float *x_out;
   int k_split;  // > 0: A columns >= k_split come from the second pair of maps
   int *status;
@@ -252,30 +255,71 @@ __device__ __forceinline__ void epi_enrich(const TcArgs &a, const CUtensorMap *m
   }
 }
 
-// The fp32 residual of one row's 32-column chunk (zeros outside the matrix).
-__device__ __forceinline__ void fuse_load_residual(const TcArgs &a, int row, int col0, float4 (&xi)[8]) {
+// The residual of one row's 32-column chunk as raw 16-byte words, zeros
+// outside the matrix: eight words of the fp32 x_in, or four words of each
+// plane of its split pair.  fuse_residual_values turns them into fp32 where
+// they are used, so that the loads stay in flight until then.
+__device__ __forceinline__ void fuse_load_residual(const TcArgs &a, int row, int col0, uint4 (&r)[8]) {
   const bool valid = row < a.rows;
-  const float4 *src = reinterpret_cast<const float4 *>(a.x_in + static_cast<long long>(row) * a.cols + col0);
+  const long long off = static_cast<long long>(row) * a.cols + col0;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  if (a.x_in != nullptr) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.x_in + off);
 #pragma unroll
-  for (int q = 0; q < 8; ++q)
-    xi[q] = (valid && col0 + 4 * q < a.cols) ? src[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < 8; ++q) r[q] = (valid && col0 + 4 * q < a.cols) ? src[q] : zero;
+  } else {
+    const uint4 *h = reinterpret_cast<const uint4 *>(a.xin_hi + off);
+    const uint4 *l = reinterpret_cast<const uint4 *>(a.xin_lo + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const bool ok = valid && col0 + 8 * q < a.cols;
+      r[q] = ok ? h[q] : zero;
+      r[4 + q] = ok ? l[q] : zero;
+    }
+  }
+}
+// hi + lo of two bf16 is exact in fp32 (the lo part sits at least 8 bits below hi).
+__device__ __forceinline__ void fuse_residual_values(const TcArgs &a, const uint4 (&r)[8], float (&x)[32]) {
+  if (a.x_in != nullptr) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      x[4 * q] = __uint_as_float(r[q].x);
+      x[4 * q + 1] = __uint_as_float(r[q].y);
+      x[4 * q + 2] = __uint_as_float(r[q].z);
+      x[4 * q + 3] = __uint_as_float(r[q].w);
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t hw[4] = {r[q].x, r[q].y, r[q].z, r[q].w};
+      const uint32_t lw[4] = {r[4 + q].x, r[4 + q].y, r[4 + q].z, r[4 + q].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 h = unpack_bf16(hw[u]), l = unpack_bf16(lw[u]);
+        x[8 * q + 2 * u] = h.x + l.x;
+        x[8 * q + 2 * u + 1] = h.y + l.y;
+      }
+    }
+  }
 }
 
-// Fuser epilogue: x_out = x_in + acc (fp32) and its split pair; one 8 KB
+// Fuser epilogue: x_out = x_in + acc (fp32) and/or its split pair; one 8 KB
 // staging buffer (fp32 4 KB, hi 2 KB, lo 2 KB).  The residual of chunk 0
-// arrives loaded (xi, issued before the accumulator wait); each chunk issues
-// the next chunk's loads before its own math, so their latency overlaps it.
+// arrives requested (xi, issued before the accumulator wait); each chunk
+// issues the next chunk's loads before its own math, so their latency
+// overlaps it.
 __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mout,
                                          const CUtensorMap *mhi, const CUtensorMap *mlo,
                                          uint32_t taddr, int row0, int lane, int nt, uint32_t stg,
-                                         int &it, float4 (&xi)[8]) {
+                                         int &it, uint4 (&xi)[8]) {
   const int row = row0 + lane;
   const bool pair = a.out_hi != nullptr;
+  const bool f32out = a.x_out != nullptr;
 #pragma unroll 1
   for (int ch = 0; ch < BN / 32; ++ch) {
     const int col0 = nt * BN + ch * 32;
     if (col0 >= a.cols) break;  // warp-uniform
-    float4 xn[8];
+    uint4 xn[8];
     if (ch + 1 < BN / 32) fuse_load_residual(a, row, col0 + 32, xn);
     float v[32];
     tmem_ld32(taddr + ch * 32, v);
@@ -284,17 +328,15 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mou
       __syncwarp();
     }
     float o[32];
+    fuse_residual_values(a, xi, o);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      o[4 * q] = xi[q].x + v[4 * q];
-      o[4 * q + 1] = xi[q].y + v[4 * q + 1];
-      o[4 * q + 2] = xi[q].z + v[4 * q + 2];
-      o[4 * q + 3] = xi[q].w + v[4 * q + 3];
+    for (int q = 0; q < 32; ++q) o[q] += v[q];
+    if (f32out) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(stg + sw128_off(lane, c), __float_as_uint(o[4 * c]), __float_as_uint(o[4 * c + 1]),
+                     __float_as_uint(o[4 * c + 2]), __float_as_uint(o[4 * c + 3]));
     }
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      st_shared_v4(stg + sw128_off(lane, c), __float_as_uint(o[4 * c]), __float_as_uint(o[4 * c + 1]),
-                   __float_as_uint(o[4 * c + 2]), __float_as_uint(o[4 * c + 3]));
     if (pair) {
       uint32_t hi[16], lo[16];
 #pragma unroll
@@ -308,7 +350,7 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mou
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_3d(mout, stg, col0, row0, 0);
+      if (f32out) tma_store_3d(mout, stg, col0, row0, 0);
       if (pair) {
         tma_store_3d(mhi, stg + 4096, col0, row0, 0);
         tma_store_3d(mlo, stg + 6144, col0, row0, 0);
@@ -715,7 +757,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = pair; tile < a.num_tiles; tile += npairs) {
       const int mt = tile / a.tiles_n, nt = tile - (tile / a.tiles_n) * a.tiles_n;
       const int row0 = mt * P::PM + static_cast<int>(rank) * 128 + quarter * 32;
-      float4 xi[8];
+      uint4 xi[8];
       if constexpr (MODE == MODE_FUSE) fuse_load_residual(a, row0 + lane, nt * BN, xi);
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
         ok = false;
@@ -877,23 +919,33 @@ avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, con
 }
 
 avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
-                           const float *x_in, float *x_out, bf16 *xo_hi, bf16 *xo_lo,
-                           cudaStream_t s, const bf16 *chi, const bf16 *clo, int k_split) {
+                           const float *x_in, const bf16 *xin_hi, const bf16 *xin_lo, float *x_out,
+                           bf16 *xo_hi, bf16 *xo_lo, cudaStream_t s, const bf16 *chi,
+                           const bf16 *clo, int k_split) {
+  if ((x_in == nullptr && (xin_hi == nullptr || xin_lo == nullptr)) ||
+      (x_out == nullptr && xo_hi == nullptr)) {
+    set_detail("fuse_tc: needs a residual (fp32 or pair) and an output (fp32 or pair)");
+    return AVEY_ERR_INVALID_ARG;
+  }
   CUtensorMap a0, a1, mb, o0, o1, o2, c0, c1;
   const uint64_t rs = static_cast<uint64_t>(m) * 2;
   const uint64_t fs = static_cast<uint64_t>(d) * 4, hs = static_cast<uint64_t>(d) * 2;
   if (!encode_bf16_map(&a0, ahi, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&a1, alo, m, T, 1, rs, rs * T, BM)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&mb, Ot, m, d, 1, rs, rs * d, 128)) return AVEY_ERR_CUDA;
-  if (!encode_map(&o0, true, x_out, d, T, 1, fs, fs * T, 32, 32, 128)) return AVEY_ERR_CUDA;
-  o1 = o0;
-  o2 = o0;
+  if (x_out != nullptr && !encode_map(&o0, true, x_out, d, T, 1, fs, fs * T, 32, 32, 128))
+    return AVEY_ERR_CUDA;
   if (xo_hi != nullptr) {
     if (!encode_map(&o1, false, xo_hi, d, T, 1, hs, hs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
     if (!encode_map(&o2, false, xo_lo, d, T, 1, hs, hs * T, 32, 32, 64)) return AVEY_ERR_CUDA;
   }
+  // the kernel never uses the map of an output it does not write
+  if (x_out == nullptr) o0 = o1;
+  if (xo_hi == nullptr) o1 = o2 = o0;
   TcArgs a = pair_args(T, d, m);
   a.x_in = x_in;
+  a.xin_hi = xin_hi;
+  a.xin_lo = xin_lo;
   a.x_out = x_out;
   a.out_hi = xo_hi;
   a.out_lo = xo_lo;

@@ -472,7 +472,10 @@ def run_ours(args):
     hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
     achieved = maxsim_flops(wl) / (rank_ms * 1e-3) / 1e12
     mix_bytes = 2.0 * T * mt * 4  # read Z_t pair, write c pair
-    comp_bytes = (wl.k + 1) * wl.T * wl.d * 2.0 + wl.T * wl.d * 8.0
+    # compression reads the k+1 gathered bf16 blocks and, ahead of at least
+    # one layer, writes only the split pair (4 bytes per element); fp32 as
+    # well (8 bytes per element) when no layer follows
+    comp_bytes = (wl.k + 1) * wl.T * wl.d * 2.0 + wl.T * wl.d * (4.0 if wl.layers else 8.0)
     kernel_src = os.path.join(ROOT, "attention_free_long_b200", "csrc", "avey_maxsim2.cu")
     result = {
         "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,

@@ -182,7 +182,9 @@ AVEY_API avey_status avey_maxsim_part(const void *x, avey_dtype dt, int B, int N
  *          range indices are rejected on the device as AVEY_ERR_DEVICE_BOUNDS
  *          and their block is treated as zero).
  * P        [S, (k+1)S], dtype dt.
- * out      [B, n*S, d] fp32 out (the residual stream entering layer 0).
+ * out      [B, n*S, d] fp32 out (the residual stream entering layer 0).  For
+ *          AVEY_BF16 it may be NULL when out_lowp is given: only the pair is
+ *          written (avey_layer_forward can then take x_in = NULL).
  * out_lowp for AVEY_BF16: NULL or an AVEY_BF16X2 pair [2][B*n*S][d] of `out`
  *          (what avey_layer_forward reads as x_in_lowp).  Ignored for F32.
  * Constraints: d % 8 == 0; k <= 32; AVEY_BF16 needs S in {16, 32, 64, 128};
@@ -275,12 +277,18 @@ AVEY_API avey_status avey_dynamic_mix(const void *zt, int64_t ld_zt, avey_dtype 
  *   V  [S, S]  static map (AVEY_STATIC, AVEY_COUPLED_CAUSAL), NULL for AVEY_DYNAMIC
  *   Ot [d, m]  the fuser matrix O stored transposed (row q holds O[:, q])
  * Activations:
- *   x_in      [T, d] fp32 residual stream in.
+ *   x_in      [T, d] fp32 residual stream in.  For AVEY_BF16 it may be NULL
+ *             when x_in_lowp is given: the residual is then hi + lo of the
+ *             pair (about 16 significant bits; exact as fp32 arithmetic).
  *   x_in_lowp AVEY_BF16 only: NULL or the AVEY_BF16X2 pair of x_in (as
  *             written by avey_compress / the previous layer).  When NULL the
  *             pair is built in the workspace.
- *   x_out     [T, d] fp32 out (may alias x_in exactly).
- *   x_out_lowp AVEY_BF16 only: NULL or an AVEY_BF16X2 pair [2][T][d] out.
+ *   x_out     [T, d] fp32 out (may alias x_in exactly).  For AVEY_BF16 it may
+ *             be NULL when x_out_lowp is given: only the pair is written.
+ *   x_out_lowp AVEY_BF16 only: NULL or an AVEY_BF16X2 pair [2][T][d] out (may
+ *             alias x_in_lowp exactly).
+ *   A stack that passes the pair alone between layers writes fp32 only after
+ *   its last layer: per token and layer it moves 4 d bytes fewer.
  *   ws        >= avey_layer_workspace_bytes(...) bytes, 256-byte aligned.
  * Constraints: T % S == 0; d, m, m_h multiples of 8 with 0 < m_h < m;
  * S in {16, 32, 64, 128} for AVEY_BF16, and also 256 or 512 for static and

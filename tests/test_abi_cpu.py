@@ -124,3 +124,21 @@ def test_layer_forward_rejects_bad_arguments():
     p.m_h, p.S = 768, 96
     assert L.avey_layer_forward(*args(T=96 * 42)) == 2  # unsupported split size
     assert L.avey_layer_forward(None, av.AVEY_BF16, 4096, FAKE, None, FAKE, None, FAKE, 1, None) == 1
+
+
+def test_fp32_activations_may_be_omitted_only_beside_the_bf16_pair():
+    # x_in / x_out (and compression's out) may be NULL only on the bf16 path
+    # and only when the split pair stands in for them
+    L = av.lib()
+    p = av.LayerParams(av.AVEY_STATIC, 768, 1536, 768, 64, 1e-8, 0, 0x10000, 0x10000, 0x10000, 0x10000)
+    call = lambda dt, xi, xil, xo, xol: L.avey_layer_forward(ctypes.byref(p), dt, 4096, xi, xil, xo, xol,
+                                                            FAKE, 1 << 34, None)
+    assert call(av.AVEY_BF16, None, None, FAKE, None) == 1   # no residual at all
+    assert call(av.AVEY_BF16, FAKE, None, None, None) == 1   # no output at all
+    assert call(av.AVEY_F32, None, FAKE, FAKE, None) == 1    # fp32 path needs x_in
+    assert call(av.AVEY_F32, FAKE, None, None, FAKE) == 1    # fp32 path needs x_out
+    assert "x_in may be NULL" in (call(av.AVEY_BF16, None, None, FAKE, None) and
+                                  L.avey_last_error_detail().decode())
+    cmp = lambda dt, out, lowp: L.avey_compress(FAKE, dt, 1, 256, 64, 64, 3, FAKE, FAKE, FAKE, out, lowp, None)
+    assert cmp(av.AVEY_BF16, None, None) == 1
+    assert cmp(av.AVEY_F32, None, FAKE) == 1

@@ -1,0 +1,81 @@
+"""The residual stream passed between bf16 calls as its split pair alone.
+
+avey_compress and avey_layer_forward may leave out the fp32 activation when
+the bf16 pair (hi, lo) stands in for it: a layer then takes its residual as
+hi + lo and may write only the pair, so a stack writes fp32 once, after its
+last layer.  The pair holds about 16 significant bits, so the result differs
+from the fp32 stream's by rounding far below the bf16 tolerance; these tests
+check that against the fp32 path on the GPU and the whole stack against the
+fp64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import attention_free_long_b200 as av
+import oracle as orc
+import synthetic as sy
+from tests.parity import TOL, check_topk, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def _pair(x):
+    hi = x.to(torch.bfloat16)
+    lo = (x - hi.float()).to(torch.bfloat16)
+    return torch.stack([hi, lo]).contiguous()
+
+
+@pytest.mark.parametrize("prenorm", [False, True])
+@pytest.mark.parametrize("kind", [sy.STATIC, sy.DYNAMIC])
+def test_layer_takes_and_gives_the_pair_alone(kind, prenorm, cuda_dev):
+    # ragged feature width (136 = 4 x 32 + 8) and 16 splits of 64 tokens
+    wl = sy.custom("pair_stream", B=1, N=1024, S=64, d=136, m=272, m_h=136, k=3, pattern=(kind,),
+                   prenorm=prenorm)
+    lay = av.device_layers(sy.gen_weights(wl), torch.bfloat16, cuda_dev)[0]
+    g = torch.Generator(device="cpu").manual_seed(5)
+    x = (torch.randn(wl.N, wl.d, generator=g) * 1.5).to(cuda_dev)
+    xp = _pair(x)
+    xr = xp[0].float() + xp[1].float()  # the value the pair represents
+    y_ref, p_ref = av.avey_layer_forward(lay, wl.S, wl.m_h, wl.eps, prenorm, xr.contiguous(), xp)
+    # residual from the pair, pair out only
+    y_none, p_only = av.avey_layer_forward(lay, wl.S, wl.m_h, wl.eps, prenorm, None, xp, fp32_out=False)
+    # residual from the pair, fp32 out only (a stack's last layer)
+    y_last, p_none = av.avey_layer_forward(lay, wl.S, wl.m_h, wl.eps, prenorm, None, xp, lowp_out=False)
+    torch.cuda.synchronize()
+    assert av.device_status() == 0
+    assert y_none is None and p_none is None
+    # the fp32 residual here is exactly hi + lo, so the fused results agree
+    # bit for bit; the pair out is the split of the same fp32 sums
+    assert torch.equal(y_last, y_ref)
+    assert torch.equal(p_only, p_ref)
+
+
+@pytest.mark.parametrize("wl", [
+    sy.custom("ps_s64_ragged", B=2, N=1000, S=64, d=136, m=272, m_h=136, k=5,
+              pattern=(sy.STATIC, sy.DYNAMIC, sy.STATIC), centers=8, sigma=0.5),
+    sy.custom("ps_s128_pre", B=1, N=3000, S=128, d=128, m=256, k=15,
+              pattern=(sy.STATIC, sy.DYNAMIC, sy.STATIC), centers=12, sigma=0.5, prenorm=True),
+    sy.custom("ps_s32", B=2, N=2053, S=32, d=96, m=192, m_h=64, k=7,
+              pattern=(sy.DYNAMIC, sy.STATIC), centers=32, sigma=0.5),
+], ids=lambda w: w.name)
+def test_encoder_stack_on_the_pair_matches_the_oracle(wl, cuda_dev):
+    E, W = sy.gen_embeddings(wl), sy.gen_weights(wl)
+    x = torch.from_numpy(E.X).to(cuda_dev, torch.bfloat16)
+    P = torch.from_numpy(W.P).to(cuda_dev, torch.bfloat16)
+    layers = av.device_layers(W, torch.bfloat16, cuda_dev)
+    ws = av.make_workspace(wl.B, wl.N, wl.d, wl.S, wl.k, wl.m, torch.bfloat16, wl.prenorm, cuda_dev)
+    out = av.encoder_forward(x, P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm, ws=ws)
+    torch.cuda.synchronize()
+    assert av.device_status() == 0
+    o = orc.forward(E.X, W, wl)
+    tol = TOL["bf16"]
+    exact = check_topk(ws.idx.cpu().numpy().reshape(-1, wl.k), ws.w.cpu().numpy().reshape(-1, wl.k),
+                       o["idx"], o["scores"], o["sel"][:, 1], tol)
+    assert exact.mean() >= 0.75
+    best = np.array([o["scores"][r, o["idx"][r, 0]] if o["idx"][r, 0] >= 0 else 1.0
+                     for r in range(o["sel"].shape[0])])
+    keep = np.repeat(exact & (best > 1e-30), wl.S)
+    got = out.cpu().numpy().reshape(-1, wl.d)
+    err = rel_err(got[keep], o["layers"][-1].reshape(-1, wl.d)[keep])
+    assert err <= tol, f"stack on the pair: err {err:.3g} > {tol}"
