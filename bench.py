@@ -80,6 +80,13 @@ def maxsim_executed_flops(wl) -> float:
     return 2.0 * wl.B * (-(-R // 128)) * (-(-R // 256)) * 128 * 256 * kpad
 
 
+def compress_bytes(wl) -> float:
+    """Algorithmic HBM bytes of the forward's compression call: the k+1
+    gathered bf16 blocks in; out, ahead of at least one layer, only the split
+    pair (4 bytes per element), else fp32 as well (8 bytes per element)."""
+    return (wl.k + 1) * wl.T * wl.d * 2.0 + wl.T * wl.d * (4.0 if wl.layers else 8.0)
+
+
 def layer_flops(wl) -> float:
     """Enricher + fuser GEMMs, 2 T d m each, per layer."""
     return wl.layers * 2 * (2.0 * wl.T * wl.d * wl.m)
@@ -472,10 +479,7 @@ def run_ours(args):
     hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
     achieved = maxsim_flops(wl) / (rank_ms * 1e-3) / 1e12
     mix_bytes = 2.0 * T * mt * 4  # read Z_t pair, write c pair
-    # compression reads the k+1 gathered bf16 blocks and, ahead of at least
-    # one layer, writes only the split pair (4 bytes per element); fp32 as
-    # well (8 bytes per element) when no layer follows
-    comp_bytes = (wl.k + 1) * wl.T * wl.d * 2.0 + wl.T * wl.d * (4.0 if wl.layers else 8.0)
+    comp_bytes = compress_bytes(wl)
     kernel_src = os.path.join(ROOT, "attention_free_long_b200", "csrc", "avey_maxsim2.cu")
     result = {
         "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,

@@ -68,3 +68,13 @@ def test_traffic_and_l2_notes_follow_the_workload(tmp_path):
     assert got is None or got > 0
     assert "larger than L2" in bench.l2_note(sy.WORKLOADS["long_bf16"])
     assert "fits" in bench.l2_note(sy.WORKLOADS["base_bf16"])
+
+
+def test_compress_bytes_count_what_the_forward_writes():
+    import bench
+    import synthetic as sy
+    wl = sy.WORKLOADS["long_bf16"]
+    # 8 gathered blocks of bf16 in, the split pair out: 1.51 GB
+    assert bench.compress_bytes(wl) == 8 * 98304 * 768 * 2 + 98304 * 768 * 4
+    no_layers = sy.custom("c0", B=1, N=1024, S=64, d=64, m=128, k=3, pattern=())
+    assert bench.compress_bytes(no_layers) == 4 * 1024 * 64 * 2 + 1024 * 64 * 8
