@@ -14,7 +14,8 @@ Entry points (same names as the C ABI):
   avey_dynamic_mix   eq. 6 row-normalised cosine mix of split blocks
   avey_layer_forward enricher -> static/dynamic mix -> fuser + residual
 and ``encoder_forward`` which strings them together (ranker once, then every
-layer), the call a user of the encoder makes.
+layer), the call a user of the encoder makes; ``processor_forward`` is the
+same forward after the ranker, for a selection the caller supplies.
 """
 from __future__ import annotations
 
@@ -65,6 +66,12 @@ def lib() -> ctypes.CDLL:
         L.avey_rank_ex.argtypes = [_vp, _i, _i, _i, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _vp,
                                    _vp, _sz, _vp]
         L.avey_rank_ex.restype = _i
+        L.avey_trace_begin.argtypes = [_vp, _i]
+        L.avey_trace_begin.restype = _i
+        L.avey_trace_end.argtypes = []
+        L.avey_trace_end.restype = _i
+        L.avey_trace_kernel_name.argtypes = [_i]
+        L.avey_trace_kernel_name.restype = ctypes.c_char_p
         L.avey_rank_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.avey_rank_workspace_bytes.restype = _sz
         L.avey_compress.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
@@ -136,6 +143,51 @@ def _ws(nbytes: int, device) -> torch.Tensor:
 
 def kernel_launches() -> int:
     return int(lib().avey_kernel_launches())
+
+
+class KernelTrace:
+    """Per-kernel device times of the library's launches on the current stream.
+
+    ``with KernelTrace(capacity) as tr: ...`` records one CUDA event after
+    every kernel the library enqueues inside the block (avey_trace_begin /
+    avey_trace_end), plus one before the first; after a synchronize,
+    ``tr.kernels()`` gives [(name, ms)] in launch order.  For launches on one
+    stream only.
+    """
+
+    def __init__(self, capacity: int = 256):
+        self.capacity = int(capacity)
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(self.capacity)]
+        self.start = torch.cuda.Event(enable_timing=True)
+        # torch creates an event's CUDA handle on its first record
+        for e in self.events:
+            e.record()
+        self.count = 0
+        self.names: List[str] = []
+
+    def __enter__(self):
+        arr = (ctypes.c_void_p * self.capacity)(*[e.cuda_event for e in self.events])
+        self.start.record()
+        _check("avey_trace_begin", lib().avey_trace_begin(arr, self.capacity))
+        return self
+
+    def __exit__(self, *exc):
+        n = int(lib().avey_trace_end())
+        if n < 0:
+            raise AveyError("avey_trace_end", 3, lib().avey_last_error_detail().decode())
+        if n > self.capacity:
+            raise RuntimeError(f"kernel trace overflow: {n} launches, capacity {self.capacity}")
+        self.count = n
+        self.names = [lib().avey_trace_kernel_name(i).decode() for i in range(n)]
+        return False
+
+    def kernels(self):
+        """[(name, ms)] of every traced launch (call after a synchronize)."""
+        out, prev = [], self.start
+        for i in range(self.count):
+            out.append((self.names[i], prev.elapsed_time(self.events[i])))
+            prev = self.events[i]
+        return out
 
 
 def device_status(stream=None) -> int:
@@ -422,22 +474,48 @@ def encoder_forward(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLay
     the current stream before the ranker and after every C-ABI call.
     """
     B, N, d = x.shape
+    m = layers[0].Ut.shape[0] if layers else d
+    if ws is None:
+        ws = make_workspace(B, N, d, S, k, m, x.dtype, prenorm, x.device)
+    dt = _dt(x)
+    L = lib()
+    st = _stream()
+    if marks is not None:
+        marks[0].record()
+    flags = AVEY_RANK_UNIDIRECTIONAL if causal else 0
+    _check("avey_rank", L.avey_rank_ex(_ptr(x), dt, B, N, d, S, k, flags, _ptr(ws.idx),
+                                       _ptr(ws.w), None, _ptr(ws.rank_ws), ws.rank_ws.numel(), st))
+    if marks is not None:
+        marks[1].record()
+    return processor_forward(x, P, layers, S, k, m_h, eps, prenorm, ws.idx, ws.w, ws, marks)
+
+
+def processor_forward(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLayer], S: int,
+                      k: int, m_h: int, eps: float, prenorm: bool, idx: torch.Tensor,
+                      w: torch.Tensor, ws: Optional[EncoderWorkspace] = None,
+                      marks=None) -> torch.Tensor:
+    """Compression and every layer for a given selection (idx int32 [B, n, k],
+    w fp32 [B, n, k], as avey_rank returns them): the part of the forward after
+    the ranker, for a caller that ranks by other means.  Returns fp32
+    [B, n*S, d].  ``marks[2 + i]`` is recorded after compression (i = 0) and
+    after every layer.
+    """
+    B, N, d = x.shape
     n = -(-N // S)
     T = B * n * S
     dt = _dt(x)
     m = layers[0].Ut.shape[0] if layers else d
     if ws is None:
         ws = make_workspace(B, N, d, S, k, m, x.dtype, prenorm, x.device)
+    for t, nm in ((idx, "idx"), (w, "w")):
+        _need(t, nm)
+        if t.numel() != B * n * k:
+            raise ValueError(f"{nm} must have B*n*k = {B * n * k} entries")
+    if idx.dtype != torch.int32 or w.dtype != torch.float32:
+        raise TypeError("idx must be int32 and w fp32")
     L = lib()
     st = _stream()
-    if marks is not None:
-        marks[0].record()
-    _check("avey_rank", L.avey_rank_ex(_ptr(x), dt, B, N, d, S, k,
-                                       AVEY_RANK_UNIDIRECTIONAL if causal else 0, _ptr(ws.idx),
-                                       _ptr(ws.w), None, _ptr(ws.rank_ws), ws.rank_ws.numel(), st))
-    if marks is not None:
-        marks[1].record()
-    _check("avey_compress", L.avey_compress(_ptr(x), dt, B, N, d, S, k, _ptr(ws.idx), _ptr(ws.w),
+    _check("avey_compress", L.avey_compress(_ptr(x), dt, B, N, d, S, k, _ptr(idx), _ptr(w),
                                             _ptr(P), None if _pair_stream(dt, layers) else _ptr(ws.x0),
                                             _ptr(ws.pair0), st))
     if marks is not None:
@@ -460,13 +538,10 @@ def encoder_forward_uncompressed(x: torch.Tensor, layers: Sequence[DeviceLayer],
     the current stream before the ranker and after every C-ABI call.
     """
     B, N, d = x.shape
-    n = -(-N // S)
-    L_ = (k + 1) * S
-    T = B * n * L_
-    dt = _dt(x)
     m = layers[0].Ut.shape[0] if layers else d
     if ws is None:
         ws = make_workspace(B, N, d, S, k, m, x.dtype, prenorm, x.device, uncompressed=True)
+    dt = _dt(x)
     L = lib()
     st = _stream()
     if marks is not None:
@@ -476,7 +551,34 @@ def encoder_forward_uncompressed(x: torch.Tensor, layers: Sequence[DeviceLayer],
                                        _ptr(ws.w), None, _ptr(ws.rank_ws), ws.rank_ws.numel(), st))
     if marks is not None:
         marks[1].record()
-    _check("avey_context", L.avey_context(_ptr(x), dt, B, N, d, S, k, _ptr(ws.idx), _ptr(ws.w),
+    return processor_forward_uncompressed(x, layers, S, k, m_h, eps, prenorm, ws.idx, ws.w, ws,
+                                          marks)
+
+
+def processor_forward_uncompressed(x: torch.Tensor, layers: Sequence[DeviceLayer], S: int, k: int,
+                                   m_h: int, eps: float, prenorm: bool, idx: torch.Tensor,
+                                   w: torch.Tensor, ws: Optional[EncoderWorkspace] = None,
+                                   marks=None) -> torch.Tensor:
+    """The uncompressed processor for a given selection (idx int32 [B, n, k],
+    w fp32 [B, n, k]): every split's context through every layer.  Returns
+    fp32 [B, n, S, d] (a view); ``marks`` as in processor_forward."""
+    B, N, d = x.shape
+    n = -(-N // S)
+    L_ = (k + 1) * S
+    T = B * n * L_
+    dt = _dt(x)
+    m = layers[0].Ut.shape[0] if layers else d
+    if ws is None:
+        ws = make_workspace(B, N, d, S, k, m, x.dtype, prenorm, x.device, uncompressed=True)
+    for t, nm in ((idx, "idx"), (w, "w")):
+        _need(t, nm)
+        if t.numel() != B * n * k:
+            raise ValueError(f"{nm} must have B*n*k = {B * n * k} entries")
+    if idx.dtype != torch.int32 or w.dtype != torch.float32:
+        raise TypeError("idx must be int32 and w fp32")
+    L = lib()
+    st = _stream()
+    _check("avey_context", L.avey_context(_ptr(x), dt, B, N, d, S, k, _ptr(idx), _ptr(w),
                                           _ptr(ws.x0), _ptr(ws.pair0), st))
     if marks is not None:
         marks[2].record()

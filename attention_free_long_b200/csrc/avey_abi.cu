@@ -1,5 +1,6 @@
 // avey_abi.cu -- host-side utilities of libavey.so: status reporting, error
-// details, launch counting, SM count, and TMA tensor-map encoding.
+// details, launch counting and the kernel trace, SM count, and TMA tensor-map
+// encoding.
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -66,7 +67,35 @@ int *device_status_word() {
   return g_status_ptr[dev];
 }
 
-void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+// Kernel trace: while active, every launch records the next caller-provided
+// event on the launch's stream and keeps the kernel's name.
+namespace {
+constexpr int kTraceName = 48;
+struct Trace {
+  std::mutex mu;
+  std::atomic<bool> on{false};
+  cudaEvent_t *events = nullptr;
+  char (*names)[kTraceName] = nullptr;
+  int capacity = 0;
+  int count = 0;       // launches seen since avey_trace_begin
+  int record_err = 0;  // first cudaEventRecord failure
+};
+Trace g_trace;
+char g_trace_names[4096][kTraceName];
+}  // namespace
+
+void count_launch(const char *name, cudaStream_t stream) {
+  g_launches.fetch_add(1);
+  if (!g_trace.on.load(std::memory_order_acquire)) return;
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  if (!g_trace.on.load(std::memory_order_relaxed)) return;
+  const int i = g_trace.count++;
+  if (i < g_trace.capacity) {
+    snprintf(g_trace.names[i], kTraceName, "%s", name ? name : "?");
+    const cudaError_t e = cudaEventRecord(g_trace.events[i], stream);
+    if (e != cudaSuccess && !g_trace.record_err) g_trace.record_err = static_cast<int>(e);
+  }
+}
 
 int sm_count() {
   const int dev = current_device();
@@ -146,7 +175,7 @@ avey_status avey_selftest_wait_timeout(uint32_t limit_us, avey_stream_t stream) 
   AVEY_REQUIRE(st != nullptr, AVEY_ERR_CUDA, "avey_selftest_wait_timeout: no device status word");
   avey::wait_timeout_probe<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(limit_us) * 1000ull, st);
-  AVEY_CHECK_LAUNCH("wait_timeout_probe");
+  AVEY_CHECK_LAUNCH("wait_timeout_probe", reinterpret_cast<cudaStream_t>(stream));
   return AVEY_OK;
 }
 
@@ -189,5 +218,44 @@ const char *avey_status_string(avey_status s) {
 const char *avey_last_error_detail(void) { return avey::t_detail; }
 
 uint64_t avey_kernel_launches(void) { return avey::g_launches.load(); }
+
+avey_status avey_trace_begin(void *const *events, int capacity) {
+  using avey::g_trace;
+  AVEY_REQUIRE(events && capacity >= 1 && capacity <= 4096, AVEY_ERR_INVALID_ARG,
+               "avey_trace_begin: need an event array and 1 <= capacity <= 4096 (got %d)",
+               capacity);
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  AVEY_REQUIRE(!g_trace.on.load(), AVEY_ERR_INVALID_ARG, "avey_trace_begin: a trace is active");
+  for (int i = 0; i < capacity; ++i)
+    AVEY_REQUIRE(events[i] != nullptr, AVEY_ERR_INVALID_ARG, "avey_trace_begin: event %d is null", i);
+  g_trace.events = reinterpret_cast<cudaEvent_t *>(const_cast<void **>(events));
+  g_trace.names = avey::g_trace_names;
+  g_trace.capacity = capacity;
+  g_trace.count = 0;
+  g_trace.record_err = 0;
+  g_trace.on.store(true, std::memory_order_release);
+  return AVEY_OK;
+}
+
+int avey_trace_end(void) {
+  using avey::g_trace;
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  if (!g_trace.on.load()) return -1;
+  g_trace.on.store(false, std::memory_order_release);
+  g_trace.events = nullptr;
+  if (g_trace.record_err) {
+    avey::set_detail("avey_trace_end: cudaEventRecord failed: %s",
+                     cudaGetErrorString(static_cast<cudaError_t>(g_trace.record_err)));
+    return -1;
+  }
+  return g_trace.count;
+}
+
+const char *avey_trace_kernel_name(int i) {
+  using avey::g_trace;
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  if (g_trace.on.load() || i < 0 || i >= g_trace.capacity || i >= g_trace.count) return nullptr;
+  return avey::g_trace_names[i];
+}
 
 }  // extern "C"

@@ -24,7 +24,9 @@ void set_detail(const char *fmt, ...);
 // Device address of the status word for the current device (nullptr on error).
 int *device_status_word();
 // Counts launches (one call per kernel launch).
-void count_launch(int n = 1);
+// Counts one launch of kernel `name` on `stream`; while a kernel trace is
+// active (avey_trace_begin), also records the trace's next event on `stream`.
+void count_launch(const char *name, cudaStream_t stream);
 // Number of SMs of the current device.
 int sm_count();
 // Encodes a bf16 3-D tiled tensor map with 128-byte swizzle:
@@ -39,14 +41,14 @@ bool encode_map(CUtensorMap *map, bool fp32, const void *base, uint64_t inner, u
                 uint64_t batch, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
                 uint32_t box_inner, uint32_t box_rows, int swizzle_bytes);
 
-#define AVEY_CHECK_LAUNCH(name)                                             \
+#define AVEY_CHECK_LAUNCH(name, stream)                                     \
   do {                                                                      \
     cudaError_t e_ = cudaGetLastError();                                    \
     if (e_ != cudaSuccess) {                                                \
       ::avey::set_detail("%s launch failed: %s", name, cudaGetErrorString(e_)); \
       return AVEY_ERR_CUDA;                                                 \
     }                                                                       \
-    ::avey::count_launch();                                                 \
+    ::avey::count_launch(name, stream);                                     \
   } while (0)
 
 #define AVEY_REQUIRE(cond, code, ...)   \

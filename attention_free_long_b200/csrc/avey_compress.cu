@@ -316,7 +316,7 @@ avey_status run_compress_bf16(const bf16 *x, int B, int N, int d, int n, int k, 
   const long long plane = static_cast<long long>(B) * nr * S * d;
   kern<<<grid, 256, C::SMEM, s>>>(x, N, d, n, k, idx, w, P, out, hi, lo, plane, t0, nr,
                                   device_status_word());
-  AVEY_CHECK_LAUNCH("compress_bf16");
+  AVEY_CHECK_LAUNCH("compress_bf16", s);
   return AVEY_OK;
 }
 
@@ -374,7 +374,7 @@ static avey_status compress_range(const void *x, avey_dtype dt, int B, int N, in
     AVEY_CF_CASE(32) AVEY_CF_CASE(64)
 #undef AVEY_CF_CASE
   }
-  AVEY_CHECK_LAUNCH("compress_f32");
+  AVEY_CHECK_LAUNCH("compress_f32", s);
   return AVEY_OK;
 }
 

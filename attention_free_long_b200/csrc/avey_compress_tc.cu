@@ -368,7 +368,7 @@ avey_status run_compress_tc(const CUtensorMap &mx, const CUtensorMap &mp, const 
     return AVEY_ERR_CUDA;
   }
   kern<<<grid, C_THR, C_SMEM, s>>>(mx, mp, mo, moh, mol, a);
-  AVEY_CHECK_LAUNCH("compress_tc");
+  AVEY_CHECK_LAUNCH("compress_tc", s);
   return AVEY_OK;
 }
 

@@ -112,6 +112,6 @@ extern "C" avey_status avey_context(const void *x, avey_dtype dt, int B, int N, 
   else
     context_rows<false><<<grid, 256, 0, s>>>(x, N, d, S, k, static_cast<int>(n), idx, w, out,
                                              nullptr, nullptr, units, device_status_word());
-  AVEY_CHECK_LAUNCH("context_rows");
+  AVEY_CHECK_LAUNCH("context_rows", s);
   return AVEY_OK;
 }

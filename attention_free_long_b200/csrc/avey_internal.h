@@ -55,6 +55,10 @@ avey_status launch_compress_tc(const bf16 *x, int B, int N, int d, int k, int t0
                                bf16 *hi, bf16 *lo, cudaStream_t s);
 
 // ---- ranker pieces (avey_rank.cu) ----
+// Shape and dtype checks of the ranker entry points (avey_rank.cu); fn names
+// the entry point in the error detail.
+avey_status check_rank_shape(const char *fn, avey_dtype dt, int B, int N, int d, int S, int k);
+
 avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, int S, void *xhat,
                              cudaStream_t s);
 avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, float *inv,

@@ -224,11 +224,11 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
     float *inv = p->prenorm ? reinterpret_cast<float *>(w + align256(static_cast<size_t>(T) * m * 4)) : nullptr;
     if (inv) {
       row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_in, T, d, inv);
-      AVEY_CHECK_LAUNCH("row_inv_rms");
+      AVEY_CHECK_LAUNCH("row_inv_rms", s);
     }
     gemm_f32<F32_ENRICH><<<dim3((m + 63) / 64, (T + 63) / 64), 256, 0, s>>>(
         x_in, static_cast<const float *>(p->Ut), T, m, d, p->bU, inv, nullptr, Z);
-    AVEY_CHECK_LAUNCH("gemm_f32_enrich");
+    AVEY_CHECK_LAUNCH("gemm_f32_enrich", s);
     if (p->kind == AVEY_STATIC)
       st = launch_static_mix_f32(static_cast<const float *>(p->V), Z + m_h, m, Z + m_h, m, blocks, S,
                                  mt, s);
@@ -240,7 +240,7 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
     if (st != AVEY_OK) return st;
     gemm_f32<F32_FUSE><<<dim3((d + 63) / 64, (T + 63) / 64), 256, 0, s>>>(
         Z, static_cast<const float *>(p->Ot), T, d, m, nullptr, nullptr, x_in, x_out);
-    AVEY_CHECK_LAUNCH("gemm_f32_fuse");
+    AVEY_CHECK_LAUNCH("gemm_f32_fuse", s);
     return AVEY_OK;
   }
 
@@ -258,7 +258,7 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
     bf16 *l = h + static_cast<long long>(T) * d;
     const long long cnt = static_cast<long long>(T) * d;
     split_rows<<<static_cast<unsigned>((cnt / 8 + 255) / 256), 256, 0, s>>>(x_in, cnt, h, l);
-    AVEY_CHECK_LAUNCH("split_rows");
+    AVEY_CHECK_LAUNCH("split_rows", s);
     xhi = h;
     xlo = l;
   }
@@ -269,7 +269,7 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
       row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_in, T, d, inv);
     else
       row_inv_rms_pair<<<(T + 7) / 8, 256, 0, s>>>(xhi, xlo, T, d, inv);
-    AVEY_CHECK_LAUNCH("row_inv_rms");
+    AVEY_CHECK_LAUNCH("row_inv_rms", s);
   }
   st = launch_enrich_tc(xhi, xlo, T, d, static_cast<const bf16 *>(p->Ut), m, p->bU, inv, Zhi, Zlo, s);
   if (st != AVEY_OK) return st;

@@ -478,7 +478,7 @@ avey_status run_pair(const CUtensorMap &mx, PairArgs a, cudaStream_t st) {
   const int mine = (a.num_tiles - a.part + a.nparts - 1) / a.nparts;  // tiles of this part
   const int pairs = std::max(1, std::min(mine, cap));
   kern<<<2 * pairs, kThreads, SMEM_BYTES, st>>>(mx, a);
-  AVEY_CHECK_LAUNCH("maxsim_pair");
+  AVEY_CHECK_LAUNCH("maxsim_pair", st);
   return AVEY_OK;
 }
 

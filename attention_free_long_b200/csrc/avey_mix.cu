@@ -476,7 +476,7 @@ avey_status run_static_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks,
   if (avey_status st = set_smem(static_mix_x2<S>, C::SMEM, "static_mix_x2")) return st;
   const dim3 grid((mt + C::NS - 1) / C::NS, blocks);
   static_mix_x2<S><<<grid, 256, C::SMEM, s>>>(V, zt, ld, mt, plane, out, ld_out, plane_out);
-  AVEY_CHECK_LAUNCH("static_mix_x2");
+  AVEY_CHECK_LAUNCH("static_mix_x2", s);
   return AVEY_OK;
 }
 
@@ -488,7 +488,7 @@ avey_status run_dynamic_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16
   if (avey_status st = set_smem(dynamic_mix_x2<S, COUPLED>, C::SMEM, "dynamic_mix_x2")) return st;
   dynamic_mix_x2<S, COUPLED><<<blocks, 256, C::SMEM, s>>>(zt, ld_zt, plane_zt, out, ld_out,
                                                           plane_out, mt, eps, V);
-  AVEY_CHECK_LAUNCH(COUPLED ? "coupled_mix_x2" : "dynamic_mix_x2");
+  AVEY_CHECK_LAUNCH(COUPLED ? "coupled_mix_x2" : "dynamic_mix_x2", s);
   return AVEY_OK;
 }
 
@@ -543,7 +543,7 @@ avey_status launch_static_mix_f32(const float *V, const float *zt, int64_t ld_zt
 #undef AVEY_SF
     default: set_detail("static mix (F32): S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
   }
-  AVEY_CHECK_LAUNCH("static_mix_f32");
+  AVEY_CHECK_LAUNCH("static_mix_f32", s);
   return AVEY_OK;
 }
 
@@ -556,7 +556,7 @@ avey_status launch_dynamic_mix_f32(const float *zt, int64_t ld_zt, float *out, i
 #undef AVEY_DF
     default: set_detail("dynamic mix (F32): S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
   }
-  AVEY_CHECK_LAUNCH("dynamic_mix_f32");
+  AVEY_CHECK_LAUNCH("dynamic_mix_f32", s);
   return AVEY_OK;
 }
 
@@ -569,7 +569,7 @@ avey_status launch_coupled_mix_f32(const float *V, const float *zt, int64_t ld_z
 #undef AVEY_CF
     default: set_detail("coupled mix (F32): S=%d unsupported", S); return AVEY_ERR_UNSUPPORTED;
   }
-  AVEY_CHECK_LAUNCH("coupled_mix_f32");
+  AVEY_CHECK_LAUNCH("coupled_mix_f32", s);
   return AVEY_OK;
 }
 

@@ -128,7 +128,7 @@ avey_status run_dynamic_gt(const bf16 *zt, int64_t ld, int blocks, int mt, float
       set_detail("long dynamic mix: m_t = %d above 1024", mt);
       return AVEY_ERR_UNSUPPORTED;
   }
-  AVEY_CHECK_LAUNCH("long_dyn_prep");
+  AVEY_CHECK_LAUNCH("long_dyn_prep", s);
   return launch_long_gram_tc(zt, ld, blocks, SL, mt, inv_n, inv_d, gt, s);
 }
 

@@ -516,7 +516,7 @@ avey_status run_mix_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUten
   }
   const int grid = std::min(args.num_tiles, sm_count());
   kern<<<grid, kThr, L::SMEM, s>>>(a0, a1, z0, z1, args);
-  AVEY_CHECK_LAUNCH("mix_tc");
+  AVEY_CHECK_LAUNCH("mix_tc", s);
   return AVEY_OK;
 }
 
@@ -592,7 +592,7 @@ avey_status launch_long_gram_tc(const bf16 *zhi, int64_t ldz, int blocks, int SL
   }
   const int grid = std::min(g.num_tiles, sm_count());
   gram_tc_kernel<<<grid, kThr, G_SMEM, s>>>(za, zb, g);
-  AVEY_CHECK_LAUNCH("gram_tc");
+  AVEY_CHECK_LAUNCH("gram_tc", s);
   return AVEY_OK;
 }
 

@@ -286,7 +286,7 @@ avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, 
   else
     normalize_rows<float, float><<<grid, 256, 0, s>>>(static_cast<const float *>(x), B, N, d, R,
                                                       static_cast<float *>(xhat));
-  AVEY_CHECK_LAUNCH("normalize_rows");
+  AVEY_CHECK_LAUNCH("normalize_rows", s);
   return AVEY_OK;
 }
 
@@ -294,7 +294,7 @@ avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, floa
                              cudaStream_t s) {
   const long long rows = static_cast<long long>(B) * rs_ld;
   inv_norms<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(x, B, N, d, rs_ld, inv);
-  AVEY_CHECK_LAUNCH("inv_norms");
+  AVEY_CHECK_LAUNCH("inv_norms", s);
   return AVEY_OK;
 }
 
@@ -305,7 +305,7 @@ avey_status launch_topk_rows(const float *scores, int B, int n, int t0, int nr, 
   const unsigned grid = static_cast<unsigned>((rows + kTopkWarps - 1) / kTopkWarps);
   const int vec4 = (n % 4 == 0 && aligned16(scores)) ? 1 : 0;
   topk_warp<<<grid, kTopkWarps * 32, 0, s>>>(scores, B, n, t0, nr, k, causal, vec4, idx, w);
-  AVEY_CHECK_LAUNCH("topk_warp");
+  AVEY_CHECK_LAUNCH("topk_warp", s);
   return AVEY_OK;
 }
 
@@ -329,7 +329,7 @@ static avey_status launch_maxsim_f32(const float *xhat, int B, int R, int d, int
       set_detail("avey_rank(F32): S=%d unsupported (powers of two up to 128)", S);
       return AVEY_ERR_UNSUPPORTED;
   }
-  AVEY_CHECK_LAUNCH("maxsim_f32");
+  AVEY_CHECK_LAUNCH("maxsim_f32", s);
   return AVEY_OK;
 }
 
@@ -414,31 +414,43 @@ extern "C" avey_status avey_maxsim_part(const void *x, avey_dtype dt, int B, int
                             static_cast<int>(n), scores, s, part, nparts);
 }
 
+// Shape and dtype checks shared by every ranker entry point (fn names the
+// entry point in the error detail).
+avey_status avey::check_rank_shape(const char *fn, avey_dtype dt, int B, int N, int d, int S,
+                                     int k) {
+  AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
+               "%s: dtype %d unsupported (F32 or BF16)", fn, int(dt));
+  AVEY_REQUIRE(B >= 1 && N >= 1 && d >= 1 && S >= 1 && k >= 1, AVEY_ERR_INVALID_ARG,
+               "%s: sizes must be >= 1 (B=%d N=%d d=%d S=%d k=%d)", fn, B, N, d, S, k);
+  AVEY_REQUIRE(d % 8 == 0, AVEY_ERR_INVALID_ARG, "%s: d=%d must be a multiple of 8", fn, d);
+  AVEY_REQUIRE(k <= 32, AVEY_ERR_UNSUPPORTED, "%s: k=%d > 32", fn, k);
+  if (dt == AVEY_BF16)
+    AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
+                 "%s(BF16): S=%d unsupported (16, 32, 64 or 128)", fn, S);
+  else
+    AVEY_REQUIRE(S <= 128 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
+                 "%s(F32): S=%d unsupported (power of two <= 128)", fn, S);
+  const long long n = (N + S - 1) / S, R = n * S;
+  AVEY_REQUIRE(n <= 46340 && static_cast<long long>(B) * R <= (1ll << 31) - 1,
+               AVEY_ERR_UNSUPPORTED, "%s: problem too large", fn);
+  return AVEY_OK;
+}
+
 extern "C" avey_status avey_rank_ex(const void *x, avey_dtype dt, int B, int N, int d, int S, int k,
                                     uint32_t flags, int32_t *idx, float *w, float *scores, void *ws,
                                     size_t ws_bytes, avey_stream_t stream) {
   AVEY_REQUIRE((flags & ~static_cast<uint32_t>(AVEY_RANK_UNIDIRECTIONAL)) == 0u,
                AVEY_ERR_INVALID_ARG, "avey_rank: unknown flags 0x%x", flags);
-  AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
-               "avey_rank: dtype %d unsupported (F32 or BF16)", int(dt));
   AVEY_REQUIRE(x && idx && w && ws, AVEY_ERR_INVALID_ARG, "avey_rank: null pointer");
-  AVEY_REQUIRE(B >= 1 && N >= 1 && d >= 1 && S >= 1 && k >= 1, AVEY_ERR_INVALID_ARG,
-               "avey_rank: sizes must be >= 1 (B=%d N=%d d=%d S=%d k=%d)", B, N, d, S, k);
-  AVEY_REQUIRE(d % 8 == 0, AVEY_ERR_INVALID_ARG, "avey_rank: d=%d must be a multiple of 8", d);
-  AVEY_REQUIRE(k <= 32, AVEY_ERR_UNSUPPORTED, "avey_rank: k=%d > 32", k);
+  {
+    const avey_status sh = check_rank_shape("avey_rank", dt, B, N, d, S, k);
+    if (sh != AVEY_OK) return sh;
+  }
   AVEY_REQUIRE(aligned16(x) && aligned16(ws) && (!scores || aligned16(scores)),
                AVEY_ERR_INVALID_ARG, "avey_rank: pointers must be 16-byte aligned");
   AVEY_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255) == 0, AVEY_ERR_INVALID_ARG,
                "avey_rank: workspace must be 256-byte aligned");
-  if (dt == AVEY_BF16)
-    AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
-                 "avey_rank(BF16): S=%d unsupported (16, 32, 64 or 128)", S);
-  else
-    AVEY_REQUIRE(S <= 128 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
-                 "avey_rank(F32): S=%d unsupported (power of two <= 128)", S);
   const long long n = (N + S - 1) / S, R = n * S;
-  AVEY_REQUIRE(n <= 46340 && static_cast<long long>(B) * R <= (1ll << 31) - 1,
-               AVEY_ERR_UNSUPPORTED, "avey_rank: problem too large");
   const size_t need = avey_rank_workspace_bytes(dt, B, N, d, S);
   AVEY_REQUIRE(ws_bytes >= need, AVEY_ERR_INVALID_ARG,
                "avey_rank: workspace %zu bytes < %zu required", ws_bytes, need);

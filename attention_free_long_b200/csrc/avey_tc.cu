@@ -831,7 +831,7 @@ avey_status run_layer_pair(const CUtensorMap &a0, const CUtensorMap &a1, const C
   }
   const int pairs = std::max(1, std::min(args.num_tiles, cap));
   kern<<<2 * pairs, kThreads, P::SMEM_BYTES, st>>>(a0, a1, b, o0, o1, o2, c0, c1, args);
-  AVEY_CHECK_LAUNCH(name);
+  AVEY_CHECK_LAUNCH(name, st);
   return AVEY_OK;
 }
 
@@ -848,7 +848,7 @@ avey_status run_maxsim_tc(const CUtensorMap &ma, const CUtensorMap &mb, TcArgs a
   }
   const int grid = std::min(args.num_tiles, sm_count());
   kern<<<grid, kThreads, L::SMEM_BYTES, st>>>(ma, mb, args);
-  AVEY_CHECK_LAUNCH("maxsim_tc");
+  AVEY_CHECK_LAUNCH("maxsim_tc", st);
   return AVEY_OK;
 }
 

@@ -4,6 +4,12 @@ One step = one full encoder forward of the long-context workload (batch 1,
 N = 98304 tokens, S = 64, d = 768, m = 1536 (768/768), k = 7, four layers
 S,D,S,D): avey_rank (normalise, MaxSim, top-k) -> avey_compress -> 4 x
 avey_layer_forward, through the C ABI, on inputs already resident in HBM.
+The timed region records one CUDA event after every kernel launch (the
+library's kernel trace), which gives the per-kernel times and the MaxSim
+roofline.  After it, the same line reports the HBM-bound kernels alone, the
+processor without compression, and a second workload (default: batch 4,
+N = 32768, S = 128, d = 1024, m = 2048, k = 15, 12 layers) with its own
+per-kernel breakdown and end-to-end figure.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -18,11 +24,9 @@ workload per step.
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import math
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -175,23 +179,6 @@ def rank_seed(rank: int) -> int:
     return rank
 
 
-def traffic_from_profile(kernel_src: str, workload: str):
-    """DRAM bytes per MaxSim launch from the committed ncu summary, or None when
-    the kernel source changed since that capture or the capture was taken on
-    another workload."""
-    path = os.path.join(ROOT, "profiles", "maxsim_long_bf16.md")
-    if not os.path.exists(path):
-        return None
-    txt = open(path).read()
-    m1 = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
-    m2 = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
-    m3 = re.search(r"traffic_workload:\s*(\S+)", txt)
-    if not (m1 and m2 and m3) or m3.group(1) != workload:
-        return None
-    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
-    return float(m1.group(1)) if sha == m2.group(1) else None
-
-
 def l2_note(wl) -> str:
     """How the timed steps stand to the 126 MB L2 (inputs larger than L2, or not)."""
     x_mb = wl.B * wl.N * wl.d * 2 / 1e6
@@ -246,16 +233,51 @@ def cpu_model() -> str:
 
 # -------------------------------------------------------------- our arm ---
 
-def run_ours(args):
+def _time_alone(call, reps, e0, e1):
+    """Mean device ms of ``call`` (returns an avey status) over ``reps`` calls."""
     import torch
-    import attention_free_long_b200 as av
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = init_dist("nccl", world)
-    barrier = (lambda: dist.barrier(device_ids=[local])) if world > 1 else (lambda: None)
+    for _ in range(3):
+        assert call() == 0
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
 
-    wl = sy.WORKLOADS[args.workload]
+
+def mixes_alone(av, wl, layers, dev, reps):
+    """The split-size static and dynamic mixes timed alone at the layer's shape
+    (in place on Z's tail columns, as inside a layer).  Returns
+    (static_ms or None, dynamic_ms, bytes): the bytes are the algorithmic read
+    of the Z_t pair plus the write of the c pair."""
+    import ctypes
+    import torch
+    T, mt = wl.T, wl.m_t
+    zpair = torch.rand((2, T, wl.m), device=dev).to(torch.bfloat16)
+    zt = zpair[:, :, wl.m_h:]
+    L = av.lib()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    zp = ctypes.c_void_p(zt.data_ptr())
+    dyn = _time_alone(lambda: L.avey_dynamic_mix(zp, wl.m, av.AVEY_BF16X2, T // wl.S, wl.S, mt,
+                                                 wl.eps, zp, wl.m, av._stream()), reps, e0, e1)
+    stat = None
+    vstat = next((l_.V for l_ in layers if l_.kind == av.AVEY_STATIC), None)
+    if vstat is not None:
+        vp = ctypes.c_void_p(vstat.data_ptr())
+        stat = _time_alone(lambda: L.avey_static_mix(vp, zp, wl.m, av.AVEY_BF16X2, T // wl.S, wl.S,
+                                                     mt, zp, wl.m, av._stream()), reps, e0, e1)
+    del zpair, zt
+    torch.cuda.empty_cache()
+    return stat, dyn, 2.0 * T * mt * 4
+
+
+def forward_leg(av, wl, dev, args, rank, world, local, barrier, e2e=True, sample_clocks=True):
+    """One workload through encoder_forward: warm-up, the device-timed region
+    (inputs resident in HBM; per-call events and a kernel trace recorded
+    live), then the same forward end to end with host buffers."""
+    import torch
     E = sy.gen_embeddings(wl, seed=rank_seed(rank))
     W = sy.gen_weights(wl)
     dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -272,74 +294,181 @@ def run_ours(args):
     torch.cuda.synchronize()
     st = av.device_status()
     if st != 0:
-        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after warm-up")
+        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after warm-up ({wl.name})")
 
-    # ---- device-timed region: inputs resident in HBM (X is 151 MB > L2) ----
+    # ---- device-timed region ----
     n_marks = 2 + wl.layers
-    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks + 1)] for _ in range(args.steps)]
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks + 1)]
+             for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    per_step = 4 + 3 * wl.layers  # upper bound of launches per forward
+    trace = av.KernelTrace(capacity=args.steps * per_step + 8)
     barrier()
     torch.cuda.synchronize()
     l0 = av.kernel_launches()
-    with ClockSampler(local) as clk:
-        start.record()
-        for s in range(args.steps):
-            step(marks[s])
-        end.record()
+    clk = ClockSampler(local) if sample_clocks else None
+    if clk is not None:
+        clk.__enter__()
+    try:
+        with trace:
+            start.record()
+            for s_ in range(args.steps):
+                step(marks[s_])
+            end.record()
         torch.cuda.synchronize()
+    finally:
+        if clk is not None:
+            clk.__exit__(None, None, None)
     launches = av.kernel_launches() - l0
     barrier()
     torch.cuda.synchronize()
     ms = start.elapsed_time(end) / args.steps
     ms_max = max_over_ranks(ms, dev)
-    stage = np.array([[marks[s][i].elapsed_time(marks[s][i + 1]) for i in range(n_marks)]
-                      for s in range(args.steps)]).mean(axis=0)
-    rank_ms, compress_ms, layer_ms = float(stage[0]), float(stage[1]), stage[2:].tolist()
+    stage = np.array([[marks[s_][i].elapsed_time(marks[s_][i + 1]) for i in range(n_marks)]
+                      for s_ in range(args.steps)]).mean(axis=0)
     st = av.device_status()
     if st != 0:
-        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after the timed region")
+        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after the timed region ({wl.name})")
+    kern = {}
+    for name, kms in trace.kernels():
+        kern.setdefault(name, []).append(kms)
+    kernels = {name: {"ms_per_launch": float(np.mean(v)), "launches_per_step": len(v) / args.steps,
+                      "ms_per_step": float(np.sum(v)) / args.steps} for name, v in kern.items()}
+    out = {"wl": wl, "ms": ms_max, "value": wl.B * wl.N * world / (ms_max * 1e-3),
+           "kernels_ms": {"rank": float(stage[0]), "compress": float(stage[1]),
+                          "layers": stage[2:].tolist()},
+           "kernels": kernels, "launches": int(launches),
+           "clocks": clk.summary() if clk is not None else None,
+           "layers": layers, "E": E, "W": W}
+    if not e2e:
+        del ws, x, P
+        torch.cuda.empty_cache()
+        return out
 
-    # ---- dynamic mix alone at the layer's shape (HBM-bound kernel) ----
-    T, mt = wl.T, wl.m_t
-    zpair = torch.rand((2, T, wl.m), device=dev).to(torch.bfloat16)
-    zt = zpair[:, :, wl.m_h:]
-    L = av.lib()
-    import ctypes
-    mix_call = lambda: L.avey_dynamic_mix(ctypes.c_void_p(zt.data_ptr()), wl.m, av.AVEY_BF16X2,
-                                          T // wl.S, wl.S, mt, wl.eps,
-                                          ctypes.c_void_p(zt.data_ptr()), wl.m, av._stream())
-    for _ in range(3):
-        assert mix_call() == 0
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = max(10, args.steps)
-    e0.record()
-    for _ in range(reps):
-        mix_call()
-    e1.record()
+    # ---- end to end through the public API with host buffers ----
+    # Every step copies its input embeddings host -> device (pinned) and its
+    # fp32 output device -> host.  Double-buffered: the copies of steps i+1 and
+    # i-1 run on their own streams while step i computes.
+    xh = torch.from_numpy(E.X).to(dt).pin_memory()
+    outh = [torch.empty((wl.B, wl.n * wl.S, wl.d), dtype=torch.float32).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x) for _ in range(2)]
+    wss = [ws, av.make_workspace(wl.B, wl.N, wl.d, wl.S, wl.k, wl.m, dt, wl.prenorm, dev)]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    started = [False, False]
+
+    def e2e_step(i):
+        j = i & 1
+        with torch.cuda.stream(s_in):
+            if started[j]:
+                s_in.wait_event(comp_done[j])  # the compute that read xd[j] is done
+            xd[j].copy_(xh, non_blocking=True)
+            h2d_done[j].record(s_in)
+        comp.wait_event(h2d_done[j])
+        if started[j]:
+            comp.wait_event(d2h_done[j])  # the output in wss[j] has been copied out
+        o = av.encoder_forward(xd[j], P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm, wss[j])
+        comp_done[j].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[j])
+            outh[j].copy_(o, non_blocking=True)
+            d2h_done[j].record(s_out)
+        started[j] = True
+
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
-    mix_ms = e0.elapsed_time(e1) / reps
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for st_ in (s_in, s_out):
+        st_.wait_event(start)
+    for i in range(args.steps):
+        e2e_step(i)
+    for st_ in (s_in, s_out):
+        e_ = ev()
+        e_.record(st_)
+        comp.wait_event(e_)
+    end.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
+    st = av.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after the e2e region ({wl.name})")
+    out["e2e"] = {"value": wl.B * wl.N * world / (e2e_ms * 1e-3), "unit": UNIT,
+                  "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
+                  "d2h_bytes_per_step": int(outh[0].numel() * outh[0].element_size()),
+                  "note": "copies of neighbouring steps overlap compute (two buffers, copy streams)"}
+    del wss, xd, outh, xh, ws, x, P
+    torch.cuda.empty_cache()
+    return out
 
-    def time_alone(call, reps_):
-        for _ in range(3):
-            assert call() == 0
-        e0.record()
-        for _ in range(reps_):
-            call()
-        e1.record()
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / reps_
 
-    # ---- static mix alone at the layer's shape (V of the first static layer) ----
-    smix_ms = None
-    vstat = next((l_.V for l_ in layers if l_.kind == av.AVEY_STATIC), None)
-    if vstat is not None:
-        smix_ms = time_alone(lambda: L.avey_static_mix(
-            ctypes.c_void_p(vstat.data_ptr()), ctypes.c_void_p(zt.data_ptr()), wl.m, av.AVEY_BF16X2,
-            T // wl.S, wl.S, mt, ctypes.c_void_p(zt.data_ptr()), wl.m, av._stream()), reps)
-    del zpair, zt
+def maxsim_roofline(wl, leg, peaks, peak_kind):
+    """MaxSim's tensor roofline from its launches inside the timed region."""
+    name = "maxsim_pair" if wl.S >= 32 else "maxsim_tc"
+    k = leg["kernels"].get(name)
+    if k is None:
+        return None
+    kms = k["ms_per_launch"]
+    burst = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    sustained = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    executed = maxsim_executed_flops(wl)
+    achieved = executed / (kms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": burst,
+            "unit": "TFLOP/s", "frac": achieved / burst,
+            "peak_kind": f"{peak_kind} bf16 burst (cuBLAS)",
+            "frac_of_sustained": achieved / sustained, "peak_sustained": sustained,
+            "kernel_ms": kms, "executed_flop_per_launch": executed,
+            "definition_flop_per_launch": maxsim_flops(wl),
+            "traffic": None,
+            "note": ("achieved = the MMA work the kernel issues (the 256x256 tiles on or right of the "
+                     "diagonal; each yields the scores of a split pair in both directions) / its "
+                     "mean launch time inside the timed region (kernel trace events on the launch "
+                     "stream); definition_flop_per_launch counts 2 (nS)^2 d, both directions in "
+                     "full; traffic is null: DRAM bytes come from an ncu capture, not this run")}
+
+
+def _hbm(ms, nbytes, peak):
+    if ms is None:
+        return None
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": ms, "gbs": gbs, "frac": gbs / peak, "bytes": nbytes}
+
+
+def run_ours(args):
+    import torch
+    import attention_free_long_b200 as av
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl", world)
+    barrier = (lambda: dist.barrier(device_ids=[local])) if world > 1 else (lambda: None)
+    peaks, peak_kind = load_peaks()
+    hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+
+    wl = sy.WORKLOADS[args.workload]
+    leg = forward_leg(av, wl, dev, args, rank, world, local, barrier)
+    layers, E, W = leg["layers"], leg["E"], leg["W"]
+    reps = max(10, args.steps)
+
+    # ---- HBM-bound kernels: the mixes alone at the layer's shape and inside
+    # the forward (kernel trace), compression inside the forward ----
+    smix_ms, mix_ms, mix_bytes = mixes_alone(av, wl, layers, dev, reps)
+    kin = leg["kernels"]
+    dyn_in = kin.get("dynamic_mix_x2", {}).get("ms_per_launch")
+    stat_in = kin.get("static_mix_x2", {}).get("ms_per_launch")
+    comp_ms = (kin.get("compress_tc") or kin.get("compress_bf16") or {}).get("ms_per_launch")
+    comp_bytes = compress_bytes(wl)
 
     # ---- top-k alone: at the workload's shape, and on a larger sweep where
     # the score matrix (5.4 GB) is far past L2 and launch latency ----
+    import ctypes
+    L = av.lib()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
     def topk_time(B_, n_, reps_):
         # timed as a captured CUDA graph of reps_ launches, so that host-side
         # call overhead does not hide the kernel at small sizes
@@ -371,70 +500,19 @@ def run_ours(args):
     sweep_B, sweep_n = 9, 12288
     sweep_ms, sweep_bytes = topk_time(sweep_B, sweep_n, 5)
     torch.cuda.empty_cache()
-
-    # ---- end to end through the public API with host buffers ----
-    # Every step copies its input embeddings host -> device (pinned) and its
-    # fp32 output device -> host.  Double-buffered: the copies of steps i+1 and
-    # i-1 run on their own streams while step i computes.
-    xh = torch.from_numpy(E.X).to(dt).pin_memory()
-    outh = [torch.empty((wl.B, wl.n * wl.S, wl.d), dtype=torch.float32).pin_memory() for _ in range(2)]
-    xd = [torch.empty_like(x) for _ in range(2)]
-    wss = [ws, av.make_workspace(wl.B, wl.N, wl.d, wl.S, wl.k, wl.m, dt, wl.prenorm, dev)]
-    comp = torch.cuda.current_stream()
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    ev = lambda: torch.cuda.Event()
-    h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
-    started = [False, False]
-
-    def e2e_step(i):
-        j = i & 1
-        with torch.cuda.stream(s_in):
-            if started[j]:
-                s_in.wait_event(comp_done[j])  # the compute that read xd[j] is done
-            xd[j].copy_(xh, non_blocking=True)
-            h2d_done[j].record(s_in)
-        comp.wait_event(h2d_done[j])
-        if started[j]:
-            comp.wait_event(d2h_done[j])  # the output in wss[j] has been copied out
-        out = av.encoder_forward(xd[j], P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm, wss[j])
-        comp_done[j].record(comp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(comp_done[j])
-            outh[j].copy_(out, non_blocking=True)
-            d2h_done[j].record(s_out)
-        started[j] = True
-
-    for i in range(2):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    start.record()
-    for st_ in (s_in, s_out):
-        st_.wait_event(start)
-    for i in range(args.steps):
-        e2e_step(i)
-    for st_ in (s_in, s_out):
-        e_ = ev()
-        e_.record(st_)
-        comp.wait_event(e_)
-    end.record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
-    st = av.device_status()
-    if st != 0:
-        raise RuntimeError(f"device status {av.STATUS.get(st, st)} after the e2e region")
-    h2d_bytes = int(xh.numel() * xh.element_size())
-    d2h_bytes = int(outh[0].numel() * outh[0].element_size())
-    del wss, xd, outh, xh
-    torch.cuda.empty_cache()
+    norms_ms = kin.get("inv_norms", {}).get("ms_per_launch")
+    norms_bytes = wl.B * wl.N * wl.d * 2.0 + wl.B * wl.n * wl.S * 4.0
 
     # ---- the processor without neural compression, same workload ----
     # Every split's (k+1)S-token context goes through the layers as one block
     # (Avey-B paperlayer summary §4.3); the pages report compression as a
     # 4.37x throughput gain over this.
     unc = None
+    n_marks = 2 + wl.layers
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if not args.no_uncompressed:
+        dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        x = torch.from_numpy(E.X).to(dev, dt)
         Wu = sy.gen_weights(wl, block=(wl.k + 1) * wl.S)
         layers_u = av.device_layers(Wu, dt, dev)
         ws_u = av.make_workspace(wl.B, wl.N, wl.d, wl.S, wl.k, wl.m, dt, wl.prenorm, dev,
@@ -464,70 +542,67 @@ def run_ours(args):
         st_u = np.array([[marks_u[r_][i].elapsed_time(marks_u[r_][i + 1]) for i in range(n_marks)]
                          for r_ in range(reps_u)]).mean(axis=0)
         unc = {"ms_per_step": ms_u, "value": wl.B * wl.N * world / (ms_u * 1e-3), "unit": UNIT,
-               "steps": reps_u, "compression_speedup": ms_u / ms_max, "pages_speedup": 4.37,
+               "steps": reps_u, "compression_speedup": ms_u / leg["ms"], "pages_speedup": 4.37,
                "kernels_ms": {"rank": float(st_u[0]), "context": float(st_u[1]),
                               "layers": st_u[2:].tolist()},
                "note": ("each split's (k+1)S-token context through every layer as one block; "
                         "compression_speedup = uncompressed / compressed ms per step on this GPU; "
                         "pages_speedup is the pages' figure (their hardware and code)")}
-        del ws_u, layers_u
+        del ws_u, layers_u, x
+        torch.cuda.empty_cache()
+
+    # ---- the large workload (batch 4, N = 32768, S = 128, d = 1024,
+    # m = 2048, k = 15, 12 layers): per-kernel breakdown and end to end ----
+    large = None
+    if args.large_workload != "none":
+        wl5 = sy.WORKLOADS[args.large_workload]
+        leg5 = forward_leg(av, wl5, dev, args, rank, world, local, barrier)
+        s5, d5, b5 = mixes_alone(av, wl5, leg5["layers"], dev, reps)
+        k5 = leg5["kernels"]
+        ksum = sum(v["ms_per_step"] for v in k5.values())
+        large = {"config": {"workload": workload_desc(wl5), "global_batch": wl5.B * world,
+                            "seq_len": wl5.N, "l2": l2_note(wl5)},
+                 "value": leg5["value"], "unit": UNIT, "ms_per_step": leg5["ms"],
+                 "steps": args.steps, "kernels_ms": leg5["kernels_ms"], "kernels": k5,
+                 "kernel_sum_ms": ksum, "e2e": leg5["e2e"],
+                 "roofline": maxsim_roofline(wl5, leg5, peaks, peak_kind),
+                 "layers_executed_tflops": layer_flops(wl5) * 2 / (sum(leg5["kernels_ms"]["layers"]) * 1e-3) / 1e12,
+                 "mixes_alone": {"static": _hbm(s5, b5, hbm), "dynamic": _hbm(d5, b5, hbm)},
+                 "clocks": leg5["clocks"], "gpu_launches": leg5["launches"]}
+        del leg5
         torch.cuda.empty_cache()
 
     tokens = wl.B * wl.N * world
-    peaks, peak_kind = load_peaks()
-    sustained = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
-    hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
-    achieved = maxsim_flops(wl) / (rank_ms * 1e-3) / 1e12
-    mix_bytes = 2.0 * T * mt * 4  # read Z_t pair, write c pair
-    comp_bytes = compress_bytes(wl)
-    kernel_src = os.path.join(ROOT, "attention_free_long_b200", "csrc", "avey_maxsim2.cu")
+    ksum = sum(v["ms_per_step"] for v in kin.values())
     result = {
-        "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "metric": METRIC, "value": leg["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": leg["ms"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian mixture, random N(0,1/fan_in) weights)",
         "config": {"workload": workload_desc(wl), "global_batch": wl.B * world, "seq_len": wl.N,
                    "parallelism": f"dp{world} (one sequence per GPU, no collective)",
                    "l2": l2_note(wl)},
-        "roofline": {"bound": "tensor", "kernel": "maxsim (avey_rank call)",
-                     "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                     "frac": achieved / sustained,
-                     "peak_kind": f"{peak_kind} bf16 sustained (kernel inside a long step)",
-                     "algorithmic_flop_per_launch": maxsim_flops(wl),
-                     "executed_flop_per_launch": maxsim_executed_flops(wl),
-                     "executed_achieved": maxsim_executed_flops(wl) / (rank_ms * 1e-3) / 1e12,
-                     "executed_frac": maxsim_executed_flops(wl) / (rank_ms * 1e-3) / 1e12 / sustained,
-                     "traffic": traffic_from_profile(kernel_src, wl.name),
-                     "note": ("duration is the whole avey_rank call (norms + MaxSim + top-k); "
-                              "achieved counts the definition's 2(nS)^2 d FLOP, the kernel executes "
-                              "about half of them (each tile yields the scores of a split pair in "
-                              "both directions), executed_* count the MMA work actually issued")},
-        "kernels_ms": {"rank": rank_ms, "compress": compress_ms, "layers": layer_ms},
-        "hbm": {"dynamic_mix": {"ms": mix_ms, "gbs": mix_bytes / (mix_ms * 1e-3) / 1e9,
-                                "frac": mix_bytes / (mix_ms * 1e-3) / 1e9 / hbm,
-                                "peak": hbm, "bytes": mix_bytes},
-                "compress": {"ms": compress_ms, "gbs": comp_bytes / (compress_ms * 1e-3) / 1e9,
-                             "frac": comp_bytes / (compress_ms * 1e-3) / 1e9 / hbm,
-                             "bytes": comp_bytes},
-                "static_mix": None if smix_ms is None else {
-                    "ms": smix_ms, "gbs": mix_bytes / (smix_ms * 1e-3) / 1e9,
-                    "frac": mix_bytes / (smix_ms * 1e-3) / 1e9 / hbm, "bytes": mix_bytes},
-                "topk": {"ms": topk_ms, "gbs": topk_bytes / (topk_ms * 1e-3) / 1e9,
-                         "frac": topk_bytes / (topk_ms * 1e-3) / 1e9 / hbm, "bytes": topk_bytes,
-                         "note": f"{topk_bytes / 1e6:.1f} MB of scores: latency-bound at this size"},
-                "topk_sweep": {"B": sweep_B, "n": sweep_n, "k": wl.k, "ms": sweep_ms,
-                               "gbs": sweep_bytes / (sweep_ms * 1e-3) / 1e9,
-                               "frac": sweep_bytes / (sweep_ms * 1e-3) / 1e9 / hbm,
-                               "bytes": sweep_bytes}},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d_bytes,
-                "d2h_bytes_per_step": d2h_bytes,
-                "note": "copies of neighbouring steps overlap compute (two buffers, copy streams)"},
-        "gpu_launches": int(launches),
-        "clocks": clk.summary(),
+        "roofline": maxsim_roofline(wl, leg, peaks, peak_kind),
+        "kernels_ms": leg["kernels_ms"], "kernels": kin, "kernel_sum_ms": ksum,
+        "hbm": {"peak": hbm, "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                "dynamic_mix": dict(_hbm(mix_ms, mix_bytes, hbm), in_forward=_hbm(dyn_in, mix_bytes, hbm)),
+                "static_mix": None if smix_ms is None else dict(
+                    _hbm(smix_ms, mix_bytes, hbm), in_forward=_hbm(stat_in, mix_bytes, hbm)),
+                "compress": _hbm(comp_ms, comp_bytes, hbm),
+                "inv_norms": _hbm(norms_ms, norms_bytes, hbm),
+                "topk": dict(_hbm(topk_ms, topk_bytes, hbm),
+                             note=f"{topk_bytes / 1e6:.1f} MB of scores: latency-bound at this size"),
+                "topk_sweep": dict(_hbm(sweep_ms, sweep_bytes, hbm), B=sweep_B, n=sweep_n, k=wl.k),
+                "note": ("mixes: alone at the layer's shape, and in_forward from the kernel trace; "
+                         "compression and inverse norms from the kernel trace; top-k alone")},
+        "e2e": leg["e2e"],
+        "gpu_launches": leg["launches"],
+        "clocks": leg["clocks"],
     }
     if unc is not None:
         result["uncompressed"] = unc
+    if large is not None:
+        result["large"] = large
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, E, W)
     if world > 1:
@@ -703,6 +778,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-uncompressed", action="store_true",
                     help="skip the measurement of the processor without compression")
+    ap.add_argument("--large-workload", default="large_bf16",
+                    choices=["none"] + sorted(sy.WORKLOADS),
+                    help="second workload measured after the first (per-kernel breakdown and "
+                         "end to end); none skips it")
     ap.add_argument("--shard", choices=["replicas", "sequence"], default="replicas",
                     help="replicas: one sequence per GPU (weak scaling, no collective); "
                          "sequence: the workload's sequence split across the GPUs (strong scaling)")

@@ -20,6 +20,9 @@
  *   - All pointers are DEVICE pointers unless a parameter says otherwise.  The
  *     caller allocates and owns every buffer, including workspaces; the
  *     library never allocates device memory and keeps no per-call state.
+ *     One exception: avey_rank_static (below) keeps its scratch in a 16 MiB
+ *     device array inside the library, held on every GPU that loads it, whose
+ *     contents persist from one call to the next.
  *   - Row-major, densely packed tensors unless an leading dimension ("ld",
  *     in elements) is given.  Base addresses must be 16-byte aligned.
  *   - Every call is asynchronous on `stream` (0 = legacy default stream).
@@ -128,8 +131,10 @@ AVEY_API avey_status avey_rank_ex(const void *x, avey_dtype dt, int B, int N, in
  *   - It allocates nothing.  A shape whose scratch
  *     (avey_rank_workspace_bytes) exceeds the array is rejected with
  *     AVEY_ERR_UNSUPPORTED before anything is enqueued.
- *   - The first call on each device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, which allocates nothing).  The first call on a
+ *     device may load the library's device code there: make that first call
+ *     before any stream capture.
  *   - All calls share the array, which keeps the previous call's contents; every
  *     call rewrites what it reads.  Calls whose kernels overlap on the GPU
  *     (e.g. on two unordered streams) race on it: order them.
@@ -343,6 +348,27 @@ AVEY_API const char *avey_last_error_detail(void);
  * device status word and the kernel returns.  The next avey_device_status()
  * reports it; the context stays usable. */
 AVEY_API avey_status avey_selftest_wait_timeout(uint32_t limit_us, avey_stream_t stream);
+
+/* Kernel trace: a measurement hook with no counterpart on the pages.  Between
+ * avey_trace_begin and avey_trace_end, every kernel the library launches
+ * records the next of the caller's events on its launch stream, right after
+ * the kernel is enqueued, and the library keeps the kernel's name.  On one
+ * stream, the time from the event before a launch (the previous launch's, or
+ * one the caller recorded) to that launch's event is the kernel's duration.
+ * events     HOST array of `capacity` cudaEvent_t handles (passed as void*),
+ *            created and owned by the caller, none NULL; 1 <= capacity <= 4096.
+ *            Launches beyond `capacity` are counted but record nothing.
+ * avey_trace_begin returns AVEY_ERR_INVALID_ARG for a bad array or while a
+ * trace is already active (one trace per process; the trace is shared by all
+ * host threads).  avey_trace_end returns the number of launches seen (which
+ * may exceed `capacity`), or -1 if no trace was active or an event record
+ * failed (detail in avey_last_error_detail).  avey_trace_kernel_name(i) is
+ * the name of traced launch i < min(count, capacity) of the last finished
+ * trace (a string owned by the library, valid until the next trace begins),
+ * or NULL. */
+AVEY_API avey_status avey_trace_begin(void *const *events, int capacity);
+AVEY_API int avey_trace_end(void);
+AVEY_API const char *avey_trace_kernel_name(int i);
 
 /* avey_kernel_launches: number of kernels this library has launched since it
  * was loaded, in this process (all threads). */

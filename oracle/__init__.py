@@ -257,19 +257,16 @@ def layer(x_splits, lw, S: int, m_h: int, eps: float, prenorm: bool) -> np.ndarr
     return x
 
 
-def forward(X, weights, wl, sel=None, idx=None, w=None, causal: bool = False):
+def forward(X, weights, wl, sel=None, causal: bool = False):
     """Ranker once, compression, then every layer, for selected targets.
 
     X [B, N, d]; weights: synthetic.Weights; wl: synthetic.Workload.
-    If idx / w are given they replace the oracle's own selection (used when a
-    near-tie lets the GPU's selection differ legitimately).
+    The oracle always uses its own selection.
     Returns dict(sel, scores, idx, w, compressed, layers=[per-layer outputs]).
     """
     X = _f64(X)
     sel, scores, oidx, ow = rank(X, wl.S, wl.k, sel, causal)
-    use_idx = oidx if idx is None else _i32(idx)
-    use_w = ow if w is None else _f64(w)
-    xc = compress(X, wl.S, wl.k, sel, use_idx, use_w, weights.P)
+    xc = compress(X, wl.S, wl.k, sel, oidx, ow, weights.P)
     outs = []
     x = xc
     for lw in weights.layers:
@@ -278,7 +275,7 @@ def forward(X, weights, wl, sel=None, idx=None, w=None, causal: bool = False):
     return dict(sel=sel, scores=scores, idx=oidx, w=ow, compressed=xc, layers=outs)
 
 
-def forward_uncompressed(X, weights, wl, sel=None, idx=None, w=None, causal: bool = False):
+def forward_uncompressed(X, weights, wl, sel=None, causal: bool = False):
     """The processor without neural compression ([AB-sum] §4.3: the ablation
     that the 4.37x throughput figure compares against).
 
@@ -292,9 +289,7 @@ def forward_uncompressed(X, weights, wl, sel=None, idx=None, w=None, causal: boo
     """
     X = _f64(X)
     sel, scores, oidx, ow = rank(X, wl.S, wl.k, sel, causal)
-    use_idx = oidx if idx is None else _i32(idx)
-    use_w = ow if w is None else _f64(w)
-    ctx = context(X, wl.S, wl.k, sel, use_idx, use_w)
+    ctx = context(X, wl.S, wl.k, sel, oidx, ow)
     L = (wl.k + 1) * wl.S
     outs = []
     x = ctx

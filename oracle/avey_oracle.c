@@ -18,7 +18,7 @@
  *   [coreui]    "Avey-B架构：无注意力机制的高效双向编码器解析", §1, §3.1
  *               (L2 normalisation before the similarity, eps about 1e-8).
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   - pad rows of the last split are zero vectors; N(0) = 0 through the
  *     floor max(||x||, 1e-12), so a pad row has cosine 0 with every row;
  *   - the candidate set is every other split of the same sequence

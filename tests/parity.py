@@ -9,6 +9,12 @@
   relative (a near tie); the GPU list must never contain the target itself
   or a repeated split, and its top-1 weight must be exactly 1 (unless the
   best score is <= 0, where the weights divide by the 1e-30 floor).
+- Downstream (compression and every layer): every compared row is checked
+  twice.  Once end to end, on the GPU's own selection, for the rows whose
+  list matches the oracle's exactly; and once with the GPU's compression and
+  layers run on the ORACLE's selection (idx and w of the sampled rows
+  replaced by the oracle's), for every row.  Values only ever flow from the
+  oracle to the GPU side, never back.
 """
 import numpy as np
 
@@ -58,3 +64,27 @@ def check_topk(g_idx, g_w, o_idx, o_scores, targets, tol_w):
             ref = s / max(s[0], 1e-30)
             assert rel_err(g_w[r, :sel.size], ref) <= tol_w, f"row {r}: weights"
     return exact
+
+
+def degenerate_rows(o_idx, o_scores):
+    """Rows whose best selected score is <= 1e-30: their weights divide by the
+    1e-30 floor, so the compressed values are meaningless (only reachable with
+    the unidirectional ranker, whose first splits have one or no candidate)."""
+    best = np.array([o_scores[r, o_idx[r, 0]] if o_idx[r, 0] >= 0 else 1.0
+                     for r in range(o_idx.shape[0])])
+    return best <= 1e-30
+
+
+def oracle_selection(g_idx, g_w, sel, o_idx, o_w):
+    """Copies of the GPU's selection tensors [B, n, k] (torch, on the device)
+    whose rows of the sampled targets ``sel`` ((b, t) pairs) hold the
+    oracle's idx / w instead; the other rows keep the GPU's, which no sampled
+    row reads."""
+    import torch
+    idx = g_idx.clone()
+    w = g_w.clone()
+    sb = torch.from_numpy(np.asarray(sel[:, 0], dtype=np.int64)).to(idx.device)
+    st = torch.from_numpy(np.asarray(sel[:, 1], dtype=np.int64)).to(idx.device)
+    idx[sb, st] = torch.from_numpy(np.asarray(o_idx, dtype=np.int32)).to(idx.device)
+    w[sb, st] = torch.from_numpy(np.asarray(o_w, dtype=np.float32)).to(idx.device)
+    return idx, w

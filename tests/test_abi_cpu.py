@@ -142,3 +142,31 @@ def test_fp32_activations_may_be_omitted_only_beside_the_bf16_pair():
     cmp = lambda dt, out, lowp: L.avey_compress(FAKE, dt, 1, 256, 64, 64, 3, FAKE, FAKE, FAKE, out, lowp, None)
     assert cmp(av.AVEY_BF16, None, None) == 1
     assert cmp(av.AVEY_F32, None, FAKE) == 1
+
+
+def test_kernel_trace_rejects_bad_arguments_and_idles_cleanly():
+    L = av.lib()
+    assert L.avey_trace_end() == -1                    # no trace active
+    assert L.avey_trace_begin(None, 4) == 1            # AVEY_ERR_INVALID_ARG
+    arr = (ctypes.c_void_p * 2)(None, None)
+    assert L.avey_trace_begin(arr, 2) == 1             # null events
+    assert L.avey_trace_begin(arr, 0) == 1             # capacity out of range
+    assert L.avey_trace_end() == -1                    # nothing was started
+    assert L.avey_trace_kernel_name(0) is None
+
+
+def test_rank_static_reports_the_shape_error_before_the_scratch_limit():
+    L = av.lib()
+    f = L.avey_rank_static
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    fake = ctypes.c_void_p(256)  # never dereferenced: rejected on the host
+    # S = 48 is unsupported, and this shape would also exceed the scratch array
+    rc = f(fake, av.AVEY_BF16, 1, 48 * 4096, 64, 48, 3, fake, fake, None)
+    assert rc == 2
+    assert "S=48" in L.avey_last_error_detail().decode()
+    # a valid shape beyond the array is rejected for its size
+    rc = f(fake, av.AVEY_BF16, 1, 64 * 4096, 64, 64, 3, fake, fake, None)
+    assert rc == 2
+    assert "scratch" in L.avey_last_error_detail().decode()

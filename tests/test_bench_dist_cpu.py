@@ -54,20 +54,12 @@ def test_single_process_is_identity():
     assert bench.max_over_ranks(3.5) == 3.5
 
 
-def test_traffic_and_l2_notes_follow_the_workload(tmp_path):
-    # the committed MaxSim DRAM traffic belongs to one workload and one kernel
-    # source: another workload, or a changed source, reports no traffic
+def test_l2_notes_follow_the_workload():
     import bench
     import synthetic as sy
-    src = os.path.join(bench.ROOT, "attention_free_long_b200", "csrc", "avey_maxsim2.cu")
-    assert bench.traffic_from_profile(src, "base_bf16") is None
-    other = tmp_path / "k.cu"
-    other.write_text("// another source\n")
-    assert bench.traffic_from_profile(str(other), "long_bf16") is None
-    got = bench.traffic_from_profile(src, "long_bf16")
-    assert got is None or got > 0
     assert "larger than L2" in bench.l2_note(sy.WORKLOADS["long_bf16"])
     assert "fits" in bench.l2_note(sy.WORKLOADS["base_bf16"])
+    assert "larger than L2" in bench.l2_note(sy.WORKLOADS["large_bf16"])
 
 
 def test_compress_bytes_count_what_the_forward_writes():

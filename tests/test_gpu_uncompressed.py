@@ -16,7 +16,7 @@ import torch
 import attention_free_long_b200 as av
 import oracle as orc
 import synthetic as sy
-from tests.parity import TOL, check_topk, rel_err
+from tests.parity import TOL, check_topk, degenerate_rows, oracle_selection, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -168,15 +168,27 @@ def test_uncompressed_long_workload_sampled(cuda_dev):
     out = av.encoder_forward_uncompressed(x, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm)
     torch.cuda.synchronize()
     assert av.device_status() == 0
-    sel = sy.sample_targets(wl, per_seq=4, seed=7)
+    sel = sy.sample_targets(wl, per_seq=16, seed=7)
     sb, st = torch.from_numpy(sel[:, 0]).long(), torch.from_numpy(sel[:, 1]).long()
     g_out = out.cpu()[sb, st].numpy()
     g_idx, g_w = av.avey_rank(x, wl.S, wl.k)
     o = orc.forward_uncompressed(E.X, W, wl, sel=sel)
     exact = check_topk(g_idx.cpu()[sb, st].numpy(), g_w.cpu()[sb, st].numpy(), o["idx"], o["scores"],
                        sel[:, 1], TOL["bf16"])
-    assert exact.any(), "no sampled row has an identical top-k list"
+    assert not degenerate_rows(o["idx"], o["scores"]).any()
+    # end to end on the GPU's own selection, rows whose list is the oracle's
     err = rel_err(g_out[exact], o["out"][exact])
-    assert err <= TOL["bf16"], f"uncompressed output err {err:.3g}"
-    del out, layers
+    assert err <= TOL["bf16"], f"uncompressed output, own selection: err {err:.3g}"
+    # every sampled row: the same processor on the oracle's selection
+    del out
+    idx2, w2 = oracle_selection(g_idx, g_w, sel, o["idx"], o["w"])
+    out2 = av.processor_forward_uncompressed(x, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm,
+                                             idx2, w2)
+    torch.cuda.synchronize()
+    assert av.device_status() == 0
+    err2 = rel_err(out2.cpu()[sb, st].numpy(), o["out"])
+    assert err2 <= TOL["bf16"], f"uncompressed output, oracle selection: err {err2:.3g}"
+    print(f"uncompressed long_bf16: {sel.shape[0]} sampled splits, "
+          f"{int((~exact).sum())} near-tie lists, all compared")
+    del out2, layers
     torch.cuda.empty_cache()

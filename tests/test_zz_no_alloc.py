@@ -1,7 +1,7 @@
 """avey_rank_static, the ranker entry point for callers that cannot allocate
 device memory (its scratch is a fixed array inside the library), against
 avey_rank with a caller workspace.  Called through the C ABI directly, twice in
-a row, on two shapes; this file is collected last so that a run stopping at the
+a row, on three shapes (the second call must leave device memory untouched); this file is collected last so that a run stopping at the
 first failure has already run every other test."""
 import ctypes
 
@@ -27,6 +27,7 @@ def _static_fn():
 
 @pytest.mark.parametrize("wl", [
     sy.custom("static_s64", B=2, N=3000, S=64, d=256, k=7, centers=24, sigma=0.5),
+    sy.custom("static_s16_bf16", B=2, N=1500, S=16, d=128, k=5, centers=24, sigma=0.4),
     sy.custom("static_s16_f32", B=1, N=500, S=16, d=64, k=3, dtype="f32", centers=16, sigma=0.3),
 ], ids=lambda w: w.name)
 def test_static_scratch_matches_workspace_entry_point(wl, cuda_dev):
@@ -36,13 +37,20 @@ def test_static_scratch_matches_workspace_entry_point(wl, cuda_dev):
     ref_idx, ref_w = av.avey_rank(x, wl.S, wl.k)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     code = av.AVEY_BF16 if wl.dtype == "bf16" else av.AVEY_F32
-    for _ in range(2):  # the second call reuses the array left by the first
+    for call in range(2):  # the second call reuses the array left by the first
         idx = torch.full_like(ref_idx, -7)
         w = torch.full_like(ref_w, -7.0)
+        torch.cuda.synchronize()
+        before = (torch.cuda.memory_allocated(cuda_dev), torch.cuda.mem_get_info(cuda_dev)[0])
         rc = f(ctypes.c_void_p(x.data_ptr()), code, wl.B, wl.N, wl.d, wl.S, wl.k,
                ctypes.c_void_p(idx.data_ptr()), ctypes.c_void_p(w.data_ptr()), stream)
         assert rc == 0, av.lib().avey_last_error_detail().decode()
         torch.cuda.synchronize()
+        after = (torch.cuda.memory_allocated(cuda_dev), torch.cuda.mem_get_info(cuda_dev)[0])
+        if call == 1:
+            # nothing allocated: neither through torch nor on the device
+            # (the first call may still load the library's device code)
+            assert after == before, (before, after)
         assert av.device_status() == 0
         assert torch.equal(idx, ref_idx)
         np.testing.assert_allclose(w.cpu().numpy(), ref_w.cpu().numpy(), rtol=1e-6, atol=0)
