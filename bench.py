@@ -458,7 +458,7 @@ def run_ours(args):
     # the forward (kernel trace), compression inside the forward ----
     smix_ms, mix_ms, mix_bytes = mixes_alone(av, wl, layers, dev, reps)
     kin = leg["kernels"]
-    dyn_in = kin.get("dynamic_mix_x2", {}).get("ms_per_launch")
+    dyn_in = kin.get("dynamic_mix_tc", {}).get("ms_per_launch")
     stat_in = kin.get("static_mix_x2", {}).get("ms_per_launch")
     comp_ms = (kin.get("compress_tc") or kin.get("compress_bf16") or {}).get("ms_per_launch")
     comp_bytes = compress_bytes(wl)

@@ -39,17 +39,22 @@ def _planes(a, split):
     return hi, (_bf16(a - hi) if split else np.zeros_like(hi))
 
 
-def emulate_layer(x, lw, m_h, eps, prenorm, split):
-    """One layer on splits x [n_sp, S, d] with the GPU's rounding points."""
+def emulate_layer(x, lw, m_h, eps, prenorm, plan):
+    """One layer on splits x [n_sp, S, d] with the GPU's rounding points.
+
+    plan = (x_pair, z_pair, fuser_pair): split pairs for the enricher input,
+    for Z / c / Gt, and for the fuser's A operand [Z_h || c] (its lo planes);
+    False keeps one bf16 plane there."""
+    x_pair, z_pair, fuser_pair = plan
     out = np.empty_like(x)
     for sp in range(x.shape[0]):
-        xh, xl = _planes(x[sp], split)
+        xh, xl = _planes(x[sp], x_pair)
         scale = 1.0
         if prenorm:
             xr = xh + xl
             scale = _f32(1.0 / np.sqrt((xr * xr).mean(axis=1, keepdims=True) + 1e-6))
         a = _f32(_f32(xh @ lw.U + xl @ lw.U) * scale + lw.bU)
-        zh, zl = _planes(np.maximum(a, 0.0) ** 2, split)
+        zh, zl = _planes(np.maximum(a, 0.0) ** 2, z_pair)
         th, tl = zh[:, m_h:], zl[:, m_h:]
         if lw.V is not None:  # static: c = V Z_t, V bf16
             c = _f32(lw.V @ (th + tl))
@@ -58,23 +63,26 @@ def emulate_layer(x, lw, m_h, eps, prenorm, split):
             nrm = np.maximum(np.sqrt(np.diag(G)), 1e-12)
             cos = _f32(G / nrm[:, None] / nrm[None, :])
             Gt = _f32(cos / (cos.sum(axis=1, keepdims=True) + eps))
-            gh, gl = _planes(Gt, split)
+            gh, gl = _planes(Gt, z_pair)
             c = _f32(gh @ th + gl @ th + gh @ tl)
-        ch, cl = _planes(c, split)
+        ch, cl = _planes(c, z_pair)
         Ah = np.concatenate([zh[:, :m_h], ch], axis=1)
-        Al = np.concatenate([zl[:, :m_h], cl], axis=1)
+        Al = np.concatenate([zl[:, :m_h], cl], axis=1) if fuser_pair else np.zeros_like(Ah)
         out[sp] = _f32(x[sp] + _f32(Ah @ lw.O + Al @ lw.O))
     return out
 
 
-def _stack_errors(wl, per_seq, split):
+ALL_BF16, PAIRS = (False, False, False), (True, True, True)
+
+
+def _stack_errors(wl, per_seq, plan):
     E, W = sy.gen_embeddings(wl), sy.gen_weights(wl)
     sel = sy.sample_targets(wl, per_seq, seed=3)
     o = orc.forward(E.X, W, wl, sel=sel)
     x = _f32(o["compressed"])
     errs = []
     for li, lw in enumerate(W.layers):
-        x = emulate_layer(x, lw, wl.m_h, wl.eps, wl.prenorm, split)
+        x = emulate_layer(x, lw, wl.m_h, wl.eps, wl.prenorm, plan)
         errs.append(rel_err(x, o["layers"][li]))
     return errs
 
@@ -90,10 +98,21 @@ def _reduced(name, n_splits):
 def test_split_pairs_hold_the_bound_and_all_bf16_does_not(name, n_splits, per_seq):
     wl = _reduced(name, n_splits)
     tol = TOL["bf16"]
-    one = _stack_errors(wl, per_seq, split=False)
-    two = _stack_errors(wl, per_seq, split=True)
+    one = _stack_errors(wl, per_seq, ALL_BF16)
+    two = _stack_errors(wl, per_seq, PAIRS)
     print(f"{name}: all bf16 {['%.2e' % e for e in one]}; split pairs {['%.2e' % e for e in two]}")
     assert max(two) < tol / 10, two
     assert one[-1] > tol, one
     if name == "long_bf16":
         assert one[0] > tol, one  # already the first layer
+
+
+@pytest.mark.parametrize("plan", [(False, True, True), (True, True, False)],
+                         ids=["enricher_input_one_plane", "fuser_input_one_plane"])
+def test_each_layer_gemm_needs_its_pair(plan):
+    # dropping the lo plane of either GEMM's A operand alone already breaks
+    # the bound within the long workload's four layers
+    wl = _reduced("long_bf16", 32)
+    errs = _stack_errors(wl, 6, plan)
+    print(plan, ['%.2e' % e for e in errs])
+    assert errs[-1] > TOL["bf16"], errs
