@@ -5,20 +5,14 @@
 //             c = Gt Z_t
 // Identity activation, no bias.
 //
-// bf16 path: Z_t is an activation split pair (hi, lo bf16 planes).  Both
-// kernels are bound by HBM (read Z_t, write c, 8 bytes per element each way):
+// bf16 path: Z_t is an activation split pair (hi, lo bf16 planes).  The
+// static mix is bound by HBM (read Z_t, write c, 8 bytes per element each way):
 //   static_mix_x2   one CTA per (block, feature slab); V and both planes of
 //                   the slab in shared memory; c = V Z_hi + V Z_lo with
 //                   mma.sync; written back in place as a split pair.
-//   dynamic_mix_x2  one CTA per block, two passes over Z_t in 64-feature
-//                   chunks (the second pass mostly hits L2):
-//                   1. from the hi plane only: Gram R = Z_hi Z_hi^T (mma.sync)
-//                      and fp32 row sums of squares, so G is the cosine matrix
-//                      of the hi vectors (within about 1e-4 of the exact one);
-//                   2. G = R / (n_i n_j), row sums, Gt in fp32, split to bf16
-//                      hi/lo in shared memory (all threads, 256 / S per row);
-//                   3. c = Gt_hi Z_hi + Gt_lo Z_hi + Gt_hi Z_lo, split pair out.
-// fp32 path: plain SIMT kernels.
+// The bf16 dynamic (and coupled causal) mix runs on tcgen05 in
+// avey_mix_dyn.cu.  fp32 path: plain SIMT kernels, and the C ABI entry points
+// of both mixes.
 #include <algorithm>
 
 #include "avey_common.cuh"
@@ -130,251 +124,6 @@ __global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V,
   }
 }
 
-// --------------------------------------------------------------- dynamic --
-
-template <int S>
-struct DynTile {
-  static constexpr int FC = 64;  // feature chunk
-  static constexpr int CLD = FC + 8;
-  static constexpr int CBYTES = S * CLD * 2;  // one plane of one chunk
-  static constexpr int BUF = 2 * CBYTES;      // hi + lo
-  // Gram tiling (S x S)
-  static constexpr int GW_M = S == 16 ? 1 : (S == 128 ? 4 : 2);
-  static constexpr int GW_N = S == 16 ? 2 : (S == 128 ? 2 : 4);
-  static constexpr int GMI = (S / GW_M) / 16, GNI = (S / GW_N) / 8;
-  // apply tiling (S x FC)
-  static constexpr int AW_M = S == 16 ? 1 : (S == 128 ? 4 : 2);
-  static constexpr int AW_N = S == 16 ? 4 : (S == 128 ? 2 : 4);
-  static constexpr int AMI = (S / AW_M) / 16, ANI = (FC / AW_N) / 8;
-  static constexpr int GLD = S + 8;             // bf16 Gt row
-  static constexpr int GBYTES = S * GLD * 2;
-  static constexpr int FLD = S + 4;             // fp32 G row
-  static constexpr int TR = 256 / S;            // threads per row (sums of squares, eq. 6)
-  static constexpr int SMEM = 2 * BUF + 2 * GBYTES;
-  static_assert(S * FLD * 4 <= 2 * BUF, "fp32 G must fit in the chunk buffers");
-};
-
-// COUPLED = false: eq. 6 (Avey-B dynamic layer).  COUPLED = true: the
-// original Avey's coupled causal map M_ij = V_ij G_ij (j <= i), no row
-// normalisation; everything else is shared.
-template <int S, bool COUPLED>
-__global__ void __launch_bounds__(256) dynamic_mix_x2(const bf16 *zt, long long ld_zt,
-                                                      long long plane_zt, bf16 *out,
-                                                      long long ld_out, long long plane_out,
-                                                      int mt, float eps,
-                                                      const bf16 *__restrict__ V) {
-  using C = DynTile<S>;
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t *bufs = smem;                       // 2 x (hi, lo) chunks; later fp32 G
-  uint8_t *gth = smem + 2 * C::BUF;           // Gt hi [S][GLD]
-  uint8_t *gtl = gth + C::GBYTES;             // Gt lo
-  __shared__ float s_ss[S * C::TR];
-  __shared__ float s_nf[S];
-  const int blk = blockIdx.x;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bf16 *zb = zt + static_cast<long long>(blk) * S * ld_zt;
-  bf16 *ob = out + static_cast<long long>(blk) * S * ld_out;
-  const int nchunks = (mt + C::FC - 1) / C::FC;
-
-  auto load_chunk = [&](int ch, int buf, bool with_lo) {
-    uint8_t *h = bufs + buf * C::BUF;
-    uint8_t *l = h + C::CBYTES;
-    for (int e = tid; e < S * (C::FC / 8); e += 256) {
-      const int row = e / (C::FC / 8), cc = e % (C::FC / 8);
-      const int f = ch * C::FC + cc * 8;
-      const bool ok = f < mt;
-      const bf16 *src = ok ? zb + row * ld_zt + f : zb;
-      cp_async16(smem_u32(h + (row * C::CLD + cc * 8) * 2), src, ok ? 16 : 0);
-      if (with_lo)
-        cp_async16(smem_u32(l + (row * C::CLD + cc * 8) * 2), ok ? src + plane_zt : zb, ok ? 16 : 0);
-    }
-    cp_async_commit();
-  };
-
-  // ---- pass 1: Gram of the hi plane and row sums of squares ----
-  const int gwm = warp / C::GW_N, gwn = warp % C::GW_N;
-  const bool gram_warp = warp < C::GW_M * C::GW_N;
-  float g[C::GMI][C::GNI][4] = {};
-  const int sr = tid % S, sp = tid / S;  // sum-of-squares row / part
-  float ss = 0.f;
-  load_chunk(0, 0, false);
-  for (int ch = 0; ch < nchunks; ++ch) {
-    if (ch + 1 < nchunks) {
-      load_chunk(ch + 1, (ch + 1) & 1, false);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint8_t *h = bufs + (ch & 1) * C::BUF;
-    {
-      constexpr int FPT = C::FC / C::TR;  // features per thread
-#pragma unroll
-      for (int q = 0; q < FPT; q += 2) {
-        const int f = sp * FPT + q;
-        const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t *>(h + (sr * C::CLD + f) * 2));
-        ss = fmaf(a.x, a.x, ss);
-        ss = fmaf(a.y, a.y, ss);
-      }
-    }
-    if (gram_warp) {
-#pragma unroll
-      for (int kk = 0; kk < C::FC; kk += 16) {
-        uint32_t af[C::GMI][4];
-#pragma unroll
-        for (int i = 0; i < C::GMI; ++i) {
-          const int row = gwm * (S / C::GW_M) + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          ldsm_x4(smem_u32(h + (row * C::CLD + kk + (lane >> 4) * 8) * 2), af[i][0], af[i][1],
-                  af[i][2], af[i][3]);
-        }
-#pragma unroll
-        for (int j = 0; j < C::GNI; ++j) {
-          uint32_t b0, b1;
-          const int jrow = gwn * (S / C::GW_N) + j * 8 + (lane & 7);
-          ldsm_x2(smem_u32(h + (jrow * C::CLD + kk + ((lane >> 3) & 1) * 8) * 2), b0, b1);
-          const uint32_t bb[2] = {b0, b1};
-#pragma unroll
-          for (int i = 0; i < C::GMI; ++i) mma16816(g[i][j], af[i], bb);
-        }
-      }
-    }
-    __syncthreads();
-  }
-
-  // ---- pass 2: eq. 6 in fp32 ----
-  float *G = reinterpret_cast<float *>(bufs);
-  if (gram_warp) {
-#pragma unroll
-    for (int i = 0; i < C::GMI; ++i)
-#pragma unroll
-      for (int j = 0; j < C::GNI; ++j)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int row = gwm * (S / C::GW_M) + i * 16 + (lane >> 2) + hh * 8;
-          const int col = gwn * (S / C::GW_N) + j * 8 + (lane & 3) * 2;
-          G[row * C::FLD + col] = g[i][j][2 * hh];
-          G[row * C::FLD + col + 1] = g[i][j][2 * hh + 1];
-        }
-  }
-  s_ss[sr * C::TR + sp] = ss;
-  __syncthreads();
-  if (tid < S) {
-    float t2 = 0.f;
-    for (int p = 0; p < C::TR; ++p) t2 += s_ss[tid * C::TR + p];
-    s_nf[tid] = fmaxf(sqrtf(t2), 1e-12f);
-  }
-  __syncthreads();
-  {
-    // All 256 threads: TR consecutive threads per row i, S / TR columns each.
-    // The cosines, the row sum (a shuffle reduction among the row's threads)
-    // and Gt = G / (row sum + eps) as a split pair, in one step.
-    constexpr int CPT = S / C::TR;
-    const int i = tid / C::TR, part = tid % C::TR;
-    const float ni = s_nf[i];
-    float v[CPT];
-    float rs = 0.f;
-#pragma unroll
-    for (int q = 0; q < CPT; ++q) {
-      const int j = part * CPT + q;
-      v[q] = G[i * C::FLD + j] / (ni * s_nf[j]);
-      rs += v[q];
-    }
-#pragma unroll
-    for (int off = 1; off < C::TR; off <<= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
-    const float den = rs + eps;
-#pragma unroll
-    for (int q = 0; q < CPT; ++q) {
-      const int j = part * CPT + q;
-      float out;
-      if constexpr (COUPLED)
-        out = j <= i ? __bfloat162float(V[i * S + j]) * v[q] : 0.f;
-      else
-        out = v[q] / den;
-      float hi, lo;
-      split_bf16(out, hi, lo);
-      reinterpret_cast<bf16 *>(gth)[i * C::GLD + j] = __float2bfloat16_rn(hi);
-      reinterpret_cast<bf16 *>(gtl)[i * C::GLD + j] = __float2bfloat16_rn(lo);
-    }
-  }
-  __syncthreads();
-
-  // ---- pass 3: c = Gt Z_t ----
-  const int awm = warp / C::AW_N, awn = warp % C::AW_N;
-  const bool apply_warp = warp < C::AW_M * C::AW_N;
-  load_chunk(0, 0, true);
-  for (int ch = 0; ch < nchunks; ++ch) {
-    if (ch + 1 < nchunks) {
-      load_chunk(ch + 1, (ch + 1) & 1, true);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    uint8_t *h = bufs + (ch & 1) * C::BUF;
-    uint8_t *l = h + C::CBYTES;
-    float acc[C::AMI][C::ANI][4] = {};
-    if (apply_warp) {
-#pragma unroll
-      for (int kk = 0; kk < S; kk += 16) {
-        uint32_t ah[C::AMI][4], al[C::AMI][4];
-#pragma unroll
-        for (int i = 0; i < C::AMI; ++i) {
-          const int row = awm * (S / C::AW_M) + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const int col = kk + (lane >> 4) * 8;
-          ldsm_x4(smem_u32(gth + (row * C::GLD + col) * 2), ah[i][0], ah[i][1], ah[i][2], ah[i][3]);
-          ldsm_x4(smem_u32(gtl + (row * C::GLD + col) * 2), al[i][0], al[i][1], al[i][2], al[i][3]);
-        }
-#pragma unroll
-        for (int j = 0; j < C::ANI; j += 2) {
-          const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const int ncol = awn * (C::FC / C::AW_N) + j * 8 + (lane >> 4) * 8;
-          uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-          ldsm_x4_t(smem_u32(h + (krow * C::CLD + ncol) * 2), h0, h1, h2, h3);
-          ldsm_x4_t(smem_u32(l + (krow * C::CLD + ncol) * 2), l0, l1, l2, l3);
-          const uint32_t hA[2] = {h0, h1}, hB[2] = {h2, h3}, lA[2] = {l0, l1}, lB[2] = {l2, l3};
-#pragma unroll
-          for (int i = 0; i < C::AMI; ++i) {
-            mma16816(acc[i][j], ah[i], hA);
-            mma16816(acc[i][j + 1], ah[i], hB);
-            mma16816(acc[i][j], al[i], hA);
-            mma16816(acc[i][j + 1], al[i], hB);
-            mma16816(acc[i][j], ah[i], lA);
-            mma16816(acc[i][j + 1], ah[i], lB);
-          }
-        }
-      }
-    }
-    // stage c (split pair) over the consumed chunk, then coalesced stores
-    __syncthreads();
-    if (apply_warp) {
-#pragma unroll
-      for (int i = 0; i < C::AMI; ++i)
-#pragma unroll
-        for (int j = 0; j < C::ANI; ++j)
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int row = awm * (S / C::AW_M) + i * 16 + (lane >> 2) + hh * 8;
-            const int fl = awn * (C::FC / C::AW_N) + j * 8 + (lane & 3) * 2;
-            uint32_t hi, lo;
-            split_pack(acc[i][j][2 * hh], acc[i][j][2 * hh + 1], hi, lo);
-            *reinterpret_cast<uint32_t *>(h + (row * C::CLD + fl) * 2) = hi;
-            *reinterpret_cast<uint32_t *>(l + (row * C::CLD + fl) * 2) = lo;
-          }
-    }
-    __syncthreads();
-    for (int e = tid; e < S * (C::FC / 8); e += 256) {
-      const int row = e / (C::FC / 8), cc = e % (C::FC / 8);
-      const int f = ch * C::FC + cc * 8;
-      if (f >= mt) continue;
-      bf16 *dst = ob + row * ld_out + f;
-      *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(h + (row * C::CLD + cc * 8) * 2);
-      *reinterpret_cast<uint4 *>(dst + plane_out) =
-          *reinterpret_cast<const uint4 *>(l + (row * C::CLD + cc * 8) * 2);
-    }
-    __syncthreads();
-  }
-}
-
 // ------------------------------------------------------------------ fp32 --
 
 template <int S>
@@ -480,18 +229,6 @@ avey_status run_static_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks,
   return AVEY_OK;
 }
 
-template <int S, bool COUPLED>
-avey_status run_dynamic_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
-                           int64_t ld_out, int64_t plane_out, int blocks, int mt, float eps,
-                           const bf16 *V, cudaStream_t s) {
-  using C = DynTile<S>;
-  if (avey_status st = set_smem(dynamic_mix_x2<S, COUPLED>, C::SMEM, "dynamic_mix_x2")) return st;
-  dynamic_mix_x2<S, COUPLED><<<blocks, 256, C::SMEM, s>>>(zt, ld_zt, plane_zt, out, ld_out,
-                                                          plane_out, mt, eps, V);
-  AVEY_CHECK_LAUNCH(COUPLED ? "coupled_mix_x2" : "dynamic_mix_x2", s);
-  return AVEY_OK;
-}
-
 }  // namespace
 
 avey_status launch_static_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks, int S,
@@ -504,32 +241,6 @@ avey_status launch_static_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld, int 
     case 128: return run_static_x2<128>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
   }
   set_detail("static mix: S=%d unsupported", S);
-  return AVEY_ERR_UNSUPPORTED;
-}
-
-avey_status launch_dynamic_mix_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
-                                  int64_t ld_out, int64_t plane_out, int blocks, int S, int mt,
-                                  float eps, cudaStream_t s) {
-  switch (S) {
-    case 16: return run_dynamic_x2<16, false>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, nullptr, s);
-    case 32: return run_dynamic_x2<32, false>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, nullptr, s);
-    case 64: return run_dynamic_x2<64, false>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, nullptr, s);
-    case 128: return run_dynamic_x2<128, false>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, eps, nullptr, s);
-  }
-  set_detail("dynamic mix: S=%d unsupported", S);
-  return AVEY_ERR_UNSUPPORTED;
-}
-
-avey_status launch_coupled_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld_zt, int64_t plane_zt,
-                                  bf16 *out, int64_t ld_out, int64_t plane_out, int blocks, int S,
-                                  int mt, cudaStream_t s) {
-  switch (S) {
-    case 16: return run_dynamic_x2<16, true>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, 0.f, V, s);
-    case 32: return run_dynamic_x2<32, true>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, 0.f, V, s);
-    case 64: return run_dynamic_x2<64, true>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, 0.f, V, s);
-    case 128: return run_dynamic_x2<128, true>(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, mt, 0.f, V, s);
-  }
-  set_detail("coupled mix: S=%d unsupported", S);
   return AVEY_ERR_UNSUPPORTED;
 }
 

@@ -1,0 +1,504 @@
+// avey_mix_dyn.cu -- the dynamic contextualizer of a split-size layer on the
+// tcgen05 tensor cores (papernotes 关键设计 2-3; paperlayer summary §4.2):
+//   G_ij = N(z_i).N(z_j)                       within each split of S tokens
+//   Gt_ij = G_ij / (sum_j G_ij + eps)          (eq. 6)
+//   c = Gt Z_t
+// and, with COUPLED, the original Avey's coupled causal map
+//   M_ij = V_ij G_ij for j <= i (0 otherwise),  c = M Z_t   (no row sums).
+// Z_t is an activation split pair (hi, lo bf16 planes); c is written as a
+// split pair, in place or to a separate buffer.
+//
+// One persistent, warp-specialised kernel, one CTA per SM.  A tile is 128
+// consecutive token rows: 128 / S whole splits (S in {16, 32, 64, 128}).
+//   1. Gram.  The tile's hi rows stream through a ring of TMA stages (128
+//      rows x 64 features, K-major, 128-byte swizzle); each stage is both
+//      operands of four 128 x 128 x 16 MMAs, so TMEM holds R = Z_hi Z_hi^T of
+//      the whole tile (the blocks outside the diagonal splits go unused).
+//   2. eq. 6 in the epilogue warps, one TMEM lane (token row i) per thread:
+//      |z_i| = sqrt(R_ii) from the diagonal, the cosines of the row's own
+//      split, their sum, and Gt = cos / (sum + eps) in fp32, split to a bf16
+//      pair and written into shared memory as the K-major A operand of step
+//      3 (block-diagonal: the zeros outside the splits are written once).
+//   3. Apply.  Z_t is read straight from the token-major activation as an
+//      MN-major B operand: TMA boxes of 64 features x 64 tokens per plane.
+//      Per 16 tokens three MMAs (Gt_hi Z_hi + Gt_lo Z_hi + Gt_hi Z_lo) into
+//      one of two 64-column accumulators; the epilogue splits c to a pair,
+//      stages it per warp in swizzled shared memory and stores it by TMA.
+// The hi rows are read twice (steps 1 and 3); the second read is close
+// enough in time to the first to be served mostly from L2.
+// Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue, warps 2-5
+// epilogue (one per TMEM lane quarter).  Every wait is bounded
+// (avey_common.cuh); a wait that runs out records AVEY_ERR_DEVICE_TIMEOUT and
+// the kernel drains and returns.
+#include <algorithm>
+
+#include "avey_common.cuh"
+#include "avey_internal.h"
+
+namespace avey {
+namespace {
+
+constexpr int DT = 128;                    // token rows per tile
+constexpr int DF = 64;                     // features per Gram chunk and per apply tile
+constexpr int D_EPI = 4;                   // epilogue warps
+constexpr int D_THR = 64 + 32 * D_EPI;
+constexpr uint32_t D_STAGE = 16384;        // 128 rows x 64 features, or 2 planes x 64 x 64
+constexpr uint32_t D_ZBOX = 8192;          // one plane of an apply stage: 64 tokens x 64 features
+constexpr int D_STAGES = 5;
+constexpr uint32_t D_GT_CHUNK = 16384;     // 128 rows x 64 tokens of one Gt plane
+constexpr uint32_t D_GT_PLANE = 2 * D_GT_CHUNK;
+constexpr uint32_t D_OUT = 4096;           // one plane of a warp's output box: 32 rows x 64
+constexpr uint32_t D_OUT_WARP = 2 * 2 * D_OUT;  // two buffers x (hi, lo)
+constexpr uint32_t D_GT_OFF = D_STAGES * D_STAGE;
+constexpr uint32_t D_OUT_OFF = D_GT_OFF + 2 * D_GT_PLANE;
+constexpr uint32_t D_CTRL_OFF = D_OUT_OFF + D_EPI * D_OUT_WARP;
+constexpr uint32_t D_CTRL = 2048;         // barriers, TMEM address, flag, norms [2][128]
+constexpr uint32_t D_SMEM = D_CTRL_OFF + D_CTRL + 1024;  // + alignment slack
+static_assert(D_SMEM <= 232448, "shared memory budget");
+static_assert(D_GT_OFF % 1024 == 0 && D_OUT_OFF % 1024 == 0 && D_CTRL_OFF % 1024 == 0,
+              "swizzled buffers need 1024-byte alignment");
+constexpr uint32_t D_COLS = 256;           // TMEM: Gram [0, 128), accumulators 128 + 64 a
+
+struct DynArgs {
+  int rows;       // T = blocks * S
+  int mt;         // mixed features
+  int nk;         // ceil(mt / 64)
+  int num_tiles;  // ceil(T / 128)
+  float eps;
+  const bf16 *V;  // COUPLED: [S, S]
+  int *status;
+};
+
+// K-major operand, 128-byte swizzle: 8-row atoms 1024 bytes apart.
+__device__ __forceinline__ uint64_t dyn_desc_k(uint32_t a) {
+  return static_cast<uint64_t>((a >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1u) << 16) |
+         (static_cast<uint64_t>(1024u >> 4) << 32) | (static_cast<uint64_t>(1u) << 46) |
+         (static_cast<uint64_t>(2u) << 61);
+}
+// MN-major operand of 64 MN elements, 128-byte swizzle: one 128-byte row per
+// K index, 8-row atoms 1024 bytes apart along K.
+__device__ __forceinline__ uint64_t dyn_desc_mn(uint32_t a) {
+  return static_cast<uint64_t>((a >> 4) & 0x3FFFu) | (static_cast<uint64_t>(D_ZBOX >> 4) << 16) |
+         (static_cast<uint64_t>(1024u >> 4) << 32) | (static_cast<uint64_t>(1u) << 46) |
+         (static_cast<uint64_t>(2u) << 61);
+}
+
+__device__ __forceinline__ void dyn_drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// Byte offset of element (row, k) of a K-major tile with 128-byte rows and
+// 128-byte swizzle (16-byte chunk c of row r sits at chunk c ^ (r % 8)).
+__device__ __forceinline__ uint32_t sw128_off(int row, int k) {
+  return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 +
+                               ((((k >> 3) ^ row) & 7) << 4) + (k & 7) * 2);
+}
+
+template <int S, bool COUPLED>
+__global__ void __launch_bounds__(D_THR, 1)
+    dyn_mix_tc_kernel(const __grid_constant__ CUtensorMap tmG,
+                      const __grid_constant__ CUtensorMap tmZh,
+                      const __grid_constant__ CUtensorMap tmZl,
+                      const __grid_constant__ CUtensorMap tmOh,
+                      const __grid_constant__ CUtensorMap tmOl, const DynArgs a) {
+  static_assert(S == 16 || S == 32 || S == 64 || S == 128, "split size");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t *base = smem_raw + pad;
+  const uint32_t sbase = raw_s + pad;
+  const uint32_t gth = sbase + D_GT_OFF, gtl = gth + D_GT_PLANE;
+  uint8_t *ctrl = base + D_CTRL_OFF;
+  const uint32_t cbase = sbase + D_CTRL_OFF;
+  // control block: full[s] @8s, empty[s] @64+8s (s < 8), tfull[2] @128,
+  // tempty[2] @144, gfull @160, gempty @168, gtready @176, gtfree @184,
+  // drain @192, tmem base @200, abort flag @204, norms [2][128] fp32 @256
+  static_assert(D_STAGES <= 8, "control block holds at most 8 stages");
+  auto full_bar = [&](int s) { return cbase + 8u * s; };
+  auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
+  auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
+  auto tempty_bar = [&](int i) { return cbase + 144u + 8u * i; };
+  const uint32_t gfull_bar = cbase + 160u, gempty_bar = cbase + 168u;
+  const uint32_t gtready_bar = cbase + 176u, gtfree_bar = cbase + 184u;
+  const uint32_t drain_bar = cbase + 192u;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 200);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 204);
+  float *s_norm = reinterpret_cast<float *>(ctrl + 256);
+  static_assert(256 + 2 * 128 * 4 <= D_CTRL, "control block size");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < D_STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), D_EPI);
+    }
+    mbar_init(gfull_bar, 1);
+    mbar_init(gempty_bar, D_EPI);
+    mbar_init(gtready_bar, D_EPI);
+    mbar_init(gtfree_bar, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(ctrl + 200), D_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmG);
+    prefetch_tmap(&tmZh);
+    prefetch_tmap(&tmZl);
+    prefetch_tmap(&tmOh);
+    prefetch_tmap(&tmOl);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // -------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      auto next = [&]() -> bool {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) return false;
+        mbar_arrive_expect_tx(full_bar(stage), D_STAGE);
+        return true;
+      };
+      auto advance = [&]() {
+        ++issued;
+        if (++stage == D_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        const int r0 = tile * DT;
+        for (int kc = 0; kc < a.nk; ++kc) {  // Gram: the hi rows, 64 features a stage
+          if (!(ok = next())) break;
+          tma_load_3d(sbase + stage * D_STAGE, &tmG, full_bar(stage), kc * DF, r0, 0);
+          advance();
+        }
+        for (int jn = 0; jn < a.nk && ok; ++jn) {  // apply: 64 features x 64 tokens x 2 planes
+          for (int kh = 0; kh < 2; ++kh) {
+            if (!(ok = next())) break;
+            const uint32_t st = sbase + stage * D_STAGE;
+            tma_load_3d(st, &tmZh, full_bar(stage), jn * DF, r0 + kh * 64, 0);
+            tma_load_3d(st + D_ZBOX, &tmZl, full_bar(stage), jn * DF, r0 + kh * 64, 0);
+            advance();
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      // wait (bounded) for the loads still in flight before the CTA exits
+      for (int s = 0; s < D_STAGES; ++s) {
+        if (issued > s) {
+          const long long last = ((issued - 1 - s) / D_STAGES) * D_STAGES + s;
+          dyn_drain_wait(full_bar(s), static_cast<uint32_t>((last / D_STAGES) & 1));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t id_gram = idesc_bf16_f32(DT, DT);
+      const uint32_t id_apply = idesc_bf16_f32(DT, DF) | (1u << 16);  // B is MN-major
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0, gphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        // Gram of the tile's hi rows into TMEM columns [0, 128)
+        if (!(ok = mbar_wait(gempty_bar, gphase ^ 1u, abort_flag))) break;
+        tc_fence_after();
+        for (int kc = 0; kc < a.nk; ++kc) {
+          if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + stage * D_STAGE;
+#pragma unroll
+          for (int kk = 0; kk < DF / 16; ++kk) {
+            const uint64_t d = dyn_desc_k(st + 32u * kk);
+            tc_mma_bf16(tmem_base, d, d, id_gram, (kc | kk) != 0);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == D_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(gfull_bar);
+        // c = Gt Z_t, 64 features at a time
+        if (!(ok = mbar_wait(gtready_bar, gphase, abort_flag))) break;
+        tc_fence_after();
+        for (int jn = 0; jn < a.nk && ok; ++jn) {
+          if (!(ok = mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + 128u + static_cast<uint32_t>(acc * DF);
+          for (int kh = 0; kh < 2; ++kh) {
+            if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t st = sbase + stage * D_STAGE;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              // 16 tokens: +32 bytes along Gt's K-major rows, +2048 bytes (two
+              // 8-token atoms) along Z's MN-major rows
+              const uint64_t ah = dyn_desc_k(gth + kh * D_GT_CHUNK + 32u * kk);
+              const uint64_t al = dyn_desc_k(gtl + kh * D_GT_CHUNK + 32u * kk);
+              const uint64_t bh = dyn_desc_mn(st + 2048u * kk);
+              const uint64_t bl = dyn_desc_mn(st + D_ZBOX + 2048u * kk);
+              tc_mma_bf16(d_tmem, ah, bh, id_apply, (kh | kk) != 0);
+              tc_mma_bf16(d_tmem, al, bh, id_apply, 1u);
+              tc_mma_bf16(d_tmem, ah, bl, id_apply, 1u);
+            }
+            tc_commit(empty_bar(stage));
+            if (++stage == D_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          tc_commit(tfull_bar(acc));
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
+        }
+        if (!ok) break;
+        tc_commit(gtfree_bar);  // the tile's MMAs no longer read Gt
+        gphase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+      }
+      tc_commit(drain_bar);
+      dyn_drain_wait(drain_bar, 0);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;          // TMEM lanes 32 quarter .. + 31
+    const int row = quarter * 32 + lane;   // token row within the tile
+    constexpr int W = S >= 32 ? S : 32;    // Gram columns a warp reads
+    const int col0 = (quarter * 32 / W) * W;
+    const int srow = row / S * S;          // first row of this row's split
+    const int sub = srow - col0;           // 0, or 16 for S = 16
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t *ob = base + D_OUT_OFF + (warp - 2) * D_OUT_WARP;
+    const uint32_t ob_s = sbase + D_OUT_OFF + (warp - 2) * D_OUT_WARP;
+    // Gt outside the diagonal splits stays zero: clear this row of both planes once
+    {
+      const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int pl = 0; pl < 2; ++pl)
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4 *>(base + D_GT_OFF + pl * D_GT_PLANE + ch * D_GT_CHUNK +
+                                       sw128_off(row, c * 8)) = z;
+    }
+    int acc = 0, obuf = 0;
+    uint32_t acc_phase = 0, gphase = 0;
+    bool ok = true;
+    // Every epilogue warp runs the same number of named barriers (one per
+    // tile): after a failed wait a warp stops waiting and working but still
+    // walks the tile loop, so the others never wait for it.
+    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+      const int r0 = tile * DT;
+      // ---- eq. 6 from the Gram ----
+      float v[W];
+      float gii = 0.f;
+      const bool got = ok && mbar_wait(gfull_bar, gphase, abort_flag);
+      if (got) {
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < W; q += 32)
+          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(col0 + q),
+                    *reinterpret_cast<float(*)[32]>(&v[q]));
+#pragma unroll
+        for (int q = 0; q < W; ++q)
+          if (col0 + q == row) gii = v[q];
+      } else {
+        ok = false;
+      }
+      float *nrm = s_norm + (gphase & 1u) * 128;
+      nrm[row] = fmaxf(sqrtf(gii), 1e-12f);
+      tc_fence_before();
+      __syncwarp();
+      if (got && lane == 0) mbar_arrive(gempty_bar);  // the Gram's TMEM may be overwritten
+      named_bar_sync(1, 32 * D_EPI);                   // every row's norm is in place
+      gphase ^= 1u;
+      if (!ok) continue;
+      const float ni = nrm[row];
+      // the row's own split, in place: v[0 .. S) (for S = 16, the warp read 32
+      // columns and this row's split is the half at `sub`)
+      if constexpr (S < 32) {
+#pragma unroll
+        for (int q = 0; q < S; ++q) v[q] = sub ? v[q + 16] : v[q];
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int q = 0; q < S; ++q) {
+        v[q] = v[q] / (ni * nrm[srow + q]);
+        rs += v[q];
+      }
+      if constexpr (COUPLED) {
+        const int i = row - srow;
+#pragma unroll
+        for (int q = 0; q < S; ++q)
+          v[q] = q <= i ? __bfloat162float(a.V[i * S + q]) * v[q] : 0.f;
+      } else {
+        const float den = rs + a.eps;
+#pragma unroll
+        for (int q = 0; q < S; ++q) v[q] = v[q] / den;
+      }
+      // the previous tile's MMAs must be done with Gt before it is rewritten
+      // (gphase now has the parity of the previous tile)
+      if (!(ok = mbar_wait(gtfree_bar, gphase, abort_flag))) continue;
+#pragma unroll
+      for (int q = 0; q < S; q += 8) {
+        uint4 h, l;
+        split_pack(v[q], v[q + 1], h.x, l.x);
+        split_pack(v[q + 2], v[q + 3], h.y, l.y);
+        split_pack(v[q + 4], v[q + 5], h.z, l.z);
+        split_pack(v[q + 6], v[q + 7], h.w, l.w);
+        const int k = srow + q;  // token column of Gt
+        const uint32_t off = (k / 64) * D_GT_CHUNK + sw128_off(row, k % 64);
+        *reinterpret_cast<uint4 *>(base + D_GT_OFF + off) = h;
+        *reinterpret_cast<uint4 *>(base + D_GT_OFF + D_GT_PLANE + off) = l;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(gtready_bar);
+      // ---- c tiles: TMEM -> split pair -> swizzled staging -> TMA store ----
+      for (int jn = 0; jn < a.nk; ++jn) {
+        if (!(ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag))) break;
+        tc_fence_after();
+        float c[64];
+        tmem_ld64(tmem_base + lane_off + 128u + static_cast<uint32_t>(acc * DF), c);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        if (r0 + quarter * 32 >= a.rows) continue;  // rows past T are never stored
+        // this buffer's previous store has finished reading it
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint8_t *bh = ob + obuf * 2 * D_OUT;
+        uint8_t *bl = bh + D_OUT;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          uint4 h, l;
+          split_pack(c[8 * g], c[8 * g + 1], h.x, l.x);
+          split_pack(c[8 * g + 2], c[8 * g + 3], h.y, l.y);
+          split_pack(c[8 * g + 4], c[8 * g + 5], h.z, l.z);
+          split_pack(c[8 * g + 6], c[8 * g + 7], h.w, l.w);
+          const uint32_t off = lane * 128 + (((g ^ lane) & 7) << 4);
+          *reinterpret_cast<uint4 *>(bh + off) = h;
+          *reinterpret_cast<uint4 *>(bl + off) = l;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t sh = ob_s + obuf * 2 * D_OUT;
+          tma_store_3d(&tmOh, sh, jn * DF, r0 + quarter * 32, 0);
+          tma_store_3d(&tmOl, sh + D_OUT, jn * DF, r0 + quarter * 32, 0);
+          bulk_commit();
+        }
+        obuf ^= 1;
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      record_status(a.status, AVEY_ERR_DEVICE_TIMEOUT);
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, D_COLS);
+  }
+}
+
+template <int S, bool COUPLED>
+avey_status run_dyn_mix_tc(const CUtensorMap *maps, const DynArgs &args, cudaStream_t s) {
+  auto kern = dyn_mix_tc_kernel<S, COUPLED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(D_SMEM));
+  if (e != cudaSuccess) {
+    set_detail("dynamic mix: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return AVEY_ERR_CUDA;
+  }
+  const int grid = std::min(args.num_tiles, sm_count());
+  kern<<<grid, D_THR, D_SMEM, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
+  AVEY_CHECK_LAUNCH(COUPLED ? "coupled_mix_tc" : "dynamic_mix_tc", s);
+  return AVEY_OK;
+}
+
+avey_status dyn_mix_tc(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
+                       int64_t ld_out, int64_t plane_out, int blocks, int S, int mt, float eps,
+                       const bf16 *V, cudaStream_t s) {
+  AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
+               "dynamic mix: S=%d unsupported (16, 32, 64 or 128)", S);
+  AVEY_REQUIRE(mt >= 8 && mt % 8 == 0 && ld_zt % 8 == 0 && ld_out % 8 == 0 && aligned16(zt) &&
+                   aligned16(out) && aligned16(zt + plane_zt) && aligned16(out + plane_out),
+               AVEY_ERR_INVALID_ARG,
+               "dynamic mix: mt, ld multiples of 8 and 16-byte aligned planes required");
+  if (blocks <= 0) return AVEY_OK;
+  const long long T = static_cast<long long>(blocks) * S;
+  AVEY_REQUIRE(T <= 0x7fffff00ll, AVEY_ERR_UNSUPPORTED, "dynamic mix: too many rows");
+  CUtensorMap maps[5];
+  const uint64_t zrow = static_cast<uint64_t>(ld_zt) * 2, orow = static_cast<uint64_t>(ld_out) * 2;
+  if (!encode_bf16_map(&maps[0], zt, mt, T, 1, zrow, zrow * T, DT)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&maps[1], zt, mt, T, 1, zrow, zrow * T, 64)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&maps[2], zt + plane_zt, mt, T, 1, zrow, zrow * T, 64)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&maps[3], out, mt, T, 1, orow, orow * T, 32)) return AVEY_ERR_CUDA;
+  if (!encode_bf16_map(&maps[4], out + plane_out, mt, T, 1, orow, orow * T, 32)) return AVEY_ERR_CUDA;
+  DynArgs args{};
+  args.rows = static_cast<int>(T);
+  args.mt = mt;
+  args.nk = (mt + DF - 1) / DF;
+  args.num_tiles = static_cast<int>((T + DT - 1) / DT);
+  args.eps = eps;
+  args.V = V;
+  args.status = device_status_word();
+  const bool cp = V != nullptr;
+  switch (S) {
+    case 16: return cp ? run_dyn_mix_tc<16, true>(maps, args, s) : run_dyn_mix_tc<16, false>(maps, args, s);
+    case 32: return cp ? run_dyn_mix_tc<32, true>(maps, args, s) : run_dyn_mix_tc<32, false>(maps, args, s);
+    case 64: return cp ? run_dyn_mix_tc<64, true>(maps, args, s) : run_dyn_mix_tc<64, false>(maps, args, s);
+    default: return cp ? run_dyn_mix_tc<128, true>(maps, args, s) : run_dyn_mix_tc<128, false>(maps, args, s);
+  }
+}
+
+}  // namespace
+
+avey_status launch_dynamic_mix_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
+                                  int64_t ld_out, int64_t plane_out, int blocks, int S, int mt,
+                                  float eps, cudaStream_t s) {
+  return dyn_mix_tc(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, S, mt, eps, nullptr, s);
+}
+
+avey_status launch_coupled_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld_zt, int64_t plane_zt,
+                                  bf16 *out, int64_t ld_out, int64_t plane_out, int blocks, int S,
+                                  int mt, cudaStream_t s) {
+  AVEY_REQUIRE(V != nullptr, AVEY_ERR_INVALID_ARG, "coupled mix: V is required");
+  return dyn_mix_tc(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, S, mt, 0.f, V, s);
+}
+
+}  // namespace avey
