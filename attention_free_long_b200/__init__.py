@@ -66,12 +66,14 @@ def lib() -> ctypes.CDLL:
         L.avey_rank_ex.argtypes = [_vp, _i, _i, _i, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _vp,
                                    _vp, _sz, _vp]
         L.avey_rank_ex.restype = _i
-        L.avey_trace_begin.argtypes = [_vp, _i]
+        L.avey_trace_begin.argtypes = [_i, _vp]
         L.avey_trace_begin.restype = _i
         L.avey_trace_end.argtypes = []
         L.avey_trace_end.restype = _i
         L.avey_trace_kernel_name.argtypes = [_i]
         L.avey_trace_kernel_name.restype = ctypes.c_char_p
+        L.avey_trace_kernel_ms.argtypes = [_i, ctypes.POINTER(ctypes.c_float)]
+        L.avey_trace_kernel_ms.restype = _i
         L.avey_rank_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.avey_rank_workspace_bytes.restype = _sz
         L.avey_compress.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
@@ -148,27 +150,20 @@ def kernel_launches() -> int:
 class KernelTrace:
     """Per-kernel device times of the library's launches on the current stream.
 
-    ``with KernelTrace(capacity) as tr: ...`` records one CUDA event after
-    every kernel the library enqueues inside the block (avey_trace_begin /
-    avey_trace_end), plus one before the first; after a synchronize,
+    ``with KernelTrace(capacity) as tr: ...`` has the library record one of its
+    own CUDA events before the block and one after every kernel it enqueues
+    inside it (avey_trace_begin / avey_trace_end); after a synchronize,
     ``tr.kernels()`` gives [(name, ms)] in launch order.  For launches on one
     stream only.
     """
 
     def __init__(self, capacity: int = 256):
         self.capacity = int(capacity)
-        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(self.capacity)]
-        self.start = torch.cuda.Event(enable_timing=True)
-        # torch creates an event's CUDA handle on its first record
-        for e in self.events:
-            e.record()
         self.count = 0
         self.names: List[str] = []
 
     def __enter__(self):
-        arr = (ctypes.c_void_p * self.capacity)(*[e.cuda_event for e in self.events])
-        self.start.record()
-        _check("avey_trace_begin", lib().avey_trace_begin(arr, self.capacity))
+        _check("avey_trace_begin", lib().avey_trace_begin(self.capacity, _stream()))
         return self
 
     def __exit__(self, *exc):
@@ -183,10 +178,11 @@ class KernelTrace:
 
     def kernels(self):
         """[(name, ms)] of every traced launch (call after a synchronize)."""
-        out, prev = [], self.start
+        out = []
+        ms = ctypes.c_float()
         for i in range(self.count):
-            out.append((self.names[i], prev.elapsed_time(self.events[i])))
-            prev = self.events[i]
+            _check("avey_trace_kernel_ms", lib().avey_trace_kernel_ms(i, ctypes.byref(ms)))
+            out.append((self.names[i], float(ms.value)))
         return out
 
 

@@ -67,21 +67,25 @@ int *device_status_word() {
   return g_status_ptr[dev];
 }
 
-// Kernel trace: while active, every launch records the next caller-provided
-// event on the launch's stream and keeps the kernel's name.
+// Kernel trace: while active, every launch records the next of the library's
+// own events on the launch's stream and keeps the kernel's name.  The events
+// are created by this library's CUDA runtime (handles made by another runtime
+// instance, such as the caller's, are not valid here) and reused.
 namespace {
 constexpr int kTraceName = 48;
+constexpr int kTraceMax = 4096;
 struct Trace {
   std::mutex mu;
   std::atomic<bool> on{false};
-  cudaEvent_t *events = nullptr;
-  char (*names)[kTraceName] = nullptr;
+  cudaEvent_t events[kTraceMax + 1] = {};  // [0] the start, [i + 1] after launch i
+  int created = 0;                         // events created so far
+  int device = -1;                         // device the events belong to
   int capacity = 0;
   int count = 0;       // launches seen since avey_trace_begin
   int record_err = 0;  // first cudaEventRecord failure
+  char names[kTraceMax][kTraceName];
 };
 Trace g_trace;
-char g_trace_names[4096][kTraceName];
 }  // namespace
 
 void count_launch(const char *name, cudaStream_t stream) {
@@ -92,7 +96,7 @@ void count_launch(const char *name, cudaStream_t stream) {
   const int i = g_trace.count++;
   if (i < g_trace.capacity) {
     snprintf(g_trace.names[i], kTraceName, "%s", name ? name : "?");
-    const cudaError_t e = cudaEventRecord(g_trace.events[i], stream);
+    const cudaError_t e = cudaEventRecord(g_trace.events[i + 1], stream);
     if (e != cudaSuccess && !g_trace.record_err) g_trace.record_err = static_cast<int>(e);
   }
 }
@@ -219,17 +223,29 @@ const char *avey_last_error_detail(void) { return avey::t_detail; }
 
 uint64_t avey_kernel_launches(void) { return avey::g_launches.load(); }
 
-avey_status avey_trace_begin(void *const *events, int capacity) {
+avey_status avey_trace_begin(int capacity, avey_stream_t stream) {
   using avey::g_trace;
-  AVEY_REQUIRE(events && capacity >= 1 && capacity <= 4096, AVEY_ERR_INVALID_ARG,
-               "avey_trace_begin: need an event array and 1 <= capacity <= 4096 (got %d)",
-               capacity);
+  AVEY_REQUIRE(capacity >= 1 && capacity <= avey::kTraceMax, AVEY_ERR_INVALID_ARG,
+               "avey_trace_begin: capacity must be in [1, %d] (got %d)", avey::kTraceMax, capacity);
   std::lock_guard<std::mutex> lk(g_trace.mu);
   AVEY_REQUIRE(!g_trace.on.load(), AVEY_ERR_INVALID_ARG, "avey_trace_begin: a trace is active");
-  for (int i = 0; i < capacity; ++i)
-    AVEY_REQUIRE(events[i] != nullptr, AVEY_ERR_INVALID_ARG, "avey_trace_begin: event %d is null", i);
-  g_trace.events = reinterpret_cast<cudaEvent_t *>(const_cast<void **>(events));
-  g_trace.names = avey::g_trace_names;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  AVEY_REQUIRE(e == cudaSuccess, AVEY_ERR_CUDA, "avey_trace_begin: cudaGetDevice: %s",
+               cudaGetErrorString(e));
+  AVEY_REQUIRE(g_trace.device < 0 || g_trace.device == dev, AVEY_ERR_UNSUPPORTED,
+               "avey_trace_begin: the trace events belong to device %d, not %d", g_trace.device,
+               dev);
+  g_trace.device = dev;
+  while (g_trace.created < capacity + 1) {
+    e = cudaEventCreate(&g_trace.events[g_trace.created]);
+    AVEY_REQUIRE(e == cudaSuccess, AVEY_ERR_CUDA, "avey_trace_begin: cudaEventCreate: %s",
+                 cudaGetErrorString(e));
+    ++g_trace.created;
+  }
+  e = cudaEventRecord(g_trace.events[0], reinterpret_cast<cudaStream_t>(stream));
+  AVEY_REQUIRE(e == cudaSuccess, AVEY_ERR_CUDA, "avey_trace_begin: cudaEventRecord: %s",
+               cudaGetErrorString(e));
   g_trace.capacity = capacity;
   g_trace.count = 0;
   g_trace.record_err = 0;
@@ -240,9 +256,11 @@ avey_status avey_trace_begin(void *const *events, int capacity) {
 int avey_trace_end(void) {
   using avey::g_trace;
   std::lock_guard<std::mutex> lk(g_trace.mu);
-  if (!g_trace.on.load()) return -1;
+  if (!g_trace.on.load()) {
+    avey::set_detail("avey_trace_end: no trace is active");
+    return -1;
+  }
   g_trace.on.store(false, std::memory_order_release);
-  g_trace.events = nullptr;
   if (g_trace.record_err) {
     avey::set_detail("avey_trace_end: cudaEventRecord failed: %s",
                      cudaGetErrorString(static_cast<cudaError_t>(g_trace.record_err)));
@@ -255,7 +273,20 @@ const char *avey_trace_kernel_name(int i) {
   using avey::g_trace;
   std::lock_guard<std::mutex> lk(g_trace.mu);
   if (g_trace.on.load() || i < 0 || i >= g_trace.capacity || i >= g_trace.count) return nullptr;
-  return avey::g_trace_names[i];
+  return g_trace.names[i];
+}
+
+avey_status avey_trace_kernel_ms(int i, float *ms) {
+  using avey::g_trace;
+  AVEY_REQUIRE(ms != nullptr, AVEY_ERR_INVALID_ARG, "avey_trace_kernel_ms: null output");
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  AVEY_REQUIRE(!g_trace.on.load(), AVEY_ERR_INVALID_ARG, "avey_trace_kernel_ms: a trace is active");
+  AVEY_REQUIRE(i >= 0 && i < g_trace.capacity && i < g_trace.count, AVEY_ERR_INVALID_ARG,
+               "avey_trace_kernel_ms: launch %d was not traced", i);
+  const cudaError_t e = cudaEventElapsedTime(ms, g_trace.events[i], g_trace.events[i + 1]);
+  AVEY_REQUIRE(e == cudaSuccess, AVEY_ERR_CUDA, "avey_trace_kernel_ms: cudaEventElapsedTime: %s",
+               cudaGetErrorString(e));
+  return AVEY_OK;
 }
 
 }  // extern "C"

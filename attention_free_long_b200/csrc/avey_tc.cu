@@ -304,14 +304,14 @@ __device__ __forceinline__ void fuse_residual_values(const TcArgs &a, const uint
 }
 
 // Fuser epilogue: x_out = x_in + acc (fp32) and/or its split pair; one 8 KB
-// staging buffer (fp32 4 KB, hi 2 KB, lo 2 KB).  The residual of chunk 0
-// arrives requested (xi, issued before the accumulator wait); each chunk
-// issues the next chunk's loads before its own math, so their latency
-// overlaps it.
+// staging buffer (fp32 4 KB, hi 2 KB, lo 2 KB).  The residuals of chunks 0
+// and 1 arrive requested (xi, xj, issued before the accumulator wait); each
+// chunk issues the loads of the chunk two ahead before its own math, so two
+// chunks' loads are always in flight behind it.
 __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mout,
                                          const CUtensorMap *mhi, const CUtensorMap *mlo,
                                          uint32_t taddr, int row0, int lane, int nt, uint32_t stg,
-                                         int &it, uint4 (&xi)[8]) {
+                                         int &it, uint4 (&xi)[8], uint4 (&xj)[8]) {
   const int row = row0 + lane;
   const bool pair = a.out_hi != nullptr;
   const bool f32out = a.x_out != nullptr;
@@ -320,7 +320,7 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mou
     const int col0 = nt * BN + ch * 32;
     if (col0 >= a.cols) break;  // warp-uniform
     uint4 xn[8];
-    if (ch + 1 < BN / 32) fuse_load_residual(a, row, col0 + 32, xn);
+    if (ch + 2 < BN / 32) fuse_load_residual(a, row, col0 + 64, xn);
     float v[32];
     tmem_ld32(taddr + ch * 32, v);
     if (it >= 1) {  // the previous chunk's stores must have read the buffer
@@ -359,7 +359,10 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mou
     }
     ++it;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) xi[q] = xn[q];
+    for (int q = 0; q < 8; ++q) {
+      xi[q] = xj[q];
+      xj[q] = xn[q];
+    }
   }
 }
 
@@ -757,8 +760,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = pair; tile < a.num_tiles; tile += npairs) {
       const int mt = tile / a.tiles_n, nt = tile - (tile / a.tiles_n) * a.tiles_n;
       const int row0 = mt * P::PM + static_cast<int>(rank) * 128 + quarter * 32;
-      uint4 xi[8];
-      if constexpr (MODE == MODE_FUSE) fuse_load_residual(a, row0 + lane, nt * BN, xi);
+      uint4 xi[8], xj[8];
+      if constexpr (MODE == MODE_FUSE) {
+        fuse_load_residual(a, row0 + lane, nt * BN, xi);
+        fuse_load_residual(a, row0 + lane, nt * BN + 32, xj);
+      }
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
         ok = false;
         break;
@@ -769,7 +775,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if constexpr (MODE == MODE_ENRICH) {
         epi_enrich(a, &tmO0, &tmO1, taddr, row0, lane, nt, stg, it);
       } else {
-        epi_fuse(a, &tmO0, &tmO1, &tmO2, taddr, row0, lane, nt, stg, it, xi);
+        epi_fuse(a, &tmO0, &tmO1, &tmO2, taddr, row0, lane, nt, stg, it, xi, xj);
       }
       tc_fence_before();
       __syncwarp();

@@ -301,7 +301,7 @@ def forward_leg(av, wl, dev, args, rank, world, local, barrier, e2e=True, sample
     marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks + 1)]
              for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    per_step = 4 + 3 * wl.layers  # upper bound of launches per forward
+    per_step = 4 + 4 * wl.layers  # upper bound of launches per forward (prenorm adds one per layer)
     trace = av.KernelTrace(capacity=args.steps * per_step + 8)
     barrier()
     torch.cuda.synchronize()
@@ -459,7 +459,7 @@ def run_ours(args):
     smix_ms, mix_ms, mix_bytes = mixes_alone(av, wl, layers, dev, reps)
     kin = leg["kernels"]
     dyn_in = kin.get("dynamic_mix_tc", {}).get("ms_per_launch")
-    stat_in = kin.get("static_mix_x2", {}).get("ms_per_launch")
+    stat_in = kin.get("static_mix_tc", {}).get("ms_per_launch")
     comp_ms = (kin.get("compress_tc") or kin.get("compress_bf16") or {}).get("ms_per_launch")
     comp_bytes = compress_bytes(wl)
 

@@ -349,26 +349,34 @@ AVEY_API const char *avey_last_error_detail(void);
  * reports it; the context stays usable. */
 AVEY_API avey_status avey_selftest_wait_timeout(uint32_t limit_us, avey_stream_t stream);
 
-/* Kernel trace: a measurement hook with no counterpart on the pages.  Between
- * avey_trace_begin and avey_trace_end, every kernel the library launches
- * records the next of the caller's events on its launch stream, right after
- * the kernel is enqueued, and the library keeps the kernel's name.  On one
- * stream, the time from the event before a launch (the previous launch's, or
- * one the caller recorded) to that launch's event is the kernel's duration.
- * events     HOST array of `capacity` cudaEvent_t handles (passed as void*),
- *            created and owned by the caller, none NULL; 1 <= capacity <= 4096.
- *            Launches beyond `capacity` are counted but record nothing.
- * avey_trace_begin returns AVEY_ERR_INVALID_ARG for a bad array or while a
- * trace is already active (one trace per process; the trace is shared by all
- * host threads).  avey_trace_end returns the number of launches seen (which
- * may exceed `capacity`), or -1 if no trace was active or an event record
- * failed (detail in avey_last_error_detail).  avey_trace_kernel_name(i) is
- * the name of traced launch i < min(count, capacity) of the last finished
- * trace (a string owned by the library, valid until the next trace begins),
- * or NULL. */
-AVEY_API avey_status avey_trace_begin(void *const *events, int capacity);
+/* Kernel trace: a measurement hook with no counterpart on the pages.
+ * avey_trace_begin records a start event on `stream`; then, until
+ * avey_trace_end, every kernel the library launches records the next event
+ * on its own launch stream right after it is enqueued, and the library keeps
+ * the kernel's name.  The events belong to the library: they are created on
+ * the current device by the first trace that needs them (no device memory),
+ * reused by later traces, and held until the process exits; all traces must
+ * run on that device (AVEY_ERR_UNSUPPORTED otherwise).
+ *   capacity  1 <= capacity <= 4096 launches are timed; later launches are
+ *             counted but record nothing.
+ * avey_trace_begin returns AVEY_ERR_INVALID_ARG for a bad capacity or while a
+ * trace is already active (one trace per process, shared by all host
+ * threads), AVEY_ERR_CUDA when an event cannot be created or recorded.
+ * avey_trace_end returns the number of launches seen (which may exceed the
+ * capacity), or -1 if no trace was active or an event record failed (detail
+ * in avey_last_error_detail).
+ * After avey_trace_end, for traced launch i < min(count, capacity):
+ *   avey_trace_kernel_name(i)  its kernel (a string owned by the library,
+ *                              valid until the next trace begins), else NULL;
+ *   avey_trace_kernel_ms(i, &ms)  the device time between the event before it
+ *                              (the start, or launch i-1's) and its own; on one
+ *                              stream that is the kernel's duration.  The
+ *                              events must have completed (synchronise the
+ *                              stream first), else AVEY_ERR_CUDA. */
+AVEY_API avey_status avey_trace_begin(int capacity, avey_stream_t stream);
 AVEY_API int avey_trace_end(void);
 AVEY_API const char *avey_trace_kernel_name(int i);
+AVEY_API avey_status avey_trace_kernel_ms(int i, float *ms);
 
 /* avey_kernel_launches: number of kernels this library has launched since it
  * was loaded, in this process (all threads). */

@@ -147,12 +147,13 @@ def test_fp32_activations_may_be_omitted_only_beside_the_bf16_pair():
 def test_kernel_trace_rejects_bad_arguments_and_idles_cleanly():
     L = av.lib()
     assert L.avey_trace_end() == -1                    # no trace active
-    assert L.avey_trace_begin(None, 4) == 1            # AVEY_ERR_INVALID_ARG
-    arr = (ctypes.c_void_p * 2)(None, None)
-    assert L.avey_trace_begin(arr, 2) == 1             # null events
-    assert L.avey_trace_begin(arr, 0) == 1             # capacity out of range
+    assert L.avey_trace_begin(0, None) == 1            # AVEY_ERR_INVALID_ARG: capacity
+    assert L.avey_trace_begin(4097, None) == 1
     assert L.avey_trace_end() == -1                    # nothing was started
     assert L.avey_trace_kernel_name(0) is None
+    ms = ctypes.c_float()
+    assert L.avey_trace_kernel_ms(0, ctypes.byref(ms)) == 1
+    assert L.avey_trace_kernel_ms(0, None) == 1
 
 
 def test_rank_static_reports_the_shape_error_before_the_scratch_limit():

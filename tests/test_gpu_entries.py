@@ -1,6 +1,6 @@
 """The single-kernel entry points avey_static_mix and avey_topk against the
 oracle, through the C ABI.  Each runs the kernel that the layer and the ranker
-launch internally (static_mix_x2 / static_mix_f32, topk_warp)."""
+launch internally (static_mix_tc / static_mix_f32, topk_warp)."""
 import numpy as np
 import pytest
 import torch
@@ -76,3 +76,31 @@ def test_smoke_entry_passes(cuda_dev):
     # cuda:0 against the oracle
     import __graft_entry__ as ge
     ge.smoke()
+
+
+def test_kernel_trace_times_every_launch_of_a_forward(cuda_dev):
+    wl = sy.custom("trace", B=1, N=2048, S=64, d=128, m=256, k=5,
+                   pattern=(sy.STATIC, sy.DYNAMIC), centers=8, sigma=0.5)
+    E, W = sy.gen_embeddings(wl), sy.gen_weights(wl)
+    x = torch.from_numpy(E.X).to(cuda_dev, torch.bfloat16)
+    P = torch.from_numpy(W.P).to(cuda_dev, torch.bfloat16)
+    layers = av.device_layers(W, torch.bfloat16, cuda_dev)
+    ws = av.make_workspace(wl.B, wl.N, wl.d, wl.S, wl.k, wl.m, torch.bfloat16, wl.prenorm, cuda_dev)
+    av.encoder_forward(x, P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm, ws)
+    before = av.kernel_launches()
+    with av.KernelTrace(64) as tr:
+        av.encoder_forward(x, P, layers, wl.S, wl.k, wl.m_h, wl.eps, wl.prenorm, ws)
+    torch.cuda.synchronize()
+    assert av.device_status() == 0
+    ks = tr.kernels()
+    assert len(ks) == av.kernel_launches() - before == 3 + 1 + 3 * len(layers)
+    names = [n for n, _ in ks]
+    assert names[:4] == ["inv_norms", "maxsim_pair", "topk_warp", "compress_tc"]
+    assert names[4:] == ["enrich_tc", "static_mix_tc", "fuse_tc",
+                         "enrich_tc", "dynamic_mix_tc", "fuse_tc"]
+    assert all(ms > 0 for _, ms in ks)
+    # a second trace reuses the library's events
+    with av.KernelTrace(8) as tr2:
+        av.avey_rank(x, wl.S, wl.k)
+    torch.cuda.synchronize()
+    assert [n for n, _ in tr2.kernels()] == ["inv_norms", "maxsim_pair", "topk_warp"]
