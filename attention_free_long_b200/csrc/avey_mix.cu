@@ -5,14 +5,9 @@
 //             c = Gt Z_t
 // Identity activation, no bias.
 //
-// bf16 path: Z_t is an activation split pair (hi, lo bf16 planes).  The
-// static mix is bound by HBM (read Z_t, write c, 8 bytes per element each way):
-//   static_mix_x2   one CTA per (block, feature slab); V and both planes of
-//                   the slab in shared memory; c = V Z_hi + V Z_lo with
-//                   mma.sync; written back in place as a split pair.
-// The bf16 dynamic (and coupled causal) mix runs on tcgen05 in
-// avey_mix_dyn.cu.  fp32 path: plain SIMT kernels, and the C ABI entry points
-// of both mixes.
+// The bf16 mixes (Z_t an activation split pair) run on tcgen05 in
+// avey_mix_dyn.cu.  This file holds the fp32 path (plain SIMT kernels) and the
+// C ABI entry points of both mixes.
 #include <algorithm>
 
 #include "avey_common.cuh"
@@ -20,109 +15,6 @@
 
 namespace avey {
 namespace {
-
-// ---------------------------------------------------------------- static --
-
-template <int S>
-struct StaticTile {
-  static constexpr int WM = S >= 32 ? 32 : 16;
-  static constexpr int WARPS_M = S / WM;
-  static constexpr int WARPS_N = 8 / WARPS_M;
-  static constexpr int WN = 32;
-  static constexpr int NS = WN * WARPS_N;
-  static constexpr int MI = WM / 16, NI = WN / 8;
-  static constexpr int ZLD = NS + 8, VLD = S + 8;
-  static constexpr int ZBYTES = S * ZLD * 2, VBYTES = S * VLD * 2;
-  static constexpr int SMEM = VBYTES + 2 * ZBYTES;
-};
-
-template <int S>
-__global__ void __launch_bounds__(256) static_mix_x2(const bf16 *__restrict__ V, const bf16 *zt,
-                                                     long long ld, int mt, long long plane,
-                                                     bf16 *out, long long ld_out,
-                                                     long long plane_out) {
-  using C = StaticTile<S>;
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t *vs = smem;
-  uint8_t *zh = smem + C::VBYTES;
-  uint8_t *zl = zh + C::ZBYTES;
-  const int slab = blockIdx.x, blk = blockIdx.y;
-  const int f0 = slab * C::NS;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wm = warp / C::WARPS_N, wn = warp % C::WARPS_N;
-  const bf16 *zbase = zt + static_cast<long long>(blk) * S * ld;
-  bf16 *obase = out + static_cast<long long>(blk) * S * ld_out;
-
-  for (int e = tid; e < S * (S / 8); e += 256) {
-    const int row = e / (S / 8), cc = e % (S / 8);
-    cp_async16(smem_u32(vs + (row * C::VLD + cc * 8) * 2), V + row * S + cc * 8, 16);
-  }
-  for (int e = tid; e < S * (C::NS / 8); e += 256) {
-    const int row = e / (C::NS / 8), cc = e % (C::NS / 8);
-    const int f = f0 + cc * 8;
-    const bool ok = f < mt;
-    const bf16 *src = ok ? zbase + row * ld + f : zbase;
-    cp_async16(smem_u32(zh + (row * C::ZLD + cc * 8) * 2), src, ok ? 16 : 0);
-    cp_async16(smem_u32(zl + (row * C::ZLD + cc * 8) * 2), ok ? src + plane : zbase, ok ? 16 : 0);
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-
-  float acc[C::MI][C::NI][4] = {};
-#pragma unroll
-  for (int kk = 0; kk < S; kk += 16) {
-    uint32_t af[C::MI][4];
-#pragma unroll
-    for (int i = 0; i < C::MI; ++i) {
-      const int row = wm * C::WM + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      ldsm_x4(smem_u32(vs + (row * C::VLD + kk + (lane >> 4) * 8) * 2), af[i][0], af[i][1], af[i][2],
-              af[i][3]);
-    }
-#pragma unroll
-    for (int j = 0; j < C::NI; j += 2) {
-      const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int ncol = wn * C::WN + j * 8 + (lane >> 4) * 8;
-#pragma unroll
-      for (int pl = 0; pl < 2; ++pl) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(smem_u32((pl ? zl : zh) + (krow * C::ZLD + ncol) * 2), b0, b1, b2, b3);
-        const uint32_t bA[2] = {b0, b1}, bB[2] = {b2, b3};
-#pragma unroll
-        for (int i = 0; i < C::MI; ++i) {
-          mma16816(acc[i][j], af[i], bA);
-          mma16816(acc[i][j + 1], af[i], bB);
-        }
-      }
-    }
-  }
-  // c as a split pair, staged over the (now consumed) input slab, then written
-  // back with coalesced 16-byte stores.
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < C::MI; ++i)
-#pragma unroll
-    for (int j = 0; j < C::NI; ++j)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = wm * C::WM + i * 16 + (lane >> 2) + h * 8;
-        const int fl = wn * C::WN + j * 8 + (lane & 3) * 2;
-        uint32_t hi, lo;
-        split_pack(acc[i][j][2 * h], acc[i][j][2 * h + 1], hi, lo);
-        *reinterpret_cast<uint32_t *>(zh + (row * C::ZLD + fl) * 2) = hi;
-        *reinterpret_cast<uint32_t *>(zl + (row * C::ZLD + fl) * 2) = lo;
-      }
-  __syncthreads();
-  for (int e = tid; e < S * (C::NS / 8); e += 256) {
-    const int row = e / (C::NS / 8), cc = e % (C::NS / 8);
-    const int f = f0 + cc * 8;
-    if (f >= mt) continue;
-    bf16 *dst = obase + row * ld_out + f;
-    *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(zh + (row * C::ZLD + cc * 8) * 2);
-    *reinterpret_cast<uint4 *>(dst + plane_out) =
-        *reinterpret_cast<const uint4 *>(zl + (row * C::ZLD + cc * 8) * 2);
-  }
-}
 
 // ------------------------------------------------------------------ fp32 --
 
@@ -206,43 +98,7 @@ __global__ void __launch_bounds__(256) dynamic_mix_f32(const float *zt, long lon
   }
 }
 
-template <typename K>
-avey_status set_smem(K kern, int bytes, const char *name) {
-  if (bytes <= 48 * 1024) return AVEY_OK;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e != cudaSuccess) {
-    set_detail("%s: %s", name, cudaGetErrorString(e));
-    return AVEY_ERR_CUDA;
-  }
-  return AVEY_OK;
-}
-
-template <int S>
-avey_status run_static_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks, int mt,
-                          int64_t plane, bf16 *out, int64_t ld_out, int64_t plane_out,
-                          cudaStream_t s) {
-  using C = StaticTile<S>;
-  if (avey_status st = set_smem(static_mix_x2<S>, C::SMEM, "static_mix_x2")) return st;
-  const dim3 grid((mt + C::NS - 1) / C::NS, blocks);
-  static_mix_x2<S><<<grid, 256, C::SMEM, s>>>(V, zt, ld, mt, plane, out, ld_out, plane_out);
-  AVEY_CHECK_LAUNCH("static_mix_x2", s);
-  return AVEY_OK;
-}
-
 }  // namespace
-
-avey_status launch_static_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks, int S,
-                                 int mt, int64_t plane, bf16 *out, int64_t ld_out,
-                                 int64_t plane_out, cudaStream_t s) {
-  switch (S) {
-    case 16: return run_static_x2<16>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
-    case 32: return run_static_x2<32>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
-    case 64: return run_static_x2<64>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
-    case 128: return run_static_x2<128>(V, zt, ld, blocks, mt, plane, out, ld_out, plane_out, s);
-  }
-  set_detail("static mix: S=%d unsupported", S);
-  return AVEY_ERR_UNSUPPORTED;
-}
 
 avey_status launch_static_mix_f32(const float *V, const float *zt, int64_t ld_zt, float *out,
                                   int64_t ld_out, int blocks, int S, int mt, cudaStream_t s) {

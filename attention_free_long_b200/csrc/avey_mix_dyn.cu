@@ -14,20 +14,24 @@
 //      rows x 64 features, K-major, 128-byte swizzle); each stage is both
 //      operands of four 128 x 128 x 16 MMAs, so TMEM holds R = Z_hi Z_hi^T of
 //      the whole tile (the blocks outside the diagonal splits go unused).
-//   2. eq. 6 in the epilogue warps, one TMEM lane (token row i) per thread:
-//      |z_i| = sqrt(R_ii) from the diagonal, the cosines of the row's own
-//      split, their sum, and Gt = cos / (sum + eps) in fp32, split to a bf16
-//      pair and written into shared memory as the K-major A operand of step
-//      3 (block-diagonal: the zeros outside the splits are written once).
+//   2. eq. 6 in the epilogue warps, two threads per TMEM lane (token row i),
+//      each on half of the row's split: 1/|z_i| = 1/sqrt(R_ii) from the
+//      diagonal, the cosines R_ij / (|z_i| |z_j|), the row sum (two halves
+//      met in shared memory) and Gt = cos / (sum + eps) in fp32, split to a
+//      bf16 pair and written into shared memory as the K-major A operand of
+//      step 3 (block-diagonal: the zeros outside the splits are written once).
 //   3. Apply.  Z_t is read straight from the token-major activation as an
 //      MN-major B operand: TMA boxes of 64 features x 64 tokens per plane.
 //      Per 16 tokens three MMAs (Gt_hi Z_hi + Gt_lo Z_hi + Gt_hi Z_lo) into
-//      one of two 64-column accumulators; the epilogue splits c to a pair,
-//      stages it per warp in swizzled shared memory and stores it by TMA.
+//      one of two 64-column accumulators; the epilogue (32 columns per warp)
+//      splits c to a pair, stages it in a 4 KB swizzled buffer per warp and
+//      stores it by TMA (a thread holds a row, so direct stores would touch 32
+//      rows per instruction: measured 1.5x slower), which leaves room for
+//      seven ring stages (112 KB of loads in flight).
 // The hi rows are read twice (steps 1 and 3); the second read is close
 // enough in time to the first to be served mostly from L2.
-// Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue, warps 2-5
-// epilogue (one per TMEM lane quarter).  Every wait is bounded
+// Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue, warps 2-9
+// epilogue (two per TMEM lane quarter).  Every wait is bounded
 // (avey_common.cuh); a wait that runs out records AVEY_ERR_DEVICE_TIMEOUT and
 // the kernel drains and returns.
 #include <algorithm>
@@ -40,19 +44,18 @@ namespace {
 
 constexpr int DT = 128;                    // token rows per tile
 constexpr int DF = 64;                     // features per Gram chunk and per apply tile
-constexpr int D_EPI = 4;                   // epilogue warps
+constexpr int D_EPI = 8;                   // epilogue warps: two per TMEM lane quarter
 constexpr int D_THR = 64 + 32 * D_EPI;
 constexpr uint32_t D_STAGE = 16384;        // 128 rows x 64 features, or 2 planes x 64 x 64
 constexpr uint32_t D_ZBOX = 8192;          // one plane of an apply stage: 64 tokens x 64 features
-constexpr int D_STAGES = 5;
+constexpr int D_STAGES = 7;
 constexpr uint32_t D_GT_CHUNK = 16384;     // 128 rows x 64 tokens of one Gt plane
 constexpr uint32_t D_GT_PLANE = 2 * D_GT_CHUNK;
-constexpr uint32_t D_OUT = 4096;           // one plane of a warp's output box: 32 rows x 64
-constexpr uint32_t D_OUT_WARP = 2 * 2 * D_OUT;  // two buffers x (hi, lo)
+constexpr uint32_t D_OUT = 2048;           // one plane of a warp's output box: 32 rows x 32
 constexpr uint32_t D_GT_OFF = D_STAGES * D_STAGE;
 constexpr uint32_t D_OUT_OFF = D_GT_OFF + 2 * D_GT_PLANE;
-constexpr uint32_t D_CTRL_OFF = D_OUT_OFF + D_EPI * D_OUT_WARP;
-constexpr uint32_t D_CTRL = 2048;         // barriers, TMEM address, flag, norms [2][128]
+constexpr uint32_t D_CTRL_OFF = D_OUT_OFF + D_EPI * 2 * D_OUT;
+constexpr uint32_t D_CTRL = 4096;  // barriers, TMEM address, flag, 1/norms [2][128], sums [2][2][128]
 constexpr uint32_t D_SMEM = D_CTRL_OFF + D_CTRL + 1024;  // + alignment slack
 static_assert(D_SMEM <= 232448, "shared memory budget");
 static_assert(D_GT_OFF % 1024 == 0 && D_OUT_OFF % 1024 == 0 && D_CTRL_OFF % 1024 == 0,
@@ -97,14 +100,20 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int k) {
                                ((((k >> 3) ^ row) & 7) << 4) + (k & 7) * 2);
 }
 
-template <int S, bool COUPLED>
+// Contextualizer kinds of the kernel: eq. 6, the coupled causal map, or the
+// static map V (shared by every split; no Gram).
+enum { MIX_DYNAMIC = 0, MIX_COUPLED = 1, MIX_STATIC = 2 };
+
+template <int S, int KIND>
 __global__ void __launch_bounds__(D_THR, 1)
-    dyn_mix_tc_kernel(const __grid_constant__ CUtensorMap tmG,
+    split_mix_tc_kernel(const __grid_constant__ CUtensorMap tmG,
                       const __grid_constant__ CUtensorMap tmZh,
                       const __grid_constant__ CUtensorMap tmZl,
                       const __grid_constant__ CUtensorMap tmOh,
                       const __grid_constant__ CUtensorMap tmOl, const DynArgs a) {
   static_assert(S == 16 || S == 32 || S == 64 || S == 128, "split size");
+  constexpr bool kGram = KIND != MIX_STATIC;     // eq. 6 / coupled: Gram per tile
+  constexpr bool kCoupled = KIND == MIX_COUPLED;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
@@ -113,21 +122,23 @@ __global__ void __launch_bounds__(D_THR, 1)
   const uint32_t gth = sbase + D_GT_OFF, gtl = gth + D_GT_PLANE;
   uint8_t *ctrl = base + D_CTRL_OFF;
   const uint32_t cbase = sbase + D_CTRL_OFF;
-  // control block: full[s] @8s, empty[s] @64+8s (s < 8), tfull[2] @128,
-  // tempty[2] @144, gfull @160, gempty @168, gtready @176, gtfree @184,
-  // drain @192, tmem base @200, abort flag @204, norms [2][128] fp32 @256
-  static_assert(D_STAGES <= 8, "control block holds at most 8 stages");
+  // control block: full[s] @8s, empty[s] @128+8s (s < 16), tfull[2] @256,
+  // tempty[2] @272, gfull @288, gempty @296, gtready @304, gtfree @312,
+  // drain @320, tmem base @328, abort flag @332, 1/norms [2][128] fp32 @512,
+  // half-row sums [2][2][128] fp32 @1536
+  static_assert(D_STAGES <= 16, "control block holds at most 16 stages");
   auto full_bar = [&](int s) { return cbase + 8u * s; };
-  auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
-  auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
-  auto tempty_bar = [&](int i) { return cbase + 144u + 8u * i; };
-  const uint32_t gfull_bar = cbase + 160u, gempty_bar = cbase + 168u;
-  const uint32_t gtready_bar = cbase + 176u, gtfree_bar = cbase + 184u;
-  const uint32_t drain_bar = cbase + 192u;
-  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 200);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 204);
-  float *s_norm = reinterpret_cast<float *>(ctrl + 256);
-  static_assert(256 + 2 * 128 * 4 <= D_CTRL, "control block size");
+  auto empty_bar = [&](int s) { return cbase + 128u + 8u * s; };
+  auto tfull_bar = [&](int i) { return cbase + 256u + 8u * i; };
+  auto tempty_bar = [&](int i) { return cbase + 272u + 8u * i; };
+  const uint32_t gfull_bar = cbase + 288u, gempty_bar = cbase + 296u;
+  const uint32_t gtready_bar = cbase + 304u, gtfree_bar = cbase + 312u;
+  const uint32_t drain_bar = cbase + 320u;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 328);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 332);
+  float *s_rn = reinterpret_cast<float *>(ctrl + 512);
+  float *s_rs = reinterpret_cast<float *>(ctrl + 1536);
+  static_assert(1536 + 4 * 128 * 4 <= D_CTRL, "control block size");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -148,7 +159,7 @@ __global__ void __launch_bounds__(D_THR, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(ctrl + 200), D_COLS);
+    tmem_alloc(smem_u32(ctrl + 328), D_COLS);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -184,7 +195,7 @@ __global__ void __launch_bounds__(D_THR, 1)
       };
       for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
         const int r0 = tile * DT;
-        for (int kc = 0; kc < a.nk; ++kc) {  // Gram: the hi rows, 64 features a stage
+        for (int kc = 0; kGram && kc < a.nk; ++kc) {  // Gram: the hi rows
           if (!(ok = next())) break;
           tma_load_3d(sbase + stage * D_STAGE, &tmG, full_bar(stage), kc * DF, r0, 0);
           advance();
@@ -220,6 +231,7 @@ __global__ void __launch_bounds__(D_THR, 1)
       uint32_t phase = 0, acc_phase = 0, gphase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        if constexpr (kGram) {
         // Gram of the tile's hi rows into TMEM columns [0, 128)
         if (!(ok = mbar_wait(gempty_bar, gphase ^ 1u, abort_flag))) break;
         tc_fence_after();
@@ -240,9 +252,13 @@ __global__ void __launch_bounds__(D_THR, 1)
         }
         if (!ok) break;
         tc_commit(gfull_bar);
-        // c = Gt Z_t, 64 features at a time
-        if (!(ok = mbar_wait(gtready_bar, gphase, abort_flag))) break;
-        tc_fence_after();
+        }
+        // c = Gt Z_t (or V Z_t), 64 features at a time; the static V is
+        // written once, before the first tile
+        if (kGram || tile == static_cast<int>(blockIdx.x)) {
+          if (!(ok = mbar_wait(gtready_bar, kGram ? gphase : 0u, abort_flag))) break;
+          tc_fence_after();
+        }
         for (int jn = 0; jn < a.nk && ok; ++jn) {
           if (!(ok = mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag))) break;
           tc_fence_after();
@@ -260,7 +276,7 @@ __global__ void __launch_bounds__(D_THR, 1)
               const uint64_t bh = dyn_desc_mn(st + 2048u * kk);
               const uint64_t bl = dyn_desc_mn(st + D_ZBOX + 2048u * kk);
               tc_mma_bf16(d_tmem, ah, bh, id_apply, (kh | kk) != 0);
-              tc_mma_bf16(d_tmem, al, bh, id_apply, 1u);
+              if constexpr (kGram) tc_mma_bf16(d_tmem, al, bh, id_apply, 1u);  // V is exact in bf16
               tc_mma_bf16(d_tmem, ah, bl, id_apply, 1u);
             }
             tc_commit(empty_bar(stage));
@@ -287,137 +303,175 @@ __global__ void __launch_bounds__(D_THR, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
+    // Eight warps, two per TMEM lane quarter: warp (quarter, h) owns token row
+    // `row` and half h of the work on it (half of the row's split in eq. 6,
+    // 32 of each 64-feature accumulator in the apply).
     const int quarter = warp & 3;          // TMEM lanes 32 quarter .. + 31
+    const int h = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;   // token row within the tile
-    constexpr int W = S >= 32 ? S : 32;    // Gram columns a warp reads
-    const int col0 = (quarter * 32 / W) * W;
+    constexpr int NQ = S / 2;              // split columns per thread
+    constexpr int LW = NQ >= 32 ? NQ : 32; // Gram columns a warp loads
     const int srow = row / S * S;          // first row of this row's split
-    const int sub = srow - col0;           // 0, or 16 for S = 16
+    const int q0 = srow + h * NQ;          // first split column of this thread
+    // warp-uniform load column: this half of the split for S >= 64, else the
+    // warp's own 32 columns (S = 32: its split; S = 16: its two splits)
+    const int lcol = S >= 64 ? q0 : quarter * 32;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    uint8_t *ob = base + D_OUT_OFF + (warp - 2) * D_OUT_WARP;
-    const uint32_t ob_s = sbase + D_OUT_OFF + (warp - 2) * D_OUT_WARP;
-    // Gt outside the diagonal splits stays zero: clear this row of both planes once
+    uint8_t *ob = base + D_OUT_OFF + (warp - 2) * 2 * D_OUT;  // staging: hi, lo
+    const uint32_t ob_s = sbase + D_OUT_OFF + (warp - 2) * 2 * D_OUT;
+    // Gt outside the diagonal splits stays zero: clear this row of both planes
+    // once (half h clears K chunk h)
     {
       const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4 *>(base + D_GT_OFF + pl * D_GT_PLANE + ch * D_GT_CHUNK +
-                                       sw128_off(row, c * 8)) = z;
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4 *>(base + D_GT_OFF + pl * D_GT_PLANE + h * D_GT_CHUNK +
+                                     sw128_off(row, c * 8)) = z;
     }
-    int acc = 0, obuf = 0;
+    if constexpr (!kGram) {
+      // the static map: V in every diagonal S x S block of the hi plane, once
+      // (after every row's zeros: the two threads of a row cleared different
+      // K chunks, and this thread's V columns may lie in the other's)
+      named_bar_sync(1, 32 * D_EPI);
+#pragma unroll
+      for (int q = 0; q < NQ; q += 8) {
+        const uint4 vv = *reinterpret_cast<const uint4 *>(a.V + (row - srow) * S + h * NQ + q);
+        const int k = q0 + q;
+        *reinterpret_cast<uint4 *>(base + D_GT_OFF + (k / 64) * D_GT_CHUNK + sw128_off(row, k % 64)) = vv;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(gtready_bar);
+    }
+    int acc = 0;
     uint32_t acc_phase = 0, gphase = 0;
     bool ok = true;
-    // Every epilogue warp runs the same number of named barriers (one per
+    // Every epilogue warp runs the same number of named barriers (two per
     // tile): after a failed wait a warp stops waiting and working but still
     // walks the tile loop, so the others never wait for it.
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
       const int r0 = tile * DT;
+      if constexpr (kGram) {
+      float *rn = s_rn + (gphase & 1u) * 128;
+      float *rs = s_rs + (gphase & 1u) * 256;
       // ---- eq. 6 from the Gram ----
-      float v[W];
-      float gii = 0.f;
+      float g[NQ];
       const bool got = ok && mbar_wait(gfull_bar, gphase, abort_flag);
       if (got) {
         tc_fence_after();
+        float v[LW];
 #pragma unroll
-        for (int q = 0; q < W; q += 32)
-          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(col0 + q),
+        for (int q = 0; q < LW; q += 32)
+          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(lcol + q),
                     *reinterpret_cast<float(*)[32]>(&v[q]));
+        // this thread's NQ split columns, at offset q0 - lcol in v
+        const int off = q0 - lcol;  // 0 for S >= 64; 0 or 16 (S = 32); 0, 8, 16, 24 (S = 16)
 #pragma unroll
-        for (int q = 0; q < W; ++q)
-          if (col0 + q == row) gii = v[q];
+        for (int q = 0; q < NQ; ++q) {
+          if constexpr (S >= 64) {
+            g[q] = v[q];
+          } else if constexpr (S == 32) {
+            g[q] = off ? v[16 + q] : v[q];
+          } else {
+            g[q] = off == 0 ? v[q] : off == 8 ? v[8 + q] : off == 16 ? v[16 + q] : v[24 + q];
+          }
+        }
+        // the diagonal R_ii sits in exactly one of the row's two threads
+        if (row >= q0 && row < q0 + NQ) {
+          float gii = 0.f;
+#pragma unroll
+          for (int q = 0; q < NQ; ++q)
+            if (q0 + q == row) gii = g[q];
+          rn[row] = 1.0f / fmaxf(sqrtf(gii), 1e-12f);
+        }
       } else {
         ok = false;
       }
-      float *nrm = s_norm + (gphase & 1u) * 128;
-      nrm[row] = fmaxf(sqrtf(gii), 1e-12f);
       tc_fence_before();
       __syncwarp();
       if (got && lane == 0) mbar_arrive(gempty_bar);  // the Gram's TMEM may be overwritten
-      named_bar_sync(1, 32 * D_EPI);                   // every row's norm is in place
+      named_bar_sync(1, 32 * D_EPI);                   // every row's 1/|z| is in place
+      float part = 0.f;
+      if (ok) {
+        const float ri = rn[row];
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          g[q] = g[q] * (ri * rn[q0 + q]);  // the cosine
+          part += g[q];
+        }
+      }
+      rs[h * 128 + row] = part;
+      named_bar_sync(1, 32 * D_EPI);                   // both halves of every row sum
       gphase ^= 1u;
       if (!ok) continue;
-      const float ni = nrm[row];
-      // the row's own split, in place: v[0 .. S) (for S = 16, the warp read 32
-      // columns and this row's split is the half at `sub`)
-      if constexpr (S < 32) {
-#pragma unroll
-        for (int q = 0; q < S; ++q) v[q] = sub ? v[q + 16] : v[q];
-      }
-      float rs = 0.f;
-#pragma unroll
-      for (int q = 0; q < S; ++q) {
-        v[q] = v[q] / (ni * nrm[srow + q]);
-        rs += v[q];
-      }
-      if constexpr (COUPLED) {
+      if constexpr (kCoupled) {
         const int i = row - srow;
 #pragma unroll
-        for (int q = 0; q < S; ++q)
-          v[q] = q <= i ? __bfloat162float(a.V[i * S + q]) * v[q] : 0.f;
+        for (int q = 0; q < NQ; ++q) {
+          const int j = h * NQ + q;
+          g[q] = j <= i ? __bfloat162float(a.V[i * S + j]) * g[q] : 0.f;
+        }
       } else {
-        const float den = rs + a.eps;
+        const float dinv = 1.0f / (rs[row] + rs[128 + row] + a.eps);
 #pragma unroll
-        for (int q = 0; q < S; ++q) v[q] = v[q] / den;
+        for (int q = 0; q < NQ; ++q) g[q] = g[q] * dinv;
       }
       // the previous tile's MMAs must be done with Gt before it is rewritten
       // (gphase now has the parity of the previous tile)
       if (!(ok = mbar_wait(gtfree_bar, gphase, abort_flag))) continue;
 #pragma unroll
-      for (int q = 0; q < S; q += 8) {
-        uint4 h, l;
-        split_pack(v[q], v[q + 1], h.x, l.x);
-        split_pack(v[q + 2], v[q + 3], h.y, l.y);
-        split_pack(v[q + 4], v[q + 5], h.z, l.z);
-        split_pack(v[q + 6], v[q + 7], h.w, l.w);
-        const int k = srow + q;  // token column of Gt
-        const uint32_t off = (k / 64) * D_GT_CHUNK + sw128_off(row, k % 64);
-        *reinterpret_cast<uint4 *>(base + D_GT_OFF + off) = h;
-        *reinterpret_cast<uint4 *>(base + D_GT_OFF + D_GT_PLANE + off) = l;
+      for (int q = 0; q < NQ; q += 8) {
+        uint4 hv, lv;
+        split_pack(g[q], g[q + 1], hv.x, lv.x);
+        split_pack(g[q + 2], g[q + 3], hv.y, lv.y);
+        split_pack(g[q + 4], g[q + 5], hv.z, lv.z);
+        split_pack(g[q + 6], g[q + 7], hv.w, lv.w);
+        const int k = q0 + q;  // token column of Gt
+        const uint32_t o = (k / 64) * D_GT_CHUNK + sw128_off(row, k % 64);
+        *reinterpret_cast<uint4 *>(base + D_GT_OFF + o) = hv;
+        *reinterpret_cast<uint4 *>(base + D_GT_OFF + D_GT_PLANE + o) = lv;
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(gtready_bar);
+      } else if (!ok) {
+        continue;
+      }
       // ---- c tiles: TMEM -> split pair -> swizzled staging -> TMA store ----
       for (int jn = 0; jn < a.nk; ++jn) {
         if (!(ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag))) break;
         tc_fence_after();
-        float c[64];
-        tmem_ld64(tmem_base + lane_off + 128u + static_cast<uint32_t>(acc * DF), c);
+        float c[32];
+        tmem_ld32(tmem_base + lane_off + 128u + static_cast<uint32_t>(acc * DF + h * 32), c);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty_bar(acc));
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
-        if (r0 + quarter * 32 >= a.rows) continue;  // rows past T are never stored
-        // this buffer's previous store has finished reading it
-        if (lane == 0) bulk_wait_read<1>();
+        const int x0 = jn * DF + h * 32;
+        // rows past T and features past m_t are never stored
+        if (r0 + quarter * 32 >= a.rows || x0 >= a.mt) continue;
+        // the warp's previous store has finished reading the staging buffer
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
-        uint8_t *bh = ob + obuf * 2 * D_OUT;
-        uint8_t *bl = bh + D_OUT;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          uint4 h, l;
-          split_pack(c[8 * g], c[8 * g + 1], h.x, l.x);
-          split_pack(c[8 * g + 2], c[8 * g + 3], h.y, l.y);
-          split_pack(c[8 * g + 4], c[8 * g + 5], h.z, l.z);
-          split_pack(c[8 * g + 6], c[8 * g + 7], h.w, l.w);
-          const uint32_t off = lane * 128 + (((g ^ lane) & 7) << 4);
-          *reinterpret_cast<uint4 *>(bh + off) = h;
-          *reinterpret_cast<uint4 *>(bl + off) = l;
+        for (int gq = 0; gq < 4; ++gq) {
+          uint32_t hv[4], lv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) split_pack(c[8 * gq + 2 * u], c[8 * gq + 2 * u + 1], hv[u], lv[u]);
+          const uint32_t o = static_cast<uint32_t>(lane * 64 + ((gq ^ ((lane >> 1) & 3)) << 4));
+          *reinterpret_cast<uint4 *>(ob + o) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          *reinterpret_cast<uint4 *>(ob + D_OUT + o) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          const uint32_t sh = ob_s + obuf * 2 * D_OUT;
-          tma_store_3d(&tmOh, sh, jn * DF, r0 + quarter * 32, 0);
-          tma_store_3d(&tmOl, sh + D_OUT, jn * DF, r0 + quarter * 32, 0);
+          tma_store_3d(&tmOh, ob_s, x0, r0 + quarter * 32, 0);
+          tma_store_3d(&tmOl, ob_s + D_OUT, x0, r0 + quarter * 32, 0);
           bulk_commit();
         }
-        obuf ^= 1;
       }
     }
     if (!ok) {
@@ -435,40 +489,56 @@ __global__ void __launch_bounds__(D_THR, 1)
   }
 }
 
-template <int S, bool COUPLED>
-avey_status run_dyn_mix_tc(const CUtensorMap *maps, const DynArgs &args, cudaStream_t s) {
-  auto kern = dyn_mix_tc_kernel<S, COUPLED>;
+template <int S, int KIND>
+avey_status run_split_mix_tc(const CUtensorMap *maps, const DynArgs &args, cudaStream_t s) {
+  auto kern = split_mix_tc_kernel<S, KIND>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(D_SMEM));
   if (e != cudaSuccess) {
-    set_detail("dynamic mix: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    set_detail("split mix: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     return AVEY_ERR_CUDA;
   }
   const int grid = std::min(args.num_tiles, sm_count());
   kern<<<grid, D_THR, D_SMEM, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
-  AVEY_CHECK_LAUNCH(COUPLED ? "coupled_mix_tc" : "dynamic_mix_tc", s);
+  AVEY_CHECK_LAUNCH(KIND == MIX_DYNAMIC ? "dynamic_mix_tc" : KIND == MIX_COUPLED ? "coupled_mix_tc"
+                                                                                : "static_mix_tc",
+                    s);
   return AVEY_OK;
 }
 
-avey_status dyn_mix_tc(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
-                       int64_t ld_out, int64_t plane_out, int blocks, int S, int mt, float eps,
-                       const bf16 *V, cudaStream_t s) {
+template <int KIND>
+avey_status run_split_mix_s(int S, const CUtensorMap *maps, const DynArgs &args, cudaStream_t s) {
+  switch (S) {
+    case 16: return run_split_mix_tc<16, KIND>(maps, args, s);
+    case 32: return run_split_mix_tc<32, KIND>(maps, args, s);
+    case 64: return run_split_mix_tc<64, KIND>(maps, args, s);
+    default: return run_split_mix_tc<128, KIND>(maps, args, s);
+  }
+}
+
+avey_status split_mix_tc(int kind, const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
+                         int64_t ld_out, int64_t plane_out, int blocks, int S, int mt, float eps,
+                         const bf16 *V, cudaStream_t s) {
   AVEY_REQUIRE(S == 16 || S == 32 || S == 64 || S == 128, AVEY_ERR_UNSUPPORTED,
-               "dynamic mix: S=%d unsupported (16, 32, 64 or 128)", S);
+               "split mix: S=%d unsupported (16, 32, 64 or 128)", S);
   AVEY_REQUIRE(mt >= 8 && mt % 8 == 0 && ld_zt % 8 == 0 && ld_out % 8 == 0 && aligned16(zt) &&
-                   aligned16(out) && aligned16(zt + plane_zt) && aligned16(out + plane_out),
+                   aligned16(out) && aligned16(zt + plane_zt) && aligned16(out + plane_out) &&
+                   (V == nullptr || aligned16(V)),
                AVEY_ERR_INVALID_ARG,
-               "dynamic mix: mt, ld multiples of 8 and 16-byte aligned planes required");
+               "split mix: mt, ld multiples of 8 and 16-byte aligned planes and V required");
+  AVEY_REQUIRE(kind == MIX_DYNAMIC || V != nullptr, AVEY_ERR_INVALID_ARG, "split mix: V is required");
   if (blocks <= 0) return AVEY_OK;
   const long long T = static_cast<long long>(blocks) * S;
-  AVEY_REQUIRE(T <= 0x7fffff00ll, AVEY_ERR_UNSUPPORTED, "dynamic mix: too many rows");
+  AVEY_REQUIRE(T <= 0x7fffff00ll, AVEY_ERR_UNSUPPORTED, "split mix: too many rows");
   CUtensorMap maps[5];
   const uint64_t zrow = static_cast<uint64_t>(ld_zt) * 2, orow = static_cast<uint64_t>(ld_out) * 2;
   if (!encode_bf16_map(&maps[0], zt, mt, T, 1, zrow, zrow * T, DT)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&maps[1], zt, mt, T, 1, zrow, zrow * T, 64)) return AVEY_ERR_CUDA;
   if (!encode_bf16_map(&maps[2], zt + plane_zt, mt, T, 1, zrow, zrow * T, 64)) return AVEY_ERR_CUDA;
-  if (!encode_bf16_map(&maps[3], out, mt, T, 1, orow, orow * T, 32)) return AVEY_ERR_CUDA;
-  if (!encode_bf16_map(&maps[4], out + plane_out, mt, T, 1, orow, orow * T, 32)) return AVEY_ERR_CUDA;
+  // c leaves in boxes of 32 features x 32 rows, 64-byte swizzle
+  if (!encode_map(&maps[3], false, out, mt, T, 1, orow, orow * T, 32, 32, 64)) return AVEY_ERR_CUDA;
+  if (!encode_map(&maps[4], false, out + plane_out, mt, T, 1, orow, orow * T, 32, 32, 64))
+    return AVEY_ERR_CUDA;
   DynArgs args{};
   args.rows = static_cast<int>(T);
   args.mt = mt;
@@ -477,13 +547,9 @@ avey_status dyn_mix_tc(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *ou
   args.eps = eps;
   args.V = V;
   args.status = device_status_word();
-  const bool cp = V != nullptr;
-  switch (S) {
-    case 16: return cp ? run_dyn_mix_tc<16, true>(maps, args, s) : run_dyn_mix_tc<16, false>(maps, args, s);
-    case 32: return cp ? run_dyn_mix_tc<32, true>(maps, args, s) : run_dyn_mix_tc<32, false>(maps, args, s);
-    case 64: return cp ? run_dyn_mix_tc<64, true>(maps, args, s) : run_dyn_mix_tc<64, false>(maps, args, s);
-    default: return cp ? run_dyn_mix_tc<128, true>(maps, args, s) : run_dyn_mix_tc<128, false>(maps, args, s);
-  }
+  if (kind == MIX_DYNAMIC) return run_split_mix_s<MIX_DYNAMIC>(S, maps, args, s);
+  if (kind == MIX_COUPLED) return run_split_mix_s<MIX_COUPLED>(S, maps, args, s);
+  return run_split_mix_s<MIX_STATIC>(S, maps, args, s);
 }
 
 }  // namespace
@@ -491,14 +557,21 @@ avey_status dyn_mix_tc(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *ou
 avey_status launch_dynamic_mix_x2(const bf16 *zt, int64_t ld_zt, int64_t plane_zt, bf16 *out,
                                   int64_t ld_out, int64_t plane_out, int blocks, int S, int mt,
                                   float eps, cudaStream_t s) {
-  return dyn_mix_tc(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, S, mt, eps, nullptr, s);
+  return split_mix_tc(MIX_DYNAMIC, zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, S, mt, eps,
+                      nullptr, s);
 }
 
 avey_status launch_coupled_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld_zt, int64_t plane_zt,
                                   bf16 *out, int64_t ld_out, int64_t plane_out, int blocks, int S,
                                   int mt, cudaStream_t s) {
-  AVEY_REQUIRE(V != nullptr, AVEY_ERR_INVALID_ARG, "coupled mix: V is required");
-  return dyn_mix_tc(zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, S, mt, 0.f, V, s);
+  return split_mix_tc(MIX_COUPLED, zt, ld_zt, plane_zt, out, ld_out, plane_out, blocks, S, mt, 0.f,
+                      V, s);
+}
+
+avey_status launch_static_mix_x2(const bf16 *V, const bf16 *zt, int64_t ld, int blocks, int S,
+                                 int mt, int64_t plane, bf16 *out, int64_t ld_out,
+                                 int64_t plane_out, cudaStream_t s) {
+  return split_mix_tc(MIX_STATIC, zt, ld, plane, out, ld_out, plane_out, blocks, S, mt, 0.f, V, s);
 }
 
 }  // namespace avey
