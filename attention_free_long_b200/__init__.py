@@ -83,6 +83,9 @@ def lib() -> ctypes.CDLL:
         L.avey_layer_forward.argtypes = [ctypes.POINTER(LayerParams), _i, _i, _vp, _vp, _vp, _vp,
                                          _vp, _sz, _vp]
         L.avey_layer_forward.restype = _i
+        L.avey_layer_forward_ex.argtypes = [ctypes.POINTER(LayerParams), _i, _i, _vp, _vp, _vp, _vp,
+                                            _vp, _vp, _vp, _sz, _vp]
+        L.avey_layer_forward_ex.restype = _i
         L.avey_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.avey_layer_workspace_bytes.restype = _sz
         L.avey_layer_workspace_bytes_ex.argtypes = [_i, _i, _i, _i, _i, _i, _i]
@@ -349,12 +352,17 @@ def avey_layer_forward(layer: DeviceLayer, S: int, m_h: int, eps: float, prenorm
                        x_in: Optional[torch.Tensor], x_in_lowp: Optional[torch.Tensor] = None,
                        x_out: Optional[torch.Tensor] = None, lowp_out: bool = True,
                        x_out_lowp: Optional[torch.Tensor] = None,
-                       ws: Optional[torch.Tensor] = None, fp32_out: bool = True):
+                       ws: Optional[torch.Tensor] = None, fp32_out: bool = True,
+                       x_in_rms: Optional[torch.Tensor] = None,
+                       x_out_rms: Optional[torch.Tensor] = None):
     """One layer on x_in fp32 [T, d] (any leading shape that flattens to T rows).
 
     For a bf16 layer, x_in may be None when x_in_lowp (the split pair
     [2, T, d]) is given: the residual is then hi + lo.  fp32_out=False writes
-    only the pair.  Returns (x_out fp32 or None, x_out_lowp pair or None).
+    only the pair.  x_in_rms / x_out_rms (fp32 [T], optional): the prenorm
+    row scales of x_in (used instead of computing them) and of x_out (written),
+    as avey_layer_forward_ex takes them.  Returns (x_out fp32 or None,
+    x_out_lowp pair or None).
     """
     m = layer.Ut.shape[0]
     dt = _dt(layer.Ut)
@@ -378,10 +386,16 @@ def avey_layer_forward(layer: DeviceLayer, S: int, m_h: int, eps: float, prenorm
     p = LayerParams(layer.kind, d, m, m_h, S, eps, int(bool(prenorm)), layer.Ut.data_ptr(),
                     layer.bU.data_ptr(), None if layer.V is None else layer.V.data_ptr(),
                     layer.Ot.data_ptr())
+    for t, nm in ((x_in_rms, "x_in_rms"), (x_out_rms, "x_out_rms")):
+        if t is not None:
+            _need(t, nm)
+            if t.dtype != torch.float32 or t.numel() != T:
+                raise TypeError(f"{nm} must be fp32 with T = {T} entries")
     _check("avey_layer_forward",
-           lib().avey_layer_forward(ctypes.byref(p), dt, T, _ptr(x_in), _ptr(x_in_lowp),
-                                    _ptr(x_out), _ptr(x_out_lowp if dt == AVEY_BF16 else None),
-                                    _ptr(ws), ws.numel(), _stream()))
+           lib().avey_layer_forward_ex(ctypes.byref(p), dt, T, _ptr(x_in), _ptr(x_in_lowp),
+                                       _ptr(x_in_rms), _ptr(x_out),
+                                       _ptr(x_out_lowp if dt == AVEY_BF16 else None), _ptr(x_out_rms),
+                                       _ptr(ws), ws.numel(), _stream()))
     return x_out, (x_out_lowp if dt == AVEY_BF16 else None)
 
 
@@ -408,6 +422,8 @@ class EncoderWorkspace:
     x1: torch.Tensor
     pair0: Optional[torch.Tensor]
     pair1: Optional[torch.Tensor]
+    rms0: Optional[torch.Tensor] = None  # per-row prenorm scales handed between layers
+    rms1: Optional[torch.Tensor] = None
 
 
 def make_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: torch.dtype, prenorm: bool,
@@ -428,7 +444,11 @@ def make_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: torch.
     if dt == AVEY_BF16:
         pair0 = torch.empty((2, T, d), dtype=torch.bfloat16, device=device)
         pair1 = torch.empty((2, T, d), dtype=torch.bfloat16, device=device)
-    return EncoderWorkspace(rank_ws, layer_ws, idx, w, x0, x1, pair0, pair1)
+    rms0 = rms1 = None
+    if prenorm:
+        rms0 = torch.empty((T,), dtype=torch.float32, device=device)
+        rms1 = torch.empty((T,), dtype=torch.float32, device=device)
+    return EncoderWorkspace(rank_ws, layer_ws, idx, w, x0, x1, pair0, pair1, rms0, rms1)
 
 
 def _pair_stream(dt: int, layers) -> bool:
@@ -439,9 +459,11 @@ def _pair_stream(dt: int, layers) -> bool:
 
 def _run_layers(L, layers, dt, T, d, m, m_h, S, eps, prenorm, ws, st, marks):
     """Every layer over the stream in (ws.x0, ws.pair0); returns the fp32 output
-    buffer.  ``marks[3 + li]`` is recorded after layer li."""
+    buffer.  ``marks[3 + li]`` is recorded after layer li.  With prenorm, each
+    layer but the last also writes its output's row scales for the next one."""
     pair_only = _pair_stream(dt, layers)
-    cur, nxt = (ws.x0, ws.pair0), (ws.x1, ws.pair1)
+    hand_rms = bool(prenorm) and ws.rms0 is not None
+    cur, nxt = (ws.x0, ws.pair0, ws.rms0), (ws.x1, ws.pair1, ws.rms1)
     for li, lay in enumerate(layers):
         last = li == len(layers) - 1
         p = LayerParams(lay.kind, d, m, m_h, S, eps, int(bool(prenorm)), lay.Ut.data_ptr(),
@@ -450,9 +472,12 @@ def _run_layers(L, layers, dt, T, d, m, m_h, S, eps, prenorm, ws, st, marks):
         x_in = None if pair_only else _ptr(cur[0])
         x_out = _ptr(nxt[0]) if (last or not pair_only) else None
         x_out_lowp = None if (last and pair_only) else _ptr(nxt[1])
+        rms_in = _ptr(cur[2]) if (hand_rms and li > 0) else None
+        rms_out = _ptr(nxt[2]) if (hand_rms and not last) else None
         _check("avey_layer_forward",
-               L.avey_layer_forward(ctypes.byref(p), dt, T, x_in, _ptr(cur[1]), x_out, x_out_lowp,
-                                    _ptr(ws.layer_ws), ws.layer_ws.numel(), st))
+               L.avey_layer_forward_ex(ctypes.byref(p), dt, T, x_in, _ptr(cur[1]), rms_in, x_out,
+                                       x_out_lowp, rms_out, _ptr(ws.layer_ws), ws.layer_ws.numel(),
+                                       st))
         if marks is not None:
             marks[3 + li].record()
         cur, nxt = nxt, cur
@@ -632,6 +657,8 @@ class ShardWorkspace:
     x1: torch.Tensor
     pair0: Optional[torch.Tensor]
     pair1: Optional[torch.Tensor]
+    rms0: Optional[torch.Tensor] = None  # per-row prenorm scales handed between layers
+    rms1: Optional[torch.Tensor] = None
 
 
 def make_shard_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: torch.dtype,
@@ -642,6 +669,8 @@ def make_shard_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: 
     dt = AVEY_BF16 if dtype == torch.bfloat16 else AVEY_F32
     pair = lambda: (torch.empty((2, T, d), dtype=torch.bfloat16, device=device)
                     if dt == AVEY_BF16 else None)
+    rms = (lambda: torch.empty((max(T, 1),), dtype=torch.float32, device=device)
+           if prenorm else None)
     return ShardWorkspace(
         t0, t1, _ws(rank_workspace_bytes(dt, B, N, d, S), device),
         torch.empty((B, n, n), dtype=torch.float32, device=device),
@@ -649,7 +678,8 @@ def make_shard_workspace(B: int, N: int, d: int, S: int, k: int, m: int, dtype: 
         torch.empty((B, t1 - t0, k), dtype=torch.int32, device=device),
         torch.empty((B, t1 - t0, k), dtype=torch.float32, device=device),
         torch.empty((max(T, 1), d), dtype=torch.float32, device=device),
-        torch.empty((max(T, 1), d), dtype=torch.float32, device=device), pair(), pair())
+        torch.empty((max(T, 1), d), dtype=torch.float32, device=device), pair(), pair(), rms(),
+        rms())
 
 
 def encoder_forward_sharded(x: torch.Tensor, P: torch.Tensor, layers: Sequence[DeviceLayer], S: int,

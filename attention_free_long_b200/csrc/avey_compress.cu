@@ -353,12 +353,13 @@ static avey_status compress_range(const void *x, avey_dtype dt, int B, int N, in
     bf16 *hi = static_cast<bf16 *>(out_lowp);
     bf16 *lo = hi ? hi + static_cast<long long>(B) * nr * S * d : nullptr;
     if (compress_tc_supported(S, d))
-      return launch_compress_tc(xb, B, N, d, k, t0, nr, idx, w, Pb, out, hi, lo, s);
+      return launch_compress_tc(xb, B, N, d, S, k, t0, nr, idx, w, Pb, out, hi, lo, s);
     switch (S) {
       case 16: return run_compress_bf16<16>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
       case 32: return run_compress_bf16<32>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
       case 64: return run_compress_bf16<64>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
       default: return run_compress_bf16<128>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
+      // (S = 64 and 128 with d % 8 == 0 run on tcgen05 above; d % 8 != 0 is rejected)
     }
   }
   AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,

@@ -41,16 +41,18 @@ avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, con
 // split pair c [T, m - k_split] instead of (ahi, alo); k_split % 64 == 0.
 // Residual: x_in (fp32) or, when x_in is null, the pair (xin_hi, xin_lo).
 // Output: x_out (fp32) and/or the pair (xo_hi, xo_lo); either may be null.
+// rms_out (nullable): also 1 / sqrt(mean(x_out^2) + 1e-6) per row, from the
+// fp32 output values (the next layer's prenorm scale).
 avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
                            const float *x_in, const bf16 *xin_hi, const bf16 *xin_lo, float *x_out,
                            bf16 *xo_hi, bf16 *xo_lo, cudaStream_t s, const bf16 *chi = nullptr,
-                           const bf16 *clo = nullptr, int k_split = 0);
+                           const bf16 *clo = nullptr, int k_split = 0, float *rms_out = nullptr);
 
-// Compression on tcgen05 (avey_compress_tc.cu) for S = 64, targets t0 ..
-// t0+nr-1 (idx, w, out as for avey_compress_rows); the split-size mma.sync
-// kernel covers the other S.
+// Compression on tcgen05 (avey_compress_tc.cu) for S = 64 and 128, targets
+// t0 .. t0+nr-1 (idx, w, out as for avey_compress_rows); the split-size
+// mma.sync kernel covers S = 16 and 32.
 bool compress_tc_supported(int S, int d);
-avey_status launch_compress_tc(const bf16 *x, int B, int N, int d, int k, int t0, int nr,
+avey_status launch_compress_tc(const bf16 *x, int B, int N, int d, int S, int k, int t0, int nr,
                                const int32_t *idx, const float *w, const bf16 *P, float *out,
                                bf16 *hi, bf16 *lo, cudaStream_t s);
 

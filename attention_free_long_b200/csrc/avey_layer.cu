@@ -168,6 +168,15 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
                                           const float *x_in, const void *x_in_lowp, float *x_out,
                                           void *x_out_lowp, void *ws, size_t ws_bytes,
                                           avey_stream_t stream) {
+  return avey_layer_forward_ex(p, dt, T, x_in, x_in_lowp, nullptr, x_out, x_out_lowp, nullptr, ws,
+                               ws_bytes, stream);
+}
+
+extern "C" avey_status avey_layer_forward_ex(const avey_layer_params *p, avey_dtype dt, int T,
+                                             const float *x_in, const void *x_in_lowp,
+                                             const float *x_in_rms, float *x_out,
+                                             void *x_out_lowp, float *x_out_rms, void *ws,
+                                             size_t ws_bytes, avey_stream_t stream) {
   AVEY_REQUIRE(p != nullptr, AVEY_ERR_INVALID_ARG, "avey_layer_forward: null params");
   AVEY_REQUIRE(dt == AVEY_F32 || dt == AVEY_BF16, AVEY_ERR_UNSUPPORTED,
                "avey_layer_forward: dtype %d unsupported (F32 or BF16)", int(dt));
@@ -196,6 +205,11 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
                AVEY_ERR_INVALID_ARG, "avey_layer_forward: pointers must be 16-byte aligned");
   AVEY_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255) == 0, AVEY_ERR_INVALID_ARG,
                "avey_layer_forward: workspace must be 256-byte aligned");
+  AVEY_REQUIRE((!x_in_rms || (reinterpret_cast<uintptr_t>(x_in_rms) & 3) == 0) &&
+                   (!x_out_rms || (reinterpret_cast<uintptr_t>(x_out_rms) & 3) == 0),
+               AVEY_ERR_INVALID_ARG, "avey_layer_forward: row scales must be 4-byte aligned");
+  AVEY_REQUIRE(!x_out_rms || x_out_rms != x_in_rms, AVEY_ERR_INVALID_ARG,
+               "avey_layer_forward: x_out_rms must not be x_in_rms");
   const size_t need = avey_layer_workspace_bytes_ex(dt, T, d, m, p->prenorm, S, p->kind);
   AVEY_REQUIRE(ws_bytes >= need, AVEY_ERR_INVALID_ARG,
                "avey_layer_forward: workspace %zu bytes < %zu required", ws_bytes, need);
@@ -221,10 +235,14 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
 
   if (dt == AVEY_F32) {
     float *Z = reinterpret_cast<float *>(w);
-    float *inv = p->prenorm ? reinterpret_cast<float *>(w + align256(static_cast<size_t>(T) * m * 4)) : nullptr;
-    if (inv) {
-      row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_in, T, d, inv);
+    const float *inv = nullptr;
+    if (p->prenorm && x_in_rms) {
+      inv = x_in_rms;  // the scales of x_in, as a previous layer wrote them
+    } else if (p->prenorm) {
+      float *iw = reinterpret_cast<float *>(w + align256(static_cast<size_t>(T) * m * 4));
+      row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_in, T, d, iw);
       AVEY_CHECK_LAUNCH("row_inv_rms", s);
+      inv = iw;
     }
     gemm_f32<F32_ENRICH><<<dim3((m + 63) / 64, (T + 63) / 64), 256, 0, s>>>(
         x_in, static_cast<const float *>(p->Ut), T, m, d, p->bU, inv, nullptr, Z);
@@ -241,6 +259,10 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
     gemm_f32<F32_FUSE><<<dim3((d + 63) / 64, (T + 63) / 64), 256, 0, s>>>(
         Z, static_cast<const float *>(p->Ot), T, d, m, nullptr, nullptr, x_in, x_out);
     AVEY_CHECK_LAUNCH("gemm_f32_fuse", s);
+    if (x_out_rms) {
+      row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_out, T, d, x_out_rms);
+      AVEY_CHECK_LAUNCH("row_inv_rms", s);
+    }
     return AVEY_OK;
   }
 
@@ -262,14 +284,17 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
     xhi = h;
     xlo = l;
   }
-  float *inv = nullptr;
-  if (p->prenorm) {
-    inv = reinterpret_cast<float *>(w + zbytes + xbytes);
+  const float *inv = nullptr;
+  if (p->prenorm && x_in_rms) {
+    inv = x_in_rms;  // the scales of x_in, as a previous layer's fuser wrote them
+  } else if (p->prenorm) {
+    float *iw = reinterpret_cast<float *>(w + zbytes + xbytes);
     if (x_in)
-      row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_in, T, d, inv);
+      row_inv_rms<<<(T + 7) / 8, 256, 0, s>>>(x_in, T, d, iw);
     else
-      row_inv_rms_pair<<<(T + 7) / 8, 256, 0, s>>>(xhi, xlo, T, d, inv);
+      row_inv_rms_pair<<<(T + 7) / 8, 256, 0, s>>>(xhi, xlo, T, d, iw);
     AVEY_CHECK_LAUNCH("row_inv_rms", s);
+    inv = iw;
   }
   st = launch_enrich_tc(xhi, xlo, T, d, static_cast<const bf16 *>(p->Ut), m, p->bU, inv, Zhi, Zlo, s);
   if (st != AVEY_OK) return st;
@@ -295,7 +320,7 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
     bf16 *ohi = static_cast<bf16 *>(x_out_lowp);
     bf16 *olo = ohi ? ohi + static_cast<long long>(T) * d : nullptr;
     return launch_fuse_tc(Zhi, Zlo, T, m, static_cast<const bf16 *>(p->Ot), d, x_in, xhi, xlo, x_out,
-                          ohi, olo, s, Chi, Clo, m_h);
+                          ohi, olo, s, Chi, Clo, m_h, x_out_rms);
   } else if (p->kind == AVEY_STATIC)
     st = launch_static_mix_x2(static_cast<const bf16 *>(p->V), Zhi + m_h, m, blocks, S, mt, plane,
                               Zhi + m_h, m, plane, s);
@@ -308,5 +333,5 @@ extern "C" avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype
   bf16 *ohi = static_cast<bf16 *>(x_out_lowp);
   bf16 *olo = ohi ? ohi + static_cast<long long>(T) * d : nullptr;
   return launch_fuse_tc(Zhi, Zlo, T, m, static_cast<const bf16 *>(p->Ot), d, x_in, xhi, xlo, x_out, ohi,
-                        olo, s);
+                        olo, s, nullptr, nullptr, 0, x_out_rms);
 }

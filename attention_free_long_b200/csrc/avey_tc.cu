@@ -71,8 +71,31 @@ struct TcArgs {
   const bf16 *xin_lo;
   float *x_out;
   int k_split;  // > 0: A columns >= k_split come from the second pair of maps
+  // fuser: when non-null, 1 / sqrt(mean(x_out^2) + 1e-6) of every output row
+  // (the next layer's prenorm scale); the pairs then walk whole row blocks
+  float *rms_out;
   int *status;
 };
+
+// The j-th output tile (row block mt, column block nt) of CTA pair `pair` of
+// `npairs`; false past the last.  Tiles are dealt round-robin, except when
+// the fuser also writes row RMS scales: then each pair takes whole row
+// blocks, all their column blocks in order, so that a row's sum of squares
+// stays in one thread.
+__device__ __forceinline__ bool pair_tile(const TcArgs &a, int pair, int npairs, int j, int &mt,
+                                          int &nt) {
+  if (a.rms_out != nullptr) {
+    const int q = j / a.tiles_n;
+    mt = pair + q * npairs;
+    nt = j - q * a.tiles_n;
+    return mt < a.tiles_m;
+  }
+  const long long tile = pair + static_cast<long long>(j) * npairs;
+  if (tile >= a.num_tiles) return false;
+  mt = static_cast<int>(tile / a.tiles_n);
+  nt = static_cast<int>(tile - static_cast<long long>(mt) * a.tiles_n);
+  return true;
+}
 
 // Single-CTA MaxSim: 128-row A tiles and 256-row B tiles of X.
 struct MaxSimLayout {
@@ -311,7 +334,7 @@ __device__ __forceinline__ void fuse_residual_values(const TcArgs &a, const uint
 __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mout,
                                          const CUtensorMap *mhi, const CUtensorMap *mlo,
                                          uint32_t taddr, int row0, int lane, int nt, uint32_t stg,
-                                         int &it, uint4 (&xi)[8], uint4 (&xj)[8]) {
+                                         int &it, uint4 (&xi)[8], uint4 (&xj)[8], float &ss) {
   const int row = row0 + lane;
   const bool pair = a.out_hi != nullptr;
   const bool f32out = a.x_out != nullptr;
@@ -331,6 +354,10 @@ __device__ __forceinline__ void epi_fuse(const TcArgs &a, const CUtensorMap *mou
     fuse_residual_values(a, xi, o);
 #pragma unroll
     for (int q = 0; q < 32; ++q) o[q] += v[q];
+    if (a.rms_out != nullptr) {
+#pragma unroll
+      for (int q = 0; q < 32; ++q) ss = fmaf(o[q], o[q], ss);
+    }
     if (f32out) {
 #pragma unroll
       for (int c = 0; c < 8; ++c)
@@ -661,8 +688,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int tile = pair; tile < a.num_tiles && ok; tile += npairs) {
-        const int mt = tile / a.tiles_n, nt = tile - (tile / a.tiles_n) * a.tiles_n;
+      int mt, nt;
+      for (int j = 0; ok && pair_tile(a, pair, npairs, j, mt, nt); ++j) {
         const int arow = mt * P::PM + static_cast<int>(rank) * 128;
         const int brow = nt * BN + static_cast<int>(rank) * 128;
         for (int kc = 0; kc < kchunks; ++kc) {
@@ -709,7 +736,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = pair; tile < a.num_tiles && ok; tile += npairs) {
+      int mt_, nt_;
+      for (int jt = 0; ok && pair_tile(a, pair, npairs, jt, mt_, nt_); ++jt) {
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -757,8 +785,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int acc = 0, it = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = pair; tile < a.num_tiles; tile += npairs) {
-      const int mt = tile / a.tiles_n, nt = tile - (tile / a.tiles_n) * a.tiles_n;
+    float ss = 0.f;  // fuser with row RMS output: this row's sum of squares so far
+    int mt, nt;
+    for (int j = 0; pair_tile(a, pair, npairs, j, mt, nt); ++j) {
       const int row0 = mt * P::PM + static_cast<int>(rank) * 128 + quarter * 32;
       uint4 xi[8], xj[8];
       if constexpr (MODE == MODE_FUSE) {
@@ -775,7 +804,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if constexpr (MODE == MODE_ENRICH) {
         epi_enrich(a, &tmO0, &tmO1, taddr, row0, lane, nt, stg, it);
       } else {
-        epi_fuse(a, &tmO0, &tmO1, &tmO2, taddr, row0, lane, nt, stg, it, xi, xj);
+        if (nt == 0) ss = 0.f;
+        epi_fuse(a, &tmO0, &tmO1, &tmO2, taddr, row0, lane, nt, stg, it, xi, xj, ss);
+        if (a.rms_out != nullptr && nt == a.tiles_n - 1 && row0 + lane < a.rows)
+          a.rms_out[row0 + lane] = 1.0f / sqrtf(ss / static_cast<float>(a.cols) + 1e-6f);
       }
       tc_fence_before();
       __syncwarp();
@@ -927,7 +959,7 @@ avey_status launch_enrich_tc(const bf16 *xhi, const bf16 *xlo, int T, int d, con
 avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const bf16 *Ot, int d,
                            const float *x_in, const bf16 *xin_hi, const bf16 *xin_lo, float *x_out,
                            bf16 *xo_hi, bf16 *xo_lo, cudaStream_t s, const bf16 *chi,
-                           const bf16 *clo, int k_split) {
+                           const bf16 *clo, int k_split, float *rms_out) {
   if ((x_in == nullptr && (xin_hi == nullptr || xin_lo == nullptr)) ||
       (x_out == nullptr && xo_hi == nullptr)) {
     set_detail("fuse_tc: needs a residual (fp32 or pair) and an output (fp32 or pair)");
@@ -956,6 +988,7 @@ avey_status launch_fuse_tc(const bf16 *ahi, const bf16 *alo, int T, int m, const
   a.out_hi = xo_hi;
   a.out_lo = xo_lo;
   a.ld_out = d;
+  a.rms_out = rms_out;
   if (chi != nullptr) {
     // columns [k_split, m) of the activation come from c [T, m - k_split]
     if (k_split <= 0 || k_split % BK != 0 || k_split >= m) {

@@ -317,6 +317,27 @@ AVEY_API avey_status avey_layer_forward(const avey_layer_params *p, avey_dtype d
                                void *x_out_lowp, void *ws, size_t ws_bytes,
                                avey_stream_t stream);
 
+/* avey_layer_forward_ex: avey_layer_forward with the per-row prenorm scales
+ * r = 1 / sqrt(mean(x^2) + 1e-6) passed between the layers of a stack, so that
+ * no layer re-reads its input to compute them.  The pages define the layer;
+ * handing its scales over is a property of this implementation only.
+ * x_in_rms   [T] fp32 or NULL: the scales of x_in (as a previous layer's
+ *            x_out_rms wrote them).  Used in place of computing them when
+ *            p->prenorm; ignored otherwise.
+ * x_out_rms  [T] fp32 or NULL: also write the scales of x_out, from its fp32
+ *            values before the split (on the bf16 path the fuser computes
+ *            them in its epilogue; on the fp32 path a separate kernel does).
+ *            Must not be x_in_rms.
+ * Both 4-byte aligned.  Everything else as avey_layer_forward, which is this
+ * call with both NULL.  The scales from x_out_rms equal a recomputation from
+ * x_out's split pair to within float rounding of the sum (about 1e-6
+ * relative), not bit for bit. */
+AVEY_API avey_status avey_layer_forward_ex(const avey_layer_params *p, avey_dtype dt, int T,
+                                           const float *x_in, const void *x_in_lowp,
+                                           const float *x_in_rms, float *x_out, void *x_out_lowp,
+                                           float *x_out_rms, void *ws, size_t ws_bytes,
+                                           avey_stream_t stream);
+
 /* Workspace of avey_layer_forward for S <= 128 (any kind). */
 AVEY_API size_t avey_layer_workspace_bytes(avey_dtype dt, int T, int d, int m, int prenorm);
 
