@@ -29,7 +29,10 @@
 //      rows per instruction: measured 1.5x slower), which leaves room for
 //      seven ring stages (112 KB of loads in flight).
 // The hi rows are read twice (steps 1 and 3); the second read is close
-// enough in time to the first to be served mostly from L2.
+// enough in time to the first to be served mostly from L2.  A tile's Gram is
+// loaded and summed while the CTA's previous tile is applied (its chunks
+// interleaved with the apply stages in the ring), so a tile waits only for
+// eq. 6 between its Gram and its apply.
 // Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue, warps 2-9
 // epilogue (two per TMEM lane quarter).  Every wait is bounded
 // (avey_common.cuh); a wait that runs out records AVEY_ERR_DEVICE_TIMEOUT and
@@ -193,13 +196,21 @@ __global__ void __launch_bounds__(D_THR, 1)
           phase ^= 1u;
         }
       };
+      // Stage order (the MMA issuer consumes the same): the first tile's Gram
+      // chunks, then for every tile its apply stages, two per 64 features,
+      // each pair followed by one Gram chunk of the CTA's next tile, so that
+      // the next Gram is loaded and summed while this tile is applied.
+      auto gram_chunk = [&](int r0, int kc) -> bool {
+        if (!next()) return false;
+        tma_load_3d(sbase + stage * D_STAGE, &tmG, full_bar(stage), kc * DF, r0, 0);
+        advance();
+        return true;
+      };
+      if (kGram && static_cast<int>(blockIdx.x) < a.num_tiles)
+        for (int kc = 0; kc < a.nk && ok; ++kc) ok = gram_chunk(blockIdx.x * DT, kc);
       for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
         const int r0 = tile * DT;
-        for (int kc = 0; kGram && kc < a.nk; ++kc) {  // Gram: the hi rows
-          if (!(ok = next())) break;
-          tma_load_3d(sbase + stage * D_STAGE, &tmG, full_bar(stage), kc * DF, r0, 0);
-          advance();
-        }
+        const int tn = tile + static_cast<int>(gridDim.x);  // this CTA's next tile
         for (int jn = 0; jn < a.nk && ok; ++jn) {  // apply: 64 features x 64 tokens x 2 planes
           for (int kh = 0; kh < 2; ++kh) {
             if (!(ok = next())) break;
@@ -208,6 +219,7 @@ __global__ void __launch_bounds__(D_THR, 1)
             tma_load_3d(st + D_ZBOX, &tmZl, full_bar(stage), jn * DF, r0 + kh * 64, 0);
             advance();
           }
+          if (ok && kGram && tn < a.num_tiles) ok = gram_chunk(tn * DT, jn);
         }
       }
       if (!ok) {
@@ -228,31 +240,34 @@ __global__ void __launch_bounds__(D_THR, 1)
       const uint32_t id_gram = idesc_bf16_f32(DT, DT);
       const uint32_t id_apply = idesc_bf16_f32(DT, DF) | (1u << 16);  // B is MN-major
       int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0, gphase = 0;
+      uint32_t phase = 0, acc_phase = 0, gphase = 0;  // gphase: parity of the tile being applied
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
-        if constexpr (kGram) {
-        // Gram of the tile's hi rows into TMEM columns [0, 128)
-        if (!(ok = mbar_wait(gempty_bar, gphase ^ 1u, abort_flag))) break;
+      // one 64-feature chunk of a tile's Gram into TMEM columns [0, 128)
+      auto gram_chunk = [&](int kc) -> bool {
+        if (!mbar_wait(full_bar(stage), phase, abort_flag)) return false;
         tc_fence_after();
-        for (int kc = 0; kc < a.nk; ++kc) {
-          if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t st = sbase + stage * D_STAGE;
+        const uint32_t st = sbase + stage * D_STAGE;
 #pragma unroll
-          for (int kk = 0; kk < DF / 16; ++kk) {
-            const uint64_t d = dyn_desc_k(st + 32u * kk);
-            tc_mma_bf16(tmem_base, d, d, id_gram, (kc | kk) != 0);
-          }
-          tc_commit(empty_bar(stage));
-          if (++stage == D_STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        for (int kk = 0; kk < DF / 16; ++kk) {
+          const uint64_t d = dyn_desc_k(st + 32u * kk);
+          tc_mma_bf16(tmem_base, d, d, id_gram, (kc | kk) != 0);
         }
-        if (!ok) break;
-        tc_commit(gfull_bar);
+        tc_commit(empty_bar(stage));
+        if (++stage == D_STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
+        return true;
+      };
+      if (kGram && static_cast<int>(blockIdx.x) < a.num_tiles) {
+        // the first tile's Gram (later tiles' Grams ride along the apply)
+        ok = mbar_wait(gempty_bar, 1u, abort_flag);
+        if (ok) tc_fence_after();
+        for (int kc = 0; kc < a.nk && ok; ++kc) ok = gram_chunk(kc);
+        if (ok) tc_commit(gfull_bar);
+      }
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        const bool next_gram = kGram && tile + static_cast<int>(gridDim.x) < a.num_tiles;
         // c = Gt Z_t (or V Z_t), 64 features at a time; the static V is
         // written once, before the first tile
         if (kGram || tile == static_cast<int>(blockIdx.x)) {
@@ -289,8 +304,18 @@ __global__ void __launch_bounds__(D_THR, 1)
           tc_commit(tfull_bar(acc));
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1u;
+          if (next_gram) {
+            // the next tile's Gram chunk jn: its TMEM was released when this
+            // tile's eq. 6 read the Gram (before gtready), so this wait passes
+            if (jn == 0) {
+              if (!(ok = mbar_wait(gempty_bar, gphase, abort_flag))) break;
+              tc_fence_after();
+            }
+            if (!(ok = gram_chunk(jn))) break;
+          }
         }
         if (!ok) break;
+        if (next_gram) tc_commit(gfull_bar);
         tc_commit(gtfree_bar);  // the tile's MMAs no longer read Gt
         gphase ^= 1u;
       }
