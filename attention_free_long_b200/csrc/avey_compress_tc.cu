@@ -14,8 +14,10 @@
 // (the residual, exact, against a 64 x 64 identity per 64 tokens), and the
 // epilogue writes fp32 and/or the split pair straight to global memory (per
 // token, the warp's 32 lanes store 32 consecutive features), so that all of
-// shared memory but the identity goes to the ring of loads: eight stages of
-// 24 KB for S = 64, three of 64 KB for S = 128.
+// shared memory but the identity (and, for S = 64 with k + 1 <= 8, all of P,
+// 64 KB, loaded once) goes to the ring of loads: nine stages of 16 KB (X
+// alone) for S = 64 with P resident, else eight of 24 KB, three of 64 KB for
+// S = 128.
 // The kernel is bound by HBM and by how many bytes of gathered blocks are in
 // flight.  Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue,
 // warps 2-9 epilogue (two per TMEM lane quarter = 32 features, each on half of
@@ -32,20 +34,26 @@ constexpr int CF = 128;                       // features per tile (M)
 constexpr int C_EPI = 8, C_THR = 64 + 32 * C_EPI;
 constexpr uint32_t C_IDENT = 64 * 64 * 2;     // 8 KB: the 64 x 64 identity (B operand)
 
-template <int S>
+template <int S, int KM>
 struct CompLayout {
   static_assert(S == 64 || S == 128, "split size");
   static constexpr uint32_t XBOX = 64 * S * 2;   // 64 features x S tokens
   static constexpr uint32_t XB = 2 * XBOX;       // the block's 128-feature slab
   static constexpr int PCH = S / 64;             // K chunks of P_r, 64 j each
   static constexpr uint32_t PBOX = S * 64 * 2;   // S i x 64 j
-  static constexpr uint32_t STAGE = XB + PCH * PBOX;
-  static constexpr int STAGES = S == 64 ? 8 : 3;
+  // For S = 64 and k + 1 <= 8, all of P (64 KB) stays in shared memory for
+  // the whole launch and the ring carries X alone; otherwise every stage also
+  // carries its block's P_r.
+  static constexpr bool PRES = S == 64 && KM == 8;
+  static constexpr uint32_t PRES_BYTES = PRES ? KM * PBOX : 0;
+  static constexpr uint32_t STAGE = XB + (PRES ? 0 : PCH * PBOX);
+  static constexpr int STAGES = PRES ? 9 : (S == 64 ? 8 : 3);
   static constexpr int NACC = 512 / S;           // TMEM buffers of S columns
   static constexpr int TOK = S / 2;              // tokens per epilogue warp
-  static constexpr uint32_t SMEM = STAGES * STAGE + C_IDENT + 1024 + 1024;
+  static constexpr uint32_t CTRL = 1024;
+  static constexpr uint32_t SMEM = STAGES * STAGE + PRES_BYTES + C_IDENT + CTRL + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(STAGES <= 8 && NACC <= 8, "the control block holds at most 8 of each");
+  static_assert(STAGES <= 16 && NACC <= 8, "the control block holds 16 stages and 8 buffers");
 };
 
 struct CompArgs {
@@ -116,28 +124,30 @@ template <int S, int KM>
 __global__ void __launch_bounds__(C_THR, 1)
     compress_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                        const CompArgs a) {
-  using L = CompLayout<S>;
+  using L = CompLayout<S, KM>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
-  uint8_t *ident = smem_raw + pad + L::STAGES * L::STAGE;
+  uint8_t *ident = smem_raw + pad + L::STAGES * L::STAGE + L::PRES_BYTES;
   uint8_t *ctrl = ident + C_IDENT;
   const uint32_t sbase = raw_s + pad;
-  const uint32_t ibase = sbase + L::STAGES * L::STAGE;
+  const uint32_t pbase = sbase + L::STAGES * L::STAGE;  // resident P (PRES)
+  const uint32_t ibase = pbase + L::PRES_BYTES;
   const uint32_t cbase = ibase + C_IDENT;
-  // control block: full[8] @0, empty[8] @64, tfull[8] @128, tempty[8] @192,
-  // drain @256, tmem base @264, abort flag @268, lfull[2] @272, lempty[2]
-  // @288, block lists [2][KM] of (split, weight) @512
-  static_assert(512 + 2 * KM * 8 <= 1024, "the block lists fit the control block");
+  // control block: full[16] @0, empty[16] @128, tfull[8] @256, tempty[8]
+  // @320, drain @384, tmem base @392, abort flag @396, lfull[2] @400,
+  // lempty[2] @416, pready @432, block lists [2][KM] of (split, weight) @512
+  static_assert(512 + 2 * KM * 8 <= L::CTRL, "the block lists fit the control block");
   auto full_bar = [&](int s) { return cbase + 8u * s; };
-  auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
-  auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
-  auto tempty_bar = [&](int i) { return cbase + 192u + 8u * i; };
-  const uint32_t drain_bar = cbase + 256u;
-  auto lfull_bar = [&](int i) { return cbase + 272u + 8u * i; };
-  auto lempty_bar = [&](int i) { return cbase + 288u + 8u * i; };
-  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 264);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 268);
+  auto empty_bar = [&](int s) { return cbase + 128u + 8u * s; };
+  auto tfull_bar = [&](int i) { return cbase + 256u + 8u * i; };
+  auto tempty_bar = [&](int i) { return cbase + 320u + 8u * i; };
+  const uint32_t drain_bar = cbase + 384u;
+  auto lfull_bar = [&](int i) { return cbase + 400u + 8u * i; };
+  auto lempty_bar = [&](int i) { return cbase + 416u + 8u * i; };
+  const uint32_t pready_bar = cbase + 432u;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(ctrl + 392);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 396);
   int *list_c = reinterpret_cast<int *>(ctrl + 512);               // [2][KM]
   float *list_w = reinterpret_cast<float *>(ctrl + 512 + 2 * KM * 4);  // [2][KM]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -156,11 +166,12 @@ __global__ void __launch_bounds__(C_THR, 1)
       mbar_init(lfull_bar(i), 1);
       mbar_init(lempty_bar(i), 1 + C_EPI);  // the MMA issuer and the epilogue warps
     }
+    mbar_init(pready_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(ctrl + 264), 512);
+    tmem_alloc(smem_u32(ctrl + 392), 512);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -195,6 +206,11 @@ __global__ void __launch_bounds__(C_THR, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
+      if constexpr (L::PRES) {  // P_0 .. P_k, once for the launch
+        mbar_arrive_expect_tx(pready_bar, static_cast<uint32_t>(a.k + 1) * L::PBOX);
+        for (int r = 0; r <= a.k; ++r)
+          tma_load_3d(pbase + r * L::PBOX, &tmP, pready_bar, r * S, 0, 0);
+      }
       int cn[KM];
       float wn[KM];
       if (static_cast<int>(blockIdx.x) < a.num_tiles) load_list<KM>(a, blockIdx.x, cn, wn);
@@ -235,9 +251,11 @@ __global__ void __launch_bounds__(C_THR, 1)
           mbar_arrive_expect_tx(full_bar(stage), L::STAGE);
           tma_load_3d(st, &tmX, full_bar(stage), slab * CF, c * S, b);
           tma_load_3d(st + L::XBOX, &tmX, full_bar(stage), slab * CF + 64, c * S, b);
+          if constexpr (!L::PRES) {
 #pragma unroll
-          for (int ch = 0; ch < L::PCH; ++ch)
-            tma_load_3d(st + L::XB + ch * L::PBOX, &tmP, full_bar(stage), r * S + ch * 64, 0, 0);
+            for (int ch = 0; ch < L::PCH; ++ch)
+              tma_load_3d(st + L::XB + ch * L::PBOX, &tmP, full_bar(stage), r * S + ch * 64, 0, 0);
+          }
           ++issued;
           if (++stage == L::STAGES) {
             stage = 0;
@@ -255,6 +273,7 @@ __global__ void __launch_bounds__(C_THR, 1)
           cwait_drain(full_bar(s), static_cast<uint32_t>((last / L::STAGES) & 1));
         }
       }
+      if constexpr (L::PRES) cwait_drain(pready_bar, 0);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -265,6 +284,7 @@ __global__ void __launch_bounds__(C_THR, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       int it = 0;
+      if constexpr (L::PRES) ok = mbar_wait(pready_bar, 0, abort_flag);
       for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x, ++it) {
         const int slot = it & 1;
         if (!mbar_wait(lfull_bar(slot), (it >> 1) & 1, abort_flag)) {
@@ -289,9 +309,11 @@ __global__ void __launch_bounds__(C_THR, 1)
           // 16 tokens j a step: +2048 bytes (two 8-token atoms) along X's
           // MN-major rows; +32 bytes along P_r's K-major rows, P box every 64 j
 #pragma unroll
-          for (int kk = 0; kk < S / 16; ++kk)
-            tc_mma_bf16(d_tmem, cdesc_mn(st + 2048u * kk, L::XBOX),
-                        cdesc_k(st + L::XB + (kk >> 2) * L::PBOX + 32u * (kk & 3)), idesc, kk != 0);
+          for (int kk = 0; kk < S / 16; ++kk) {
+            const uint32_t pb = L::PRES ? pbase + r * L::PBOX : st + L::XB + (kk >> 2) * L::PBOX;
+            tc_mma_bf16(d_tmem, cdesc_mn(st + 2048u * kk, L::XBOX), cdesc_k(pb + 32u * (kk & 3)),
+                        idesc, kk != 0);
+          }
           if (r == 0) {  // + X_t^T: the residual, one 64-token half at a time
 #pragma unroll
             for (int hh = 0; hh < S / 64; ++hh)
@@ -409,7 +431,7 @@ __global__ void __launch_bounds__(C_THR, 1)
 template <int S, int KM>
 avey_status run_compress_tc(const CUtensorMap &mx, const CUtensorMap &mp, const CompArgs &a,
                             int grid, cudaStream_t s) {
-  using L = CompLayout<S>;
+  using L = CompLayout<S, KM>;
   auto kern = compress_tc_kernel<S, KM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));

@@ -96,6 +96,13 @@ __device__ __forceinline__ void dyn_drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Gram chunks of the next tile to have issued after the apply pair jn of the
+// current one (nk pairs, nk chunks): none in the first half, then two per
+// pair, all by the last.
+__host__ __device__ constexpr int gram_chunks_after(int jn, int nk) {
+  return 2 * (jn + 1) - nk < 0 ? 0 : (2 * (jn + 1) - nk > nk ? nk : 2 * (jn + 1) - nk);
+}
+
 // Byte offset of element (row, k) of a K-major tile with 128-byte rows and
 // 128-byte swizzle (16-byte chunk c of row r sits at chunk c ^ (r % 8)).
 __device__ __forceinline__ uint32_t sw128_off(int row, int k) {
@@ -198,8 +205,9 @@ __global__ void __launch_bounds__(D_THR, 1)
       };
       // Stage order (the MMA issuer consumes the same): the first tile's Gram
       // chunks, then for every tile its apply stages, two per 64 features,
-      // each pair followed by one Gram chunk of the CTA's next tile, so that
-      // the next Gram is loaded and summed while this tile is applied.
+      // with the Gram chunks of the CTA's next tile placed after the pairs of
+      // the second half (gram_chunks_after), so that the next Gram is loaded
+      // and summed while this tile is applied.
       auto gram_chunk = [&](int r0, int kc) -> bool {
         if (!next()) return false;
         tma_load_3d(sbase + stage * D_STAGE, &tmG, full_bar(stage), kc * DF, r0, 0);
@@ -211,6 +219,7 @@ __global__ void __launch_bounds__(D_THR, 1)
       for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
         const int r0 = tile * DT;
         const int tn = tile + static_cast<int>(gridDim.x);  // this CTA's next tile
+        int g = 0;                                           // its Gram chunks issued
         for (int jn = 0; jn < a.nk && ok; ++jn) {  // apply: 64 features x 64 tokens x 2 planes
           for (int kh = 0; kh < 2; ++kh) {
             if (!(ok = next())) break;
@@ -219,7 +228,11 @@ __global__ void __launch_bounds__(D_THR, 1)
             tma_load_3d(st + D_ZBOX, &tmZl, full_bar(stage), jn * DF, r0 + kh * 64, 0);
             advance();
           }
-          if (ok && kGram && tn < a.num_tiles) ok = gram_chunk(tn * DT, jn);
+          // the next Gram's chunks ride along the second half of this apply,
+          // two per 64 features, so that their second read (the next apply)
+          // follows soon enough to come from L2
+          if (kGram && tn < a.num_tiles)
+            for (; ok && g < gram_chunks_after(jn, a.nk); ++g) ok = gram_chunk(tn * DT, g);
         }
       }
       if (!ok) {
@@ -268,6 +281,7 @@ __global__ void __launch_bounds__(D_THR, 1)
       }
       for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
         const bool next_gram = kGram && tile + static_cast<int>(gridDim.x) < a.num_tiles;
+        int g = 0;  // the next tile's Gram chunks issued
         // c = Gt Z_t (or V Z_t), 64 features at a time; the static V is
         // written once, before the first tile
         if (kGram || tile == static_cast<int>(blockIdx.x)) {
@@ -305,13 +319,15 @@ __global__ void __launch_bounds__(D_THR, 1)
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1u;
           if (next_gram) {
-            // the next tile's Gram chunk jn: its TMEM was released when this
+            // the next tile's Gram chunks: its TMEM was released when this
             // tile's eq. 6 read the Gram (before gtready), so this wait passes
-            if (jn == 0) {
+            const int upto = gram_chunks_after(jn, a.nk);
+            if (g == 0 && upto > 0) {
               if (!(ok = mbar_wait(gempty_bar, gphase, abort_flag))) break;
               tc_fence_after();
             }
-            if (!(ok = gram_chunk(jn))) break;
+            for (; ok && g < upto; ++g) ok = gram_chunk(g);
+            if (!ok) break;
           }
         }
         if (!ok) break;
