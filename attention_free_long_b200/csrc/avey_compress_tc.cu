@@ -365,31 +365,57 @@ __global__ void __launch_bounds__(C_THR, 1)
 #pragma unroll
       for (int i = 0; i < TOK; ++i) o[i] = 0.f;
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-#pragma unroll 1
-      for (int r = 0; r <= a.k && r < KM; ++r) {
-        if (!((mask >> r) & 1u)) continue;
-        const float wr = list_w[slot * KM + r];
-        if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        float v[TOK];
-        const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * S + half * TOK) + lane_off;
-        if constexpr (TOK == 64) {
-          tmem_ld64(taddr, v);
-        } else {
-          tmem_ld32(taddr, v);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(acc));
-#pragma unroll
-        for (int i = 0; i < TOK; ++i) o[i] = fmaf(wr, v[i], o[i]);
+      const uint32_t col = static_cast<uint32_t>(half * TOK) + lane_off;
+      auto take = [&]() {  // the next accumulator in the MMA issuer's order
+        const uint32_t t = static_cast<uint32_t>(acc);
         if (++acc == L::NACC) {
           acc = 0;
           acc_phase ^= 1u;
         }
+        return t;
+      };
+      uint32_t left = mask;  // present blocks not yet added
+#pragma unroll 1
+      while (left != 0u && ok) {
+        const int r1 = __ffs(static_cast<int>(left)) - 1;
+        left &= left - 1u;
+        const float w1 = list_w[slot * KM + r1];
+        if (!(ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag))) break;
+        const uint32_t a1 = take();
+        if constexpr (TOK == 32) {
+          if (left != 0u) {
+            // two blocks per TMEM wait: the second load's latency overlaps the first's
+            const int r2 = __ffs(static_cast<int>(left)) - 1;
+            left &= left - 1u;
+            const float w2 = list_w[slot * KM + r2];
+            if (!(ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag))) break;
+            const uint32_t a2 = take();
+            tc_fence_after();
+            float v1[32], v2[32];
+            tmem_ld32x2(tmem_base + a1 * S + col, tmem_base + a2 * S + col, v1, v2);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(tempty_bar(static_cast<int>(a1)));
+              mbar_arrive(tempty_bar(static_cast<int>(a2)));
+            }
+#pragma unroll
+            for (int i = 0; i < TOK; ++i) o[i] = fmaf(w2, v2[i], fmaf(w1, v1[i], o[i]));
+            continue;
+          }
+        }
+        tc_fence_after();
+        float v[TOK];
+        if constexpr (TOK == 64) {
+          tmem_ld64(tmem_base + a1 * S + col, v);
+        } else {
+          tmem_ld32(tmem_base + a1 * S + col, v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(static_cast<int>(a1)));
+#pragma unroll
+        for (int i = 0; i < TOK; ++i) o[i] = fmaf(w1, v[i], o[i]);
       }
       // the list slot is no longer read by this warp
       __syncwarp();
