@@ -7,7 +7,8 @@
 // blocks stacked in rank order; the weight multiplies the fp32 partial
 // product of its block, so the bf16 embeddings are never re-rounded.
 //
-// bf16 kernel: one CTA per (target split, column slab of d).  Each retrieved
+// bf16 kernel (S = 16 and 32; S = 64 and 128 run on tcgen05 in
+// avey_compress_tc.cu): one CTA per (target split, column slab of d).  Each retrieved
 // block (S rows x slab) and its P_r are staged in shared memory with
 // cp.async, double-buffered over r; 8 warps compute the S x slab product with
 // mma.sync m16n8k16 (P_r from ldmatrix, X from ldmatrix.trans).  The kernel is
@@ -352,15 +353,12 @@ static avey_status compress_range(const void *x, avey_dtype dt, int B, int N, in
     const bf16 *Pb = static_cast<const bf16 *>(P);
     bf16 *hi = static_cast<bf16 *>(out_lowp);
     bf16 *lo = hi ? hi + static_cast<long long>(B) * nr * S * d : nullptr;
+    // S = 64 and 128 run on tcgen05 (d % 8 == 0 is checked above), the
+    // smaller splits on the mma.sync kernel
     if (compress_tc_supported(S, d))
       return launch_compress_tc(xb, B, N, d, S, k, t0, nr, idx, w, Pb, out, hi, lo, s);
-    switch (S) {
-      case 16: return run_compress_bf16<16>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
-      case 32: return run_compress_bf16<32>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
-      case 64: return run_compress_bf16<64>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
-      default: return run_compress_bf16<128>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
-      // (S = 64 and 128 with d % 8 == 0 run on tcgen05 above; d % 8 != 0 is rejected)
-    }
+    if (S == 16) return run_compress_bf16<16>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
+    return run_compress_bf16<32>(xb, B, N, d, n, k, t0, nr, idx, w, Pb, out, hi, lo, s);
   }
   AVEY_REQUIRE(S <= 64 && (S & (S - 1)) == 0, AVEY_ERR_UNSUPPORTED,
                "%s(F32): S=%d unsupported (power of two <= 64)", fn, S);
