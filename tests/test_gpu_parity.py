@@ -114,6 +114,11 @@ SMALL = [
               pattern=(sy.STATIC, sy.DYNAMIC, sy.STATIC), centers=12, sigma=0.5, prenorm=True),
     sy.custom("bf16_k_gt_n", B=2, N=200, S=64, d=64, m=128, k=7, pattern=(sy.DYNAMIC,),
               centers=2, sigma=0.5),
+    # compression with P streamed per block (k + 1 > 8 at S = 64) and S = 128 with few blocks
+    sy.custom("bf16_s64_k9", B=2, N=1500, S=64, d=192, m=256, k=9, pattern=(sy.STATIC, sy.DYNAMIC),
+              centers=10, sigma=0.5),
+    sy.custom("bf16_s128_k3", B=1, N=2000, S=128, d=256, m=256, k=3, pattern=(sy.DYNAMIC,),
+              centers=6, sigma=0.5),
 ]
 
 
