@@ -45,7 +45,7 @@ constexpr int kRedCands = 16;
 constexpr uint32_t HALF_BYTES = 128 * BK * 2;  // 16 KB: 128 rows x 64 bf16
 constexpr uint32_t STAGE_BYTES = 2 * HALF_BYTES;
 constexpr uint32_t TILES_BYTES = kStages * STAGE_BYTES;
-constexpr uint32_t CTRL_BYTES = 10240;
+constexpr uint32_t CTRL_BYTES = 14336;
 constexpr uint32_t SMEM_BYTES = TILES_BYTES + CTRL_BYTES + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -132,7 +132,8 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-// One epilogue warp: its 32 rows (TMEM lanes) x its 128 columns.  With
+// One epilogue warp: its 32 rows (TMEM lanes) x its 128 columns, whose
+// scales c_j sit in the warp's shared-memory copy cs.  With
 // v = x_i . x_j, r_i = 1/|x_i| and c_j = 1/|x_j| (both >= 0), the cosine's
 // row maximum is r_i * max_j (v c_j) and its column maximum c_j * max_i (v r_i);
 // each direction takes one packed product per two entries.  Row maxima per
@@ -141,15 +142,15 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
 // they are summed).
 template <int S>
 __device__ __forceinline__ void pair_rows(uint32_t taddr, int lane, int quarter, int half, float *red,
-                                          float *cm, const float *__restrict__ col_scale,
-                                          float row_scale, bool need_col) {
+                                          float *cm, const float *cs, float row_scale,
+                                          bool need_col) {
   constexpr int CH_PER_CAND = S / 32;
   const float2 r2 = make_float2(row_scale, row_scale);
   float m = -INFINITY;
 #pragma unroll 1
   for (int pr = 0; pr < 2; ++pr) {
     const int ch0 = 4 * half + 2 * pr;  // 32-column chunk index inside the 256-column tile
-    const float4 *cs4 = reinterpret_cast<const float4 *>(col_scale + ch0 * 32);
+    const float4 *cs4 = reinterpret_cast<const float4 *>(cs + 2 * pr * 32);
     float v[64];
     tmem_ld64(taddr + ch0 * 32, v);
 #pragma unroll
@@ -158,7 +159,7 @@ __device__ __forceinline__ void pair_rows(uint32_t taddr, int lane, int quarter,
       float p[32];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const float4 c = __ldg(cs4 + 8 * u + q);
+        const float4 c = cs4[8 * u + q];  // the same address in every lane: a broadcast
         const float2 a = fmul2(make_float2(v[32 * u + 4 * q], v[32 * u + 4 * q + 1]), make_float2(c.x, c.y));
         const float2 b = fmul2(make_float2(v[32 * u + 4 * q + 2], v[32 * u + 4 * q + 3]), make_float2(c.z, c.w));
         p[4 * q] = a.x;
@@ -192,10 +193,10 @@ __device__ __forceinline__ void pair_rows(uint32_t taddr, int lane, int quarter,
 // Leader warp of one half: scores of this CTA's target splits against the
 // half's candidate splits (row maxima), and, right of the diagonal, of the
 // half's splits as targets against this CTA's splits (column maxima times
-// 1/|x_j|, summed over the candidate's columns).
+// 1/|x_j| from the warp's copy cs, summed over the candidate's columns).
 template <int S>
 __device__ __forceinline__ void pair_write(const PairArgs &a, const float *red, const float *cm,
-                                           const float *__restrict__ col_scale, int lane, int b,
+                                           const float *cs, int lane, int b,
                                            int t0, int c0, int half, bool need_col) {
   constexpr int TS = 128 / S, PER = S / 32, CB = 128 / S;
   float *scores = a.scores + static_cast<long long>(b) * a.n * a.n;
@@ -217,7 +218,7 @@ __device__ __forceinline__ void pair_write(const PairArgs &a, const float *red, 
         float mx = cm[((ts * PER) * 8 + ch) * 32 + lane];
 #pragma unroll
         for (int q = 1; q < PER; ++q) mx = fmaxf(mx, cm[((ts * PER + q) * 8 + ch) * 32 + lane]);
-        sum += mx * __ldg(col_scale + ch * 32 + lane);
+        sum += mx * cs[(cl * PER + u) * 32 + lane];
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
@@ -239,7 +240,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   static_assert(kStages <= 8, "the control block holds at most 8 stages");
   // control block: full[6] @0, empty[6] @64, tfull[2] @128, tempty[2] @144,
   // redbar[4] @160, redfree[4] @192, drain @224, tmem base @232, abort @236,
-  // red @256, column maxima @2048
+  // red @256, column maxima @2048, column scales [8 epilogue warps][128] @10240
   auto full_bar = [&](int s) { return cbase + 8u * s; };
   auto empty_bar = [&](int s) { return cbase + 64u + 8u * s; };
   auto tfull_bar = [&](int i) { return cbase + 128u + 8u * i; };
@@ -251,6 +252,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 236);
   float *red = reinterpret_cast<float *>(ctrl + 256);
   float *cmx = reinterpret_cast<float *>(ctrl + 2048);
+  float *csx = reinterpret_cast<float *>(ctrl + 10240);
+  static_assert(10240 + 8 * 128 * 4 <= CTRL_BYTES, "control block size");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -390,11 +393,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int mt, nt;
       if (!cursor_tile(cur, mt, nt)) continue;
       const int b = cur.b;
+      const int row0 = mt * PT + static_cast<int>(rank) * 128;  // this CTA's rows of the tile
+      const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
+      // the scales of this warp's rows and of its half's 128 columns, loaded
+      // before the accumulator wait so that their latency hides behind it
+      const float row_scale = rs[row0 + quarter * 32 + lane];
+      const float4 col4 = __ldg(reinterpret_cast<const float4 *>(rs + nt * PT + half * 128) + lane);
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      float *cs = csx + (warp - 2) * 128;  // read by this warp alone, after this store
+      reinterpret_cast<float4 *>(cs)[lane] = col4;
+      __syncwarp();
       const int rb = acc * 2 + half;
       if (!mbar_wait(red_free(rb), acc_phase ^ 1u, abort_flag)) {
         ok = false;
@@ -402,13 +414,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       const uint32_t taddr =
           tmem_base + static_cast<uint32_t>(acc * PT) + (static_cast<uint32_t>(quarter * 32) << 16);
-      const int row0 = mt * PT + static_cast<int>(rank) * 128;  // this CTA's rows of the tile
       const bool need_col = nt > mt;
       float *red_acc = red + acc * 8 * kRedCands;
       float *cm_acc = cmx + acc * (4 * 8 * 32);
-      const float *rs = a.inv_norm + static_cast<long long>(b) * a.rs_ld;
-      pair_rows<S>(taddr, lane, quarter, half, red_acc, cm_acc, rs + nt * PT, rs[row0 + quarter * 32 + lane],
-                   need_col);
+      pair_rows<S>(taddr, lane, quarter, half, red_acc, cm_acc, cs, row_scale, need_col);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -419,7 +428,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!mbar_wait(red_bar(rb), acc_phase, abort_flag)) {
           ok = false;
         } else {
-          pair_write<S>(a, red_acc, cm_acc, rs + nt * PT, lane, b, row0 / S,
+          pair_write<S>(a, red_acc, cm_acc, cs, lane, b, row0 / S,
                         (nt * PT + half * 128) / S, half, need_col);
         }
         __syncwarp();

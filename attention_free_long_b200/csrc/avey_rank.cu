@@ -3,14 +3,15 @@
 // Background and App. H; papernotes 整体框架).
 //
 //   inv_norms        (bf16) 1/max(||x||, 1e-12) per token, 0 for the pad rows
-//                    of the last split; the tcgen05 MaxSim (avey_tc.cu) reads
-//                    the raw bf16 rows and applies these scales in its epilogue.
+//                    of the last split; the tcgen05 MaxSim (avey_maxsim2.cu,
+//                    and avey_tc.cu for S = 16) reads the raw bf16 rows and
+//                    applies these scales in its epilogue.
 //   normalize_rows   (fp32) N(x) = x / max(||x||, 1e-12) per token, padded to
 //                    n*S rows per sequence (pad rows zero).
 //   maxsim_f32       SIMT fp32 version (one CTA per target/candidate pair).
-//   topk_warp        one warp per target split: k rounds of a warp-wide
-//                    argmax over the split's score row held in shared memory,
-//                    order (score desc, index asc), self excluded, then
+//   topk_warp        one warp per target split, one pass over its score row
+//                    keeping a warp-wide sorted list of the k best, order
+//                    (score desc, index asc), self excluded, then
 //                    w_r = s_r / s_1 with IEEE division (s_1 / s_1 == 1).
 #include <algorithm>
 
@@ -140,34 +141,61 @@ __global__ void __launch_bounds__(256) maxsim_f32(const float *__restrict__ xhat
   }
 }
 
-// One warp per row of inv [B, rs_ld]: rows < N get 1/max(||x||, 1e-12),
-// rows >= N (split padding and tile padding) get 0.
+// Rows of inv [B, rs_ld]: rows < N get 1/max(||x||, 1e-12), rows >= N (split
+// padding and tile padding) get 0.  A persistent grid of resident blocks; each
+// warp takes two rows per step (rows w and w + warps, then on by 2 * warps)
+// and issues the 16-byte loads of both rows, four per lane and row for every
+// 1024 features, before any use, so that enough bytes are in flight to cover
+// HBM latency.  Each lane sums its features in the same order for any grid.
 __global__ void __launch_bounds__(256) inv_norms(const bf16 *__restrict__ x, int B, int N, int d,
                                                  int rs_ld, float *__restrict__ inv) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= static_cast<long long>(B) * rs_ld) return;
-  const int b = static_cast<int>(row / rs_ld);
-  const int tok = static_cast<int>(row - static_cast<long long>(b) * rs_ld);
-  if (tok >= N) {
-    if (lane == 0) inv[row] = 0.f;
-    return;
-  }
-  const bf16 *src = x + (static_cast<long long>(b) * N + tok) * d;
-  float ss = 0.f;
-  for (int j = lane * 8; j < d; j += 256) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(src + j);
-    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+  const long long warps = static_cast<long long>(gridDim.x) * 8;
+  const long long total = static_cast<long long>(B) * rs_ld;
+  for (long long r0 = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); r0 < total;
+       r0 += 2 * warps) {
+    const bf16 *src[2];
+    bool live[2];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 f = unpack_bf16(w4[q]);
-      ss = fmaf(f.x, f.x, ss);
-      ss = fmaf(f.y, f.y, ss);
+    for (int h = 0; h < 2; ++h) {
+      const long long row = r0 + h * warps;
+      const int b = static_cast<int>(row / rs_ld);
+      const int tok = static_cast<int>(row - static_cast<long long>(b) * rs_ld);
+      live[h] = row < total && tok < N;
+      src[h] = x + (live[h] ? (static_cast<long long>(b) * N + tok) * d : 0);
+    }
+    float ss[2] = {0.f, 0.f};
+    for (int j0 = lane * 8; j0 < d; j0 += 4 * 256) {
+      uint4 u[2][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          u[h][r] = live[h] && j0 + r * 256 < d
+                        ? *reinterpret_cast<const uint4 *>(src[h] + j0 + r * 256)
+                        : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const uint32_t w4[4] = {u[h][r].x, u[h][r].y, u[h][r].z, u[h][r].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = unpack_bf16(w4[q]);
+            ss[h] = fmaf(f.x, f.x, ss[h]);
+            ss[h] = fmaf(f.y, f.y, ss[h]);
+          }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float t = ss[h];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+      const long long row = r0 + h * warps;
+      if (lane == 0 && row < total) inv[row] = live[h] ? 1.0f / fmaxf(sqrtf(t), 1e-12f) : 0.f;
     }
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  if (lane == 0) inv[row] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
 }
 
 constexpr int kTopkWarps = 8;
@@ -293,7 +321,9 @@ avey_status launch_normalize(const void *x, avey_dtype dt, int B, int N, int d, 
 avey_status launch_inv_norms(const bf16 *x, int B, int N, int d, int rs_ld, float *inv,
                              cudaStream_t s) {
   const long long rows = static_cast<long long>(B) * rs_ld;
-  inv_norms<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(x, B, N, d, rs_ld, inv);
+  const long long blocks = std::min<long long>((rows + 15) / 16, 8ll * sm_count());
+  if (blocks <= 0) return AVEY_OK;
+  inv_norms<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, B, N, d, rs_ld, inv);
   AVEY_CHECK_LAUNCH("inv_norms", s);
   return AVEY_OK;
 }

@@ -329,11 +329,22 @@ def forward_leg(av, wl, dev, args, rank, world, local, barrier, e2e=True, sample
     st = av.device_status()
     if st != 0:
         raise RuntimeError(f"device status {av.STATUS.get(st, st)} after the timed region ({wl.name})")
-    kern = {}
-    for name, kms in trace.kernels():
-        kern.setdefault(name, []).append(kms)
-    kernels = {name: {"ms_per_launch": float(np.mean(v)), "launches_per_step": len(v) / args.steps,
-                      "ms_per_step": float(np.sum(v)) / args.steps} for name, v in kern.items()}
+    # the first interval runs from the trace's opening event, recorded before
+    # the host had enqueued the first kernel, so it holds the host's lead-in:
+    # it counts as a launch but is left out of the per-launch time
+    kern, count, lead = {}, {}, {}
+    for i, (name, kms) in enumerate(trace.kernels()):
+        count[name] = count.get(name, 0) + 1
+        kern.setdefault(name, [])
+        if i > 0:
+            kern[name].append(kms)
+        else:
+            lead[name] = kms
+    kernels = {}
+    for name, v in kern.items():
+        per = float(np.mean(v)) if v else float(lead[name])  # one launch only: keep it
+        kernels[name] = {"ms_per_launch": per, "launches_per_step": count[name] / args.steps,
+                         "ms_per_step": per * count[name] / args.steps}
     out = {"wl": wl, "ms": ms_max, "value": wl.B * wl.N * world / (ms_max * 1e-3),
            "kernels_ms": {"rank": float(stage[0]), "compress": float(stage[1]),
                           "layers": stage[2:].tolist()},
