@@ -2,7 +2,7 @@
 
 Small shapes are compared in full; they span several tiles, ragged token
 tails (N not a multiple of S), contraction tails (d not a multiple of 64),
-partial output tiles and k > n-1.  The five named workloads run at full size
+partial output tiles, k > n-1 and sequences shorter than one split.  The five named workloads run at full size
 in the same launch configuration as the benchmark; the oracle checks a seeded
 sample of target splits (a split's scores, selection, compression and layer
 outputs depend only on its own row of scores and its retrieved splits, so the
@@ -119,6 +119,14 @@ SMALL = [
               centers=10, sigma=0.5),
     sy.custom("bf16_s128_k3", B=1, N=2000, S=128, d=256, m=256, k=3, pattern=(sy.DYNAMIC,),
               centers=6, sigma=0.5),
+    # sequences shorter than one split (n = 1): no candidate anywhere, eq. 8
+    # keeps the target's own block alone
+    sy.custom("bf16_one_split", B=2, N=40, S=64, d=64, m=128, k=3, pattern=(sy.STATIC, sy.DYNAMIC),
+              centers=2, sigma=0.5),
+    sy.custom("bf16_s16_one_split", B=3, N=16, S=16, d=64, m=128, k=2,
+              pattern=(sy.DYNAMIC, sy.STATIC), centers=2),
+    sy.custom("f32_one_split", B=1, N=5, S=8, d=32, m=48, m_h=24, k=2, pattern=(sy.DYNAMIC,),
+              dtype="f32"),
 ]
 
 
@@ -128,8 +136,13 @@ def test_small_shapes_full(wl, cuda_dev):
     compare(wl, E, W, orc.all_targets(wl.B, wl.n), cuda_dev)
 
 
+def _small(name):
+    return next(w for w in SMALL if w.name == name)
+
+
 def test_rank_scores_optional_and_padding(cuda_dev):
-    wl = SMALL[-1]
+    wl = _small("bf16_k_gt_n")  # k > n - 1: the lists end in padding
+    assert wl.k > wl.n - 1
     E = sy.gen_embeddings(wl)
     x = torch.from_numpy(E.X).to(cuda_dev, dtype=torch.bfloat16)
     i1, w1 = av.avey_rank(x, wl.S, wl.k)
@@ -196,7 +209,7 @@ def test_dynamic_mix_entry_point(dtype, S, cuda_dev):
 
 def test_kernels_launched_through_the_library(cuda_dev):
     before = av.kernel_launches()
-    wl = SMALL[2]
+    wl = _small("bf16_s16")
     E, W = sy.gen_embeddings(wl), sy.gen_weights(wl)
     run_gpu(wl, E, W, orc.all_targets(1, 2), cuda_dev)
     # rank: normalize + maxsim + topk; compress; per layer: enrich + mix + fuse

@@ -337,6 +337,23 @@ def test_forward_matches_bruteforce_end_to_end():
         np.testing.assert_allclose(res["layers"][-1][r], np.array(x), rtol=1e-10, atol=1e-10)
 
 
+@pytest.mark.parametrize("N,S", [(5, 8), (8, 8), (40, 64)])
+def test_sequence_shorter_than_one_split_has_no_candidates(N, S):
+    # n = 1: the only split is the target itself, which never selects itself;
+    # every slot is empty (index -1, weight 0) and eq. 8 keeps only the
+    # target's own block: P_0 X_t + X_t over the zero-padded split
+    w = sy.custom(B=2, N=N, S=S, d=8, m=16, k=3, pattern=(sy.DYNAMIC,), dtype="f32", centers=2)
+    E, W = sy.gen_embeddings(w), sy.gen_weights(w)
+    res = orc.forward(E.X, W, w)
+    assert res["idx"].tolist() == [[-1] * 3] * 2
+    assert not res["w"].any()
+    X = np.zeros((w.B, S, w.d))
+    X[:, :N] = E.X
+    P0 = W.P.astype(np.float64)[:, :S]
+    want = np.stack([P0 @ X[b] + X[b] for b in range(w.B)])
+    np.testing.assert_allclose(res["compressed"].reshape(want.shape), want, rtol=1e-12, atol=1e-12)
+
+
 def test_large_stack_needs_prenorm():
     """The literal residual stack overflows within 12 layers at the large
     workload's shapes; the prenorm reading keeps it finite."""
