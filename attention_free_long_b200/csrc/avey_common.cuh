@@ -110,14 +110,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed
+// sleeps until it does or until kWaitSuspendNs pass, instead of returning at
+// once and taking issue slots from the warps it waits for.
+constexpr uint32_t kWaitSuspendNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(kWaitSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase with the given parity of barrier `bar` completes.
-// Returns false if `*abort` becomes non-zero or `limit_ns` expires.
+// Returns false if `*abort` becomes non-zero or `limit_ns` expires (checked
+// every 128 tries, so within about 128 suspend hints of the limit).
 __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, volatile int *abort,
                                                 uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity)) return true;
     if ((it & 127u) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) return false;
