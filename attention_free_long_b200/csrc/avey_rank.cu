@@ -11,8 +11,9 @@
 //   maxsim_f32       SIMT fp32 version (one CTA per target/candidate pair).
 //   topk_warp        one warp per target split, one pass over its score row
 //                    keeping a warp-wide sorted list of the k best, order
-//                    (score desc, index asc), self excluded, then
-//                    w_r = s_r / s_1 with IEEE division (s_1 / s_1 == 1).
+//                    (score desc, index asc), self excluded, behind a bar
+//                    seeded from the first batch, then w_r = s_r / s_1 with
+//                    IEEE division (s_1 / s_1 == 1).
 #include <algorithm>
 
 #include "avey_common.cuh"
@@ -206,12 +207,14 @@ constexpr int kTopkWarps = 8;
 // list's k-th key; the (rare, about k ln(n/k) per row) elements that beat it
 // are inserted one at a time, warp-wide: lanes behind the insertion point take
 // their predecessor's entry.  Self, and c > t for the unidirectional ranker,
-// never enter; -inf and NaN scores never beat the empty list's -inf.
+// never enter; -inf and NaN scores never beat the empty list's -inf.  Five
+// blocks stay resident per SM (at most 48 registers), which a score matrix
+// far past L2 needs to keep HBM busy.
 __device__ __forceinline__ bool key_gt(float a, int ia, float b, int ib) {
   return a > b || (a == b && ia < ib);
 }
 
-__global__ void __launch_bounds__(kTopkWarps * 32)
+__global__ void __launch_bounds__(kTopkWarps * 32, 5)
     topk_warp(const float *__restrict__ scores, int B, int n, int t0, int nr, int k, int causal,
               int vec4, int32_t *__restrict__ idx, float *__restrict__ w) {
   // rows of this launch: targets t0 .. t0+nr-1 of every sequence; outputs are
@@ -225,8 +228,10 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
   const int lim = causal ? t : n;  // candidates c < lim, c != t
   float lv = -INFINITY;  // this lane's list entry (q = lane)
   int lc = 0x7fffffff;
-  float tv = -INFINITY;  // the k-th entry: the bar a new candidate must clear
-  int tc = 0x7fffffff;
+  float tv = -INFINITY;  // the bar a new candidate must clear: the list's k-th
+  int tc = 0x7fffffff;   // entry, or the seed while the list is not yet full
+  float sv = -INFINITY;  // the seed bar (see seed below)
+  int sc = 0x7fffffff;
   auto consider = [&](float v, int c) {
     const bool ok = c < lim && c != t && key_gt(v, c, tv, tc);
     unsigned mask = __ballot_sync(0xffffffffu, ok);
@@ -246,8 +251,47 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
         lv = pv;
         lc = pc;
       }
-      tv = __shfl_sync(0xffffffffu, lv, k - 1);
-      tc = __shfl_sync(0xffffffffu, lc, k - 1);
+      const float kv = __shfl_sync(0xffffffffu, lv, k - 1);
+      const int kc = __shfl_sync(0xffffffffu, lc, k - 1);
+      // every entry cleared the seed, so a full list's k-th is at least the seed
+      if (key_gt(kv, kc, sv, sc)) {
+        tv = kv;
+        tc = kc;
+      }
+    }
+  };
+  // The seed: every lane offers its best candidate of the first batch, a
+  // bitonic network sorts the 32 offers (key order, descending) and the k-th
+  // becomes the bar.  k distinct candidates are at least that good, so nothing
+  // below it can be chosen; without it the empty list takes nearly every
+  // element of the first batch one warp-wide insertion at a time.  The bar is
+  // set just below the seed's own key, so the seed itself still enters.
+  auto seed = [&](float bv, int bc) {
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, stride);
+        const int oc = __shfl_xor_sync(0xffffffffu, bc, stride);
+        const bool desc = (lane & size) == 0 || size == 32;
+        const bool keep_greater = desc == ((lane & stride) == 0);
+        if (keep_greater == key_gt(ov, oc, bv, bc)) {
+          bv = ov;
+          bc = oc;
+        }
+      }
+    }
+    const float kv = __shfl_sync(0xffffffffu, bv, k - 1);
+    const int kc = __shfl_sync(0xffffffffu, bc, k - 1);
+    if (kc != 0x7fffffff) {  // k real offers: the k-th is a valid bar
+      sv = tv = kv;
+      sc = tc = kc + 1;
+    }
+  };
+  auto offer = [&](float v, int c, float &bv, int &bc) {
+    if (c < lim && c != t && key_gt(v, c, bv, bc)) {
+      bv = v;
+      bc = c;
     }
   };
   if (vec4) {
@@ -260,6 +304,19 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
       for (int u = 0; u < 4; ++u) {
         const int g = g0 + 32 * u + lane;
         v[u] = g < n4 ? __ldg(s4 + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+      if (g0 == 0) {
+        float bv = -INFINITY;
+        int bc = 0x7fffffff;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = 4 * (32 * u + lane);
+          offer(v[u].x, c, bv, bc);
+          offer(v[u].y, c + 1, bv, bc);
+          offer(v[u].z, c + 2, bv, bc);
+          offer(v[u].w, c + 3, bv, bc);
+        }
+        seed(bv, bc);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -282,6 +339,13 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
       for (int u = 0; u < 4; ++u) {
         const int c = c0 + 32 * u + lane;
         v[u] = c < lim ? __ldg(src + c) : -INFINITY;
+      }
+      if (c0 == 0) {
+        float bv = -INFINITY;
+        int bc = 0x7fffffff;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) offer(v[u], 32 * u + lane, bv, bc);
+        seed(bv, bc);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) consider(v[u], c0 + 32 * u + lane);
