@@ -15,13 +15,15 @@
 // epilogue writes fp32 and/or the split pair straight to global memory (per
 // token, the warp's 32 lanes store 32 consecutive features), so that all of
 // shared memory but the identity (and, for S = 64 with k + 1 <= 8, all of P,
-// 64 KB, loaded once) goes to the ring of loads: nine stages of 16 KB (X
-// alone) for S = 64 with P resident, else eight of 24 KB, three of 64 KB for
-// S = 128.
-// The kernel is bound by HBM and by how many bytes of gathered blocks are in
-// flight.  Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue,
-// warps 2-9 epilogue (two per TMEM lane quarter = 32 features, each on half of
-// the split's S tokens).  Every wait is bounded.
+// 64 KB, loaded once) goes to the ring of loads.  A stage holds a group of
+// consecutive present blocks of one tile, two for S = 64 and one for S = 128:
+// the single MMA-issuing thread pays a fixed cost per stage (its waits, fence,
+// first MMA and commits) that exceeds the tensor time of a 16 KB block, so a
+// pair of blocks per stage halves it.  Four stages of 32 KB (X alone) for
+// S = 64 with P resident, else four of 48 KB; three of 64 KB for S = 128.
+// Roles: warp 0 TMA producer, warp 1 TMEM allocation and MMA issue, warps 2-9
+// epilogue (two per TMEM lane quarter = 32 features, each on half of the
+// split's S tokens).  Every wait is bounded.
 #include <algorithm>
 
 #include "avey_common.cuh"
@@ -46,14 +48,22 @@ struct CompLayout {
   // carries its block's P_r.
   static constexpr bool PRES = S == 64 && KM == 8;
   static constexpr uint32_t PRES_BYTES = PRES ? KM * PBOX : 0;
-  static constexpr uint32_t STAGE = XB + (PRES ? 0 : PCH * PBOX);
-  static constexpr int STAGES = PRES ? 9 : (S == 64 ? 8 : 3);
+  // A stage holds a group of G consecutive present blocks of one tile (the
+  // last group of a tile may hold fewer): every per-stage cost of the single
+  // MMA-issuing thread (its waits, fence and commits) is paid once per group.
+  // S = 128 blocks are too large for two per stage.
+  static constexpr int G = S == 64 ? 2 : 1;
+  static constexpr uint32_t SLOT = XB + (PRES ? 0 : PCH * PBOX);  // one block of a stage
+  static constexpr uint32_t STAGE = G * SLOT;
+  static constexpr int STAGES = S == 64 ? 4 : 3;
   static constexpr int NACC = 512 / S;           // TMEM buffers of S columns
+  static constexpr int NGRP = NACC / G;          // groups of buffers in flight
   static constexpr int TOK = S / 2;              // tokens per epilogue warp
   static constexpr uint32_t CTRL = 1024;
   static constexpr uint32_t SMEM = STAGES * STAGE + PRES_BYTES + C_IDENT + CTRL + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(STAGES <= 16 && NACC <= 8, "the control block holds 16 stages and 8 buffers");
+  static_assert(G == 1 || TOK == 32, "the epilogue reads a pair of blocks with one wait");
 };
 
 struct CompArgs {
@@ -157,7 +167,7 @@ __global__ void __launch_bounds__(C_THR, 1)
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int i = 0; i < L::NACC; ++i) {
+    for (int i = 0; i < L::NGRP; ++i) {
       mbar_init(tfull_bar(i), 1);
       mbar_init(tempty_bar(i), C_EPI);
     }
@@ -239,22 +249,42 @@ __global__ void __launch_bounds__(C_THR, 1)
           list_w[slot * KM + r] = wl[r];
         }
         mbar_arrive(lfull_bar(slot));
+        uint32_t left = 0;  // the tile's present blocks
+#pragma unroll
+        for (int r = 0; r < KM; ++r) left |= (cl[r] >= 0 ? 1u : 0u) << r;
 #pragma unroll 1
-        for (int r = 0; r <= a.k && r < KM; ++r) {
-          const int c = list_c[slot * KM + r];
-          if (c < 0) continue;
+        while (left != 0u) {
+          // the next group: up to G present blocks in rank order
+          int rg[L::G];
+          int nb = 0;
+#pragma unroll
+          for (int j = 0; j < L::G; ++j) {
+            rg[j] = -1;
+            if (left != 0u) {
+              rg[j] = __ffs(static_cast<int>(left)) - 1;
+              left &= left - 1u;
+              ++nb;
+            }
+          }
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           const uint32_t st = sbase + stage * L::STAGE;
-          mbar_arrive_expect_tx(full_bar(stage), L::STAGE);
-          tma_load_3d(st, &tmX, full_bar(stage), slab * CF, c * S, b);
-          tma_load_3d(st + L::XBOX, &tmX, full_bar(stage), slab * CF + 64, c * S, b);
-          if constexpr (!L::PRES) {
+          mbar_arrive_expect_tx(full_bar(stage), static_cast<uint32_t>(nb) * L::SLOT);
 #pragma unroll
-            for (int ch = 0; ch < L::PCH; ++ch)
-              tma_load_3d(st + L::XB + ch * L::PBOX, &tmP, full_bar(stage), r * S + ch * 64, 0, 0);
+          for (int j = 0; j < L::G; ++j) {
+            if (rg[j] < 0) continue;
+            const int r = rg[j];
+            const int c = list_c[slot * KM + r];
+            const uint32_t sl = st + j * L::SLOT;
+            tma_load_3d(sl, &tmX, full_bar(stage), slab * CF, c * S, b);
+            tma_load_3d(sl + L::XBOX, &tmX, full_bar(stage), slab * CF + 64, c * S, b);
+            if constexpr (!L::PRES) {
+#pragma unroll
+              for (int ch = 0; ch < L::PCH; ++ch)
+                tma_load_3d(sl + L::XB + ch * L::PBOX, &tmP, full_bar(stage), r * S + ch * 64, 0, 0);
+            }
           }
           ++issued;
           if (++stage == L::STAGES) {
@@ -280,8 +310,8 @@ __global__ void __launch_bounds__(C_THR, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(CF, S) | (1u << 15);       // A is MN-major
       const uint32_t idesc_res = idesc_bf16_f32(CF, 64) | (1u << 15);  // residual, 64 tokens
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int stage = 0, grp = 0;
+      uint32_t phase = 0, grp_phase = 0;
       bool ok = true;
       int it = 0;
       if constexpr (L::PRES) ok = mbar_wait(pready_bar, 0, abort_flag);
@@ -291,46 +321,60 @@ __global__ void __launch_bounds__(C_THR, 1)
           ok = false;
           break;
         }
-        uint32_t mask = 0;  // blocks present
+        uint32_t left = 0;  // blocks present
 #pragma unroll
-        for (int r = 0; r < KM; ++r) mask |= (list_c[slot * KM + r] >= 0 ? 1u : 0u) << r;
+        for (int r = 0; r < KM; ++r) left |= (list_c[slot * KM + r] >= 0 ? 1u : 0u) << r;
         mbar_arrive(lempty_bar(slot));
 #pragma unroll 1
-        for (int r = 0; r <= a.k && r < KM; ++r) {
-          if (!((mask >> r) & 1u)) continue;
-          if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag) ||
+        while (left != 0u) {
+          int rg[L::G];  // the group: the producer's pairing of the same present blocks
+#pragma unroll
+          for (int j = 0; j < L::G; ++j) {
+            rg[j] = -1;
+            if (left != 0u) {
+              rg[j] = __ffs(static_cast<int>(left)) - 1;
+              left &= left - 1u;
+            }
+          }
+          if (!mbar_wait(tempty_bar(grp), grp_phase ^ 1u, abort_flag) ||
               !mbar_wait(full_bar(stage), phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t st = sbase + stage * L::STAGE;
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S);
-          // 16 tokens j a step: +2048 bytes (two 8-token atoms) along X's
-          // MN-major rows; +32 bytes along P_r's K-major rows, P box every 64 j
 #pragma unroll
-          for (int kk = 0; kk < S / 16; ++kk) {
-            const uint32_t pb = L::PRES ? pbase + r * L::PBOX : st + L::XB + (kk >> 2) * L::PBOX;
-            tc_mma_bf16(d_tmem, cdesc_mn(st + 2048u * kk, L::XBOX), cdesc_k(pb + 32u * (kk & 3)),
-                        idesc, kk != 0);
-          }
-          if (r == 0) {  // + X_t^T: the residual, one 64-token half at a time
+          for (int j = 0; j < L::G; ++j) {
+            if (rg[j] < 0) continue;
+            const int r = rg[j];
+            const uint32_t sl = st + j * L::SLOT;
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((grp * L::G + j) * S);
+            // 16 tokens j a step: +2048 bytes (two 8-token atoms) along X's
+            // MN-major rows; +32 bytes along P_r's K-major rows, P box every 64 j
 #pragma unroll
-            for (int hh = 0; hh < S / 64; ++hh)
+            for (int kk = 0; kk < S / 16; ++kk) {
+              const uint32_t pb = L::PRES ? pbase + r * L::PBOX : sl + L::XB + (kk >> 2) * L::PBOX;
+              tc_mma_bf16(d_tmem, cdesc_mn(sl + 2048u * kk, L::XBOX), cdesc_k(pb + 32u * (kk & 3)),
+                          idesc, kk != 0);
+            }
+            if (r == 0) {  // + X_t^T: the residual, one 64-token half at a time
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                tc_mma_bf16(d_tmem + 64u * hh, cdesc_mn(st + 8192u * hh + 2048u * kk, L::XBOX),
-                            cdesc_k(ibase + 32u * kk), idesc_res, 1u);
+              for (int hh = 0; hh < S / 64; ++hh)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  tc_mma_bf16(d_tmem + 64u * hh, cdesc_mn(sl + 8192u * hh + 2048u * kk, L::XBOX),
+                              cdesc_k(ibase + 32u * kk), idesc_res, 1u);
+            }
           }
           tc_commit(empty_bar(stage));
-          tc_commit(tfull_bar(acc));
+          tc_commit(tfull_bar(grp));
           if (++stage == L::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
-          if (++acc == L::NACC) {
-            acc = 0;
-            acc_phase ^= 1u;
+          if (++grp == L::NGRP) {
+            grp = 0;
+            grp_phase ^= 1u;
           }
         }
       }
@@ -346,8 +390,8 @@ __global__ void __launch_bounds__(C_THR, 1)
     constexpr int TOK = L::TOK;
     const int quarter = warp & 3;      // TMEM lanes = features 32*quarter .. +31 of the slab
     const int half = (warp - 2) >> 2;  // TMEM columns = tokens TOK*half .. +TOK-1 of the split
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    int grp = 0;
+    uint32_t grp_phase = 0;
     bool ok = true;
     int it = 0;
     for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x, ++it) {
@@ -366,54 +410,52 @@ __global__ void __launch_bounds__(C_THR, 1)
       for (int i = 0; i < TOK; ++i) o[i] = 0.f;
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
       const uint32_t col = static_cast<uint32_t>(half * TOK) + lane_off;
-      auto take = [&]() {  // the next accumulator in the MMA issuer's order
-        const uint32_t t = static_cast<uint32_t>(acc);
-        if (++acc == L::NACC) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
-        return t;
-      };
-      uint32_t left = mask;  // present blocks not yet added
+      uint32_t left = mask;  // present blocks not yet added, taken in the MMA issuer's groups
 #pragma unroll 1
       while (left != 0u && ok) {
         const int r1 = __ffs(static_cast<int>(left)) - 1;
         left &= left - 1u;
         const float w1 = list_w[slot * KM + r1];
-        if (!(ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag))) break;
-        const uint32_t a1 = take();
-        if constexpr (TOK == 32) {
+        int r2 = -1;
+        float w2 = 0.f;
+        if constexpr (L::G == 2) {
           if (left != 0u) {
-            // two blocks per TMEM wait: the second load's latency overlaps the first's
-            const int r2 = __ffs(static_cast<int>(left)) - 1;
+            r2 = __ffs(static_cast<int>(left)) - 1;
             left &= left - 1u;
-            const float w2 = list_w[slot * KM + r2];
-            if (!(ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag))) break;
-            const uint32_t a2 = take();
-            tc_fence_after();
+            w2 = list_w[slot * KM + r2];
+          }
+        }
+        if (!(ok = mbar_wait(tfull_bar(grp), grp_phase, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t t1 = tmem_base + static_cast<uint32_t>(grp * L::G * S) + col;
+        const int g = grp;
+        if (++grp == L::NGRP) {
+          grp = 0;
+          grp_phase ^= 1u;
+        }
+        if constexpr (L::G == 2) {
+          if (r2 >= 0) {
+            // both blocks of the group with one wait: the second load's latency
+            // overlaps the first's
             float v1[32], v2[32];
-            tmem_ld32x2(tmem_base + a1 * S + col, tmem_base + a2 * S + col, v1, v2);
+            tmem_ld32x2(t1, t1 + S, v1, v2);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-              mbar_arrive(tempty_bar(static_cast<int>(a1)));
-              mbar_arrive(tempty_bar(static_cast<int>(a2)));
-            }
+            if (lane == 0) mbar_arrive(tempty_bar(g));
 #pragma unroll
             for (int i = 0; i < TOK; ++i) o[i] = fmaf(w2, v2[i], fmaf(w1, v1[i], o[i]));
             continue;
           }
         }
-        tc_fence_after();
         float v[TOK];
         if constexpr (TOK == 64) {
-          tmem_ld64(tmem_base + a1 * S + col, v);
+          tmem_ld64(t1, v);
         } else {
-          tmem_ld32(tmem_base + a1 * S + col, v);
+          tmem_ld32(t1, v);
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(static_cast<int>(a1)));
+        if (lane == 0) mbar_arrive(tempty_bar(g));
 #pragma unroll
         for (int i = 0; i < TOK; ++i) o[i] = fmaf(w1, v[i], o[i]);
       }
