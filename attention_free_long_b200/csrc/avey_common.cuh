@@ -347,8 +347,8 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // TMA load into this CTA's shared memory whose completion is counted on a
-// barrier of either CTA of the pair (bar is a shared::cluster address).  No
-// multicast.
+// barrier of either CTA of the pair (bar is a shared::cluster address).  It
+// fills only the issuing CTA's own shared memory.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                                  int x, int y, int z) {
   asm volatile(

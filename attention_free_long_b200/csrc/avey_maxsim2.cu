@@ -22,7 +22,8 @@
 //   * Barriers: each CTA's loads complete on CTA 0's "full" barrier; the MMA
 //     commit frees the stage in both CTAs and publishes the accumulator to
 //     both; both CTAs' epilogue warps release the accumulator to CTA 0.
-//     Every wait is bounded (avey_common.cuh); no load uses multicast.
+//     Every wait is bounded (avey_common.cuh); every load fills only the
+//     issuing CTA's own shared memory.
 //   * Tiles are visited in groups of 32 row blocks (the group's rows stay in
 //     L2 while its column blocks stream past); a launch may compute only the
 //     tiles t with t % nparts == part (one long sequence across GPUs).

@@ -599,8 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 //
 // Barriers: both CTAs' loads complete on CTA 0's "full" barrier; the MMA
 // commit frees the stage in both CTAs and publishes the accumulator to both;
-// both CTAs' epilogue warps release the accumulator to CTA 0.  No load uses
-// multicast.
+// both CTAs' epilogue warps release the accumulator to CTA 0.  Every load
+// fills only the issuing CTA's own shared memory.
 
 struct PairLayout {
   static constexpr int PM = 256;                        // rows per pair tile
