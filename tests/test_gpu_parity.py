@@ -119,6 +119,13 @@ SMALL = [
               centers=10, sigma=0.5),
     sy.custom("bf16_s128_k3", B=1, N=2000, S=128, d=256, m=256, k=3, pattern=(sy.DYNAMIC,),
               centers=6, sigma=0.5),
+    # an odd number of blocks per tile at S = 64, where compression takes the
+    # blocks two per ring stage: the last group holds one block (P resident
+    # for k + 1 = 5, streamed per block for k + 1 = 11)
+    sy.custom("bf16_s64_k4", B=2, N=1300, S=64, d=128, m=256, k=4, pattern=(sy.STATIC, sy.DYNAMIC),
+              centers=8, sigma=0.5),
+    sy.custom("bf16_s64_k10", B=1, N=1500, S=64, d=192, m=256, k=10, pattern=(sy.DYNAMIC,),
+              centers=6, sigma=0.5),
     # sequences shorter than one split (n = 1): no candidate anywhere, eq. 8
     # keeps the target's own block alone
     sy.custom("bf16_one_split", B=2, N=40, S=64, d=64, m=128, k=3, pattern=(sy.STATIC, sy.DYNAMIC),
