@@ -189,16 +189,19 @@ def l2_note(wl) -> str:
 
 # ----------------------------------------------------------- CPU baseline ---
 
-def cpu_baseline(wl, E, W, budget_s: float = 15.0, max_splits: int = 64):
+def cpu_baseline(wl, E, W, budget_s: float = 12.0, max_splits: int = 256):
     """The fp64 oracle as it stands, on this host's cores, on a bounded sample
-    of target splits of the same workload (rank, compression, every layer)."""
+    of target splits of the same workload (rank, compression, every layer),
+    sized to about budget_s of wall time from a batch of 8 splits run the
+    same way."""
     import oracle as orc
     X64 = E.X.astype(np.float64)
     one = sy.sample_targets(wl, 1, seed=100)[:1]
+    cal = sy.sample_targets(wl, 8, seed=99)[:8]
     t0 = time.perf_counter()
-    orc.forward(X64, W, wl, sel=one)
-    t_one = time.perf_counter() - t0
-    count = int(max(1, min(max_splits, budget_s / max(t_one, 1e-3))))
+    orc.forward(X64, W, wl, sel=cal)
+    per = (time.perf_counter() - t0) / cal.shape[0]
+    count = int(max(1, min(max_splits, budget_s / max(per, 1e-3))))
     sel = sy.sample_targets(wl, count, seed=101)[:count]
     t0 = time.perf_counter()
     orc.forward(X64, W, wl, sel=sel)
