@@ -59,7 +59,8 @@ struct CompLayout {
   static constexpr int NACC = 512 / S;           // TMEM buffers of S columns
   static constexpr int NGRP = NACC / G;          // groups of buffers in flight
   static constexpr int TOK = S / 2;              // tokens per epilogue warp
-  static constexpr uint32_t CTRL = 1024;
+  // barriers and flags in the first 512 bytes, then two block lists of KM (split, weight)
+  static constexpr uint32_t CTRL = (512 + 2 * KM * 8 + 1023) / 1024 * 1024;
   static constexpr uint32_t SMEM = STAGES * STAGE + PRES_BYTES + C_IDENT + CTRL + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(STAGES <= 16 && NACC <= 8, "the control block holds 16 stages and 8 buffers");
@@ -249,9 +250,9 @@ __global__ void __launch_bounds__(C_THR, 1)
           list_w[slot * KM + r] = wl[r];
         }
         mbar_arrive(lfull_bar(slot));
-        uint32_t left = 0;  // the tile's present blocks
+        uint64_t left = 0;  // the tile's present blocks (k + 1 <= 33)
 #pragma unroll
-        for (int r = 0; r < KM; ++r) left |= (cl[r] >= 0 ? 1u : 0u) << r;
+        for (int r = 0; r < KM; ++r) left |= (cl[r] >= 0 ? 1ull : 0ull) << r;
 #pragma unroll 1
         while (left != 0u) {
           // the next group: up to G present blocks in rank order
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(C_THR, 1)
           for (int j = 0; j < L::G; ++j) {
             rg[j] = -1;
             if (left != 0u) {
-              rg[j] = __ffs(static_cast<int>(left)) - 1;
+              rg[j] = __ffsll(static_cast<long long>(left)) - 1;
               left &= left - 1u;
               ++nb;
             }
@@ -321,9 +322,9 @@ __global__ void __launch_bounds__(C_THR, 1)
           ok = false;
           break;
         }
-        uint32_t left = 0;  // blocks present
+        uint64_t left = 0;  // blocks present
 #pragma unroll
-        for (int r = 0; r < KM; ++r) left |= (list_c[slot * KM + r] >= 0 ? 1u : 0u) << r;
+        for (int r = 0; r < KM; ++r) left |= (list_c[slot * KM + r] >= 0 ? 1ull : 0ull) << r;
         mbar_arrive(lempty_bar(slot));
 #pragma unroll 1
         while (left != 0u) {
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(C_THR, 1)
           for (int j = 0; j < L::G; ++j) {
             rg[j] = -1;
             if (left != 0u) {
-              rg[j] = __ffs(static_cast<int>(left)) - 1;
+              rg[j] = __ffsll(static_cast<long long>(left)) - 1;
               left &= left - 1u;
             }
           }
@@ -402,25 +403,25 @@ __global__ void __launch_bounds__(C_THR, 1)
         ok = false;
         break;
       }
-      uint32_t mask = 0;
+      uint64_t mask = 0;
 #pragma unroll 1
-      for (int r = 0; r <= a.k && r < KM; ++r) mask |= (list_c[slot * KM + r] >= 0 ? 1u : 0u) << r;
+      for (int r = 0; r <= a.k && r < KM; ++r) mask |= (list_c[slot * KM + r] >= 0 ? 1ull : 0ull) << r;
       float o[TOK];
 #pragma unroll
       for (int i = 0; i < TOK; ++i) o[i] = 0.f;
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
       const uint32_t col = static_cast<uint32_t>(half * TOK) + lane_off;
-      uint32_t left = mask;  // present blocks not yet added, taken in the MMA issuer's groups
+      uint64_t left = mask;  // present blocks not yet added, taken in the MMA issuer's groups
 #pragma unroll 1
       while (left != 0u && ok) {
-        const int r1 = __ffs(static_cast<int>(left)) - 1;
+        const int r1 = __ffsll(static_cast<long long>(left)) - 1;
         left &= left - 1u;
         const float w1 = list_w[slot * KM + r1];
         int r2 = -1;
         float w2 = 0.f;
         if constexpr (L::G == 2) {
           if (left != 0u) {
-            r2 = __ffs(static_cast<int>(left)) - 1;
+            r2 = __ffsll(static_cast<long long>(left)) - 1;
             left &= left - 1u;
             w2 = list_w[slot * KM + r2];
           }
@@ -517,7 +518,8 @@ avey_status run_compress_tc_k(int k, const CUtensorMap &mx, const CUtensorMap &m
                               const CompArgs &a, int grid, cudaStream_t s) {
   if (k + 1 <= 8) return run_compress_tc<S, 8>(mx, mp, a, grid, s);
   if (k + 1 <= 16) return run_compress_tc<S, 16>(mx, mp, a, grid, s);
-  return run_compress_tc<S, 32>(mx, mp, a, grid, s);
+  if (k + 1 <= 32) return run_compress_tc<S, 32>(mx, mp, a, grid, s);
+  return run_compress_tc<S, 33>(mx, mp, a, grid, s);  // k = 32: the target and 32 candidates
 }
 
 }  // namespace

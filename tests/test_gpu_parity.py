@@ -126,6 +126,12 @@ SMALL = [
               centers=8, sigma=0.5),
     sy.custom("bf16_s64_k10", B=1, N=1500, S=64, d=192, m=256, k=10, pattern=(sy.DYNAMIC,),
               centers=6, sigma=0.5),
+    # the largest k the ranker takes: 33 blocks per target (the target and 32
+    # candidates) for compression
+    sy.custom("bf16_s64_k32", B=1, N=2560, S=64, d=64, m=128, k=32, pattern=(sy.DYNAMIC,),
+              centers=4, sigma=0.5),
+    sy.custom("bf16_s128_k32", B=1, N=4608, S=128, d=128, m=256, k=32, pattern=(sy.STATIC,),
+              centers=4, sigma=0.5),
     # sequences shorter than one split (n = 1): no candidate anywhere, eq. 8
     # keeps the target's own block alone
     sy.custom("bf16_one_split", B=2, N=40, S=64, d=64, m=128, k=3, pattern=(sy.STATIC, sy.DYNAMIC),
