@@ -132,6 +132,16 @@ SMALL = [
               centers=4, sigma=0.5),
     sy.custom("bf16_s128_k32", B=1, N=4608, S=128, d=128, m=256, k=32, pattern=(sy.STATIC,),
               centers=4, sigma=0.5),
+    # 16 < k + 1 <= 32 (the 32-block lists) at S = 64 and 128, and large k on
+    # the smaller splits' kernel
+    sy.custom("bf16_s64_k20", B=1, N=1920, S=64, d=128, m=256, k=20, pattern=(sy.STATIC,),
+              centers=4, sigma=0.5),
+    sy.custom("bf16_s128_k24", B=1, N=3840, S=128, d=128, m=256, k=24, pattern=(sy.DYNAMIC,),
+              centers=4, sigma=0.5),
+    sy.custom("bf16_s32_k32", B=1, N=1280, S=32, d=96, m=192, m_h=64, k=32, pattern=(sy.DYNAMIC,),
+              centers=4, sigma=0.5),
+    sy.custom("bf16_s16_k20", B=2, N=480, S=16, d=64, m=128, k=20, pattern=(sy.STATIC,),
+              centers=4, sigma=0.4),
     # sequences shorter than one split (n = 1): no candidate anywhere, eq. 8
     # keeps the target's own block alone
     sy.custom("bf16_one_split", B=2, N=40, S=64, d=64, m=128, k=3, pattern=(sy.STATIC, sy.DYNAMIC),
