@@ -142,6 +142,14 @@ SMALL = [
               centers=4, sigma=0.5),
     sy.custom("bf16_s16_k20", B=2, N=480, S=16, d=64, m=128, k=20, pattern=(sy.STATIC,),
               centers=4, sigma=0.4),
+    # the narrowest widths the layer takes: an 8-feature head, an 8-feature
+    # tail (the contextualized part), and d = 8
+    sy.custom("bf16_head8", B=1, N=700, S=64, d=64, m=144, m_h=8, k=3,
+              pattern=(sy.STATIC, sy.DYNAMIC), centers=4, sigma=0.5),
+    sy.custom("bf16_tail8", B=1, N=700, S=32, d=64, m=72, m_h=64, k=3,
+              pattern=(sy.DYNAMIC, sy.STATIC), centers=4, sigma=0.5),
+    sy.custom("bf16_d8", B=1, N=300, S=16, d=8, m=16, m_h=8, k=2, pattern=(sy.DYNAMIC,),
+              centers=3, sigma=0.4),
     # sequences shorter than one split (n = 1): no candidate anywhere, eq. 8
     # keeps the target's own block alone
     sy.custom("bf16_one_split", B=2, N=40, S=64, d=64, m=128, k=3, pattern=(sy.STATIC, sy.DYNAMIC),
