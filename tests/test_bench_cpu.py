@@ -32,3 +32,25 @@ def test_hbm_byte_counts():
     h = bench._hbm(2.0, 4e9, 8000.0)
     assert abs(h["gbs"] - 2000.0) < 1e-9 and abs(h["frac"] - 0.25) < 1e-12
     assert bench._hbm(None, 1.0, 1.0) is None
+
+
+def test_reference_arm_prints_the_contract_line():
+    # the reference arm (the fp64 oracle on the host cores) as the driver runs
+    # it, on the smallest workload: one JSON line with the contract's keys
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3",
+                        "--workload", "tiny_f32"], cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 2
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert "tiny_f32" in line["config"]["workload"]
