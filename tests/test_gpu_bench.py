@@ -43,3 +43,18 @@ def test_bench_line_carries_the_contract(cuda_dev):
     hbm = line["hbm"]
     assert hbm["compress"]["frac"] > 0 and hbm["compress"]["in_forward"]["frac"] > 0
     assert hbm["dynamic_mix"]["frac"] > 0 and hbm["topk_sweep"]["frac"] > 0
+
+
+def test_sequence_sharded_bench_line(cuda_dev):
+    # --shard sequence at one rank: the same path the multi-GPU run takes (the
+    # score all-reduce is a no-op), with its own JSON line
+    r = subprocess.run([sys.executable, "bench.py", "--shard", "sequence", "--workload", "base_bf16",
+                        "--steps", "3", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stderr[-3000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "scaling", "e2e",
+                "config"):
+        assert key in line, key
+    assert line["n_gpus"] == 1 and line["value"] > 0 and line["e2e"]["value"] > 0
+    assert line["scaling"] == "strong"
